@@ -1,0 +1,389 @@
+"""Benchmark of the EFLA forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl efla|reference]
+
+One step = one efla_chunk_fwd call over the 1.3B-layer workload (B=4, H=16, T=2048,
+d_k=d_v=128, chunk 64, bf16 in / fp32 state): the gate, the intra-chunk UT transform and
+the inter-chunk state propagation, fused.  Multi-GPU (torchrun, one rank per GPU) is data
+parallel over independent (b, h) streams: every rank runs its own batch with no data-path
+collective (weak scaling); the timing is the max over ranks.  The single-token decode step
+(N=256, H=16, d=128, fp32 state, in place) is measured in the same run and reported under
+"decode".  Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+WORKLOAD = workloads.CHUNK_WORKLOADS["lm1p3b_bf16"]
+DECODE = workloads.DECODE_WORKLOAD
+METRIC = "EFLA fwd tokens/s (B4 H16 T2048 d128 bf16)"
+N_ROTATE = 4            # rotating input sets: 4 x 139 MB > 126 MB L2, so no set is L2-resident
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return 6650.0, 1590.0, "fallback"
+
+
+def chunk_alg(w):
+    """Algorithmic bytes and flops of one forward call.
+
+    Bytes: read q, k, v, beta and write o (2 bytes each) plus S_T (fp32) and S0 if given.
+    Flops per (stream, chunk): KK^T, QK^T, TK, TV, P Delta (5 x 2 C^2 d) and WS, QS, K^T Delta
+    (3 x 2 C d^2), with C = 64, d = d_k = d_v.
+    """
+    es = 2 if w.dtype == torch.bfloat16 else 4
+    BH, T, d = w.B * w.H, w.T, w.dk
+    nbytes = BH * T * (3 * d * es + es + d * es) + BH * d * d * 4
+    if w.s0_std is not None:
+        nbytes += BH * d * d * 4
+    chunks = (T + 63) // 64
+    flops = BH * chunks * (5 * 2 * 64 * 64 * d + 3 * 2 * 64 * d * d)
+    return nbytes, flops
+
+
+def decode_alg(w):
+    """One decode step: read + write the fp32 state, read q, k, v, beta, write o."""
+    NH, d = w.N * w.H, w.dk
+    return NH * (2 * d * d * 4 + (3 * d + 1 + d) * 4), NH * 6 * d * d
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "delta_rule_linear_02_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel: str):
+    """dram bytes per launch recorded in profiles/traffic.md for the current kernel sources."""
+    path = os.path.join(ROOT, "profiles", "traffic.md")
+    try:
+        lines = open(path).read().splitlines()
+    except OSError:
+        return None
+    src = kernel_source_hash()
+    for ln in lines:
+        if ln.startswith("traffic|"):
+            _, name, nbytes, sha = ln.split("|")[:4]
+            if name == kernel and sha.strip() == src:
+                return int(nbytes)
+    return None
+
+
+class Clocks:
+    """SM clock and throttle-reason sampler (NVML, a background thread polling every ~2 ms)
+    running during the timed region."""
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
+
+    def __init__(self, index: int):
+        self.index = index
+        self.samples = []
+        self.max_mhz = None
+        self._stop = None
+
+    def __enter__(self):
+        try:
+            import threading
+            import pynvml
+            pynvml.nvmlInit()
+            h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            self._stop = threading.Event()
+
+            def run():
+                while not self._stop.is_set():
+                    try:
+                        mhz = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+                        rs = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                        self.samples.append((mhz, rs))
+                    except Exception:  # pragma: no cover
+                        pass
+                    time.sleep(0.002)
+
+            self._thread = threading.Thread(target=run, daemon=True)
+            self._thread.start()
+            time.sleep(0.02)
+        except Exception:
+            self._stop = None
+        return self
+
+    def __exit__(self, *exc):
+        if self._stop is not None:
+            self._stop.set()
+            self._thread.join(timeout=5)
+
+    def summary(self):
+        if not self.samples:
+            return None
+        reasons = sorted({n for _, rs in self.samples for n, bit in self.REASONS.items() if rs & bit})
+        return {"sm_mhz": statistics.median(m for m, _ in self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(self.samples), "source": "NVML, ~2 ms polling"}
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return rank, world, local
+
+
+def barrier(world):
+    torch.cuda.synchronize()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def shard_seed(rank: int) -> int:
+    """Each rank draws its own independent batch of streams (weak scaling)."""
+    return WORKLOAD.seed + 1000 * rank
+
+
+def cpu_baseline(w, cpu_seconds: float = 12.0):
+    """The fp64 oracle, as it stands, on the workload's streams: whole passes over all
+    B*H streams, repeated until about `cpu_seconds` of CPU work (wall x threads) is done."""
+    import oracle
+    inp = workloads.make_chunk_inputs(w)
+    threads = oracle.default_threads()
+    passes, t0 = 0, time.perf_counter()
+    while True:
+        oracle.fwd(inp["q"], inp["k"], inp["v"], inp["beta"], inp["S0"], threads=threads)
+        passes += 1
+        dt = time.perf_counter() - t0
+        if dt * threads >= cpu_seconds or dt >= 60.0:
+            break
+    tokens = passes * w.B * w.T                 # a token spans all H heads
+    return {"value": tokens / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{passes} full pass(es) over all {w.B * w.H} (b,h) streams of the workload "
+                      f"(T={w.T}), {dt:.1f} s wall on {threads} threads"}
+
+
+def run_reference(args):
+    """The oracle as the reference arm: rank 0 only, each step a bounded sample."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    w = WORKLOAD
+    streams = 8
+    inp = workloads.make_chunk_inputs(w.replace(B=1, H=streams))
+    threads = oracle.default_threads()
+    for _ in range(args.warmup):
+        oracle.fwd(inp["q"], inp["k"], inp["v"], inp["beta"], inp["S0"], threads=threads)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.fwd(inp["q"], inp["k"], inp["v"], inp["beta"], inp["S0"], threads=threads)
+    dt = (time.perf_counter() - t0) / args.steps
+    tokens = streams * w.T / w.H
+    value = tokens / dt
+    sample = f"{streams} of {w.B * w.H} (b,h) streams at full T={w.T} per step"
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "d_k": w.dk, "d_v": w.dv,
+                   "chunk": w.chunk, "parallelism": f"dp{args.gpus}"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="efla", choices=["efla", "reference"])
+    ap.add_argument("--decode-steps", type=int, default=1000)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    if args.impl == "reference":
+        run_reference(args)
+        return
+
+    import delta_rule_linear_02_b200 as efla
+    rank, world, local = dist_setup(args)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    w = WORKLOAD.replace(seed=shard_seed(rank))
+    hbm, tc, peak_kind = peaks()
+
+    # ---- device-resident inputs: N_ROTATE independent sets, so every step misses L2
+    sets = []
+    for i in range(N_ROTATE):
+        inp = workloads.make_chunk_inputs(w.replace(seed=w.seed + 97 * i))
+        sets.append({k: (None if v is None else v.to(dev)) for k, v in inp.items()})
+    B, H, T, d = w.B, w.H, w.T, w.dk
+    ws = efla.new_workspace(B, H, T, d, d, 64, w.dtype, dev)
+    outs = [(torch.empty(B, H, T, d, dtype=w.dtype, device=dev),
+             torch.empty(B, H, d, d, dtype=torch.float32, device=dev)) for _ in range(N_ROTATE)]
+
+    def step(i):
+        s, (o, ST) = sets[i % N_ROTATE], outs[i % N_ROTATE]
+        efla.efla_chunk_fwd(s["q"], s["k"], s["v"], s["beta"], s["S0"], o=o, S_T=ST,
+                            workspace=ws, stream=stream)
+
+    for i in range(args.warmup):
+        step(i)
+    barrier(world)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * args.steps + 2)]
+    with Clocks(local) as clk:
+        ev[0].record(stream)
+        for i in range(args.steps):
+            ev[2 + 2 * i].record(stream)
+            step(i)
+            ev[3 + 2 * i].record(stream)
+        ev[1].record(stream)
+        barrier(world)
+    total_ms = max_over_ranks(ev[0].elapsed_time(ev[1]), world)
+    launch_ms = statistics.mean(ev[2 + 2 * i].elapsed_time(ev[3 + 2 * i]) for i in range(args.steps))
+    launch_ms = max_over_ranks(launch_ms, world)
+    status = efla.efla_workspace_status(ws, clear=True, stream=stream)
+    if status != efla.EFLA_OK:
+        raise SystemExit(f"device reported {efla.efla_status_string(status)}")
+    ms_per_step = total_ms / args.steps
+    tokens = w.tokens * world
+    value = tokens / (ms_per_step * 1e-3)
+
+    nbytes, flops = chunk_alg(w)
+    achieved = nbytes / (launch_ms * 1e-3) / 1e9
+    t_star = max(nbytes / (hbm * 1e9), flops / (tc * 1e12))
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                "frac": achieved / hbm, "traffic": ncu_traffic("efla_chunk_fwd"),
+                "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
+                "alg_bytes_per_launch": nbytes, "alg_flops_per_launch": flops,
+                "tensor_tflops": flops / (launch_ms * 1e-3) / 1e12,
+                "roofline_time_us": t_star * 1e6, "roofline_frac": t_star / (launch_ms * 1e-3)}
+
+    # ---- end to end through the public API with host buffers (pinned), copies timed
+    host = {k: (None if v is None else v.cpu().pin_memory()) for k, v in sets[0].items()}
+    o_h = torch.empty(B, H, T, d, dtype=w.dtype).pin_memory()
+    ST_h = torch.empty(B, H, d, d, dtype=torch.float32).pin_memory()
+    dbuf = {k: (None if v is None else torch.empty_like(v, device=dev)) for k, v in host.items()}
+    o_d, ST_d = outs[0]
+    h2d = sum(v.numel() * v.element_size() for v in host.values() if v is not None)
+    d2h = o_h.numel() * o_h.element_size() + ST_h.numel() * ST_h.element_size()
+
+    def e2e_step():
+        for k, v in host.items():
+            if v is not None:
+                dbuf[k].copy_(v, non_blocking=True)
+        efla.efla_chunk_fwd(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["beta"], dbuf["S0"], o=o_d,
+                            S_T=ST_d, workspace=ws, stream=stream)
+        o_h.copy_(o_d, non_blocking=True)
+        ST_h.copy_(ST_d, non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 20))
+    for _ in range(3):
+        e2e_step()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    barrier(world)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / e2e_steps
+    e2e = {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+           "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+    del sets, outs, dbuf
+
+    # ---- decode step (N=256, H=16, d=128, fp32 state updated in place)
+    dec = None
+    if args.decode_steps > 0:
+        wd = DECODE.replace(seed=DECODE.seed + 1000 * rank)
+        S = workloads.make_decode_state(wd, device=dev)
+        nd = args.decode_steps
+        st = workloads.make_decode_steps(wd, steps=nd + args.warmup, device=dev)
+        o_dec = torch.empty(wd.N, wd.H, wd.dv, device=dev)
+        for i in range(args.warmup):
+            efla.efla_recurrent_step(st["q"][i], st["k"][i], st["v"][i], st["beta"][i], S, o=o_dec,
+                                     stream=stream)
+        barrier(world)
+        d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        d0.record(stream)
+        for i in range(args.warmup, args.warmup + nd):
+            efla.efla_recurrent_step(st["q"][i], st["k"][i], st["v"][i], st["beta"][i], S, o=o_dec,
+                                     stream=stream)
+        d1.record(stream)
+        barrier(world)
+        dms = max_over_ranks(d0.elapsed_time(d1), world) / nd
+        dbytes, dflops = decode_alg(wd)
+        dach = dbytes / (dms * 1e-3) / 1e9
+        dec = {"metric": "EFLA decode tokens/s (N256 H16 d128 fp32 state, in place)",
+               "value": wd.N * world / (dms * 1e-3), "unit": "tokens/s", "us_per_step": dms * 1e3,
+               "steps": nd, "dtype": "f32",
+               "roofline": {"bound": "hbm", "achieved": dach, "peak": hbm, "unit": "GB/s",
+                            "frac": dach / hbm, "traffic": ncu_traffic("efla_recurrent_step"),
+                            "alg_bytes_per_launch": dbytes},
+               "gpu_launches": nd}
+        del S, st
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(WORKLOAD)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded; q,k unit direction x LogNormal(0,0.5) norm, v~N(0,1), beta=sigmoid(N(0,1)))",
+            "config": {"workload": w.name, "B": B, "H": H, "T": T, "d_k": d, "d_v": d, "chunk": 64,
+                       "global_batch": B * world, "seq_len": T, "parallelism": f"dp{world}",
+                       "l2": f"{N_ROTATE} rotating input sets ({N_ROTATE * nbytes / 1e6:.0f} MB) > 126 MB L2"},
+            "roofline": roofline, "e2e": e2e, "gpu_launches": args.steps,
+            "clocks": clk.summary(), "decode": dec, "cpu_baseline": cpu,
+            "kernel_source": kernel_source_hash(),
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

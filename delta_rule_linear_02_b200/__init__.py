@@ -1,0 +1,168 @@
+"""Python binding of libefla.so, the B200 Exact Flow Linear Attention forward.
+
+Argument marshalling only: every step of the computation runs in the library's CUDA
+kernels.  PyTorch provides device memory and streams.  The names mirror the C ABI of
+include/efla.h.  Importing this package loads the in-tree libefla.so and fails loudly if
+it has not been built (python delta_rule_linear_02_b200/build.py).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libefla.so")
+
+EFLA_OK, EFLA_ERR_INVALID_ARG, EFLA_ERR_UNSUPPORTED, EFLA_ERR_CUDA, EFLA_ERR_TIMEOUT = range(5)
+EFLA_DTYPE_F32, EFLA_DTYPE_BF16 = 0, 1
+CHUNK = 64
+
+_DTYPES = {torch.float32: EFLA_DTYPE_F32, torch.bfloat16: EFLA_DTYPE_BF16}
+
+
+class EflaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {efla_status_string(status)} ({status})")
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libefla.so is not built at {LIB_PATH}; run "
+                          "`python delta_rule_linear_02_b200/build.py` (nvcc, sm_100a)")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, I, L, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_long, ctypes.c_size_t
+    lib.efla_status_string.argtypes = [I]
+    lib.efla_status_string.restype = ctypes.c_char_p
+    lib.efla_gate.argtypes = [vp, vp, vp, L, I, I, vp]
+    lib.efla_gate.restype = I
+    lib.efla_chunk_fwd_workspace_bytes.argtypes = [I, I, I, I, I, I, I]
+    lib.efla_chunk_fwd_workspace_bytes.restype = Z
+    lib.efla_chunk_fwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, I, I, I, I, I, I, I, vp, Z, vp]
+    lib.efla_chunk_fwd.restype = I
+    lib.efla_workspace_status.argtypes = [vp, I, vp]
+    lib.efla_workspace_status.restype = I
+    lib.efla_selftest_wait_timeout.argtypes = [vp, ctypes.c_longlong, vp]
+    lib.efla_selftest_wait_timeout.restype = I
+    lib.efla_recurrent_step.argtypes = [vp, vp, vp, vp, vp, vp, I, I, I, I, I, vp]
+    lib.efla_recurrent_step.restype = I
+    return lib
+
+
+lib = _load()
+
+
+def efla_status_string(status: int) -> str:
+    return lib.efla_status_string(int(status)).decode()
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _check(t: torch.Tensor, name: str, dtype=None):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def _raise(status: int, where: str):
+    if status != EFLA_OK:
+        raise EflaError(status, where)
+
+
+def efla_gate(k: torch.Tensor, beta: torch.Tensor, out: Optional[torch.Tensor] = None,
+              stream=None) -> torch.Tensor:
+    """alpha [...] float32 from keys k [..., d_k] and gates beta [...] (same dtype)."""
+    _check(k, "k"); _check(beta, "beta", k.dtype)
+    n = beta.numel()
+    if out is None:
+        out = torch.empty(beta.shape, device=k.device, dtype=torch.float32)
+    _check(out, "out", torch.float32)
+    _raise(lib.efla_gate(_ptr(k), _ptr(beta), _ptr(out), n, k.shape[-1], _DTYPES[k.dtype],
+                         _stream(stream)), "efla_gate")
+    return out
+
+
+def efla_chunk_fwd_workspace_bytes(B, H, T, d_k, d_v, chunk=CHUNK, dtype=torch.bfloat16) -> int:
+    return int(lib.efla_chunk_fwd_workspace_bytes(B, H, T, d_k, d_v, chunk, _DTYPES[dtype]))
+
+
+def new_workspace(B, H, T, d_k, d_v, chunk=CHUNK, dtype=torch.bfloat16, device="cuda"):
+    """A zeroed workspace tensor (uint8) sized for efla_chunk_fwd."""
+    n = efla_chunk_fwd_workspace_bytes(B, H, T, d_k, d_v, chunk, dtype)
+    if n == 0:
+        raise EflaError(EFLA_ERR_UNSUPPORTED, "efla_chunk_fwd_workspace_bytes")
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def efla_chunk_fwd(q, k, v, beta, S0=None, chunk: int = CHUNK, o=None, S_T=None,
+                   workspace=None, want_state: bool = True, stream=None
+                   ) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Chunked EFLA forward. q, k [B,H,T,d_k], v [B,H,T,d_v], beta [B,H,T] (one dtype),
+    S0 [B,H,d_k,d_v] float32 or None.  Returns (o [B,H,T,d_v], S_T or None)."""
+    dt = k.dtype
+    for t, nme in ((q, "q"), (k, "k"), (v, "v"), (beta, "beta")):
+        _check(t, nme, dt)
+    B, H, T, d_k = k.shape
+    d_v = v.shape[-1]
+    if S0 is not None:
+        _check(S0, "S0", torch.float32)
+    if o is None:
+        o = torch.empty((B, H, T, d_v), device=k.device, dtype=dt)
+    _check(o, "o", dt)
+    if S_T is None and want_state:
+        S_T = torch.empty((B, H, d_k, d_v), device=k.device, dtype=torch.float32)
+    if S_T is not None:
+        _check(S_T, "S_T", torch.float32)
+    if workspace is None:
+        workspace = new_workspace(B, H, T, d_k, d_v, chunk, dt, k.device)
+    st = lib.efla_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(S0), _ptr(o), _ptr(S_T),
+                            B, H, T, d_k, d_v, chunk, _DTYPES.get(dt, -1), _ptr(workspace),
+                            workspace.numel(), _stream(stream))
+    _raise(st, "efla_chunk_fwd")
+    return o, S_T
+
+
+def efla_workspace_status(workspace: torch.Tensor, clear: bool = False, stream=None) -> int:
+    return int(lib.efla_workspace_status(_ptr(workspace), int(clear), _stream(stream)))
+
+
+def efla_selftest_wait_timeout(workspace: torch.Tensor, limit_ns: int = 1_000_000, stream=None) -> None:
+    _raise(lib.efla_selftest_wait_timeout(_ptr(workspace), int(limit_ns), _stream(stream)),
+           "efla_selftest_wait_timeout")
+
+
+def efla_recurrent_step(q, k, v, beta, S, o=None, stream=None) -> torch.Tensor:
+    """One decode token: q, k [N,H,d_k], v [N,H,d_v], beta [N,H]; S [N,H,d_k,d_v] float32
+    updated in place.  Returns o [N,H,d_v]."""
+    dt = k.dtype
+    for t, nme in ((q, "q"), (k, "k"), (v, "v"), (beta, "beta")):
+        _check(t, nme, dt)
+    _check(S, "S", torch.float32)
+    N, H, d_k = k.shape
+    d_v = v.shape[-1]
+    if o is None:
+        o = torch.empty((N, H, d_v), device=k.device, dtype=dt)
+    _check(o, "o", dt)
+    _raise(lib.efla_recurrent_step(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(S), _ptr(o),
+                                   N, H, d_k, d_v, _DTYPES.get(dt, -1), _stream(stream)),
+           "efla_recurrent_step")
+    return o
+
+
+__all__ = ["efla_gate", "efla_chunk_fwd", "efla_chunk_fwd_workspace_bytes", "efla_recurrent_step",
+           "efla_workspace_status", "efla_status_string", "efla_selftest_wait_timeout", "new_workspace", "EflaError", "lib",
+           "LIB_PATH", "CHUNK"]

@@ -1,0 +1,147 @@
+// efla_api.cu -- the C ABI declared in include/efla.h: argument checks, then launches.
+#include <stdint.h>
+#include <string.h>
+
+#include "../../include/efla.h"
+#include "efla_common.cuh"
+#include "efla_kernels.h"
+
+namespace {
+
+constexpr size_t kWorkspaceHeader = 256;   // device error word + reserved
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+    if (!a || !b || na == 0 || nb == 0) return false;
+    const uintptr_t a0 = (uintptr_t)a, b0 = (uintptr_t)b;
+    return a0 < b0 + nb && b0 < a0 + na;
+}
+
+size_t elem_size(int dtype) { return dtype == EFLA_DTYPE_BF16 ? 2 : 4; }
+
+int from_cuda(cudaError_t e) { return e == cudaSuccess ? EFLA_OK : EFLA_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+const char* efla_status_string(int status) {
+    switch (status) {
+        case EFLA_OK: return "EFLA_OK";
+        case EFLA_ERR_INVALID_ARG: return "EFLA_ERR_INVALID_ARG";
+        case EFLA_ERR_UNSUPPORTED: return "EFLA_ERR_UNSUPPORTED";
+        case EFLA_ERR_CUDA: return "EFLA_ERR_CUDA";
+        case EFLA_ERR_TIMEOUT: return "EFLA_ERR_TIMEOUT";
+        default: return "EFLA_ERR_UNKNOWN";
+    }
+}
+
+int efla_gate(const void* k, const void* beta, float* alpha, long n, int d_k, int dtype,
+              efla_stream_t stream) {
+    if (dtype != EFLA_DTYPE_F32 && dtype != EFLA_DTYPE_BF16) return EFLA_ERR_UNSUPPORTED;
+    if (n < 0 || d_k < 1 || d_k > 4096) return EFLA_ERR_INVALID_ARG;
+    if ((d_k * elem_size(dtype)) % 16 != 0) return EFLA_ERR_UNSUPPORTED;
+    if (n == 0) return EFLA_OK;
+    if (!k || !beta || !alpha || !aligned16(k) || !aligned16(beta) || !aligned16(alpha))
+        return EFLA_ERR_INVALID_ARG;
+    return from_cuda(efla::launch_gate(k, beta, alpha, n, d_k, dtype == EFLA_DTYPE_BF16,
+                                       (cudaStream_t)stream));
+}
+
+static int check_chunk_shape(int B, int H, int T, int d_k, int d_v, int chunk, int dtype) {
+    if (B < 0 || H < 0 || T < 0 || d_k <= 0 || d_v <= 0 || chunk <= 0) return EFLA_ERR_INVALID_ARG;
+    if (dtype != EFLA_DTYPE_F32 && dtype != EFLA_DTYPE_BF16) return EFLA_ERR_UNSUPPORTED;
+    if (d_k != d_v || (d_k != 64 && d_k != 128) || chunk != 64) return EFLA_ERR_UNSUPPORTED;
+    if ((long long)B * H * 2 >= (1ll << 31)) return EFLA_ERR_UNSUPPORTED;
+    return EFLA_OK;
+}
+
+size_t efla_chunk_fwd_workspace_bytes(int B, int H, int T, int d_k, int d_v, int chunk, int dtype) {
+    if (check_chunk_shape(B, H, T, d_k, d_v, chunk, dtype) != EFLA_OK) return 0;
+    return kWorkspaceHeader;
+}
+
+int efla_chunk_fwd(const void* q, const void* k, const void* v, const void* beta, const float* S0,
+                   void* o, float* S_T, int B, int H, int T, int d_k, int d_v, int chunk, int dtype,
+                   void* workspace, size_t workspace_bytes, efla_stream_t stream) {
+    int st = check_chunk_shape(B, H, T, d_k, d_v, chunk, dtype);
+    if (st != EFLA_OK) return st;
+    if (!workspace || !aligned16(workspace) ||
+        workspace_bytes < efla_chunk_fwd_workspace_bytes(B, H, T, d_k, d_v, chunk, dtype))
+        return EFLA_ERR_INVALID_ARG;
+    const long BH = (long)B * H;
+    if (BH == 0) return EFLA_OK;
+    const size_t es = elem_size(dtype);
+    const size_t nqk = (size_t)BH * T * d_k * es, nv = (size_t)BH * T * d_v * es;
+    const size_t nb = (size_t)BH * T * es, ns = (size_t)BH * d_k * d_v * sizeof(float);
+    if ((S0 && !aligned16(S0)) || (S_T && !aligned16(S_T))) return EFLA_ERR_INVALID_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (T == 0) {   // empty sequence: the state passes through unchanged
+        if (!S_T || S_T == S0) return EFLA_OK;
+        return from_cuda(S0 ? cudaMemcpyAsync(S_T, S0, ns, cudaMemcpyDeviceToDevice, s)
+                            : cudaMemsetAsync(S_T, 0, ns, s));
+    }
+    if (!q || !k || !v || !beta || !o) return EFLA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(beta) || !aligned16(o))
+        return EFLA_ERR_INVALID_ARG;
+    if (overlaps(o, nv, q, nqk) || overlaps(o, nv, k, nqk) || overlaps(o, nv, v, nv) ||
+        overlaps(o, nv, beta, nb) || overlaps(o, nv, S0, ns) || overlaps(o, nv, S_T, ns) ||
+        overlaps(o, nv, workspace, workspace_bytes))
+        return EFLA_ERR_INVALID_ARG;
+    if (S_T && S_T != S0 &&
+        (overlaps(S_T, ns, q, nqk) || overlaps(S_T, ns, k, nqk) || overlaps(S_T, ns, v, nv) ||
+         overlaps(S_T, ns, beta, nb) || overlaps(S_T, ns, S0, ns)))
+        return EFLA_ERR_INVALID_ARG;
+    if (dtype == EFLA_DTYPE_BF16 && d_k == 128)
+        return from_cuda(efla::launch_chunk_tc(q, k, v, beta, S0, o, S_T, BH, T,
+                                               static_cast<uint32_t*>(workspace), s));
+    return from_cuda(efla::launch_chunk_simt(q, k, v, beta, S0, o, S_T, BH, T, d_k,
+                                             dtype == EFLA_DTYPE_BF16, s));
+}
+
+int efla_workspace_status(void* workspace, int clear, efla_stream_t stream) {
+    if (!workspace || !aligned16(workspace)) return EFLA_ERR_INVALID_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+    uint32_t word = 0;
+    if (cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return EFLA_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return EFLA_ERR_CUDA;
+    if (clear) {
+        if (cudaMemsetAsync(workspace, 0, sizeof(word), s) != cudaSuccess) return EFLA_ERR_CUDA;
+        if (cudaStreamSynchronize(s) != cudaSuccess) return EFLA_ERR_CUDA;
+    }
+    return word == efla::kDevOk ? EFLA_OK : EFLA_ERR_TIMEOUT;
+}
+
+int efla_selftest_wait_timeout(void* workspace, long long limit_ns, efla_stream_t stream) {
+    if (!workspace || !aligned16(workspace) || limit_ns < 0) return EFLA_ERR_INVALID_ARG;
+    return from_cuda(efla::launch_wait_timeout_selftest(static_cast<uint32_t*>(workspace),
+                                                        (unsigned long long)limit_ns,
+                                                        (cudaStream_t)stream));
+}
+
+int efla_recurrent_step(const void* q, const void* k, const void* v, const void* beta, float* S,
+                        void* o, int N, int H, int d_k, int d_v, int dtype, efla_stream_t stream) {
+    if (N < 0 || H < 0 || d_k <= 0 || d_v <= 0) return EFLA_ERR_INVALID_ARG;
+    if (dtype != EFLA_DTYPE_F32 && dtype != EFLA_DTYPE_BF16) return EFLA_ERR_UNSUPPORTED;
+    if (d_k != d_v || (d_k != 64 && d_k != 128)) return EFLA_ERR_UNSUPPORTED;
+    const long NH = (long)N * H;
+    if (NH == 0) return EFLA_OK;
+    if (NH * (d_k / 32) >= (1l << 31)) return EFLA_ERR_UNSUPPORTED;
+    if (!q || !k || !v || !beta || !S || !o) return EFLA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(beta) || !aligned16(S) ||
+        !aligned16(o))
+        return EFLA_ERR_INVALID_ARG;
+    const size_t es = elem_size(dtype);
+    const size_t nq = (size_t)NH * d_k * es, nv = (size_t)NH * d_v * es, nb = (size_t)NH * es;
+    const size_t ns = (size_t)NH * d_k * d_v * sizeof(float);
+    if (overlaps(o, nv, S, ns) || overlaps(o, nv, q, nq) || overlaps(o, nv, k, nq) ||
+        overlaps(o, nv, v, nv) || overlaps(o, nv, beta, nb) || overlaps(S, ns, q, nq) ||
+        overlaps(S, ns, k, nq) || overlaps(S, ns, v, nv) || overlaps(S, ns, beta, nb))
+        return EFLA_ERR_INVALID_ARG;
+    return from_cuda(efla::launch_decode(q, k, v, beta, S, o, NH, d_k, dtype == EFLA_DTYPE_BF16,
+                                         (cudaStream_t)stream));
+}
+
+}  // extern "C"

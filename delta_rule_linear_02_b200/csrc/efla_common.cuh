@@ -1,0 +1,60 @@
+// efla_common.cuh -- element access and the exact-flow gate, shared by the kernels.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace efla {
+
+// ---------------------------------------------------------------- element access
+template <typename T> struct Elem;
+
+template <> struct Elem<float> {
+    static __device__ __forceinline__ float to_f(float x) { return x; }
+    static __device__ __forceinline__ float from_f(float x) { return x; }
+};
+
+template <> struct Elem<__nv_bfloat16> {
+    static __device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
+    static __device__ __forceinline__ __nv_bfloat16 from_f(float x) { return __float2bfloat16_rn(x); }
+};
+
+// Load 4 consecutive elements (16-byte aligned for float, 8-byte for bf16) as floats.
+__device__ __forceinline__ float4 load4(const float* p) { return *reinterpret_cast<const float4*>(p); }
+__device__ __forceinline__ float4 load4(const __nv_bfloat16* p) {
+    uint2 u = *reinterpret_cast<const uint2*>(p);
+    float2 a = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&u.x));
+    float2 b = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&u.y));
+    return make_float4(a.x, a.y, b.x, b.y);
+}
+
+__device__ __forceinline__ void store4(float* p, float4 v) { *reinterpret_cast<float4*>(p) = v; }
+__device__ __forceinline__ void store4(__nv_bfloat16* p, float4 v) {
+    __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y);
+    __nv_bfloat162 b = __floats2bfloat162_rn(v.z, v.w);
+    uint2 u;
+    u.x = *reinterpret_cast<uint32_t*>(&a);
+    u.y = *reinterpret_cast<uint32_t*>(&b);
+    *reinterpret_cast<uint2*>(p) = u;
+}
+
+// ---------------------------------------------------------------- the gate
+// Exact Flow Linear Attention, Section 3.2: the closed-form flow keeps the delta rule's
+// rank-1 write with beta replaced by alpha = (1 - exp(-beta*lambda)) / lambda, where
+// lambda = ||k||^2 (Section 3.4; the nonzero eigenvalue of A = k k^T, App. D).
+// For |x| = |beta*lambda| < 2^-10 the series 1 - x/2 + x^2/6 of (1 - e^{-x})/x is used
+// (truncation error below x^3/24 < 4e-11 relative): it keeps full precision when x is
+// subnormal and gives alpha = beta exactly at lambda = 0, the limit of the formula.
+__device__ __forceinline__ float gate_alpha(float beta, float lambda) {
+    const float x = beta * lambda;
+    if (fabsf(x) < 0.0009765625f) {
+        return beta * (1.0f - x * (0.5f - x * (1.0f / 6.0f)));
+    }
+    return -expm1f(-x) / lambda;
+}
+
+// Device error word values (kept in the caller's workspace).
+enum : uint32_t { kDevOk = 0u, kDevTimeout = 1u };
+
+}  // namespace efla

@@ -1,0 +1,25 @@
+// efla_kernels.h -- internal launchers (not part of the C ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace efla {
+
+cudaError_t launch_gate(const void* k, const void* beta, float* alpha, long n, int dk, bool bf16,
+                        cudaStream_t stream);
+
+cudaError_t launch_decode(const void* q, const void* k, const void* v, const void* beta, float* S,
+                          void* o, long NH, int D, bool bf16, cudaStream_t stream);
+
+cudaError_t launch_chunk_simt(const void* q, const void* k, const void* v, const void* beta,
+                              const float* S0, void* o, float* S_T, long BH, int T, int D, bool bf16,
+                              cudaStream_t stream);
+
+cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const void* beta, const float* S0,
+                            void* o, float* S_T, long BH, int T, uint32_t* err, cudaStream_t stream);
+
+cudaError_t launch_wait_timeout_selftest(uint32_t* err, unsigned long long limit_ns, cudaStream_t stream);
+
+}  // namespace efla

@@ -1,0 +1,136 @@
+/*
+ * efla.h -- C ABI of the B200 (sm_100a) Exact Flow Linear Attention forward.
+ *
+ * The method (Exact Flow Linear Attention, arXiv 2512.12602): the delta-rule write
+ * S_t = S_{t-1} - beta_t k_t (k_t^T S_{t-1} - v_t^T) is one explicit Euler step of
+ * dS/dtau = -k k^T S + k v^T (summary page, Section 2 and Section 3.1).  Solving that
+ * zero-order-hold ODE in closed form keeps the rank-1 write with beta_t replaced by the
+ * gate (Section 3.2, with the denominator of Section 3.4 and the rank-1 algebra of App. D/E)
+ *
+ *     alpha_t = (1 - exp(-beta_t * lambda_t)) / lambda_t,   lambda_t = ||k_t||^2,
+ *
+ * and the read-out is o_t = S_t^T q_t, taken after the write.
+ *
+ * Conventions shared by every entry point:
+ *   - Row convention: the state S of one (batch, head) stream is a d_k x d_v row-major
+ *     float32 matrix and o_t^T = q_t^T S_t (the transpose of the pages' column form).
+ *   - Tensors are contiguous, row-major, head-major: q, k [B, H, T, d_k]; v, o [B, H, T, d_v];
+ *     beta [B, H, T]; states [B, H, d_k, d_v] float32.
+ *   - q, k, v, beta and o share one element type (efla_dtype); states are always float32.
+ *   - All data pointers are DEVICE pointers owned by the caller.  The library keeps no
+ *     global state and never allocates: calls on different streams may run concurrently
+ *     as long as their buffers do not overlap.
+ *   - Every pointer must be 16-byte aligned.
+ *   - Calls are asynchronous on `stream` (NULL: the legacy default stream) and never
+ *     synchronise the host.  A non-OK status from argument checking means nothing was
+ *     launched.  EFLA_ERR_CUDA reports a launch error (cudaGetLastError).
+ *   - Errors detected on the device (a bounded wait that ran out) are recorded in the
+ *     workspace of efla_chunk_fwd and read back with efla_workspace_status.
+ */
+#ifndef EFLA_H
+#define EFLA_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    EFLA_OK = 0,
+    EFLA_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, non-positive size, bad workspace */
+    EFLA_ERR_UNSUPPORTED = 2,  /* valid but unsupported shape (d_k, d_v, chunk) or dtype */
+    EFLA_ERR_CUDA = 3,         /* a CUDA call or kernel launch failed */
+    EFLA_ERR_TIMEOUT = 4       /* a device-side bounded wait ran out (see efla_workspace_status) */
+} efla_status;
+
+typedef enum {
+    EFLA_DTYPE_F32 = 0,   /* float32 q, k, v, beta, o */
+    EFLA_DTYPE_BF16 = 1   /* bfloat16 q, k, v, beta, o (fp32 accumulation and state) */
+} efla_dtype;
+
+/* Same type as cudaStream_t, declared here so this header needs no CUDA include. */
+typedef struct CUstream_st *efla_stream_t;
+
+/* Human-readable name of a status code (static storage). */
+const char *efla_status_string(int status);
+
+/*
+ * efla_gate -- the exact-flow gate alone (Section 3.2 gate, Section 3.4 denominator).
+ *   k     [n, d_k] (dtype), beta [n] (dtype)  ->  alpha [n] float32
+ *   lambda = sum_i k_i^2 accumulated in float32; alpha = -expm1(-beta*lambda)/lambda, and
+ *   alpha = beta exactly when lambda == 0.
+ * Supports any d_k in [1, 4096] with d_k*sizeof(dtype) a multiple of 16 bytes.
+ */
+int efla_gate(const void *k, const void *beta, float *alpha, long n, int d_k, int dtype,
+              efla_stream_t stream);
+
+/*
+ * efla_chunk_fwd_workspace_bytes -- bytes of device workspace efla_chunk_fwd needs for
+ * this problem (always > 0: it holds at least the device error word).  Returns 0 for
+ * arguments efla_chunk_fwd would reject.
+ */
+size_t efla_chunk_fwd_workspace_bytes(int B, int H, int T, int d_k, int d_v, int chunk,
+                                      int dtype);
+
+/*
+ * efla_chunk_fwd -- chunkwise-parallel forward over B*H independent streams of T tokens
+ * (Section 3.3: tokens stacked per chunk, causal lower-triangular mask, UT transform).
+ *
+ *   q, k [B,H,T,d_k], v [B,H,T,d_v], beta [B,H,T]         inputs, `dtype`
+ *   S0   [B,H,d_k,d_v] float32 or NULL (zero initial state)
+ *   o    [B,H,T,d_v]  output, `dtype`
+ *   S_T  [B,H,d_k,d_v] float32 final state, or NULL (not written).  S_T may alias S0.
+ *   o must not overlap any input.
+ *   workspace: device memory of at least efla_chunk_fwd_workspace_bytes(...) bytes,
+ *   16-byte aligned, owned by the caller; its first bytes hold a sticky device error word
+ *   (zero it once before first use, e.g. with cudaMemset).
+ *
+ * Supported: d_k = d_v in {64, 128}, chunk = 64, any T >= 1 (the tail chunk is padded with
+ * k = 0, beta = 0 tokens, which are exact no-ops), B*H >= 1.
+ * bf16 runs on the 5th-generation tensor cores (bf16 operands, fp32 accumulation, fp32
+ * state); f32 runs on fp32 CUDA cores.
+ */
+int efla_chunk_fwd(const void *q, const void *k, const void *v, const void *beta,
+                   const float *S0, void *o, float *S_T, int B, int H, int T, int d_k,
+                   int d_v, int chunk, int dtype, void *workspace, size_t workspace_bytes,
+                   efla_stream_t stream);
+
+/*
+ * efla_workspace_status -- waits for `stream`, then returns EFLA_ERR_TIMEOUT if any
+ * efla_chunk_fwd that used `workspace` gave up on a device wait since the word was last
+ * cleared (its outputs are then invalid), else EFLA_OK.  clear != 0 resets the word.
+ * This is the one call that synchronises the host.
+ */
+int efla_workspace_status(void *workspace, int clear, efla_stream_t stream);
+
+/*
+ * efla_selftest_wait_timeout -- failure-detection self test.  Launches one CTA that waits
+ * on a barrier nothing will ever arrive on, with the device-side bound `limit_ns`
+ * (nanoseconds); when the bound runs out the CTA records the timeout in `workspace`'s
+ * error word and exits.  efla_workspace_status then reports EFLA_ERR_TIMEOUT.  The same
+ * bounded wait guards every barrier wait of efla_chunk_fwd (bound: 2 s per wait).
+ */
+int efla_selftest_wait_timeout(void *workspace, long long limit_ns, efla_stream_t stream);
+
+/*
+ * efla_recurrent_step -- one decode token for N*H streams, state updated in place
+ * (the recurrent form: Section 3.2 update, o_t = S_t^T q_t).
+ *
+ *   q, k [N,H,d_k], v [N,H,d_v], beta [N,H]   inputs, `dtype`
+ *   S    [N,H,d_k,d_v] float32, read and overwritten with the new state
+ *   o    [N,H,d_v] output, `dtype`; must not overlap S or any input
+ *
+ * One pass over S: r = k^T S, p = q^T S and c = q.k are formed together, then
+ * S <- S - alpha k (r - v)^T and o = p - alpha c (r - v).
+ * Supported: d_k = d_v in {64, 128}; dtype f32 or bf16.
+ */
+int efla_recurrent_step(const void *q, const void *k, const void *v, const void *beta,
+                        float *S, void *o, int N, int H, int d_k, int d_v, int dtype,
+                        efla_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EFLA_H */

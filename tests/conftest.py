@@ -20,3 +20,29 @@ def pytest_configure(config):
 def oracle_lib():
     import oracle
     return oracle.load()
+
+
+def _build_library():
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "efla_build", os.path.join(ROOT, "delta_rule_linear_02_b200", "build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod.build()
+
+
+@pytest.fixture(scope="session")
+def efla():
+    """The library binding (builds libefla.so in-tree first if it is missing or stale)."""
+    _build_library()
+    import delta_rule_linear_02_b200 as m
+    return m
+
+
+@pytest.fixture(scope="session")
+def cuda(efla):
+    import torch
+    if not torch.cuda.is_available():
+        pytest.fail("GPU test selected but no CUDA device is visible")
+    torch.backends.cuda.matmul.allow_tf32 = False
+    return torch.device("cuda", 0)

@@ -1,0 +1,116 @@
+"""The C ABI library loads, exports every declared symbol and rejects bad arguments
+without launching anything (CPU only: no call here reaches a kernel)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "efla.h")
+
+# validation codes
+OK, INVALID, UNSUPPORTED = 0, 1, 2
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(efla_[a-z_]+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for want in ("efla_chunk_fwd", "efla_recurrent_step", "efla_gate", "efla_status_string",
+                 "efla_chunk_fwd_workspace_bytes", "efla_workspace_status"):
+        assert want in names
+
+
+def test_library_exports_every_declared_symbol(efla):
+    lib = ctypes.CDLL(efla.LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(lib, name), f"libefla.so does not export {name}"
+
+
+def test_status_strings(efla):
+    assert efla.efla_status_string(0) == "EFLA_OK"
+    assert efla.efla_status_string(4) == "EFLA_ERR_TIMEOUT"
+    assert efla.efla_status_string(99) == "EFLA_ERR_UNKNOWN"
+
+
+def test_workspace_bytes(efla):
+    L = efla.lib
+    assert L.efla_chunk_fwd_workspace_bytes(4, 16, 2048, 128, 128, 64, 1) >= 16
+    assert L.efla_chunk_fwd_workspace_bytes(1, 1, 1, 64, 64, 64, 0) >= 16
+    assert L.efla_chunk_fwd_workspace_bytes(1, 1, 1, 96, 96, 64, 0) == 0      # unsupported d
+    assert L.efla_chunk_fwd_workspace_bytes(1, 1, 1, 128, 64, 64, 1) == 0     # d_k != d_v
+    assert L.efla_chunk_fwd_workspace_bytes(1, 1, 1, 128, 128, 32, 1) == 0    # chunk
+    assert L.efla_chunk_fwd_workspace_bytes(-1, 1, 1, 128, 128, 64, 1) == 0   # negative
+
+
+def _fwd(L, ptrs, B=1, H=1, T=64, d=128, chunk=64, dtype=1, ws=256):
+    q, k, v, b, s0, o, st, w = ptrs
+    return L.efla_chunk_fwd(q, k, v, b, s0, o, st, B, H, T, d, d, chunk, dtype, w, ws, None)
+
+
+# fake, well-separated, 16-byte aligned device addresses: validation never dereferences them
+GOOD = [ctypes.c_void_p(0x10000000 * (i + 1)) for i in range(8)]
+
+
+def test_chunk_fwd_rejects_bad_arguments(efla):
+    L = efla.lib
+    assert _fwd(L, GOOD, d=96) == UNSUPPORTED
+    assert _fwd(L, GOOD, chunk=32) == UNSUPPORTED
+    assert _fwd(L, GOOD, dtype=7) == UNSUPPORTED
+    assert _fwd(L, GOOD, T=-1) == INVALID
+    assert _fwd(L, GOOD, B=-2) == INVALID
+    for i in (0, 1, 2, 3, 5):                     # q, k, v, beta, o may not be NULL
+        bad = list(GOOD); bad[i] = None
+        assert _fwd(L, bad) == INVALID, i
+    for i in range(8):                            # every pointer must be 16-byte aligned
+        bad = list(GOOD); bad[i] = ctypes.c_void_p(GOOD[i].value + 8)
+        assert _fwd(L, bad) == INVALID, i
+    bad = list(GOOD); bad[7] = None               # workspace required
+    assert _fwd(L, bad) == INVALID
+    assert _fwd(L, GOOD, ws=8) == INVALID         # workspace too small
+    bad = list(GOOD); bad[5] = GOOD[0]            # o aliases q
+    assert _fwd(L, bad) == INVALID
+    assert _fwd(L, GOOD, B=0) == OK               # nothing to do, nothing launched
+    assert _fwd(L, GOOD, H=0) == OK
+
+
+def test_recurrent_step_rejects_bad_arguments(efla):
+    L = efla.lib
+    P = GOOD
+    f = lambda ptrs=P, N=4, H=2, d=128, dt=0: L.efla_recurrent_step(*ptrs[:6], N, H, d, d, dt, None)
+    assert f(d=32) == UNSUPPORTED
+    assert f(dt=3) == UNSUPPORTED
+    assert f(N=-1) == INVALID
+    assert f(N=0) == OK
+    for i in range(6):
+        bad = list(P); bad[i] = None
+        assert f(bad) == INVALID, i
+        bad = list(P); bad[i] = ctypes.c_void_p(P[i].value + 4)
+        assert f(bad) == INVALID, i
+    bad = list(P); bad[5] = P[4]                  # o aliases S
+    assert f(bad) == INVALID
+    assert L.efla_recurrent_step(P[0], P[1], P[2], P[3], P[4], P[5], 4, 2, 128, 64, 0, None) == UNSUPPORTED
+
+
+def test_gate_rejects_bad_arguments(efla):
+    L = efla.lib
+    assert L.efla_gate(GOOD[0], GOOD[1], GOOD[2], 10, 6, 0, None) == UNSUPPORTED   # 24-byte rows
+    assert L.efla_gate(GOOD[0], GOOD[1], GOOD[2], -1, 64, 0, None) == INVALID
+    assert L.efla_gate(None, GOOD[1], GOOD[2], 10, 64, 0, None) == INVALID
+    assert L.efla_gate(GOOD[0], GOOD[1], GOOD[2], 0, 64, 0, None) == OK
+
+
+def test_binding_fails_loudly_without_the_library(tmp_path):
+    """The product path has no fallback: a missing libefla.so is an import error."""
+    import subprocess, sys, shutil
+    pkg = tmp_path / "delta_rule_linear_02_b200"
+    shutil.copytree(os.path.join(ROOT, "delta_rule_linear_02_b200"), pkg,
+                    ignore=shutil.ignore_patterns("*.so", "__pycache__"))
+    r = subprocess.run([sys.executable, "-c", "import delta_rule_linear_02_b200"], cwd=tmp_path,
+                       capture_output=True, text=True)
+    assert r.returncode != 0 and "libefla.so is not built" in r.stderr
