@@ -43,6 +43,8 @@ def _load() -> ctypes.CDLL:
     lib.efla_chunk_fwd_workspace_bytes.restype = Z
     lib.efla_chunk_fwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, I, I, I, I, I, I, I, vp, Z, vp]
     lib.efla_chunk_fwd.restype = I
+    lib.efla_chunk_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, I, I, I, I, I, I, I, vp]
+    lib.efla_chunk_fwd_noalloc.restype = I
     lib.efla_workspace_status.argtypes = [vp, I, vp]
     lib.efla_workspace_status.restype = I
     lib.efla_selftest_wait_timeout.argtypes = [vp, ctypes.c_longlong, vp]
@@ -136,6 +138,32 @@ def efla_chunk_fwd(q, k, v, beta, S0=None, chunk: int = CHUNK, o=None, S_T=None,
     return o, S_T
 
 
+def efla_chunk_fwd_noalloc(q, k, v, beta, S0=None, chunk: int = CHUNK, o=None, S_T=None,
+                           want_state: bool = True, stream=None
+                           ) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """efla_chunk_fwd using the library's internal static scratch instead of a workspace.
+    o and S_T are allocated here when not given (pass them in to allocate nothing)."""
+    dt = k.dtype
+    for t, nme in ((q, "q"), (k, "k"), (v, "v"), (beta, "beta")):
+        _check(t, nme, dt)
+    B, H, T, d_k = k.shape
+    d_v = v.shape[-1]
+    if S0 is not None:
+        _check(S0, "S0", torch.float32)
+    if o is None:
+        o = torch.empty((B, H, T, d_v), device=k.device, dtype=dt)
+    _check(o, "o", dt)
+    if S_T is None and want_state:
+        S_T = torch.empty((B, H, d_k, d_v), device=k.device, dtype=torch.float32)
+    if S_T is not None:
+        _check(S_T, "S_T", torch.float32)
+    st = lib.efla_chunk_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(S0), _ptr(o),
+                                    _ptr(S_T), B, H, T, d_k, d_v, chunk, _DTYPES.get(dt, -1),
+                                    _stream(stream))
+    _raise(st, "efla_chunk_fwd_noalloc")
+    return o, S_T
+
+
 def efla_workspace_status(workspace: torch.Tensor, clear: bool = False, stream=None) -> int:
     return int(lib.efla_workspace_status(_ptr(workspace), int(clear), _stream(stream)))
 
@@ -163,6 +191,6 @@ def efla_recurrent_step(q, k, v, beta, S, o=None, stream=None) -> torch.Tensor:
     return o
 
 
-__all__ = ["efla_gate", "efla_chunk_fwd", "efla_chunk_fwd_workspace_bytes", "efla_recurrent_step",
+__all__ = ["efla_gate", "efla_chunk_fwd", "efla_chunk_fwd_noalloc", "efla_chunk_fwd_workspace_bytes", "efla_recurrent_step",
            "efla_workspace_status", "efla_status_string", "efla_selftest_wait_timeout", "new_workspace", "EflaError", "lib",
            "LIB_PATH", "CHUNK"]

@@ -100,6 +100,47 @@ int efla_chunk_fwd(const void* q, const void* k, const void* v, const void* beta
                                              dtype == EFLA_DTYPE_BF16, s));
 }
 
+// ---------------------------------------------------------------- allocation-free variant
+// Scratch for efla_chunk_fwd_noalloc: a file-scope device array, so that callers who
+// cannot allocate device memory still get the chunked forward.  Every GPU that loads
+// this library holds it until the process exits.  Host code cannot use the symbol
+// itself as a device address; the address is looked up once per device below.
+static constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;   // 16 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+static void* noalloc_scratch(int* status) {
+    constexpr int kMaxDevices = 64;
+    static void* addr[kMaxDevices] = {};
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        *status = EFLA_ERR_CUDA;
+        return nullptr;
+    }
+    if (!addr[dev]) {   // first call on this device (with it current): resolve the address
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
+            *status = EFLA_ERR_CUDA;
+            return nullptr;
+        }
+        addr[dev] = p;
+    }
+    return addr[dev];
+}
+
+int efla_chunk_fwd_noalloc(const void* q, const void* k, const void* v, const void* beta,
+                           const float* S0, void* o, float* S_T, int B, int H, int T, int d_k,
+                           int d_v, int chunk, int dtype, efla_stream_t stream) {
+    int st = check_chunk_shape(B, H, T, d_k, d_v, chunk, dtype);
+    if (st != EFLA_OK) return st;
+    const size_t need = efla_chunk_fwd_workspace_bytes(B, H, T, d_k, d_v, chunk, dtype);
+    if (need > kNoAllocScratchBytes) return EFLA_ERR_UNSUPPORTED;
+    void* ws = noalloc_scratch(&st);
+    if (!ws) return st;
+    // the scratch keeps the previous call's contents: the device error word starts at zero
+    if (cudaMemsetAsync(ws, 0, 16, (cudaStream_t)stream) != cudaSuccess) return EFLA_ERR_CUDA;
+    return efla_chunk_fwd(q, k, v, beta, S0, o, S_T, B, H, T, d_k, d_v, chunk, dtype, ws, need, stream);
+}
+
 int efla_workspace_status(void* workspace, int clear, efla_stream_t stream) {
     if (!workspace || !aligned16(workspace)) return EFLA_ERR_INVALID_ARG;
     cudaStream_t s = (cudaStream_t)stream;

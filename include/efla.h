@@ -97,6 +97,28 @@ int efla_chunk_fwd(const void *q, const void *k, const void *v, const void *beta
                    efla_stream_t stream);
 
 /*
+ * efla_chunk_fwd_noalloc -- efla_chunk_fwd without a caller-provided workspace.
+ * The paper has no counterpart: this is an integration variant for callers that cannot
+ * allocate device memory, e.g. code embedded in a host runtime that owns every device
+ * allocation and hands over only the input and output tensors, or latency-critical
+ * paths where cudaMalloc (which may synchronise the device) is not acceptable.
+ *
+ * Arguments, layouts, supported shapes and results are those of efla_chunk_fwd.  The
+ * scratch is a 16 MiB static device array inside the library (held on every GPU that
+ * loads it, until exit): a problem whose efla_chunk_fwd_workspace_bytes exceeds 16 MiB
+ * returns EFLA_ERR_UNSUPPORTED and launches nothing.  No device memory is allocated.
+ * The first call on a device looks up the array's device address (with that device
+ * current); make that first call before any stream capture.  Every call shares the one
+ * array and each call clears its error word first, so calls that overlap on the GPU
+ * (different streams, or different host threads) race on it and must be serialised by
+ * the caller.  A device-side wait timeout in this variant is recorded only in the
+ * internal scratch and is not reported to the caller.
+ */
+int efla_chunk_fwd_noalloc(const void *q, const void *k, const void *v, const void *beta,
+                           const float *S0, void *o, float *S_T, int B, int H, int T, int d_k,
+                           int d_v, int chunk, int dtype, efla_stream_t stream);
+
+/*
  * efla_workspace_status -- waits for `stream`, then returns EFLA_ERR_TIMEOUT if any
  * efla_chunk_fwd that used `workspace` gave up on a device wait since the word was last
  * cleared (its outputs are then invalid), else EFLA_OK.  clear != 0 resets the word.
