@@ -59,6 +59,8 @@ static int check_chunk_shape(int B, int H, int T, int d_k, int d_v, int chunk, i
 
 size_t efla_chunk_fwd_workspace_bytes(int B, int H, int T, int d_k, int d_v, int chunk, int dtype) {
     if (check_chunk_shape(B, H, T, d_k, d_v, chunk, dtype) != EFLA_OK) return 0;
+    if (dtype == EFLA_DTYPE_BF16 && d_k == 128)   // + the per-chunk UT transforms
+        return kWorkspaceHeader + efla::chunk_tc_workspace_bytes((long)B * H, T);
     return kWorkspaceHeader;
 }
 
@@ -95,7 +97,8 @@ int efla_chunk_fwd(const void* q, const void* k, const void* v, const void* beta
         return EFLA_ERR_INVALID_ARG;
     if (dtype == EFLA_DTYPE_BF16 && d_k == 128)
         return from_cuda(efla::launch_chunk_tc(q, k, v, beta, S0, o, S_T, BH, T,
-                                               static_cast<uint32_t*>(workspace), s));
+                                               static_cast<uint32_t*>(workspace),
+                                               static_cast<char*>(workspace) + kWorkspaceHeader, s));
     return from_cuda(efla::launch_chunk_simt(q, k, v, beta, S0, o, S_T, BH, T, d_k,
                                              dtype == EFLA_DTYPE_BF16, s));
 }
@@ -105,7 +108,7 @@ int efla_chunk_fwd(const void* q, const void* k, const void* v, const void* beta
 // cannot allocate device memory still get the chunked forward.  Every GPU that loads
 // this library holds it until the process exits.  Host code cannot use the symbol
 // itself as a device address; the address is looked up once per device below.
-static constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;   // 16 MiB
+static constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;   // 32 MiB
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 static void* noalloc_scratch(int* status) {

@@ -1,0 +1,253 @@
+// efla_ut.cu -- the UT transform of every 64-token chunk of every stream (bf16, d_k = 128).
+//
+// Exact Flow Linear Attention, Section 3.3: inside a chunk the rank-1 writes satisfy
+// (I + A) Delta = diag(alpha) (V - K S) with A = strictly-lower(diag(alpha) K K^T), so
+// Delta = T (V - K S) with T = (I + A)^{-1} diag(alpha).  T depends on K and beta only,
+// not on the state, so it is computed here for all chunks at once, in parallel, and the
+// chain kernel (efla_chunk_tc.cu) reads it back as a bf16 operand.
+//
+// Per tile (stream bh, chunk c):
+//   G = K K^T                                   tcgen05 MMA (bf16 in, fp32 in TMEM)
+//   lambda_r = G_rr, alpha_r = gate(beta_r, lambda_r)   (Section 3.2 / 3.4)
+//   A^T rows = alpha (.) G rows                 (G is symmetric)
+//   X = (I + A)^{-1}                            efla_ut_tf32.cuh (fp32 + TF32 merges)
+//   T = X diag(alpha) -> bf16, row-major 64 x 64, at Tout + 4096 * (bh * nchunks + c)
+// Tokens past T are zero-filled by TMA (k = 0, beta = 0: alpha = 0, their rows and
+// columns of T are zero).
+//
+// A persistent grid of several CTAs per SM walks the tiles; each CTA double-buffers its
+// K tiles (the next tile's TMA is in flight while the current one is solved), and the
+// CTAs on an SM overlap each other's latency.  Warp 0 issues the TMA copies and the MMA;
+// warps 1-4 compute the gate, the solve and the bf16 store.  Every wait is bounded.
+#include "efla_common.cuh"
+#include "efla_kernels.h"
+#include "efla_tma.cuh"
+#include "efla_ut_tf32.cuh"
+#include "sm100.cuh"
+
+namespace efla {
+
+namespace {
+using namespace sm100;
+using ut::LDX;
+
+constexpr int kThreads = 160;
+constexpr int kCtasPerSm = 3;
+constexpr uint32_t TILE = 8192;
+constexpr uint32_t OFF_K = 0;                          // 2 stages x [K a0 | K a1]
+constexpr uint32_t F32_TILE = 64 * LDX * 4;
+constexpr uint32_t OFF_AT = OFF_K + 4 * TILE;          // also the (unused) rows 64..127 of stage 1's MMA
+constexpr uint32_t OFF_X = OFF_AT + F32_TILE;
+constexpr uint32_t OFF_ALPHA = OFF_X + F32_TILE;
+constexpr uint32_t OFF_BETA = OFF_ALPHA + 256;
+constexpr uint32_t OFF_BAR = OFF_BETA + 256;
+constexpr uint32_t NBAR = 8;
+constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
+constexpr uint32_t SMEM_USED = OFF_MISC + 16;
+constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;
+static_assert(kCtasPerSm * SMEM_BYTES <= 232448, "UT kernel: shared memory for the target occupancy");
+
+enum : int { B_FULL = 0 /* [2] */, B_GP_FULL = 2, B_GP_FREE = 3, B_DRAIN = 4 };
+constexpr uint32_t TM_COLS = 64;
+constexpr uint32_t ID_G = idesc_bf16(128, 64, false, false);
+constexpr int NB_W = 1;                                // named barrier of the 128 worker threads
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+
+__device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                             unsigned long long limit) {
+    if (mbar_try_wait_sleep(bar, parity, 20000)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait_sleep(bar, parity, 20000)) {
+        if (*abort) return false;
+        if (globaltimer_ns() - t0 > limit) {
+            *abort = 1;
+            return false;
+        }
+    }
+    return true;
+}
+
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+ut_kernel(const __grid_constant__ CUtensorMap tm_k, const __nv_bfloat16* __restrict__ beta,
+          __nv_bfloat16* __restrict__ Tout, int T, int nchunks, long ntiles, uint32_t* __restrict__ err,
+          unsigned long long limit_ns) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sb = smem_u32(sm);
+    float* At = reinterpret_cast<float*>(sm + OFF_AT);
+    float* X = reinterpret_cast<float*>(sm + OFF_X);
+    float* al = reinterpret_cast<float*>(sm + OFF_ALPHA);
+    float* bt = reinterpret_cast<float*>(sm + OFF_BETA);
+    uint64_t* bar = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + OFF_MISC);
+    volatile int* abort = reinterpret_cast<volatile int*>(sm + OFF_MISC + 4);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const long first = blockIdx.x, step = gridDim.x;
+    const int ntile = first < ntiles ? (int)((ntiles - first + step - 1) / step) : 0;
+
+    if (tid == 0) {
+        for (int i = 0; i < (int)NBAR; ++i) mbar_init(bar + i, 1);
+        *abort = 0;
+        fence_mbar_init();
+        tma_prefetch_desc(&tm_k);
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, TM_COLS);
+        tmem_relinquish();
+    }
+    // X's strictly-upper 16 x 16 blocks stay zero for the whole kernel
+    for (int e = tid; e < 6 * 256; e += kThreads) {
+        const int blk = e >> 8, rr = (e >> 4) & 15, cc = e & 15;
+        const int R = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
+        const int C = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
+        X[(16 * R + rr) * LDX + 16 * C + cc] = 0.f;
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA + MMA issue
+        if (lane == 0) {
+            auto load = [&](int j) {
+                const long tile = first + (long)j * step;
+                const int bh = (int)(tile / nchunks), c = (int)(tile % nchunks);
+                uint8_t* st = sm + OFF_K + (j & 1) * 2 * TILE;
+                mbar_arrive_expect_tx(bar + B_FULL + (j & 1), 2 * TILE);
+                tma_load_3d(st, &tm_k, bar + B_FULL + (j & 1), 0, c * 64, bh);
+                tma_load_3d(st + TILE, &tm_k, bar + B_FULL + (j & 1), 64, c * 64, bh);
+            };
+            for (int j = 0; j < min(2, ntile); ++j) load(j);
+            bool ok = true;
+            for (int j = 0; j < ntile && ok; ++j) {
+                const int s = j & 1;
+                ok = wait_bounded(bar + B_FULL + s, (j >> 1) & 1, abort, limit_ns) &&
+                     (j == 0 || wait_bounded(bar + B_GP_FREE, (j - 1) & 1, abort, limit_ns));
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t st = sb + OFF_K + s * 2 * TILE;
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) {
+                    const uint32_t a = st + (ks >> 2) * TILE + (ks & 3) * 32;
+                    mma_bf16(tmem, sdesc_sw128(a, 16, 1024), sdesc_sw128(a, 16, 1024), ID_G, ks > 0);
+                }
+                mma_commit(bar + B_GP_FULL);
+                if (j + 2 < ntile) {        // the stage is free once this MMA has read it
+                    if (!(ok = wait_bounded(bar + B_GP_FULL, j & 1, abort, limit_ns))) break;
+                    load(j + 2);
+                }
+            }
+            mma_commit(bar + B_DRAIN);
+            mbar_wait(bar + B_DRAIN, 0, limit_ns);
+            for (int j = max(0, ntile - 2); j < ntile; ++j) mbar_wait(bar + B_FULL + (j & 1), (j >> 1) & 1, limit_ns);
+        }
+    } else {
+        // ------------------------------------------------------------ workers (128 threads)
+        const int wt = tid - 32;
+        const int q = warp & 3;                       // TMEM lane quarter of this warp
+        const int r = 32 * q + lane;                  // G row held by quarters 0 and 1
+        const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
+        auto beta_of = [&](int j) -> float {
+            if (j >= ntile || wt >= 64) return 0.f;
+            const long tile = first + (long)j * step;
+            const long bh = tile / nchunks;
+            const int t = (int)(tile % nchunks) * 64 + wt;
+            return t < T ? __bfloat162float(beta[bh * T + t]) : 0.f;
+        };
+        float beta_next = beta_of(0);
+        bool ok = true;
+        for (int j = 0; j < ntile; ++j) {
+            if (wt < 64) {
+                bt[wt] = beta_next;
+                beta_next = beta_of(j + 1);
+            }
+            ok = bar_and(NB_W, 128, ok && wait_bounded(bar + B_GP_FULL, j & 1, abort, limit_ns));
+            if (!ok) break;
+            tc_fence_after();
+            float g[64];
+            if (q < 2) {
+#pragma unroll
+                for (int m = 0; m < 4; ++m) {
+                    float t16[16];
+                    tmem_ld16(tmem + lane_off + 16 * m, t16);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) g[16 * m + e] = t16[e];
+                }
+                float lam = 0.f;
+#pragma unroll
+                for (int e = 0; e < 64; ++e) lam = (e == r) ? g[e] : lam;
+                al[r] = gate_alpha(bt[r], lam);
+            }
+            tc_fence_before();
+            bar_sync(NB_W, 128);                     // alpha visible, G read
+            if (wt == 0) mbar_arrive(bar + B_GP_FREE);
+            if (q < 2) {
+                // A^T[r][i] = A[i][r] = alpha_i G[i][r] = alpha_i G[r][i]; only i > r is read
+#pragma unroll
+                for (int m = 0; m < 16; ++m) {
+                    const float4 a = *reinterpret_cast<const float4*>(al + 4 * m);
+                    *reinterpret_cast<float4*>(At + r * LDX + 4 * m) =
+                        make_float4(a.x * g[4 * m], a.y * g[4 * m + 1], a.z * g[4 * m + 2], a.w * g[4 * m + 3]);
+                }
+            }
+            bar_sync(NB_W, 128);
+            ut::ut_solve<NB_W, 128>(At, X, wt);
+            {   // T = X diag(alpha) -> bf16, 64 bytes per thread
+                const long tile = first + (long)j * step;
+                const int rr = wt >> 1, h = wt & 1;
+                uint4* dst = reinterpret_cast<uint4*>(Tout + (tile * 64 + rr) * 64 + 32 * h);
+#pragma unroll
+                for (int m = 0; m < 4; ++m) {
+                    const float4 x0 = *reinterpret_cast<const float4*>(X + rr * LDX + 32 * h + 8 * m);
+                    const float4 x1 = *reinterpret_cast<const float4*>(X + rr * LDX + 32 * h + 8 * m + 4);
+                    const float4 a0 = *reinterpret_cast<const float4*>(al + 32 * h + 8 * m);
+                    const float4 a1 = *reinterpret_cast<const float4*>(al + 32 * h + 8 * m + 4);
+                    uint4 u;
+                    u.x = pack_bf16x2(x0.x * a0.x, x0.y * a0.y);
+                    u.y = pack_bf16x2(x0.z * a0.z, x0.w * a0.w);
+                    u.z = pack_bf16x2(x1.x * a1.x, x1.y * a1.y);
+                    u.w = pack_bf16x2(x1.z * a1.z, x1.w * a1.w);
+                    dst[m] = u;
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0 && *abort) atomicOr(err, kDevTimeout);
+    if (warp == 0) tmem_dealloc(tmem, TM_COLS);
+}
+
+int sm_count() {
+    static int n[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (!n[dev] && cudaDeviceGetAttribute(&n[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) n[dev] = 148;
+    return n[dev];
+}
+}  // namespace
+
+cudaError_t launch_ut(const void* k, const void* beta, void* Tout, long BH, int T, uint32_t* err,
+                      unsigned long long limit_ns, cudaStream_t stream) {
+    CUtensorMap mk;
+    if (!tma_map_tokens(&mk, k, 128, T, BH)) return cudaErrorInvalidValue;
+    const int nchunks = (T + 63) / 64;
+    const long ntiles = BH * nchunks;
+    const long grid = std::min<long>(ntiles, (long)sm_count() * kCtasPerSm);
+    cudaError_t e = cudaFuncSetAttribute(ut_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    ut_kernel<<<(unsigned)grid, kThreads, SMEM_BYTES, stream>>>(mk, (const __nv_bfloat16*)beta,
+                                                                (__nv_bfloat16*)Tout, T, nchunks, ntiles, err,
+                                                                limit_ns);
+    return cudaGetLastError();
+}
+
+}  // namespace efla

@@ -1,0 +1,139 @@
+// efla_ut_tf32.cuh -- the UT transform of one 64-token chunk: X = (I + A)^{-1}.
+//
+// Exact Flow Linear Attention, Section 3.3 applies the UT transform to the chunk
+// recurrence: with A = strictly-lower(diag(alpha) K K^T), the chunk's rank-1 writes are
+// Delta = T (V - K S) for T = (I + A)^{-1} diag(alpha) (row convention).  This header
+// builds X = (I + A)^{-1}; the caller applies diag(alpha).
+#pragma once
+
+#include <stdint.h>
+
+#include "sm100.cuh"
+
+namespace efla {
+namespace ut {
+
+using sm100::bar_sync;
+constexpr int LDX = 68;          // fp32 row stride of At and X (16-byte aligned rows)
+
+// X = (I + A)^{-1} for the 64 x 64 strictly-lower A, by NT >= 128 threads (ptid, named barrier NB),
+// with
+//   At[j * LDX + i] = A[i][j] (i > j)  -- only that part of At is read;
+//   the merge products are kept in At's other triangle (At[r * LDX + c], r > c).
+// X's strictly-upper 16 x 16 blocks are zero from the start of the kernel.
+//   (1) 16 x 16 diagonal blocks by forward substitution, one thread per column (fp32);
+//   (2) 32 x 32 merges X21 = -X22 (A21 X11);  (3) the 64 x 64 merge the same way.
+// The merge products run as warp-level TF32 tensor-core tiles (m16n8k8, fp32
+// accumulation): operands are read from shared memory once per warp fragment instead of
+// once per output, which is what bounds a CUDA-core solve.  TF32 operands (10-bit
+// mantissa, round-to-nearest) are finer than the bf16 rounding T receives afterwards.
+// Tiles that multiply a structural zero block of a triangular factor are skipped.
+
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+
+// D += A(16x8, row) B(8x8, col), TF32 in, fp32 accumulate
+__device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+// One warp: C(16 x 16) = sum over k-steps [k0, k1) of A(16 x 8) B(8 x 16).
+//   A(r, k) = a_base[k * a_ks + r * a_rs]      B(k, n) = b_base[k * LDX + n]
+// Output fragment: rows g, g + 8 (g = lane / 4), columns 8 nt + 2 t, + 1 (t = lane % 4).
+__device__ __forceinline__ void warp_mm16x16(float (&c)[2][4], const float* __restrict__ a_base, int a_ks,
+                                             int a_rs, const float* __restrict__ b_base, int k0, int k1,
+                                             int lane) {
+    const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) c[nt][e] = 0.f;
+    for (int ks = k0; ks < k1; ++ks) {
+        const int k = 8 * ks + t;
+        uint32_t a[4];
+        a[0] = to_tf32(a_base[k * a_ks + g * a_rs]);
+        a[1] = to_tf32(a_base[k * a_ks + (g + 8) * a_rs]);
+        a[2] = to_tf32(a_base[(k + 4) * a_ks + g * a_rs]);
+        a[3] = to_tf32(a_base[(k + 4) * a_ks + (g + 8) * a_rs]);
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+            uint32_t b[2];
+            b[0] = to_tf32(b_base[k * LDX + 8 * nt + g]);
+            b[1] = to_tf32(b_base[(k + 4) * LDX + 8 * nt + g]);
+            mma_tf32(c[nt], a, b);
+        }
+    }
+}
+
+// Store a 16 x 16 fragment (times `scale`) at dst[r * LDX + c].
+__device__ __forceinline__ void warp_st16x16(float* __restrict__ dst, const float (&c)[2][4], float scale, int lane) {
+    const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+        *reinterpret_cast<float2*>(dst + g * LDX + 8 * nt + 2 * t) = make_float2(scale * c[nt][0], scale * c[nt][1]);
+        *reinterpret_cast<float2*>(dst + (g + 8) * LDX + 8 * nt + 2 * t) = make_float2(scale * c[nt][2], scale * c[nt][3]);
+    }
+}
+
+template <int NB, int NT>
+__device__ __forceinline__ void ut_solve(float* __restrict__ At, float* __restrict__ X, int ptid) {
+    static_assert(NT >= 128, "the solve uses four warps");
+    const int pw = ptid >> 5, lane = ptid & 31;
+    if (ptid < 64) {   // (1) column c of diagonal block b; A rows read four at a time
+        const int b = ptid >> 4, c = ptid & 15;
+        const float* Ab = At + (16 * b) * LDX + 16 * b;
+        float x[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) x[i] = (i == c) ? 1.f : 0.f;
+#pragma unroll
+        for (int j = 0; j < 15; ++j) {
+            const float xj = x[j];
+#pragma unroll
+            for (int m = (j + 1) >> 2; m < 4; ++m) {
+                const float4 a = *reinterpret_cast<const float4*>(Ab + j * LDX + 4 * m);
+                const float av[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    if (4 * m + e > j) x[4 * m + e] = fmaf(-av[e], xj, x[4 * m + e]);
+            }
+        }
+        float* Xb = X + (16 * b) * LDX + 16 * b + c;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) Xb[i * LDX] = x[i];
+    }
+    bar_sync(NB, NT);
+    float acc[2][4];
+    if (pw < 2) {      // (2a) Y = A21 X11 for super-block pw (16 x 16 x 16; X11 lower: k >= n)
+        const int r0 = 32 * pw + 16, c0 = 32 * pw;
+        warp_mm16x16(acc, At + c0 * LDX + r0, LDX, 1, X + c0 * LDX + c0, 0, 2, lane);
+        warp_st16x16(At + r0 * LDX + c0, acc, 1.f, lane);
+    }
+    bar_sync(NB, NT);
+    if (pw < 2) {      // (2b) X21 = -X22 Y
+        const int r0 = 32 * pw + 16, c0 = 32 * pw;
+        warp_mm16x16(acc, X + r0 * LDX + r0, 1, LDX, At + r0 * LDX + c0, 0, 2, lane);
+        warp_st16x16(X + r0 * LDX + c0, acc, -1.f, lane);
+    }
+    bar_sync(NB, NT);
+    if (pw < 4) {      // (3a) Y = A21 X11 (32 x 32 x 32); tile (wr, wc), X11[k][n] = 0 for k < 16 wc
+        const int wr = pw >> 1, wc = pw & 1;
+        warp_mm16x16(acc, At + 32 + 16 * wr, LDX, 1, X + 16 * wc, 2 * wc, 4, lane);
+        warp_st16x16(At + (32 + 16 * wr) * LDX + 16 * wc, acc, 1.f, lane);
+    }
+    bar_sync(NB, NT);
+    if (pw < 4) {      // (3b) X21 = -X22 Y; X22[m][k] = 0 for k > 16 wr + 15
+        const int wr = pw >> 1, wc = pw & 1;
+        warp_mm16x16(acc, X + (32 + 16 * wr) * LDX + 32, 1, LDX, At + 32 * LDX + 16 * wc, 0, 2 * wr + 2, lane);
+        warp_st16x16(X + (32 + 16 * wr) * LDX + 16 * wc, acc, -1.f, lane);
+    }
+    bar_sync(NB, NT);
+}
+
+}  // namespace ut
+}  // namespace efla

@@ -84,7 +84,9 @@ size_t efla_chunk_fwd_workspace_bytes(int B, int H, int T, int d_k, int d_v, int
  *   o must not overlap any input.
  *   workspace: device memory of at least efla_chunk_fwd_workspace_bytes(...) bytes,
  *   16-byte aligned, owned by the caller; its first bytes hold a sticky device error word
- *   (zero it once before first use, e.g. with cudaMemset).
+ *   (zero it once before first use, e.g. with cudaMemset).  For bf16 with d = 128 it also
+ *   holds every chunk's UT transform T (8 KiB per (stream, chunk)); calls that overlap
+ *   on the GPU must not share a workspace.
  *
  * Supported: d_k = d_v in {64, 128}, chunk = 64, any T >= 1 (the tail chunk is padded with
  * k = 0, beta = 0 tokens, which are exact no-ops), B*H >= 1.
@@ -104,9 +106,10 @@ int efla_chunk_fwd(const void *q, const void *k, const void *v, const void *beta
  * paths where cudaMalloc (which may synchronise the device) is not acceptable.
  *
  * Arguments, layouts, supported shapes and results are those of efla_chunk_fwd.  The
- * scratch is a 16 MiB static device array inside the library (held on every GPU that
- * loads it, until exit): a problem whose efla_chunk_fwd_workspace_bytes exceeds 16 MiB
- * returns EFLA_ERR_UNSUPPORTED and launches nothing.  No device memory is allocated.
+ * scratch is a 32 MiB static device array inside the library (held on every GPU that
+ * loads it, until exit): a problem whose efla_chunk_fwd_workspace_bytes exceeds 32 MiB
+ * (for bf16, d = 128: more than 4095 (stream, 64-token chunk) tiles) returns
+ * EFLA_ERR_UNSUPPORTED and launches nothing.  No device memory is allocated.
  * The first call on a device looks up the array's device address (with that device
  * current); make that first call before any stream capture.  Every call shares the one
  * array and each call clears its error word first, so calls that overlap on the GPU
