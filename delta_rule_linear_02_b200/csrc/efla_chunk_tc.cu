@@ -6,31 +6,35 @@
 // transform T of every chunk comes precomputed from efla_ut.cu (bf16, via TMA).
 //
 // Per 64-token chunk (Exact Flow Linear Attention, Section 3.3; row convention):
-//   [. ; P~] = [K; Q] K^T                   M=128 MMA  (P = P~ with the causal mask, diagonal kept)
-//   [. ; W | U] = [P; T] [K | V]            M=128, N=192 MMA
-//   [QS; WS] = [Q; W] S                     M=128 MMA
-//   Delta = U - WS                          fp32, then a bf16 operand
-//   S += K^T Delta;  [O; .] = [QS; .] + [P; T] Delta               two M=128 MMAs
+//   [W | U] = T [K | V]                      (M=64, N=192)
+//   WS = W S                                 (M=64)      -- on the state chain
+//   Delta = U - WS                           fp32, then a bf16 operand
+//   S += K^T Delta                           (M=128)     -- on the state chain
+//   P~ = Q K^T, P = P~ masked causally (diagonal kept)              (M=64)
+//   O = Q S + P Delta                        (M=64, two MMAs into one accumulator)
 // Tokens past T are zero-filled by TMA (k = 0, and T's rows/columns are zero there).
 //
-// Warp roles (12 warps).  Only S -> [Q;W]S -> Delta -> K^T Delta -> S is sequential;
-// everything that does not depend on S runs a chunk ahead on other warps:
-//   warp 0       one thread polls its barriers and issues whatever is ready: the TMA
-//                copies (K, Q, V, T of chunk c into a 2-deep stage ring), [K;Q]K^T and
-//                [P;T][K|V]
-//   warp 1       chain MMA issue: [Q;W]S, K^T Delta, [P;T]Delta
-//   warps 2-3    converter: TMEM rows 64..127 -> the masked P operand, the bf16 W operand
-//                and fp32 U
-//   warps 4-11   chain, two warps per TMEM lane quarter (one per 32-column half): Delta,
-//                the state's bf16 copy, O and the final state
+// One warp issues every MMA in a fixed order per chunk c:
+//   W S(c), Q S(c), [W|U](c+1), K^T Delta(c) (after Delta), P Delta(c), Q K^T(c+1)
+// so the two MMAs of the state chain never queue behind work that could have waited:
+// the others fill the tensor pipe while the chain's epilogues run.  The M=64 products
+// leave lanes 16..31 of each TMEM lane quarter unused (row r is in lane (r%16) + 32(r/16)).
+//
+// Warp roles (14 warps):
+//   warp 0       TMA: K, V, Q, T of chunk c into a 3-deep stage ring, L2 prefetch ahead
+//   warp 1       the MMA issuer (warp-uniform control flow, one elected lane issues)
+//   warps 2-5    converter (one per TMEM lane quarter): the bf16 W operand, fp32 U and
+//                the masked P operand, in that order (W is on the state chain, P is not)
+//   warps 6-13   chain, two per lane quarter (one per 32-column half): Delta, the state's
+//                bf16 copy, O and the final state
 // Operands are staged by TMA (128-byte swizzle, no multicast) or written in the same
 // swizzled layouts.  Every wait is bounded (2 s); a wait that runs out sets a CTA-wide
 // abort flag, every role winds down, and the caller's workspace records the timeout.
 // `dbg` (null in the library) receives CTA 0's chunk-0 intermediates for diagnosis:
 // W [8256,16448) U [16448,20544) WS [20544,24640) S after the chunk [24640,32832); and
 // per chunk c < 64 the cycle at which each role passed its milestones, at
-// [40000 + 16 c + k): k = 0..3 MMA issue of [K;Q]K^T, [P;T][K|V], [Q;W]S, S-update;
-// 4 P ready; 6 W ready; 7 U ready; 8 Delta ready; 9 new S ready; 10 O stored; 11 TMA.
+// [40000 + 16 c + k): k = 0 QK^T, 1 [W|U], 2 WS, 3 K^T Delta issued; 4 P ready; 6 W ready;
+// 7 U ready; 8 Delta ready; 9 new S ready; 10 O stored; 11 TMA issued.
 #include <cudaTypedefs.h>
 
 #include "efla_common.cuh"
@@ -43,20 +47,22 @@ namespace efla {
 namespace {
 using namespace sm100;
 
-constexpr int kThreads = 384;
+constexpr int kThreads = 448;
 constexpr int kD = 128;          // d_k = d_v
 constexpr int LDU = 68;          // fp32 row stride of the U rows (16-byte aligned, conflict-free)
+constexpr int kStages = 3;
 
 // ---- shared-memory map (bytes from a 1024-aligned base)
-// stage s (x2): [K a0 | Q a0 | W a0 | K a1 | Q a1 | W a1 | V | P | T]: 9 tiles of 64 x 64 bf16
+// stage s (x3): [K a0 | K a1 | V | Q a0 | Q a1 | T]: 6 tiles of 64 x 64 bf16, 128-byte swizzle
 constexpr uint32_t TILE = 8192;
-constexpr uint32_t ATOM_STRIDE = 3 * TILE;          // a0 -> a1 (one 64-column half of d_k)
-constexpr uint32_t ST_K = 0, ST_Q = TILE, ST_W = 2 * TILE, ST_V = 6 * TILE, ST_P = 7 * TILE, ST_T = 8 * TILE;
-constexpr uint32_t STAGE_BYTES = 9 * TILE;
+constexpr uint32_t ST_K = 0, ST_V = 2 * TILE, ST_Q = 3 * TILE, ST_T = 5 * TILE;
+constexpr uint32_t STAGE_BYTES = 6 * TILE;
 constexpr uint32_t OFF_STAGE = 0;
-constexpr uint32_t OFF_DL = OFF_STAGE + 2 * STAGE_BYTES;   // Delta, MN-major 64 x 64
-constexpr uint32_t OFF_SB = OFF_DL + TILE;                 // S bf16, MN-major 128 x 64
-constexpr uint32_t OFF_U = OFF_SB + 2 * TILE;              // U rows, fp32
+constexpr uint32_t OFF_W = OFF_STAGE + kStages * STAGE_BYTES;   // W bf16, K-major 64 x 128
+constexpr uint32_t OFF_P = OFF_W + 2 * TILE;                    // P bf16, K-major 64 x 64
+constexpr uint32_t OFF_DL = OFF_P + TILE;                       // Delta, MN-major 64 x 64
+constexpr uint32_t OFF_SB = OFF_DL + TILE;                      // S bf16, MN-major 128 x 64
+constexpr uint32_t OFF_U = OFF_SB + 2 * TILE;                   // U rows, fp32
 constexpr uint32_t OFF_BAR = OFF_U + 64 * LDU * 4;
 constexpr uint32_t NBAR = 24;
 constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
@@ -66,28 +72,32 @@ static_assert(SMEM_BYTES <= 232448, "shared-memory map exceeds 227 KB");
 
 // ---- mbarriers (all count 1)
 enum : int {
-    B_FULL = 0,        // [2] TMA landed stage s
-    B_STAGE_FREE = 2,  // [2] last MMA reading stage s done
-    B_GP_FULL = 4, B_GP_FREE, B_P_READY, B_WU_FULL, B_WU_FREE, B_W_READY, B_U_READY, B_U_FREE,
-    B_Y_FULL = 12,     // [2]
-    B_D_READY = 14, B_S_FULL,
-    B_O_FULL = 16,     // [2]
-    B_SB_READY = 18,
-    B_Y_FREE = 19,     // [2]
-    B_DRAIN = 21,      // [2] one per issuing thread
+    B_FULL = 0,         // [3] TMA landed stage s
+    B_STAGE_FREE = 3,   // [3] last MMA reading stage s done
+    B_GP_FULL = 6, B_GP_FREE, B_P_READY, B_WU_FULL, B_WU_FREE, B_W_READY, B_U_READY, B_U_FREE,
+    B_WS_FULL = 14, B_D_READY, B_S_FULL,
+    B_O_FULL = 17,      // [2]
+    B_O_FREE = 19,      // [2]
+    B_SB_READY = 21,
+    B_DRAIN = 22,       // [2] one per issuing thread
 };
 
-// ---- TMEM columns (fp32 accumulators, lanes 0..127)
-constexpr uint32_t TM_S = 0, TM_Y = 64 /* x2 */, TM_GP = 192, TM_WU = 256, TM_COLS = 512;
+// ---- TMEM columns (fp32 accumulators)
+constexpr uint32_t TM_S = 0;          // M=128: S (d_k x 64)
+constexpr uint32_t TM_WS = 64;        // M=64:  W S
+constexpr uint32_t TM_O = 128;        // M=64, x2: Q S + P Delta
+constexpr uint32_t TM_GP = 256;       // M=64:  Q K^T
+constexpr uint32_t TM_WU = 320;       // M=64, N=192: [W | U]
+constexpr uint32_t TM_COLS = 512;
 
-constexpr uint32_t ID_GP = idesc_bf16(128, 64, false, false);
-constexpr uint32_t ID_WU = idesc_bf16(128, 192, false, true);
-constexpr uint32_t ID_Y = idesc_bf16(128, 64, false, true);
+constexpr uint32_t ID_QK = idesc_bf16(64, 64, false, false);
+constexpr uint32_t ID_XS = idesc_bf16(64, 64, false, true);     // W S, Q S, P Delta
+constexpr uint32_t ID_WU = idesc_bf16(64, 192, false, true);
 constexpr uint32_t ID_S = idesc_bf16(128, 64, true, true);
 
 // ---- named barriers
-constexpr int NB_CHAIN = 1, NB_DELTA = 2, NB_OUT = 3, NB_CONV = 5;
-constexpr int kChainThreads = 256;   // warps 4..11: two per TMEM lane quarter, one per column half
+constexpr int NB_CHAIN = 1, NB_CONV = 2;
+constexpr int kChainThreads = 256, kConvThreads = 128;
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
     __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
@@ -124,6 +134,20 @@ struct Ctl {
     }
 };
 
+// One accumulator tile: nk tcgen05.mma of K = 16, issued by a converged warp.  Operand k-step ks starts at
+// base + (ks / 4) * atom + (ks % 4) * step (a K-major operand walks 32 bytes within a
+// 64-column swizzle atom and jumps `atom` bytes between atoms; an MN-major operand walks
+// 16 rows = 2048 bytes, atom = 8192).
+__device__ __forceinline__ void mma_group(uint32_t d, uint32_t a, uint32_t a_atom, uint32_t a_step, uint32_t a_lbo,
+                                       uint32_t b, uint32_t b_atom, uint32_t b_step, uint32_t b_lbo, uint32_t idesc,
+                                       int nk, uint32_t acc) {
+#pragma unroll
+    for (int ks = 0; ks < nk; ++ks) {
+        mma_bf16_elect(d, sdesc_sw128(a + (ks >> 2) * a_atom + (ks & 3) * a_step, a_lbo, 1024),
+                       sdesc_sw128(b + (ks >> 2) * b_atom + (ks & 3) * b_step, b_lbo, 1024), idesc, (acc | ks) != 0);
+    }
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_t,
@@ -137,9 +161,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     Ctl ctl{reinterpret_cast<uint64_t*>(sm + OFF_BAR), reinterpret_cast<volatile int*>(sm + OFF_MISC + 4), limit_ns};
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int q = warp & 3;                                                  // TMEM lane quarter
+    const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
     const int bh = blockIdx.x >> 1;
     const int col0 = (blockIdx.x & 1) * 64;
-    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;   // this warp's TMEM lanes
     const int nchunks = (T + 63) / 64;
     const size_t tok0 = (size_t)bh * T;
     const long long t_start = clock64();
@@ -167,200 +192,182 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const uint32_t tmem = *tmem_slot;
 
     if (warp == 0) {
-        // ================================================================ TMA + [K;Q]K^T + [P;T][K|V]
-        if (lane == 0) {
-            int it = 0, ia = 0, ic = 0;       // next chunk to load / to issue [K;Q]K^T / [P;T][K|V] for
-            unsigned idle = 0;
-            uint64_t last = globaltimer_ns();
-            while (ic < nchunks) {
-                if (*ctl.abort) break;
-                bool did = true;
-                if (ic < ia && mbar_test_wait(ctl.b(B_P_READY), ic & 1) &&
-                    (ic == 0 || mbar_test_wait(ctl.b(B_WU_FREE), (ic - 1) & 1))) {
-                    // [. ; W | U] = [P; T] [K | V]
-                    tc_fence_after();
-                    const uint32_t st = sb + OFF_STAGE + (ic & 1) * STAGE_BYTES;
-#pragma unroll
-                    for (int ks = 0; ks < 4; ++ks)
-                        mma_bf16(tmem + TM_WU, sdesc_sw128(st + ST_P + ks * 32, 16, 1024),
-                                 sdesc_sw128(st + ST_K + ks * 2048, ATOM_STRIDE, 1024), ID_WU, ks > 0);
-                    mma_commit(ctl.b(B_WU_FULL));
-                    EFLA_STAMP(ic, 1);
-                    ++ic;
-                } else if (ia < it && mbar_test_wait(ctl.b(B_FULL + (ia & 1)), (ia >> 1) & 1) &&
-                           (ia == 0 || mbar_test_wait(ctl.b(B_GP_FREE), (ia - 1) & 1))) {
-                    // [. ; P~] = [K; Q] K^T
-                    tc_fence_after();
-                    const uint32_t sa = sb + OFF_STAGE + (ia & 1) * STAGE_BYTES;
-#pragma unroll
-                    for (int ks = 0; ks < 8; ++ks) {
-                        const uint32_t aa = sa + (ks >> 2) * ATOM_STRIDE + ST_K + (ks & 3) * 32;
-                        mma_bf16(tmem + TM_GP, sdesc_sw128(aa, 16, 1024), sdesc_sw128(aa, 16, 1024), ID_GP, ks > 0);
-                    }
-                    mma_commit(ctl.b(B_GP_FULL));
-                    EFLA_STAMP(ia, 0);
-                    ++ia;
-                } else if (it < nchunks && (it < 2 || mbar_test_wait(ctl.b(B_STAGE_FREE + (it & 1)), ((it - 2) >> 1) & 1))) {
-                    const int s = it & 1;
-                    uint8_t* st = sm + OFF_STAGE + s * STAGE_BYTES;
-                    uint64_t* full = ctl.b(B_FULL + s);
-                    mbar_arrive_expect_tx(full, 6 * TILE);
-                    const int t0 = it * 64;
-                    tma_load_3d(st + ST_K, &tm_k, full, 0, t0, bh);
-                    tma_load_3d(st + ST_Q, &tm_q, full, 0, t0, bh);
-                    tma_load_3d(st + ATOM_STRIDE + ST_K, &tm_k, full, 64, t0, bh);
-                    tma_load_3d(st + ATOM_STRIDE + ST_Q, &tm_q, full, 64, t0, bh);
-                    tma_load_3d(st + ST_V, &tm_v, full, col0, t0, bh);
-                    tma_load_2d(st + ST_T, &tm_t, full, 0, (bh * nchunks + it) * 64);
-                    EFLA_STAMP(it, 11);
-                    if (it + 2 < nchunks) {   // its stage frees only after this chunk: warm L2 now
-                        const int t2 = t0 + 128;
-                        tma_prefetch_l2_3d(&tm_k, 0, t2, bh);
-                        tma_prefetch_l2_3d(&tm_q, 0, t2, bh);
-                        tma_prefetch_l2_3d(&tm_k, 64, t2, bh);
-                        tma_prefetch_l2_3d(&tm_q, 64, t2, bh);
-                        tma_prefetch_l2_3d(&tm_v, col0, t2, bh);
-                        tma_prefetch_l2_2d(&tm_t, 0, (bh * nchunks + it + 2) * 64);
-                    }
-                    ++it;
-                } else {
-                    did = false;
-                }
-                if (did) {
-                    idle = 0;
-                } else if (++idle >= 512) {   // read the clock only now and then
-                    idle = 0;
-                    const uint64_t now = globaltimer_ns();
-                    if (now - last > limit_ns) {
-                        *ctl.abort = 1;
-                        break;
-                    }
-                    continue;
-                }
-                if (did) last = globaltimer_ns();
-            }
-            // every copy and MMA this thread issued has landed before the CTA can exit
-            mma_commit(ctl.b(B_DRAIN));
-            mbar_wait(ctl.b(B_DRAIN), 0, limit_ns);
-            for (int c = max(0, it - 2); c < it; ++c) mbar_wait(ctl.b(B_FULL + (c & 1)), (c >> 1) & 1, limit_ns);
-        }
-    } else if (warp == 1) {
-        // ================================================================ chain issuer
+        // ================================================================ TMA producer
         if (lane == 0) {
             bool ok = true;
+            int issued = 0;
             for (int c = 0; c < nchunks && ok; ++c) {
-                const int s = c & 1;
-                const uint32_t st = sb + OFF_STAGE + s * STAGE_BYTES;
-                // [QS; WS] = [Q; W] S
-                ok = ctl.wait(B_W_READY, c & 1) && ctl.wait(B_SB_READY, c & 1) &&
-                     (c < 2 || ctl.wait(B_Y_FREE + s, ((c - 2) >> 1) & 1));
-                if (!ok) break;
-                tc_fence_after();
-#pragma unroll
-                for (int ks = 0; ks < 8; ++ks) {
-                    const uint32_t aa = st + (ks >> 2) * ATOM_STRIDE + ST_Q + (ks & 3) * 32;
-                    mma_bf16(tmem + TM_Y + 64 * s, sdesc_sw128(aa, 16, 1024),
-                             sdesc_sw128(sb + OFF_SB + ks * 2048, TILE, 1024), ID_Y, ks > 0);
+                const int s = c % kStages;
+                if (c >= kStages && !(ok = ctl.wait(B_STAGE_FREE + s, ((c - kStages) / kStages) & 1))) break;
+                uint8_t* st = sm + OFF_STAGE + s * STAGE_BYTES;
+                uint64_t* full = ctl.b(B_FULL + s);
+                mbar_arrive_expect_tx(full, 6 * TILE);
+                const int t0 = c * 64;
+                tma_load_3d(st + ST_K, &tm_k, full, 0, t0, bh);
+                tma_load_3d(st + ST_K + TILE, &tm_k, full, 64, t0, bh);
+                tma_load_3d(st + ST_V, &tm_v, full, col0, t0, bh);
+                tma_load_3d(st + ST_Q, &tm_q, full, 0, t0, bh);
+                tma_load_3d(st + ST_Q + TILE, &tm_q, full, 64, t0, bh);
+                tma_load_2d(st + ST_T, &tm_t, full, 0, (bh * nchunks + c) * 64);
+                EFLA_STAMP(c, 11);
+                issued = c + 1;
+                if (c + kStages < nchunks) {  // its stage frees only after this chunk: warm L2 now
+                    const int t2 = t0 + 64 * kStages;
+                    tma_prefetch_l2_3d(&tm_k, 0, t2, bh);
+                    tma_prefetch_l2_3d(&tm_k, 64, t2, bh);
+                    tma_prefetch_l2_3d(&tm_v, col0, t2, bh);
+                    tma_prefetch_l2_3d(&tm_q, 0, t2, bh);
+                    tma_prefetch_l2_3d(&tm_q, 64, t2, bh);
+                    tma_prefetch_l2_2d(&tm_t, 0, (bh * nchunks + c + kStages) * 64);
                 }
-                mma_commit(ctl.b(B_Y_FULL + s));
-                EFLA_STAMP(c, 2);
-                // S += K^T Delta, then [O; .] += [P; T] Delta
-                if (!(ok = ctl.wait(B_D_READY, c & 1))) break;
-                tc_fence_after();
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    mma_bf16(tmem + TM_S, sdesc_sw128(st + ST_K + ks * 2048, ATOM_STRIDE, 1024),
-                             sdesc_sw128(sb + OFF_DL + ks * 2048, TILE, 1024), ID_S, 1);
-                mma_commit(ctl.b(B_S_FULL));
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    mma_bf16(tmem + TM_Y + 64 * s, sdesc_sw128(st + ST_P + ks * 32, 16, 1024),
-                             sdesc_sw128(sb + OFF_DL + ks * 2048, TILE, 1024), ID_Y, 1);
-                mma_commit(ctl.b(B_O_FULL + s));
-                mma_commit(ctl.b(B_STAGE_FREE + s));
-                EFLA_STAMP(c, 3);
             }
-            mma_commit(ctl.b(B_DRAIN + 1));
-            mbar_wait(ctl.b(B_DRAIN + 1), 0, limit_ns);
+            for (int c = max(0, issued - kStages); c < issued; ++c)   // no copy may land after exit
+                mbar_wait(ctl.b(B_FULL + c % kStages), (c / kStages) & 1, limit_ns);
         }
-    } else if (warp < 4) {
-        // ================================================================ converter (TMEM lanes 64..127)
-        const int r = tid - 64;                       // chunk row
+    } else if (warp == 1) {
+        // ================================================================ MMA issuer (whole warp)
+        // Control flow stays warp-uniform: every lane polls the barrier (a converged wait)
+        // and the warp votes on the outcome; elect.sync inside each MMA and commit picks
+        // the issuing lane.
+        auto wait = [&](int i, uint32_t parity) { return __all_sync(0xffffffffu, ctl.wait(i, parity)); };
+        auto stage = [&](int c) { return sb + OFF_STAGE + (c % kStages) * STAGE_BYTES; };
+        auto issue_qk = [&](int c) {      // P~ = Q K^T (M = 64)
+            tc_fence_after();
+            const uint32_t st = stage(c);
+            mma_group(tmem + TM_GP, st + ST_Q, TILE, 32, 16, st + ST_K, TILE, 32, 16, ID_QK, 8, 0);
+            mma_commit_elect(ctl.b(B_GP_FULL));
+            EFLA_STAMP(c, 0);
+        };
+        auto issue_wu = [&](int c) {      // [W | U] = T [K | V] (M = 64, N = 192)
+            tc_fence_after();
+            const uint32_t st = stage(c);
+            mma_group(tmem + TM_WU, st + ST_T, TILE, 32, 16, st + ST_K, 8192, 2048, TILE, ID_WU, 4, 0);
+            mma_commit_elect(ctl.b(B_WU_FULL));
+            EFLA_STAMP(c, 1);
+        };
+        bool ok = wait(B_FULL, 0);
+        if (ok) {
+            issue_qk(0);
+            issue_wu(0);
+        }
+        for (int c = 0; c < nchunks && ok; ++c) {
+            const uint32_t st = stage(c);
+            const int b = c & 1;
+            // W S (state chain)
+            if (!(ok = wait(B_W_READY, c & 1) && wait(B_SB_READY, c & 1))) break;
+            tc_fence_after();
+            mma_group(tmem + TM_WS, sb + OFF_W, TILE, 32, 16, sb + OFF_SB, 8192, 2048, TILE, ID_XS, 8, 0);
+            mma_commit_elect(ctl.b(B_WS_FULL));
+            EFLA_STAMP(c, 2);
+            // Q S into O[b]
+            if (c >= 2 && !(ok = wait(B_O_FREE + b, ((c - 2) >> 1) & 1))) break;
+            tc_fence_after();
+            mma_group(tmem + TM_O + 64 * b, st + ST_Q, TILE, 32, 16, sb + OFF_SB, 8192, 2048, TILE, ID_XS, 8, 0);
+            // the next chunk's [W | U] fills the pipe while Delta is formed
+            if (c + 1 < nchunks) {
+                if (!(ok = wait(B_FULL + (c + 1) % kStages, ((c + 1) / kStages) & 1) && wait(B_WU_FREE, c & 1))) break;
+                issue_wu(c + 1);
+            }
+            // S += K^T Delta (state chain)
+            if (!(ok = wait(B_D_READY, c & 1))) break;
+            tc_fence_after();
+            mma_group(tmem + TM_S, st + ST_K, 8192, 2048, TILE, sb + OFF_DL, 8192, 2048, TILE, ID_S, 4, 1);
+            mma_commit_elect(ctl.b(B_S_FULL));
+            EFLA_STAMP(c, 3);
+            // O += P Delta
+            if (!(ok = wait(B_P_READY, c & 1))) break;
+            tc_fence_after();
+            mma_group(tmem + TM_O + 64 * b, sb + OFF_P, TILE, 32, 16, sb + OFF_DL, 8192, 2048, TILE, ID_XS, 4, 1);
+            mma_commit_elect(ctl.b(B_O_FULL + b));
+            mma_commit_elect(ctl.b(B_STAGE_FREE + c % kStages));
+            // the next chunk's Q K^T
+            if (c + 1 < nchunks) {
+                if (!(ok = wait(B_GP_FREE, c & 1))) break;
+                issue_qk(c + 1);
+            }
+        }
+        mma_commit_elect(ctl.b(B_DRAIN));
+        if (lane == 0) mbar_wait(ctl.b(B_DRAIN), 0, limit_ns);
+        __syncwarp();
+    } else if (warp < 6) {
+        // ================================================================ converter (one warp per lane quarter)
+        const int r = 16 * q + lane;                  // chunk row held by lanes 0..15
+        const bool act = lane < 16;
         bool ok = true;
         for (int c = 0; c < nchunks && ok; ++c) {
-            const int s = c & 1;
-            uint8_t* st = sm + OFF_STAGE + s * STAGE_BYTES;
-            // P = P~ with the causal mask (diagonal kept) -> bf16 K-major rows
-            ok = bar_and(NB_CONV, 64, ctl.wait(B_GP_FULL, c & 1));
-            if (!ok) break;
-            tc_fence_after();
-#pragma unroll
-            for (int qd = 0; qd < 4; ++qd) {
-                float t16[16];
-                tmem_ld16(tmem + lane_off + TM_GP + 16 * qd, t16);
-                tmem_wait_ld();
-#pragma unroll
-                for (int j = 0; j < 16; ++j) t16[j] = (16 * qd + j <= r) ? t16[j] : 0.f;
-                st_chunk(st + ST_P + sw128_off(r, 2 * qd), t16);
-                st_chunk(st + ST_P + sw128_off(r, 2 * qd + 1), t16 + 8);
-            }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            bar_sync(NB_CONV, 64);
-            if (r == 0) {
-                mbar_arrive(ctl.b(B_GP_FREE));
-                mbar_arrive(ctl.b(B_P_READY));
-                EFLA_STAMP(c, 4);
-            }
             // W row r -> bf16, K-major, two 64-column atoms
-            ok = bar_and(NB_CONV, 64, ctl.wait(B_WU_FULL, c & 1));
+            ok = bar_and(NB_CONV, kConvThreads, ctl.wait(B_WU_FULL, c & 1));
             if (!ok) break;
             tc_fence_after();
 #pragma unroll
-            for (int qd = 0; qd < 8; ++qd) {
-                float w16[16];
-                tmem_ld16(tmem + lane_off + TM_WU + 16 * qd, w16);
-                tmem_wait_ld();
-                uint8_t* dst = st + (qd >> 2) * ATOM_STRIDE + ST_W;
-                st_chunk(dst + sw128_off(r, (qd & 3) * 2), w16);
-                st_chunk(dst + sw128_off(r, (qd & 3) * 2 + 1), w16 + 8);
-                if (dbg && blockIdx.x == 0 && c == 0)
-                    for (int j = 0; j < 16; ++j) dbg[8256 + r * 128 + 16 * qd + j] = w16[j];
+            for (int h = 0; h < 2; ++h) {
+                float w[64];
+                tmem_ld64_wait(tmem + lane_off + TM_WU + 64 * h, w);
+                if (act) {
+                    uint8_t* dst = sm + OFF_W + h * TILE;
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) st_chunk(dst + sw128_off(r, j), w + 8 * j);
+                    if (dbg && blockIdx.x == 0 && c == 0)
+                        for (int j = 0; j < 64; ++j) dbg[8256 + r * 128 + 64 * h + j] = w[j];
+                }
             }
             fence_proxy_async_smem();
-            bar_sync(NB_CONV, 64);
-            if (r == 0) {
+            bar_sync(NB_CONV, kConvThreads);
+            if (warp == 2 && lane == 0) {
                 mbar_arrive(ctl.b(B_W_READY));
                 EFLA_STAMP(c, 6);
             }
             // U row r stays fp32 (after the chain has read the previous chunk's)
-            ok = bar_and(NB_CONV, 64, c == 0 || ctl.wait(B_U_FREE, (c - 1) & 1));
+            ok = bar_and(NB_CONV, kConvThreads, c == 0 || ctl.wait(B_U_FREE, (c - 1) & 1));
             if (!ok) break;
+            {
+                float u[64];
+                tmem_ld64_wait(tmem + lane_off + TM_WU + 128, u);
+                if (act) {
 #pragma unroll
-            for (int qd = 0; qd < 4; ++qd) {
-                float u16[16];
-                tmem_ld16(tmem + lane_off + TM_WU + 128 + 16 * qd, u16);
-                tmem_wait_ld();
-#pragma unroll
-                for (int j = 0; j < 16; j += 4)
-                    *reinterpret_cast<float4*>(Us + r * LDU + 16 * qd + j) = make_float4(u16[j], u16[j + 1], u16[j + 2], u16[j + 3]);
-                if (dbg && blockIdx.x == 0 && c == 0)
-                    for (int j = 0; j < 16; ++j) dbg[16448 + r * 64 + 16 * qd + j] = u16[j];
+                    for (int j = 0; j < 64; j += 4)
+                        *reinterpret_cast<float4*>(Us + r * LDU + j) = make_float4(u[j], u[j + 1], u[j + 2], u[j + 3]);
+                    if (dbg && blockIdx.x == 0 && c == 0)
+                        for (int j = 0; j < 64; ++j) dbg[16448 + r * 64 + j] = u[j];
+                }
             }
             tc_fence_before();
-            bar_sync(NB_CONV, 64);
-            if (r == 0) {
+            bar_sync(NB_CONV, kConvThreads);
+            if (warp == 2 && lane == 0) {
                 mbar_arrive(ctl.b(B_U_READY));
                 mbar_arrive(ctl.b(B_WU_FREE));
                 EFLA_STAMP(c, 7);
             }
+            // P = P~ with the causal mask (diagonal kept) -> bf16 K-major rows
+            ok = bar_and(NB_CONV, kConvThreads, ctl.wait(B_GP_FULL, c & 1));
+            if (!ok) break;
+            tc_fence_after();
+            {
+                float t[64];
+                tmem_ld64_wait(tmem + lane_off + TM_GP, t);
+                if (act) {
+#pragma unroll
+                    for (int j = 0; j < 64; ++j) t[j] = (j <= r) ? t[j] : 0.f;
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) st_chunk(sm + OFF_P + sw128_off(r, j), t + 8 * j);
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            bar_sync(NB_CONV, kConvThreads);
+            if (warp == 2 && lane == 0) {
+                mbar_arrive(ctl.b(B_GP_FREE));
+                mbar_arrive(ctl.b(B_P_READY));
+                EFLA_STAMP(c, 4);
+            }
         }
     } else {
-        // ================================================================ chain (TMEM lanes 0..127)
-        const int q = warp & 3;                       // TMEM lane quarter
-        const int ch = (warp - 4) >> 2;               // column half: 32 of this CTA's 64 columns
-        const int ct = 32 * q + lane;                 // d_k row for S; rows of Y by quarter
-        const int cc = 32 * ch;                       // first column of this thread's half
+        // ================================================================ chain (two warps per lane quarter)
+        const int ch = (warp - 6) >> 2;               // column half: 32 of this CTA's 64 columns
+        const int cc = 32 * ch;
+        const int ct = 32 * q + lane;                 // d_k row of S (M=128 accumulator)
+        const int r = 16 * q + lane;                  // chunk row of the M=64 accumulators
+        const bool act = lane < 16;
         {   // initial state
             const float* src = S0 ? S0 + ((size_t)bh * kD + ct) * kD + col0 + cc : nullptr;
 #pragma unroll
@@ -379,106 +386,94 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             fence_proxy_async_smem();
             tc_fence_before();
             bar_sync(NB_CHAIN, kChainThreads);
-            if (warp == 4 && lane == 0) mbar_arrive(ctl.b(B_SB_READY));
+            if (warp == 6 && lane == 0) mbar_arrive(ctl.b(B_SB_READY));
         }
         bool ok = true;
         for (int c = 0; c < nchunks; ++c) {
             const int b = c & 1;
-            const uint32_t tY = tmem + lane_off + TM_Y + 64 * b + cc;
-            if (q >= 2) {                             // Delta = U - WS (rows 64..127 of Y)
-                const int r = ct - 64;
-                bool w = ok && ctl.wait(B_Y_FULL + b, (c >> 1) & 1) && ctl.wait(B_U_READY, c & 1);
-                w = bar_and(NB_DELTA, 128, w);
-                if (w) {
-                    tc_fence_after();
-#pragma unroll
-                    for (int qd = 0; qd < 2; ++qd) {
-                        float t16[16];
-                        tmem_ld16(tY + 16 * qd, t16);
-                        tmem_wait_ld();
-                        if (dbg && blockIdx.x == 0 && c == 0)
-                            for (int j = 0; j < 16; ++j) dbg[20544 + r * 64 + cc + 16 * qd + j] = t16[j];
-#pragma unroll
-                        for (int j = 0; j < 16; j += 4) {
-                            const float4 u = *reinterpret_cast<const float4*>(Us + r * LDU + cc + 16 * qd + j);
-                            t16[j] = u.x - t16[j];
-                            t16[j + 1] = u.y - t16[j + 1];
-                            t16[j + 2] = u.z - t16[j + 2];
-                            t16[j + 3] = u.w - t16[j + 3];
-                        }
-                        st_chunk(sm + OFF_DL + sw128_off(r, 4 * ch + 2 * qd), t16);
-                        st_chunk(sm + OFF_DL + sw128_off(r, 4 * ch + 2 * qd + 1), t16 + 8);
-                    }
-                    fence_proxy_async_smem();
-                    tc_fence_before();
-                    bar_sync(NB_DELTA, 128);
-                    if (warp == 6 && lane == 0) {
-                        mbar_arrive(ctl.b(B_D_READY));
-                        mbar_arrive(ctl.b(B_U_FREE));
-                        EFLA_STAMP(c, 8);
-                    }
-                }
-                ok = w;
-            }
-            // the new state: bf16 operand for the next chunk (and S_T after the last)
-            ok = bar_and(NB_CHAIN, kChainThreads, ok && ctl.wait(B_S_FULL, c & 1));
+            // Delta = U - W S
+            ok = bar_and(NB_CHAIN, kChainThreads, ok && ctl.wait(B_WS_FULL, c & 1) && ctl.wait(B_U_READY, c & 1));
             if (!ok) break;
             tc_fence_after();
-            const bool last = (c == nchunks - 1);
+            {
+                float t[32];
+                tmem_ld32_wait(tmem + lane_off + TM_WS + cc, t);
+                if (act) {
+                    if (dbg && blockIdx.x == 0 && c == 0)
+                        for (int j = 0; j < 32; ++j) dbg[20544 + r * 64 + cc + j] = t[j];
 #pragma unroll
-            for (int qd = 0; qd < 2; ++qd) {
-                float t16[16];
-                tmem_ld16(tmem + lane_off + TM_S + cc + 16 * qd, t16);
-                tmem_wait_ld();
-                st_chunk(sm + OFF_SB + sw128_off(ct, 4 * ch + 2 * qd), t16);
-                st_chunk(sm + OFF_SB + sw128_off(ct, 4 * ch + 2 * qd + 1), t16 + 8);
-                if (dbg && blockIdx.x == 0 && c == 0)
-                    for (int j = 0; j < 16; ++j) dbg[24640 + ct * 64 + cc + 16 * qd + j] = t16[j];
-                if (last && S_T) {
-                    float* dst = S_T + ((size_t)bh * kD + ct) * kD + col0 + cc + 16 * qd;
+                    for (int j = 0; j < 32; j += 4) {
+                        const float4 u = *reinterpret_cast<const float4*>(Us + r * LDU + cc + j);
+                        t[j] = u.x - t[j];
+                        t[j + 1] = u.y - t[j + 1];
+                        t[j + 2] = u.z - t[j + 2];
+                        t[j + 3] = u.w - t[j + 3];
+                    }
 #pragma unroll
-                    for (int j = 0; j < 16; j += 4)
-                        *reinterpret_cast<float4*>(dst + j) = make_float4(t16[j], t16[j + 1], t16[j + 2], t16[j + 3]);
+                    for (int j = 0; j < 4; ++j) st_chunk(sm + OFF_DL + sw128_off(r, 4 * ch + j), t + 8 * j);
                 }
             }
             fence_proxy_async_smem();
             tc_fence_before();
             bar_sync(NB_CHAIN, kChainThreads);
-            if (warp == 4 && lane == 0) {
+            if (warp == 6 && lane == 0) {
+                mbar_arrive(ctl.b(B_D_READY));
+                mbar_arrive(ctl.b(B_U_FREE));
+                EFLA_STAMP(c, 8);
+            }
+            // the new state: bf16 operand for the next chunk (and S_T after the last)
+            ok = bar_and(NB_CHAIN, kChainThreads, ctl.wait(B_S_FULL, c & 1));
+            if (!ok) break;
+            tc_fence_after();
+            const bool last = (c == nchunks - 1);
+            {
+                float t[32];
+                tmem_ld32_wait(tmem + lane_off + TM_S + cc, t);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) st_chunk(sm + OFF_SB + sw128_off(ct, 4 * ch + j), t + 8 * j);
+                if (dbg && blockIdx.x == 0 && c == 0)
+                    for (int j = 0; j < 32; ++j) dbg[24640 + ct * 64 + cc + j] = t[j];
+                if (last && S_T) {
+                    float* dst = S_T + ((size_t)bh * kD + ct) * kD + col0 + cc;
+#pragma unroll
+                    for (int j = 0; j < 32; j += 4)
+                        *reinterpret_cast<float4*>(dst + j) = make_float4(t[j], t[j + 1], t[j + 2], t[j + 3]);
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            bar_sync(NB_CHAIN, kChainThreads);
+            if (warp == 6 && lane == 0) {
                 mbar_arrive(ctl.b(B_SB_READY));
                 EFLA_STAMP(c, 9);
             }
-            if (q < 2) {                              // O rows (lanes 0..63 of Y)
-                const int r = ct;
-                bool w = bar_and(NB_OUT, 128, ctl.wait(B_O_FULL + b, (c >> 1) & 1));
-                if (w) {
-                    tc_fence_after();
-                    const int t0 = c * 64;
-                    const bool live = r < min(64, T - t0);
+            // O = Q S + P Delta -> bf16 global
+            ok = bar_and(NB_CHAIN, kChainThreads, ctl.wait(B_O_FULL + b, (c >> 1) & 1));
+            if (!ok) break;
+            tc_fence_after();
+            {
+                const int t0 = c * 64;
+                const bool live = act && r < min(64, T - t0);
+                float t[32];
+                tmem_ld32_wait(tmem + lane_off + TM_O + 64 * b + cc, t);
+                if (live) {
+                    uint4* dst = reinterpret_cast<uint4*>(o + (tok0 + t0 + r) * kD + col0 + cc);
 #pragma unroll
-                    for (int qd = 0; qd < 2; ++qd) {
-                        float t16[16];
-                        tmem_ld16(tY + 16 * qd, t16);
-                        tmem_wait_ld();
-                        if (live) {
-                            uint4* dst = reinterpret_cast<uint4*>(o + (tok0 + t0 + r) * kD + col0 + cc + 16 * qd);
-                            uint4 a, bb;
-                            a.x = pack_bf16x2(t16[0], t16[1]); a.y = pack_bf16x2(t16[2], t16[3]);
-                            a.z = pack_bf16x2(t16[4], t16[5]); a.w = pack_bf16x2(t16[6], t16[7]);
-                            bb.x = pack_bf16x2(t16[8], t16[9]); bb.y = pack_bf16x2(t16[10], t16[11]);
-                            bb.z = pack_bf16x2(t16[12], t16[13]); bb.w = pack_bf16x2(t16[14], t16[15]);
-                            dst[0] = a;
-                            dst[1] = bb;
-                        }
-                    }
-                    tc_fence_before();
-                    bar_sync(NB_OUT, 128);
-                    if (warp == 4 && lane == 0) {
-                        mbar_arrive(ctl.b(B_Y_FREE + b));
-                        EFLA_STAMP(c, 10);
+                    for (int j = 0; j < 4; ++j) {
+                        uint4 x;
+                        x.x = pack_bf16x2(t[8 * j], t[8 * j + 1]);
+                        x.y = pack_bf16x2(t[8 * j + 2], t[8 * j + 3]);
+                        x.z = pack_bf16x2(t[8 * j + 4], t[8 * j + 5]);
+                        x.w = pack_bf16x2(t[8 * j + 6], t[8 * j + 7]);
+                        dst[j] = x;
                     }
                 }
-                ok = w;
+            }
+            tc_fence_before();
+            bar_sync(NB_CHAIN, kChainThreads);
+            if (warp == 6 && lane == 0) {
+                mbar_arrive(ctl.b(B_O_FREE + b));
+                EFLA_STAMP(c, 10);
             }
         }
     }
