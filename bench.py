@@ -142,32 +142,40 @@ class Clocks:
                 "reasons": reasons, "samples": len(self.samples), "source": "NVML, ~2 ms polling"}
 
 
-def dist_setup(args):
+def dist_setup(backend: str = "nccl"):
+    """Rank, world size and local rank from the torchrun environment; joins the process
+    group when there is more than one rank (NCCL on GPUs, gloo for host-only use)."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        kw = {}
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            kw["device_id"] = torch.device("cuda", local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120), **kw)
     return rank, world, local
 
 
 def barrier(world):
-    torch.cuda.synchronize()
+    if torch.cuda.is_available():
+        torch.cuda.synchronize()
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
-    torch.cuda.synchronize()
+    if torch.cuda.is_available():
+        torch.cuda.synchronize()
 
 
-def max_over_ranks(x: float, world: int) -> float:
+def max_over_ranks(x: float, world: int, device: str = "cuda") -> float:
+    """The largest of the ranks' values (every rank gets it): device times are reported
+    as the slowest rank's."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
@@ -175,6 +183,14 @@ def max_over_ranks(x: float, world: int) -> float:
 def shard_seed(rank: int) -> int:
     """Each rank draws its own independent batch of streams (weak scaling)."""
     return WORKLOAD.seed + 1000 * rank
+
+
+def rank_workload(rank: int, world: int):
+    """The rank's share of the job and the job's total tokens per step: every rank runs a
+    full bench workload of its own streams (weak scaling; streams never interact, so no
+    data-path collective exists)."""
+    w = WORKLOAD.replace(seed=shard_seed(rank))
+    return w, w.tokens * world
 
 
 def cpu_baseline(w, cpu_seconds: float = 12.0):
@@ -243,11 +259,11 @@ def main():
         return
 
     import delta_rule_linear_02_b200 as efla
-    rank, world, local = dist_setup(args)
+    rank, world, local = dist_setup("nccl")
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream(dev)
-    w = WORKLOAD.replace(seed=shard_seed(rank))
+    w, tokens = rank_workload(rank, world)
     hbm, tc, peak_kind = peaks()
 
     # ---- device-resident inputs: N_ROTATE independent sets, so every step misses L2
@@ -284,7 +300,6 @@ def main():
     if status != efla.EFLA_OK:
         raise SystemExit(f"device reported {efla.efla_status_string(status)}")
     ms_per_step = total_ms / args.steps
-    tokens = w.tokens * world
     value = tokens / (ms_per_step * 1e-3)
 
     nbytes, flops = chunk_alg(w)
