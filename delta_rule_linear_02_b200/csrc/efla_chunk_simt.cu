@@ -222,7 +222,8 @@ cudaError_t launch_t(const void* q, const void* k, const void* v, const void* be
                      void* o, float* S_T, long BH, int T, cudaStream_t stream) {
     using L = SimtSmem<D>;
     auto kern = chunk_simt_kernel<Tin, D>;
-    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::kBytes);
+    static std::atomic<uint64_t> smem_set{0};
+    cudaError_t err = set_smem_limit_once(kern, (int)L::kBytes, smem_set);
     if (err != cudaSuccess) return err;
     kern<<<(unsigned)(BH * (D / 64)), kNT, L::kBytes, stream>>>((const Tin*)q, (const Tin*)k, (const Tin*)v,
                                                                  (const Tin*)beta, S0, (Tin*)o, S_T, T);

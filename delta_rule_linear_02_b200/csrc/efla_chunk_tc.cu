@@ -27,7 +27,8 @@
 // (K, V, T, Q), Delta and the bf16 copy of S.
 //
 // One warp issues every MMA, in a fixed order per chunk c:
-//   [W;Q] S(c), [W|U](c+1), K^T Delta(c) (after Delta), P Delta(c), Q K^T(c+1)
+//   [W;Q] S(c), [W|U](c+1), half of Q K^T(c+1) if its Q is in place, K^T Delta(c) (after
+//   Delta), P Delta(c), the rest of Q K^T(c+1)
 // Issue is by a converged warp with elect.sync (warp-uniform control flow keeps the
 // descriptors in uniform registers; a one-lane issuer in a data-dependent loop issues
 // several times slower).
@@ -36,10 +37,11 @@
 //   warp 0       TMA producer (no multicast), L2 prefetch ahead
 //   warp 1       MMA issuer
 //   warps 4-5    W: fp32 accumulator rows 0-63 -> bf16 A operand rows 0-63
-//   warps 2-3    Q rows -> A operand rows 64-127; P~ rows 64-127 -> masked bf16 P
+//   warps 2-3    Q rows -> A operand rows 64-127; P~ rows 64-127 -> masked bf16 P; O
+//                (X rows 64-127) -> global, X released as soon as O is in registers
 //   warps 6-13   chain, two per lane quarter (32-column halves).  Quarters 0-1 form Delta
-//                (U taken from its accumulator as soon as it lands); quarters 2-3 store O;
-//                all eight rebuild the bf16 S and S_T.
+//                (U taken from its accumulator as soon as it lands); all eight rebuild the
+//                bf16 S and S_T.
 // Every wait is bounded (2 s); a wait that runs out sets a CTA-wide abort flag, every
 // role winds down, and the caller's workspace records the timeout.
 // `dbg` (null in the library) receives CTA 0's chunk-0 intermediates for diagnosis:
@@ -118,7 +120,7 @@ constexpr uint32_t ID_GP = idesc_bf16(128, 64, false, false);     // [W;Q] K^T
 constexpr uint32_t ID_S = idesc_bf16(128, 64, true, true);        // K^T Delta
 
 // ---- named barriers
-constexpr int NB_CW = 1, NB_CQ = 2, NB_DELTA = 3, NB_OUT = 4, NB_CHAIN = 5;
+constexpr int NB_CW = 1, NB_CQ = 2, NB_DELTA = 3, NB_CHAIN = 4;
 constexpr int kPair = 64, kHalfChain = 128, kChainThreads = 256;
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
@@ -277,11 +279,17 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         // Warp-uniform control flow: every lane polls the barrier and the warp votes;
         // elect.sync inside each MMA and commit picks the issuing lane.
         auto wait = [&](int i, uint32_t parity) { return __all_sync(0xffffffffu, ctl.wait(i, parity)); };
-        auto issue_qk = [&](int c) {      // [W;Q] K^T: rows 64-127 are Q K^T
+        auto ready = [&](int i, uint32_t parity) { return __all_sync(0xffffffffu, mbar_test_wait(ctl.b(i), parity)); };
+        auto issue_qk = [&](int c, int k0, int k1) {      // [W;Q] K^T, k-steps [k0, k1): rows 64-127 are Q K^T
             tc_fence_after();
-            mma_ts(tmem + TM_GP, tmem + TM_AWQ, sb + kvt(c) + KVT_K, TILE, 32, 16, ID_GP, 8, 0);
-            mma_commit_elect(ctl.b(B_GP_FULL));
-            EFLA_STAMP(c, 0);
+            const uint64_t db = sdesc_sw128(sb + kvt(c) + KVT_K, 16, 1024);
+            for (int ks = k0; ks < k1; ++ks)
+                mma_bf16_ts_elect(tmem + TM_GP, tmem + TM_AWQ + 8 * ks, db + (((ks >> 2) * TILE + (ks & 3) * 32) >> 4),
+                                  ID_GP, ks > 0);
+            if (k1 == 8) {
+                mma_commit_elect(ctl.b(B_GP_FULL));
+                EFLA_STAMP(c, 0);
+            }
         };
         auto issue_wu = [&](int c) {      // [W | U] = [T; *] [K | V]
             tc_fence_after();
@@ -292,7 +300,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         };
         bool ok = wait(B_KVT_FULL, 0) && wait(B_Q_READY, 0);
         if (ok) {
-            issue_qk(0);
+            issue_qk(0, 0, 8);
             issue_wu(0);
         }
         for (int c = 0; c < nchunks && ok; ++c) {
@@ -309,6 +317,12 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                            wait(B_WU_FREE, c & 1))) break;
                 issue_wu(c + 1);
             }
+            // half of the next chunk's Q K^T too, if its Q is already in place (never wait here)
+            int qk_half = 0;
+            if (c + 1 < nchunks && ready(B_Q_READY, (c + 1) & 1) && ready(B_GP_FREE, c & 1)) {
+                issue_qk(c + 1, 0, 4);
+                qk_half = 4;
+            }
             // S += K^T Delta (state chain)
             if (!(ok = wait(B_D_READY, c & 1))) break;
             tc_fence_after();
@@ -322,10 +336,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             tc_fence_after();
             mma_ts(tmem + TM_X, tmem + TM_AP, sb + OFF_DL, 4 * 2048, 2048, TILE, ID_N64, 4, 1);
             mma_commit_elect(ctl.b(B_O_FULL));
-            // the next chunk's Q K^T
+            // the (rest of the) next chunk's Q K^T
             if (c + 1 < nchunks) {
-                if (!(ok = wait(B_Q_READY, (c + 1) & 1) && wait(B_GP_FREE, c & 1))) break;
-                issue_qk(c + 1);
+                if (qk_half == 0 && !(ok = wait(B_Q_READY, (c + 1) & 1) && wait(B_GP_FREE, c & 1))) break;
+                issue_qk(c + 1, qk_half, 8);
             }
         }
         mma_commit_elect(ctl.b(B_DRAIN));
@@ -384,11 +398,41 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 EFLA_STAMP(c, 5);
             }
         };
+        // O(c) = X rows 64-127 once P Delta(c) has landed: taken into registers, X released
+        // at once for [W;Q] S(c+1), then stored to global as bf16 (rows past T skipped)
+        auto store_o = [&](int c) {
+            bool fine = bar_and(NB_CQ, kPair, ctl.wait(B_O_FULL, c & 1));
+            if (!fine) return false;
+            tc_fence_after();
+            float t[64];
+            tmem_ld64_wait(tmem + lane_off + TM_X, t);
+            tc_fence_before();
+            bar_sync(NB_CQ, kPair);
+            if (warp == 2 && lane == 0) {
+                mbar_arrive(ctl.b(B_X_FREE));
+                EFLA_STAMP(c, 10);
+            }
+            const int t0 = c * 64;
+            if (r < min(64, T - t0)) {
+                uint4* dst = reinterpret_cast<uint4*>(o + (tok0 + t0 + r) * kD + col0);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    uint4 y;
+                    y.x = pack_bf16x2(t[8 * j], t[8 * j + 1]);
+                    y.y = pack_bf16x2(t[8 * j + 2], t[8 * j + 3]);
+                    y.z = pack_bf16x2(t[8 * j + 4], t[8 * j + 5]);
+                    y.w = pack_bf16x2(t[8 * j + 6], t[8 * j + 7]);
+                    dst[j] = y;
+                }
+            }
+            return true;
+        };
         bool ok = bar_and(NB_CQ, kPair, ctl.wait(B_Q_FULL, 0));
         if (ok) copy_q(0);
         for (int c = 0; c < nchunks && ok; ++c) {
-            // P = Q K^T masked causally (diagonal kept) -> A rows 64-127, once P Delta(c-1) is done
-            ok = bar_and(NB_CQ, kPair, ctl.wait(B_GP_FULL, c & 1) && (c == 0 || ctl.wait(B_O_FULL, (c - 1) & 1)));
+            if (c > 0 && !(ok = store_o(c - 1))) break;
+            // P = Q K^T masked causally (diagonal kept) -> A rows 64-127 (P Delta(c-1) is done)
+            ok = bar_and(NB_CQ, kPair, ctl.wait(B_GP_FULL, c & 1));
             if (!ok) break;
             tc_fence_after();
             {
@@ -417,11 +461,12 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 copy_q(c + 1);
             }
         }
+        if (ok) store_o(nchunks - 1);
     } else {
         // ================================================================ chain (two warps per lane quarter)
-        // Quarters 0-1 (X rows 0-63, W S) form Delta; quarters 2-3 (X rows 64-127) store O.
-        // The groups meet at the S epilogue; a group that gives up still reaches the next
-        // S-epilogue barrier with ok = false, so both groups stop together.
+        // Quarters 0-1 (X rows 0-63, W S) form Delta; all eight rebuild the bf16 S.  A group
+        // that gives up still reaches the next S-epilogue barrier with ok = false, so both
+        // stop together.
         const int ch = (warp - 6) >> 2;               // column half: 32 of this CTA's 64 columns
         const int cc = 32 * ch;
         const int ct = 32 * q + lane;                 // d_k row of S, and row of X / [W | U]
@@ -510,34 +555,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 mbar_arrive(ctl.b(B_SB_READY));
                 EFLA_STAMP(c, 9);
             }
-            if (!delta_group) {
-                // O = Q S + P Delta (X rows 64-127) -> bf16 global
-                ok = bar_and(NB_OUT, kHalfChain, ctl.wait(B_O_FULL, c & 1));
-                if (ok) {
-                    tc_fence_after();
-                    const int r = ct - 64, t0 = c * 64;
-                    float t[32];
-                    tmem_ld32_wait(tmem + lane_off + TM_X + cc, t);
-                    if (r < min(64, T - t0)) {
-                        uint4* dst = reinterpret_cast<uint4*>(o + (tok0 + t0 + r) * kD + col0 + cc);
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            uint4 y;
-                            y.x = pack_bf16x2(t[8 * j], t[8 * j + 1]);
-                            y.y = pack_bf16x2(t[8 * j + 2], t[8 * j + 3]);
-                            y.z = pack_bf16x2(t[8 * j + 4], t[8 * j + 5]);
-                            y.w = pack_bf16x2(t[8 * j + 6], t[8 * j + 7]);
-                            dst[j] = y;
-                        }
-                    }
-                    tc_fence_before();
-                    bar_sync(NB_OUT, kHalfChain);
-                    if (warp == 6 && lane == 0) {
-                        mbar_arrive(ctl.b(B_X_FREE));
-                        EFLA_STAMP(c, 10);
-                    }
-                }
-            }
         }
     }
 
@@ -580,7 +597,8 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const v
     if (!tma_map_tokens(&mq, q, kD, T, BH) || !tma_map_tokens(&mk, k, kD, T, BH) ||
         !tma_map_tokens(&mv, v, kD, T, BH) || !tma_map_rows64(&mt, scratch, BH * nchunks * 64))
         return cudaErrorInvalidValue;
-    e = cudaFuncSetAttribute(chunk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+    static std::atomic<uint64_t> smem_set{0};
+    e = set_smem_limit_once(chunk_tc_kernel, (int)SMEM_BYTES, smem_set);
     if (e != cudaSuccess) return e;
     chunk_tc_kernel<<<(unsigned)(BH * 2), kThreads, SMEM_BYTES, stream>>>(mq, mk, mv, mt, S0, (__nv_bfloat16*)o,
                                                                           S_T, T, err, kWaitLimitNs, nullptr);

@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 namespace efla {
 
 // ---------------------------------------------------------------- element access
@@ -56,5 +58,20 @@ __device__ __forceinline__ float gate_alpha(float beta, float lambda) {
 
 // Device error word values (kept in the caller's workspace).
 enum : uint32_t { kDevOk = 0u, kDevTimeout = 1u };
+
+// A kernel's dynamic shared-memory limit is a per-device attribute that persists, so it
+// is set once per device (bit `dev` of `done`); setting it on every launch would add a
+// driver call to each forward.
+template <typename Kernel>
+inline cudaError_t set_smem_limit_once(Kernel kernel, int bytes, std::atomic<uint64_t>& done) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const uint64_t bit = (dev >= 0 && dev < 64) ? (1ull << dev) : 0;
+    if (bit && (done.load(std::memory_order_relaxed) & bit)) return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_relaxed);
+    return e;
+}
 
 }  // namespace efla

@@ -242,7 +242,8 @@ cudaError_t launch_ut(const void* k, const void* beta, void* Tout, long BH, int 
     const int nchunks = (T + 63) / 64;
     const long ntiles = BH * nchunks;
     const long grid = std::min<long>(ntiles, (long)sm_count() * kCtasPerSm);
-    cudaError_t e = cudaFuncSetAttribute(ut_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+    static std::atomic<uint64_t> smem_set{0};
+    cudaError_t e = set_smem_limit_once(ut_kernel, (int)SMEM_BYTES, smem_set);
     if (e != cudaSuccess) return e;
     ut_kernel<<<(unsigned)grid, kThreads, SMEM_BYTES, stream>>>(mk, (const __nv_bfloat16*)beta,
                                                                 (__nv_bfloat16*)Tout, T, nchunks, ntiles, err,
