@@ -7,7 +7,8 @@
 // chain kernel (efla_chunk_tc.cu) reads it back as a bf16 operand.
 //
 // Per tile (stream bh, chunk c):
-//   G = K K^T                                   tcgen05 MMA (bf16 in, fp32 in TMEM)
+//   G = K K^T                                   tcgen05 MMA, M = 64 (bf16 in, fp32 in TMEM;
+//                                                row r in lane (r % 16) + 32 (r / 16))
 //   lambda_r = G_rr, alpha_r = gate(beta_r, lambda_r)   (Section 3.2 / 3.4)
 //   A^T rows = alpha (.) G rows                 (G is symmetric)
 //   X = (I + A)^{-1}                            efla_ut_tf32.cuh (fp32 + TF32 merges)
@@ -36,7 +37,7 @@ constexpr int kCtasPerSm = 3;
 constexpr uint32_t TILE = 8192;
 constexpr uint32_t OFF_K = 0;                          // 2 stages x [K a0 | K a1]
 constexpr uint32_t F32_TILE = 64 * LDX * 4;
-constexpr uint32_t OFF_AT = OFF_K + 4 * TILE;          // also the (unused) rows 64..127 of stage 1's MMA
+constexpr uint32_t OFF_AT = OFF_K + 4 * TILE;
 constexpr uint32_t OFF_X = OFF_AT + F32_TILE;
 constexpr uint32_t OFF_ALPHA = OFF_X + F32_TILE;
 constexpr uint32_t OFF_BETA = OFF_ALPHA + 256;
@@ -49,7 +50,7 @@ static_assert(kCtasPerSm * SMEM_BYTES <= 232448, "UT kernel: shared memory for t
 
 enum : int { B_FULL = 0 /* [2] */, B_GP_FULL = 2, B_GP_FREE = 3, B_DRAIN = 4 };
 constexpr uint32_t TM_COLS = 64;
-constexpr uint32_t ID_G = idesc_bf16(128, 64, false, false);
+constexpr uint32_t ID_G = idesc_bf16(64, 64, false, false);
 constexpr int NB_W = 1;                                // named barrier of the 128 worker threads
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
@@ -151,7 +152,8 @@ ut_kernel(const __grid_constant__ CUtensorMap tm_k, const __nv_bfloat16* __restr
         // ------------------------------------------------------------ workers (128 threads)
         const int wt = tid - 32;
         const int q = warp & 3;                       // TMEM lane quarter of this warp
-        const int r = 32 * q + lane;                  // G row held by quarters 0 and 1
+        const int r = 16 * q + lane;                  // G row held by lanes 0-15 of each quarter
+        const bool grow = lane < 16;
         const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
         auto beta_of = [&](int j) -> float {
             if (j >= ntile || wt >= 64) return 0.f;
@@ -171,15 +173,8 @@ ut_kernel(const __grid_constant__ CUtensorMap tm_k, const __nv_bfloat16* __restr
             if (!ok) break;
             tc_fence_after();
             float g[64];
-            if (q < 2) {
-#pragma unroll
-                for (int m = 0; m < 4; ++m) {
-                    float t16[16];
-                    tmem_ld16(tmem + lane_off + 16 * m, t16);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) g[16 * m + e] = t16[e];
-                }
+            tmem_ld64_wait(tmem + lane_off, g);
+            if (grow) {
                 float lam = 0.f;
 #pragma unroll
                 for (int e = 0; e < 64; ++e) lam = (e == r) ? g[e] : lam;
@@ -188,7 +183,7 @@ ut_kernel(const __grid_constant__ CUtensorMap tm_k, const __nv_bfloat16* __restr
             tc_fence_before();
             bar_sync(NB_W, 128);                     // alpha visible, G read
             if (wt == 0) mbar_arrive(bar + B_GP_FREE);
-            if (q < 2) {
+            if (grow) {
                 // A^T[r][i] = A[i][r] = alpha_i G[i][r] = alpha_i G[r][i]; only i > r is read
 #pragma unroll
                 for (int m = 0; m < 16; ++m) {
@@ -199,9 +194,10 @@ ut_kernel(const __grid_constant__ CUtensorMap tm_k, const __nv_bfloat16* __restr
             }
             bar_sync(NB_W, 128);
             ut::ut_solve<NB_W, 128>(At, X, wt);
-            {   // T = X diag(alpha) -> bf16, 64 bytes per thread
+            {   // T = X diag(alpha) -> bf16, 64 bytes per thread (a warp reads 32 consecutive
+                // rows of one column half: conflict-free with the 68-float row stride)
                 const long tile = first + (long)j * step;
-                const int rr = wt >> 1, h = wt & 1;
+                const int rr = wt & 63, h = wt >> 6;
                 uint4* dst = reinterpret_cast<uint4*>(Tout + (tile * 64 + rr) * 64 + 32 * h);
 #pragma unroll
                 for (int m = 0; m < 4; ++m) {
