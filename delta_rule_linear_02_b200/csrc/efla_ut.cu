@@ -16,9 +16,10 @@
 // Tokens past T are zero-filled by TMA (k = 0, beta = 0: alpha = 0, their rows and
 // columns of T are zero).
 //
-// A persistent grid of several CTAs per SM walks the tiles; each CTA double-buffers its
-// K tiles (the next tile's TMA is in flight while the current one is solved), and the
-// CTAs on an SM overlap each other's latency.  Warp 0 issues the TMA copies and the MMA;
+// A persistent grid of four CTAs per SM walks the tiles.  Each CTA holds kStages K tiles
+// (the next tile's TMA is in flight while the current one is solved); one stage and four
+// CTAs per SM measured faster than two stages and three CTAs, since the CTAs on an SM
+// overlap each other's latency.  Warp 0 issues the TMA copies and the MMA;
 // warps 1-4 compute the gate, the solve and the bf16 store.  Every wait is bounded.
 #include "efla_common.cuh"
 #include "efla_kernels.h"
@@ -33,11 +34,12 @@ using namespace sm100;
 using ut::LDX;
 
 constexpr int kThreads = 160;
-constexpr int kCtasPerSm = 3;
+constexpr int kCtasPerSm = 4;
+constexpr int kStages = 1;                             // K tiles in flight per CTA
 constexpr uint32_t TILE = 8192;
-constexpr uint32_t OFF_K = 0;                          // 2 stages x [K a0 | K a1]
+constexpr uint32_t OFF_K = 0;                          // kStages x [K a0 | K a1]
 constexpr uint32_t F32_TILE = 64 * LDX * 4;
-constexpr uint32_t OFF_AT = OFF_K + 4 * TILE;
+constexpr uint32_t OFF_AT = OFF_K + kStages * 2 * TILE;
 constexpr uint32_t OFF_X = OFF_AT + F32_TILE;
 constexpr uint32_t OFF_ALPHA = OFF_X + F32_TILE;
 constexpr uint32_t OFF_BETA = OFF_ALPHA + 256;
@@ -48,7 +50,8 @@ constexpr uint32_t SMEM_USED = OFF_MISC + 16;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;
 static_assert(kCtasPerSm * SMEM_BYTES <= 232448, "UT kernel: shared memory for the target occupancy");
 
-enum : int { B_FULL = 0 /* [2] */, B_GP_FULL = 2, B_GP_FREE = 3, B_DRAIN = 4 };
+enum : int { B_FULL = 0 /* [kStages] */, B_GP_FULL = 2, B_GP_FREE = 3, B_DRAIN = 4 };
+static_assert(kStages <= 2, "barrier map holds two stages");
 constexpr uint32_t TM_COLS = 64;
 constexpr uint32_t ID_G = idesc_bf16(64, 64, false, false);
 constexpr int NB_W = 1;                                // named barrier of the 128 worker threads
@@ -119,16 +122,16 @@ ut_kernel(const __grid_constant__ CUtensorMap tm_k, const __nv_bfloat16* __restr
             auto load = [&](int j) {
                 const long tile = first + (long)j * step;
                 const int bh = (int)(tile / nchunks), c = (int)(tile % nchunks);
-                uint8_t* st = sm + OFF_K + (j & 1) * 2 * TILE;
-                mbar_arrive_expect_tx(bar + B_FULL + (j & 1), 2 * TILE);
-                tma_load_3d(st, &tm_k, bar + B_FULL + (j & 1), 0, c * 64, bh);
-                tma_load_3d(st + TILE, &tm_k, bar + B_FULL + (j & 1), 64, c * 64, bh);
+                uint8_t* st = sm + OFF_K + (j % kStages) * 2 * TILE;
+                mbar_arrive_expect_tx(bar + B_FULL + (j % kStages), 2 * TILE);
+                tma_load_3d(st, &tm_k, bar + B_FULL + (j % kStages), 0, c * 64, bh);
+                tma_load_3d(st + TILE, &tm_k, bar + B_FULL + (j % kStages), 64, c * 64, bh);
             };
-            for (int j = 0; j < min(2, ntile); ++j) load(j);
+            for (int j = 0; j < min(kStages, ntile); ++j) load(j);
             bool ok = true;
             for (int j = 0; j < ntile && ok; ++j) {
-                const int s = j & 1;
-                ok = wait_bounded(bar + B_FULL + s, (j >> 1) & 1, abort, limit_ns) &&
+                const int s = j % kStages;
+                ok = wait_bounded(bar + B_FULL + s, (j / kStages) & 1, abort, limit_ns) &&
                      (j == 0 || wait_bounded(bar + B_GP_FREE, (j - 1) & 1, abort, limit_ns));
                 if (!ok) break;
                 tc_fence_after();
@@ -139,14 +142,15 @@ ut_kernel(const __grid_constant__ CUtensorMap tm_k, const __nv_bfloat16* __restr
                     mma_bf16(tmem, sdesc_sw128(a, 16, 1024), sdesc_sw128(a, 16, 1024), ID_G, ks > 0);
                 }
                 mma_commit(bar + B_GP_FULL);
-                if (j + 2 < ntile) {        // the stage is free once this MMA has read it
+                if (j + kStages < ntile) {  // the stage is free once this MMA has read it
                     if (!(ok = wait_bounded(bar + B_GP_FULL, j & 1, abort, limit_ns))) break;
-                    load(j + 2);
+                    load(j + kStages);
                 }
             }
             mma_commit(bar + B_DRAIN);
             mbar_wait(bar + B_DRAIN, 0, limit_ns);
-            for (int j = max(0, ntile - 2); j < ntile; ++j) mbar_wait(bar + B_FULL + (j & 1), (j >> 1) & 1, limit_ns);
+            for (int j = max(0, ntile - kStages); j < ntile; ++j)
+                mbar_wait(bar + B_FULL + j % kStages, (j / kStages) & 1, limit_ns);
         }
     } else {
         // ------------------------------------------------------------ workers (128 threads)
