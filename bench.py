@@ -389,7 +389,9 @@ def main():
             "config": {"workload": w.name, "B": B, "H": H, "T": T, "d_k": d, "d_v": d, "chunk": 64,
                        "global_batch": B * world, "seq_len": T, "parallelism": f"dp{world}",
                        "l2": f"{N_ROTATE} rotating input sets ({N_ROTATE * nbytes / 1e6:.0f} MB) > 126 MB L2"},
-            "roofline": roofline, "e2e": e2e, "gpu_launches": args.steps,
+            "roofline": roofline, "e2e": e2e,
+            # bf16, d = 128: each efla_chunk_fwd launches the UT kernel and the chain kernel
+            "gpu_launches": 2 * args.steps,
             "clocks": clk.summary(), "decode": dec, "cpu_baseline": cpu,
             "kernel_source": kernel_source_hash(),
         }
