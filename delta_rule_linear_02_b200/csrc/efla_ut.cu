@@ -19,7 +19,8 @@
 // A persistent grid of four CTAs per SM walks the tiles.  Each CTA holds kStages K tiles
 // (the next tile's TMA is in flight while the current one is solved); one stage and four
 // CTAs per SM measured faster than two stages and three CTAs, since the CTAs on an SM
-// overlap each other's latency.  Warp 0 issues the TMA copies and the MMA;
+// overlap each other's latency.  Warp 0 (whole-warp control flow, elect.sync) issues the
+// TMA copies and the MMA;
 // warps 1-4 compute the gate, the solve and the bf16 store.  Every wait is bounded.
 #include "efla_common.cuh"
 #include "efla_kernels.h"
@@ -117,41 +118,50 @@ ut_kernel(const __grid_constant__ CUtensorMap tm_k, const __nv_bfloat16* __restr
     const uint32_t tmem = *tmem_slot;
 
     if (warp == 0) {
-        // ------------------------------------------------------------ TMA + MMA issue
-        if (lane == 0) {
-            auto load = [&](int j) {
+        // ------------------------------------------------------------ TMA + MMA issue (whole warp)
+        // Warp-uniform control flow (every lane polls, the warp votes); lane 0 issues the
+        // TMA copies, elect.sync the MMAs and commits.
+        auto wait = [&](uint64_t* b, uint32_t parity) {
+            return __all_sync(0xffffffffu, wait_bounded(b, parity, abort, limit_ns));
+        };
+        auto load = [&](int j) {
+            if (lane == 0) {
                 const long tile = first + (long)j * step;
                 const int bh = (int)(tile / nchunks), c = (int)(tile % nchunks);
                 uint8_t* st = sm + OFF_K + (j % kStages) * 2 * TILE;
                 mbar_arrive_expect_tx(bar + B_FULL + (j % kStages), 2 * TILE);
                 tma_load_3d(st, &tm_k, bar + B_FULL + (j % kStages), 0, c * 64, bh);
                 tma_load_3d(st + TILE, &tm_k, bar + B_FULL + (j % kStages), 64, c * 64, bh);
-            };
-            for (int j = 0; j < min(kStages, ntile); ++j) load(j);
-            bool ok = true;
-            for (int j = 0; j < ntile && ok; ++j) {
-                const int s = j % kStages;
-                ok = wait_bounded(bar + B_FULL + s, (j / kStages) & 1, abort, limit_ns) &&
-                     (j == 0 || wait_bounded(bar + B_GP_FREE, (j - 1) & 1, abort, limit_ns));
-                if (!ok) break;
-                tc_fence_after();
-                const uint32_t st = sb + OFF_K + s * 2 * TILE;
-#pragma unroll
-                for (int ks = 0; ks < 8; ++ks) {
-                    const uint32_t a = st + (ks >> 2) * TILE + (ks & 3) * 32;
-                    mma_bf16(tmem, sdesc_sw128(a, 16, 1024), sdesc_sw128(a, 16, 1024), ID_G, ks > 0);
-                }
-                mma_commit(bar + B_GP_FULL);
-                if (j + kStages < ntile) {  // the stage is free once this MMA has read it
-                    if (!(ok = wait_bounded(bar + B_GP_FULL, j & 1, abort, limit_ns))) break;
-                    load(j + kStages);
-                }
             }
-            mma_commit(bar + B_DRAIN);
+            __syncwarp();
+        };
+        for (int j = 0; j < min(kStages, ntile); ++j) load(j);
+        bool ok = true;
+        for (int j = 0; j < ntile && ok; ++j) {
+            const int s = j % kStages;
+            ok = wait(bar + B_FULL + s, (j / kStages) & 1) && (j == 0 || wait(bar + B_GP_FREE, (j - 1) & 1));
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t st = sb + OFF_K + s * 2 * TILE;
+            const uint64_t d0 = sdesc_sw128(st, 16, 1024);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                const uint64_t d = d0 + (((ks >> 2) * TILE + (ks & 3) * 32) >> 4);
+                mma_bf16_elect(tmem, d, d, ID_G, ks > 0);
+            }
+            mma_commit_elect(bar + B_GP_FULL);
+            if (j + kStages < ntile) {  // the stage is free once this MMA has read it
+                if (!(ok = wait(bar + B_GP_FULL, j & 1))) break;
+                load(j + kStages);
+            }
+        }
+        mma_commit_elect(bar + B_DRAIN);
+        if (lane == 0) {
             mbar_wait(bar + B_DRAIN, 0, limit_ns);
             for (int j = max(0, ntile - kStages); j < ntile; ++j)
                 mbar_wait(bar + B_FULL + j % kStages, (j / kStages) & 1, limit_ns);
         }
+        __syncwarp();
     } else {
         // ------------------------------------------------------------ workers (128 threads)
         const int wt = tid - 32;
