@@ -18,6 +18,7 @@ LIB_PATH = os.path.join(_PKG, "libefla.so")
 
 EFLA_OK, EFLA_ERR_INVALID_ARG, EFLA_ERR_UNSUPPORTED, EFLA_ERR_CUDA, EFLA_ERR_TIMEOUT = range(5)
 EFLA_DTYPE_F32, EFLA_DTYPE_BF16 = 0, 1
+EFLA_RULE_EXACT, EFLA_RULE_EULER = 0, 1     # exact-flow gate, or alpha = beta (the delta rule)
 CHUNK = 64
 
 _DTYPES = {torch.float32: EFLA_DTYPE_F32, torch.bfloat16: EFLA_DTYPE_BF16}
@@ -43,6 +44,8 @@ def _load() -> ctypes.CDLL:
     lib.efla_chunk_fwd_workspace_bytes.restype = Z
     lib.efla_chunk_fwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, I, I, I, I, I, I, I, vp, Z, vp]
     lib.efla_chunk_fwd.restype = I
+    lib.efla_chunk_fwd_ex.argtypes = [vp, vp, vp, vp, vp, vp, vp, I, I, I, I, I, I, I, I, vp, Z, vp]
+    lib.efla_chunk_fwd_ex.restype = I
     lib.efla_chunk_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, I, I, I, I, I, I, I, vp]
     lib.efla_chunk_fwd_noalloc.restype = I
     lib.efla_workspace_status.argtypes = [vp, I, vp]
@@ -51,6 +54,8 @@ def _load() -> ctypes.CDLL:
     lib.efla_selftest_wait_timeout.restype = I
     lib.efla_recurrent_step.argtypes = [vp, vp, vp, vp, vp, vp, I, I, I, I, I, vp]
     lib.efla_recurrent_step.restype = I
+    lib.efla_recurrent_step_ex.argtypes = [vp, vp, vp, vp, vp, vp, I, I, I, I, I, I, vp]
+    lib.efla_recurrent_step_ex.restype = I
     return lib
 
 
@@ -111,10 +116,11 @@ def new_workspace(B, H, T, d_k, d_v, chunk=CHUNK, dtype=torch.bfloat16, device="
 
 
 def efla_chunk_fwd(q, k, v, beta, S0=None, chunk: int = CHUNK, o=None, S_T=None,
-                   workspace=None, want_state: bool = True, stream=None
+                   workspace=None, want_state: bool = True, stream=None, rule: int = EFLA_RULE_EXACT
                    ) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
     """Chunked EFLA forward. q, k [B,H,T,d_k], v [B,H,T,d_v], beta [B,H,T] (one dtype),
-    S0 [B,H,d_k,d_v] float32 or None.  Returns (o [B,H,T,d_v], S_T or None)."""
+    S0 [B,H,d_k,d_v] float32 or None.  Returns (o [B,H,T,d_v], S_T or None).
+    rule: EFLA_RULE_EXACT (the method) or EFLA_RULE_EULER (the delta rule, alpha = beta)."""
     dt = k.dtype
     for t, nme in ((q, "q"), (k, "k"), (v, "v"), (beta, "beta")):
         _check(t, nme, dt)
@@ -131,9 +137,9 @@ def efla_chunk_fwd(q, k, v, beta, S0=None, chunk: int = CHUNK, o=None, S_T=None,
         _check(S_T, "S_T", torch.float32)
     if workspace is None:
         workspace = new_workspace(B, H, T, d_k, d_v, chunk, dt, k.device)
-    st = lib.efla_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(S0), _ptr(o), _ptr(S_T),
-                            B, H, T, d_k, d_v, chunk, _DTYPES.get(dt, -1), _ptr(workspace),
-                            workspace.numel(), _stream(stream))
+    st = lib.efla_chunk_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(S0), _ptr(o), _ptr(S_T),
+                               B, H, T, d_k, d_v, chunk, _DTYPES.get(dt, -1), int(rule), _ptr(workspace),
+                               workspace.numel(), _stream(stream))
     _raise(st, "efla_chunk_fwd")
     return o, S_T
 
@@ -173,9 +179,9 @@ def efla_selftest_wait_timeout(workspace: torch.Tensor, limit_ns: int = 1_000_00
            "efla_selftest_wait_timeout")
 
 
-def efla_recurrent_step(q, k, v, beta, S, o=None, stream=None) -> torch.Tensor:
+def efla_recurrent_step(q, k, v, beta, S, o=None, stream=None, rule: int = EFLA_RULE_EXACT) -> torch.Tensor:
     """One decode token: q, k [N,H,d_k], v [N,H,d_v], beta [N,H]; S [N,H,d_k,d_v] float32
-    updated in place.  Returns o [N,H,d_v]."""
+    updated in place.  Returns o [N,H,d_v].  rule as in efla_chunk_fwd."""
     dt = k.dtype
     for t, nme in ((q, "q"), (k, "k"), (v, "v"), (beta, "beta")):
         _check(t, nme, dt)
@@ -185,12 +191,12 @@ def efla_recurrent_step(q, k, v, beta, S, o=None, stream=None) -> torch.Tensor:
     if o is None:
         o = torch.empty((N, H, d_v), device=k.device, dtype=dt)
     _check(o, "o", dt)
-    _raise(lib.efla_recurrent_step(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(S), _ptr(o),
-                                   N, H, d_k, d_v, _DTYPES.get(dt, -1), _stream(stream)),
+    _raise(lib.efla_recurrent_step_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(S), _ptr(o),
+                                      N, H, d_k, d_v, _DTYPES.get(dt, -1), int(rule), _stream(stream)),
            "efla_recurrent_step")
     return o
 
 
-__all__ = ["efla_gate", "efla_chunk_fwd", "efla_chunk_fwd_noalloc", "efla_chunk_fwd_workspace_bytes", "efla_recurrent_step",
+__all__ = ["EFLA_RULE_EXACT", "EFLA_RULE_EULER", "efla_gate", "efla_chunk_fwd", "efla_chunk_fwd_noalloc", "efla_chunk_fwd_workspace_bytes", "efla_recurrent_step",
            "efla_workspace_status", "efla_status_string", "efla_selftest_wait_timeout", "new_workspace", "EflaError", "lib",
            "LIB_PATH", "CHUNK"]

@@ -64,11 +64,12 @@ size_t efla_chunk_fwd_workspace_bytes(int B, int H, int T, int d_k, int d_v, int
     return kWorkspaceHeader;
 }
 
-int efla_chunk_fwd(const void* q, const void* k, const void* v, const void* beta, const float* S0,
-                   void* o, float* S_T, int B, int H, int T, int d_k, int d_v, int chunk, int dtype,
-                   void* workspace, size_t workspace_bytes, efla_stream_t stream) {
+int efla_chunk_fwd_ex(const void* q, const void* k, const void* v, const void* beta, const float* S0,
+                      void* o, float* S_T, int B, int H, int T, int d_k, int d_v, int chunk, int dtype,
+                      int rule, void* workspace, size_t workspace_bytes, efla_stream_t stream) {
     int st = check_chunk_shape(B, H, T, d_k, d_v, chunk, dtype);
     if (st != EFLA_OK) return st;
+    if (rule != EFLA_RULE_EXACT && rule != EFLA_RULE_EULER) return EFLA_ERR_INVALID_ARG;
     if (!workspace || !aligned16(workspace) ||
         workspace_bytes < efla_chunk_fwd_workspace_bytes(B, H, T, d_k, d_v, chunk, dtype))
         return EFLA_ERR_INVALID_ARG;
@@ -98,9 +99,16 @@ int efla_chunk_fwd(const void* q, const void* k, const void* v, const void* beta
     if (dtype == EFLA_DTYPE_BF16 && d_k == 128)
         return from_cuda(efla::launch_chunk_tc(q, k, v, beta, S0, o, S_T, BH, T,
                                                static_cast<uint32_t*>(workspace),
-                                               static_cast<char*>(workspace) + kWorkspaceHeader, s));
+                                               static_cast<char*>(workspace) + kWorkspaceHeader, rule, s));
     return from_cuda(efla::launch_chunk_simt(q, k, v, beta, S0, o, S_T, BH, T, d_k,
-                                             dtype == EFLA_DTYPE_BF16, s));
+                                             dtype == EFLA_DTYPE_BF16, rule, s));
+}
+
+int efla_chunk_fwd(const void* q, const void* k, const void* v, const void* beta, const float* S0,
+                   void* o, float* S_T, int B, int H, int T, int d_k, int d_v, int chunk, int dtype,
+                   void* workspace, size_t workspace_bytes, efla_stream_t stream) {
+    return efla_chunk_fwd_ex(q, k, v, beta, S0, o, S_T, B, H, T, d_k, d_v, chunk, dtype, EFLA_RULE_EXACT,
+                             workspace, workspace_bytes, stream);
 }
 
 // ---------------------------------------------------------------- allocation-free variant
@@ -165,9 +173,10 @@ int efla_selftest_wait_timeout(void* workspace, long long limit_ns, efla_stream_
                                                         (cudaStream_t)stream));
 }
 
-int efla_recurrent_step(const void* q, const void* k, const void* v, const void* beta, float* S,
-                        void* o, int N, int H, int d_k, int d_v, int dtype, efla_stream_t stream) {
+int efla_recurrent_step_ex(const void* q, const void* k, const void* v, const void* beta, float* S,
+                           void* o, int N, int H, int d_k, int d_v, int dtype, int rule, efla_stream_t stream) {
     if (N < 0 || H < 0 || d_k <= 0 || d_v <= 0) return EFLA_ERR_INVALID_ARG;
+    if (rule != EFLA_RULE_EXACT && rule != EFLA_RULE_EULER) return EFLA_ERR_INVALID_ARG;
     if (dtype != EFLA_DTYPE_F32 && dtype != EFLA_DTYPE_BF16) return EFLA_ERR_UNSUPPORTED;
     if (d_k != d_v || (d_k != 64 && d_k != 128)) return EFLA_ERR_UNSUPPORTED;
     const long NH = (long)N * H;
@@ -184,8 +193,13 @@ int efla_recurrent_step(const void* q, const void* k, const void* v, const void*
         overlaps(o, nv, v, nv) || overlaps(o, nv, beta, nb) || overlaps(S, ns, q, nq) ||
         overlaps(S, ns, k, nq) || overlaps(S, ns, v, nv) || overlaps(S, ns, beta, nb))
         return EFLA_ERR_INVALID_ARG;
-    return from_cuda(efla::launch_decode(q, k, v, beta, S, o, NH, d_k, dtype == EFLA_DTYPE_BF16,
+    return from_cuda(efla::launch_decode(q, k, v, beta, S, o, NH, d_k, dtype == EFLA_DTYPE_BF16, rule,
                                          (cudaStream_t)stream));
+}
+
+int efla_recurrent_step(const void* q, const void* k, const void* v, const void* beta, float* S,
+                        void* o, int N, int H, int d_k, int d_v, int dtype, efla_stream_t stream) {
+    return efla_recurrent_step_ex(q, k, v, beta, S, o, N, H, d_k, d_v, dtype, EFLA_RULE_EXACT, stream);
 }
 
 }  // extern "C"

@@ -74,7 +74,7 @@ __global__ void __launch_bounds__(kNT, 1) chunk_simt_kernel(const Tin* __restric
                                                             const Tin* __restrict__ beta,
                                                             const float* __restrict__ S0,
                                                             Tin* __restrict__ o,
-                                                            float* __restrict__ S_T, int T) {
+                                                            float* __restrict__ S_T, int T, int rule) {
     using L = SimtSmem<D>;
     constexpr int NSL = D / 64;                 // d_v slices per stream
     extern __shared__ float smem[];
@@ -133,7 +133,7 @@ __global__ void __launch_bounds__(kNT, 1) chunk_simt_kernel(const Tin* __restric
             for (int d = part; d < D; d += 4) lam = fmaf(Ks[r * L::kKD + d], Ks[r * L::kKD + d], lam);
             lam += __shfl_xor_sync(0xffffffffu, lam, 1);
             lam += __shfl_xor_sync(0xffffffffu, lam, 2);
-            if (part == 0) al[r] = gate_alpha(bt[r], lam);
+            if (part == 0) al[r] = rule_alpha(rule, bt[r], lam);
         }
         // ---- G = K K^T and P = Q K^T
         float g[4][4], p[4][4];
@@ -219,26 +219,26 @@ __global__ void __launch_bounds__(kNT, 1) chunk_simt_kernel(const Tin* __restric
 
 template <typename Tin, int D>
 cudaError_t launch_t(const void* q, const void* k, const void* v, const void* beta, const float* S0,
-                     void* o, float* S_T, long BH, int T, cudaStream_t stream) {
+                     void* o, float* S_T, long BH, int T, int rule, cudaStream_t stream) {
     using L = SimtSmem<D>;
     auto kern = chunk_simt_kernel<Tin, D>;
     static std::atomic<uint64_t> smem_set{0};
     cudaError_t err = set_smem_limit_once(kern, (int)L::kBytes, smem_set);
     if (err != cudaSuccess) return err;
     kern<<<(unsigned)(BH * (D / 64)), kNT, L::kBytes, stream>>>((const Tin*)q, (const Tin*)k, (const Tin*)v,
-                                                                 (const Tin*)beta, S0, (Tin*)o, S_T, T);
+                                                                 (const Tin*)beta, S0, (Tin*)o, S_T, T, rule);
     return cudaGetLastError();
 }
 }  // namespace
 
 cudaError_t launch_chunk_simt(const void* q, const void* k, const void* v, const void* beta,
                               const float* S0, void* o, float* S_T, long BH, int T, int D, bool bf16,
-                              cudaStream_t stream) {
+                              int rule, cudaStream_t stream) {
     if (bf16)
-        return D == 128 ? launch_t<__nv_bfloat16, 128>(q, k, v, beta, S0, o, S_T, BH, T, stream)
-                        : launch_t<__nv_bfloat16, 64>(q, k, v, beta, S0, o, S_T, BH, T, stream);
-    return D == 128 ? launch_t<float, 128>(q, k, v, beta, S0, o, S_T, BH, T, stream)
-                    : launch_t<float, 64>(q, k, v, beta, S0, o, S_T, BH, T, stream);
+        return D == 128 ? launch_t<__nv_bfloat16, 128>(q, k, v, beta, S0, o, S_T, BH, T, rule, stream)
+                        : launch_t<__nv_bfloat16, 64>(q, k, v, beta, S0, o, S_T, BH, T, rule, stream);
+    return D == 128 ? launch_t<float, 128>(q, k, v, beta, S0, o, S_T, BH, T, rule, stream)
+                    : launch_t<float, 64>(q, k, v, beta, S0, o, S_T, BH, T, rule, stream);
 }
 
 }  // namespace efla

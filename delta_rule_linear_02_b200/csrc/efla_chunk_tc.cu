@@ -589,9 +589,9 @@ size_t chunk_tc_workspace_bytes(long BH, int T) {
 
 cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const void* beta, const float* S0,
                             void* o, float* S_T, long BH, int T, uint32_t* err, void* scratch,
-                            cudaStream_t stream) {
+                            int rule, cudaStream_t stream) {
     const int nchunks = (T + 63) / 64;
-    cudaError_t e = launch_ut(k, beta, scratch, BH, T, err, kWaitLimitNs, stream);
+    cudaError_t e = launch_ut(k, beta, scratch, BH, T, err, kWaitLimitNs, rule, stream);
     if (e != cudaSuccess) return e;
     CUtensorMap mq, mk, mv, mt;
     if (!tma_map_tokens(&mq, q, kD, T, BH) || !tma_map_tokens(&mk, k, kD, T, BH) ||

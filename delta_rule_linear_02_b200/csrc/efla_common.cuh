@@ -48,6 +48,14 @@ __device__ __forceinline__ void store4(__nv_bfloat16* p, float4 v) {
 // For |x| = |beta*lambda| < 2^-10 the series 1 - x/2 + x^2/6 of (1 - e^{-x})/x is used
 // (truncation error below x^3/24 < 4e-11 relative): it keeps full precision when x is
 // subnormal and gives alpha = beta exactly at lambda = 0, the limit of the formula.
+// The step size the rule writes with: the exact flow's gate, or beta itself for the Euler
+// (delta-rule) step the exact flow replaces (Exact Flow Linear Attention, Section 2).
+constexpr int kRuleExact = 0, kRuleEuler = 1;
+__device__ __forceinline__ float gate_alpha(float beta, float lambda);
+__device__ __forceinline__ float rule_alpha(int rule, float beta, float lambda) {
+    return rule == kRuleEuler ? beta : gate_alpha(beta, lambda);
+}
+
 __device__ __forceinline__ float gate_alpha(float beta, float lambda) {
     const float x = beta * lambda;
     if (fabsf(x) < 0.0009765625f) {

@@ -22,7 +22,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const Tin* __restrict_
                                                           const Tin* __restrict__ v,
                                                           const Tin* __restrict__ beta,
                                                           float* __restrict__ S,
-                                                          Tin* __restrict__ o) {
+                                                          Tin* __restrict__ o, int rule) {
     constexpr int RPT = D / 32;                 // rows per thread
     constexpr int SLICES = D / kCols;
     const int t = threadIdx.x;
@@ -67,7 +67,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const Tin* __restrict_
             c += __shfl_xor_sync(0xffffffffu, c, off);
         }
         if (lane == 0) {
-            sh_alpha = gate_alpha(Elem<Tin>::to_f(beta[head]), lam);
+            sh_alpha = rule_alpha(rule, Elem<Tin>::to_f(beta[head]), lam);
             sh_c = c;
         }
     }
@@ -125,22 +125,22 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const Tin* __restrict_
 
 template <typename Tin, int D>
 cudaError_t launch_decode_t(const void* q, const void* k, const void* v, const void* beta,
-                            float* S, void* o, long NH, cudaStream_t stream) {
+                            float* S, void* o, long NH, int rule, cudaStream_t stream) {
     const long blocks = NH * (D / kCols);
     decode_kernel<Tin, D><<<(unsigned)blocks, kThreads, 0, stream>>>(
-        (const Tin*)q, (const Tin*)k, (const Tin*)v, (const Tin*)beta, S, (Tin*)o);
+        (const Tin*)q, (const Tin*)k, (const Tin*)v, (const Tin*)beta, S, (Tin*)o, rule);
     return cudaGetLastError();
 }
 }  // namespace
 
 cudaError_t launch_decode(const void* q, const void* k, const void* v, const void* beta, float* S,
-                          void* o, long NH, int D, bool bf16, cudaStream_t stream) {
+                          void* o, long NH, int D, bool bf16, int rule, cudaStream_t stream) {
     if (bf16) {
-        return D == 128 ? launch_decode_t<__nv_bfloat16, 128>(q, k, v, beta, S, o, NH, stream)
-                        : launch_decode_t<__nv_bfloat16, 64>(q, k, v, beta, S, o, NH, stream);
+        return D == 128 ? launch_decode_t<__nv_bfloat16, 128>(q, k, v, beta, S, o, NH, rule, stream)
+                        : launch_decode_t<__nv_bfloat16, 64>(q, k, v, beta, S, o, NH, rule, stream);
     }
-    return D == 128 ? launch_decode_t<float, 128>(q, k, v, beta, S, o, NH, stream)
-                    : launch_decode_t<float, 64>(q, k, v, beta, S, o, NH, stream);
+    return D == 128 ? launch_decode_t<float, 128>(q, k, v, beta, S, o, NH, rule, stream)
+                    : launch_decode_t<float, 64>(q, k, v, beta, S, o, NH, rule, stream);
 }
 
 }  // namespace efla

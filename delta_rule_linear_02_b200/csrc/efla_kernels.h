@@ -10,21 +10,22 @@ namespace efla {
 cudaError_t launch_gate(const void* k, const void* beta, float* alpha, long n, int dk, bool bf16,
                         cudaStream_t stream);
 
+// rule: kRuleExact (the exact-flow gate) or kRuleEuler (alpha = beta, the delta rule)
 cudaError_t launch_decode(const void* q, const void* k, const void* v, const void* beta, float* S,
-                          void* o, long NH, int D, bool bf16, cudaStream_t stream);
+                          void* o, long NH, int D, bool bf16, int rule, cudaStream_t stream);
 
 cudaError_t launch_chunk_simt(const void* q, const void* k, const void* v, const void* beta,
                               const float* S0, void* o, float* S_T, long BH, int T, int D, bool bf16,
-                              cudaStream_t stream);
+                              int rule, cudaStream_t stream);
 
 // bf16, d_k = d_v = 128: the UT kernel (efla_ut.cu) writes every chunk's T into `scratch`
 // (chunk_tc_workspace_bytes bytes, 16-byte aligned), then the chain kernel runs.
 size_t chunk_tc_workspace_bytes(long BH, int T);
 cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const void* beta, const float* S0,
                             void* o, float* S_T, long BH, int T, uint32_t* err, void* scratch,
-                            cudaStream_t stream);
+                            int rule, cudaStream_t stream);
 cudaError_t launch_ut(const void* k, const void* beta, void* Tout, long BH, int T, uint32_t* err,
-                      unsigned long long limit_ns, cudaStream_t stream);
+                      unsigned long long limit_ns, int rule, cudaStream_t stream);
 
 cudaError_t launch_wait_timeout_selftest(uint32_t* err, unsigned long long limit_ns, cudaStream_t stream);
 

@@ -9,7 +9,8 @@
 // Per tile (stream bh, chunk c):
 //   G = K K^T                                   tcgen05 MMA, M = 64 (bf16 in, fp32 in TMEM;
 //                                                row r in lane (r % 16) + 32 (r / 16))
-//   lambda_r = G_rr, alpha_r = gate(beta_r, lambda_r)   (Section 3.2 / 3.4)
+//   lambda_r = G_rr, alpha_r = gate(beta_r, lambda_r)   (Section 3.2 / 3.4; beta_r itself
+//                                                under the Euler rule, Section 2)
 //   A^T rows = alpha (.) G rows                 (G is symmetric)
 //   X = (I + A)^{-1}                            efla_ut_tf32.cuh (fp32 + TF32 merges)
 //   T = X diag(alpha) -> bf16, row-major 64 x 64, at Tout + 4096 * (bh * nchunks + c)
@@ -79,7 +80,7 @@ __device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, vol
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 ut_kernel(const __grid_constant__ CUtensorMap tm_k, const __nv_bfloat16* __restrict__ beta,
           __nv_bfloat16* __restrict__ Tout, int T, int nchunks, long ntiles, uint32_t* __restrict__ err,
-          unsigned long long limit_ns) {
+          unsigned long long limit_ns, int rule) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sb = smem_u32(sm);
@@ -192,7 +193,7 @@ ut_kernel(const __grid_constant__ CUtensorMap tm_k, const __nv_bfloat16* __restr
                 float lam = 0.f;
 #pragma unroll
                 for (int e = 0; e < 64; ++e) lam = (e == r) ? g[e] : lam;
-                al[r] = gate_alpha(bt[r], lam);
+                al[r] = rule_alpha(rule, bt[r], lam);
             }
             tc_fence_before();
             bar_sync(NB_W, 128);                     // alpha visible, G read
@@ -246,7 +247,7 @@ int sm_count() {
 }  // namespace
 
 cudaError_t launch_ut(const void* k, const void* beta, void* Tout, long BH, int T, uint32_t* err,
-                      unsigned long long limit_ns, cudaStream_t stream) {
+                      unsigned long long limit_ns, int rule, cudaStream_t stream) {
     CUtensorMap mk;
     if (!tma_map_tokens(&mk, k, 128, T, BH)) return cudaErrorInvalidValue;
     const int nchunks = (T + 63) / 64;
@@ -257,7 +258,7 @@ cudaError_t launch_ut(const void* k, const void* beta, void* Tout, long BH, int 
     if (e != cudaSuccess) return e;
     ut_kernel<<<(unsigned)grid, kThreads, SMEM_BYTES, stream>>>(mk, (const __nv_bfloat16*)beta,
                                                                 (__nv_bfloat16*)Tout, T, nchunks, ntiles, err,
-                                                                limit_ns);
+                                                                limit_ns, rule);
     return cudaGetLastError();
 }
 

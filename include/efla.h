@@ -49,6 +49,17 @@ typedef enum {
     EFLA_DTYPE_BF16 = 1   /* bfloat16 q, k, v, beta, o (fp32 accumulation and state) */
 } efla_dtype;
 
+/*
+ * The step size each token writes with.  EFLA_RULE_EXACT is the method: the exact-flow
+ * gate alpha = (1 - exp(-beta lambda)) / lambda (Section 3.2).  EFLA_RULE_EULER is the
+ * delta rule the method replaces (alpha = beta: one explicit Euler step of the same ODE,
+ * Section 2), run through the same kernels for comparison.
+ */
+typedef enum {
+    EFLA_RULE_EXACT = 0,
+    EFLA_RULE_EULER = 1
+} efla_rule;
+
 /* Same type as cudaStream_t, declared here so this header needs no CUDA include. */
 typedef struct CUstream_st *efla_stream_t;
 
@@ -97,6 +108,18 @@ int efla_chunk_fwd(const void *q, const void *k, const void *v, const void *beta
                    const float *S0, void *o, float *S_T, int B, int H, int T, int d_k,
                    int d_v, int chunk, int dtype, void *workspace, size_t workspace_bytes,
                    efla_stream_t stream);
+
+/*
+ * efla_chunk_fwd_ex -- efla_chunk_fwd with the step rule chosen: `rule` is an efla_rule
+ * (any other value: EFLA_ERR_INVALID_ARG, nothing launched).  efla_chunk_fwd is this call
+ * with EFLA_RULE_EXACT.  Under EFLA_RULE_EULER the forward is the chunked delta rule
+ * (DeltaNet form): the same UT-transform algebra with alpha = beta.  Every other argument
+ * and behaviour is that of efla_chunk_fwd.
+ */
+int efla_chunk_fwd_ex(const void *q, const void *k, const void *v, const void *beta,
+                      const float *S0, void *o, float *S_T, int B, int H, int T, int d_k,
+                      int d_v, int chunk, int dtype, int rule, void *workspace,
+                      size_t workspace_bytes, efla_stream_t stream);
 
 /*
  * efla_chunk_fwd_noalloc -- efla_chunk_fwd without a caller-provided workspace.
@@ -153,6 +176,15 @@ int efla_selftest_wait_timeout(void *workspace, long long limit_ns, efla_stream_
 int efla_recurrent_step(const void *q, const void *k, const void *v, const void *beta,
                         float *S, void *o, int N, int H, int d_k, int d_v, int dtype,
                         efla_stream_t stream);
+
+/*
+ * efla_recurrent_step_ex -- efla_recurrent_step with the step rule chosen (`rule` an
+ * efla_rule, else EFLA_ERR_INVALID_ARG and nothing launched).  efla_recurrent_step is
+ * this call with EFLA_RULE_EXACT; EFLA_RULE_EULER writes with alpha = beta.
+ */
+int efla_recurrent_step_ex(const void *q, const void *k, const void *v, const void *beta,
+                           float *S, void *o, int N, int H, int d_k, int d_v, int dtype,
+                           int rule, efla_stream_t stream);
 
 #ifdef __cplusplus
 }

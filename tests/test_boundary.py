@@ -97,6 +97,27 @@ def test_recurrent_step_rejects_bad_arguments(efla):
     assert L.efla_recurrent_step(P[0], P[1], P[2], P[3], P[4], P[5], 4, 2, 128, 64, 0, None) == UNSUPPORTED
 
 
+def test_rule_entry_points_validate_the_rule(efla):
+    """The _ex entry points take the step rule; anything but EXACT (0) or EULER (1) is an
+    invalid argument and launches nothing.  With a valid rule the other checks are those
+    of the plain entry points."""
+    L = efla.lib
+    q, k, v, b, s0, o, st, w = GOOD
+    B, H, T, d, ws = 1, 2, 128, 128, 1 << 24
+    fwd = lambda rule, ptrs=GOOD, **kw: L.efla_chunk_fwd_ex(*ptrs[:7], kw.get("B", B), H, T, d, d, 64, 1, rule,
+                                                             ptrs[7], ws, None)
+    for rule in (-1, 2, 7):
+        assert fwd(rule) == INVALID
+    assert fwd(0, B=0) == OK and fwd(1, B=0) == OK
+    bad = list(GOOD); bad[0] = None
+    assert fwd(1, bad) == INVALID
+    step = lambda rule, N=4: L.efla_recurrent_step_ex(*GOOD[:6], N, 2, 128, 128, 0, rule, None)
+    for rule in (-1, 2):
+        assert step(rule) == INVALID
+    assert step(0, N=0) == OK and step(1, N=0) == OK
+    assert efla.EFLA_RULE_EXACT == 0 and efla.EFLA_RULE_EULER == 1
+
+
 def test_gate_rejects_bad_arguments(efla):
     L = efla.lib
     assert L.efla_gate(GOOD[0], GOOD[1], GOOD[2], 10, 6, 0, None) == UNSUPPORTED   # 24-byte rows
