@@ -252,6 +252,8 @@ def main():
     ap.add_argument("--impl", default="efla", choices=["efla", "reference"])
     ap.add_argument("--decode-steps", type=int, default=1000)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--other-steps", type=int, default=10,
+                    help="forwards timed on each of the long-context and stiff workloads (0: skip)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.impl == "reference":
@@ -376,6 +378,40 @@ def main():
                "gpu_launches": nd}
         del S, st
 
+    # ---- the other forward workloads (long context, stiff keys): tokens/s and roofline
+    # fraction of a few forwards each, inputs resident in HBM, CUDA events around the calls
+    others = {}
+    for name in ([] if args.other_steps <= 0 else ["longctx_bf16", "stiff_bf16"]):
+        wo = workloads.CHUNK_WORKLOADS[name]
+        wo = wo.replace(seed=wo.seed + 1000 * rank)
+        xo = {k_: (None if v_ is None else v_.to(dev)) for k_, v_ in workloads.make_chunk_inputs(wo).items()}
+        wso = efla.new_workspace(wo.B, wo.H, wo.T, wo.dk, wo.dv, 64, wo.dtype, dev)
+        oo = torch.empty(wo.B, wo.H, wo.T, wo.dv, dtype=wo.dtype, device=dev)
+        So = torch.empty(wo.B, wo.H, wo.dk, wo.dv, dtype=torch.float32, device=dev)
+        call = lambda: efla.efla_chunk_fwd(xo["q"], xo["k"], xo["v"], xo["beta"], xo["S0"], o=oo, S_T=So,
+                                           workspace=wso, stream=stream)
+        for _ in range(args.warmup):
+            call()
+        barrier(world)
+        o0, o1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        o0.record(stream)
+        for _ in range(args.other_steps):
+            call()
+        o1.record(stream)
+        barrier(world)
+        oms = max_over_ranks(o0.elapsed_time(o1), world) / args.other_steps
+        if efla.efla_workspace_status(wso, clear=True, stream=stream) != efla.EFLA_OK:
+            raise SystemExit(f"device reported a timeout on {name}")
+        ob, of = chunk_alg(wo)
+        ot = max(ob / (hbm * 1e9), of / (tc * 1e12))
+        others[name] = {"value": wo.tokens * world / (oms * 1e-3), "unit": "tokens/s", "ms_per_step": oms,
+                        "steps": args.other_steps,
+                        "config": {"B": wo.B, "H": wo.H, "T": wo.T, "d_k": wo.dk, "d_v": wo.dv, "chunk": 64},
+                        "roofline": {"bound": "hbm", "achieved": ob / (oms * 1e-3) / 1e9, "peak": hbm,
+                                     "unit": "GB/s", "frac": ot / (oms * 1e-3), "roofline_time_us": ot * 1e6},
+                        "gpu_launches": 2 * args.other_steps}
+        del xo, wso, oo, So
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(WORKLOAD)
@@ -392,7 +428,7 @@ def main():
             "roofline": roofline, "e2e": e2e,
             # bf16, d = 128: each efla_chunk_fwd launches the UT kernel and the chain kernel
             "gpu_launches": 2 * args.steps,
-            "clocks": clk.summary(), "decode": dec, "cpu_baseline": cpu,
+            "clocks": clk.summary(), "decode": dec, "other_workloads": others, "cpu_baseline": cpu,
             "kernel_source": kernel_source_hash(),
         }
         print(json.dumps(line), flush=True)
