@@ -27,8 +27,8 @@
 // (K, V, T, Q), Delta and the bf16 copy of S.
 //
 // One warp issues every MMA, in a fixed order per chunk c:
-//   [W;Q] S(c), [W|U](c+1), half of Q K^T(c+1) if its Q is in place, K^T Delta(c) (after
-//   Delta), P Delta(c), the rest of Q K^T(c+1)
+//   [W;Q] S(c), Q K^T(c), [W|U](c+1), K^T Delta(c) (after Delta), P Delta(c)
+// so that only P Delta(c) is in the pipe ahead of the next [W;Q] S.
 // Issue is by a converged warp with elect.sync (warp-uniform control flow keeps the
 // descriptors in uniform registers; a one-lane issuer in a data-dependent loop issues
 // several times slower).
@@ -279,7 +279,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         // Warp-uniform control flow: every lane polls the barrier and the warp votes;
         // elect.sync inside each MMA and commit picks the issuing lane.
         auto wait = [&](int i, uint32_t parity) { return __all_sync(0xffffffffu, ctl.wait(i, parity)); };
-        auto ready = [&](int i, uint32_t parity) { return __all_sync(0xffffffffu, mbar_test_wait(ctl.b(i), parity)); };
         auto issue_qk = [&](int c, int k0, int k1) {      // [W;Q] K^T, k-steps [k0, k1): rows 64-127 are Q K^T
             tc_fence_after();
             const uint64_t db = sdesc_sw128(sb + kvt(c) + KVT_K, 16, 1024);
@@ -298,30 +297,26 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             mma_commit_elect(ctl.b(B_WU_FULL));
             EFLA_STAMP(c, 1);
         };
-        bool ok = wait(B_KVT_FULL, 0) && wait(B_Q_READY, 0);
-        if (ok) {
-            issue_qk(0, 0, 8);
-            issue_wu(0);
-        }
+        bool ok = wait(B_KVT_FULL, 0);
+        if (ok) issue_wu(0);
         for (int c = 0; c < nchunks && ok; ++c) {
             // X = [W; Q] S (state chain)
-            if (!(ok = wait(B_W_READY, c & 1) && wait(B_SB_READY, c & 1) && (c == 0 || wait(B_X_FREE, (c - 1) & 1))))
+            if (!(ok = wait(B_W_READY, c & 1) && wait(B_Q_READY, c & 1) && wait(B_SB_READY, c & 1) &&
+                       (c == 0 || wait(B_X_FREE, (c - 1) & 1))))
                 break;
             tc_fence_after();
             mma_ts(tmem + TM_X, tmem + TM_AWQ, sb + OFF_SB, 4 * 2048, 2048, TILE, ID_N64, 8, 0);
             mma_commit_elect(ctl.b(B_XS_FULL));
             EFLA_STAMP(c, 2);
-            // the next chunk's [W | U] fills the pipe while Delta is formed
+            // this chunk's Q K^T (its Q has been in place since the last chunk) and the next
+            // chunk's [W | U] fill the pipe while Delta is formed; after K^T Delta only
+            // P Delta remains ahead of the next [W;Q] S
+            if (!(ok = c == 0 || wait(B_GP_FREE, (c - 1) & 1))) break;
+            issue_qk(c, 0, 8);
             if (c + 1 < nchunks) {
                 if (!(ok = wait(B_KVT_FULL + (c + 1) % kKvtStages, ((c + 1) / kKvtStages) & 1) &&
                            wait(B_WU_FREE, c & 1))) break;
                 issue_wu(c + 1);
-            }
-            // half of the next chunk's Q K^T too, if its Q is already in place (never wait here)
-            int qk_half = 0;
-            if (c + 1 < nchunks && ready(B_Q_READY, (c + 1) & 1) && ready(B_GP_FREE, c & 1)) {
-                issue_qk(c + 1, 0, 4);
-                qk_half = 4;
             }
             // S += K^T Delta (state chain)
             if (!(ok = wait(B_D_READY, c & 1))) break;
@@ -336,11 +331,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             tc_fence_after();
             mma_ts(tmem + TM_X, tmem + TM_AP, sb + OFF_DL, 4 * 2048, 2048, TILE, ID_N64, 4, 1);
             mma_commit_elect(ctl.b(B_O_FULL));
-            // the (rest of the) next chunk's Q K^T
-            if (c + 1 < nchunks) {
-                if (qk_half == 0 && !(ok = wait(B_Q_READY, (c + 1) & 1) && wait(B_GP_FREE, c & 1))) break;
-                issue_qk(c + 1, qk_half, 8);
-            }
         }
         mma_commit_elect(ctl.b(B_DRAIN));
         if (lane == 0) mbar_wait(ctl.b(B_DRAIN), 0, limit_ns);
