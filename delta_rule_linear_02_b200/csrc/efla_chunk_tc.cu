@@ -152,9 +152,14 @@ struct Ctl {
     unsigned long long limit;
     __device__ uint64_t* b(int i) const { return bar + i; }
     // bounded wait; gives up early once another role has aborted.  A phase that has
-    // already completed is seen by one non-blocking probe.
-    __device__ bool wait(int i, uint32_t parity) const {
+    // already completed is seen by one inlined non-blocking probe; the sleeping, timed
+    // part is one out-of-line copy, which keeps the role loops small in the
+    // instruction cache.
+    __device__ __forceinline__ bool wait(int i, uint32_t parity) const {
         if (mbar_test_wait(bar + i, parity)) return true;
+        return wait_slow(i, parity);
+    }
+    __device__ __noinline__ bool wait_slow(int i, uint32_t parity) const {
         if (mbar_try_wait_sleep(bar + i, parity, 20000)) return true;
         const uint64_t t0 = globaltimer_ns();
         while (!mbar_try_wait_sleep(bar + i, parity, 20000)) {
