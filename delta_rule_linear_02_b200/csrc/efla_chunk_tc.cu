@@ -44,10 +44,11 @@
 //                bf16 S and S_T.
 // Every wait is bounded (2 s); a wait that runs out sets a CTA-wide abort flag, every
 // role winds down, and the caller's workspace records the timeout.
-// Built with EFLA_CHUNK_TRACE=1 (never in the library), `dbg` receives CTA 0's chunk-0
+// Built with EFLA_CHUNK_TRACE=2 (never in the library), `dbg` receives CTA 0's chunk-0
 // intermediates for diagnosis:
 // W [8256,16448) U [16448,20544) WS [20544,24640) S after the chunk [24640,32832); and
-// per chunk c < 64 the cycle at which each role passed its milestones, at
+// with EFLA_CHUNK_TRACE >= 1, per chunk c < 64 the cycle at which each role passed its
+// milestones, at
 // [40000 + 16 c + k): k = 0 QK^T, 1 [W|U], 2 [W;Q]S, 3 K^T Delta issued; 4 P ready;
 // 5 Q ready; 6 W ready; 7 U taken; 8 Delta ready; 9 new S ready; 10 O stored; 11 TMA.
 #include <cudaTypedefs.h>
@@ -62,9 +63,11 @@ namespace efla {
 #ifndef EFLA_CHUNK_TRACE
 #define EFLA_CHUNK_TRACE 0
 #endif
-// diagnosis stores compiled in only for tracing builds: they cost instruction-cache
-// space in the role loops even when never taken
-constexpr bool kTrace = EFLA_CHUNK_TRACE != 0;
+// diagnosis stores compiled in only for tracing builds (1: milestone cycles, 2: also
+// chunk-0 intermediates): they cost instruction-cache space in the role loops even when
+// never taken
+constexpr bool kTrace = EFLA_CHUNK_TRACE >= 1;
+constexpr bool kTraceDump = EFLA_CHUNK_TRACE >= 2;
 
 namespace {
 using namespace sm100;
@@ -365,7 +368,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
                 for (int j = 0; j < 32; ++j) pk[j] = pack_bf16x2(w[2 * j], w[2 * j + 1]);
                 tmem_st32(tmem + lane_off + TM_AWQ + 32 * h, pk);
-                if (kTrace && dbg && blockIdx.x == 0 && c == 0)
+                if (kTraceDump && dbg && blockIdx.x == 0 && c == 0)
                     for (int j = 0; j < 64; ++j) dbg[8256 + r * 128 + 64 * h + j] = w[j];
             }
             tmem_wait_st();
@@ -509,7 +512,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         mbar_arrive(ctl.b(B_WU_FREE));
                         EFLA_STAMP(c, 7);
                     }
-                    if (kTrace && dbg && blockIdx.x == 0 && c == 0)
+                    if (kTraceDump && dbg && blockIdx.x == 0 && c == 0)
                         for (int j = 0; j < 32; ++j) dbg[16448 + ct * 64 + cc + j] = u[j];
                     // Delta = U - W S (X rows 0-63)
                     ok = bar_and(NB_DELTA, kHalfChain, ctl.wait(B_XS_FULL, c & 1));
@@ -518,7 +521,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     tc_fence_after();
                     float t[32];
                     tmem_ld32_wait(tmem + lane_off + TM_X + cc, t);
-                    if (kTrace && dbg && blockIdx.x == 0 && c == 0)
+                    if (kTraceDump && dbg && blockIdx.x == 0 && c == 0)
                         for (int j = 0; j < 32; ++j) dbg[20544 + ct * 64 + cc + j] = t[j];
 #pragma unroll
                     for (int j = 0; j < 32; ++j) t[j] = u[j] - t[j];
@@ -542,7 +545,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 tmem_ld32_wait(tmem + lane_off + TM_S + cc, t);
 #pragma unroll
                 for (int j = 0; j < 4; ++j) st_chunk(sm + OFF_SB + sw128_off(ct, 4 * ch + j), t + 8 * j);
-                if (kTrace && dbg && blockIdx.x == 0 && c == 0)
+                if (kTraceDump && dbg && blockIdx.x == 0 && c == 0)
                     for (int j = 0; j < 32; ++j) dbg[24640 + ct * 64 + cc + j] = t[j];
                 if (c == nchunks - 1 && S_T) {
                     float* dst = S_T + ((size_t)bh * kD + ct) * kD + col0 + cc;
