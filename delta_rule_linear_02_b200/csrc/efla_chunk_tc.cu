@@ -16,15 +16,17 @@
 //   X += [*; P] Delta                        (rows 64-127 become O = Q S + P Delta)
 // Tokens past T are zero-filled by TMA (k = 0, and T's rows/columns are zero there).
 //
-// What bounds a chunk step is shared memory: an N = 64 MMA reads about 6 KB of smem
-// operands in the ~47 cycles it takes, close to the SM's shared-memory bandwidth, and
-// while it runs the CUDA-core epilogues' shared loads and stores (and every mbarrier
-// probe) wait several times longer than on an idle pipe.  So the A operands [W; Q] and
-// [*; P] live in tensor memory (bf16, K-major: TMEM column j of lane m holds elements
-// 2j and 2j + 1 of row m): W goes from its fp32 accumulator to the A operand without
-// touching shared memory, P likewise, Q is copied in once, and U is read by the Delta
-// warps straight from its accumulator.  Shared memory then holds only the TMA tiles
-// (K, V, T, Q), Delta and the bf16 copy of S.
+// The A operands [W; Q] and [*; P] live in tensor memory (bf16, K-major: TMEM column j of
+// lane m holds elements 2j and 2j + 1 of row m): an N = 64 MMA with A in tensor memory
+// runs at the tensor core's math rate (~33 cycles), one with both operands in shared
+// memory at the shared-memory bandwidth (~49 cycles).  W goes from its fp32 accumulator
+// to the A operand without touching shared memory, P likewise, Q is copied in once, and
+// U is read by the Delta warps straight from its accumulator.  Shared memory then holds
+// only the TMA tiles (K, V, T, Q), Delta and the bf16 copy of S.
+//
+// A chunk step is bound by latency, not by a unit's throughput: its MMAs take ~1,240
+// tensor-pipe cycles, and the rest of a step is the hand-offs of the chain
+// [W;Q] S -> Delta -> K^T Delta -> bf16 S -> the next [W;Q] S between roles.
 //
 // One warp issues every MMA, in a fixed order per chunk c:
 //   [W;Q] S(c), Q K^T(c), [W|U](c+1), K^T Delta(c) (after Delta), P Delta(c)
