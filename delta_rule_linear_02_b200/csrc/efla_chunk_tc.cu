@@ -590,6 +590,11 @@ __global__ void wait_timeout_selftest_kernel(uint32_t* err, unsigned long long l
 
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;   // 2 s per wait
 
+#if EFLA_CHUNK_TRACE
+// tracing builds only: the diagnosis record of CTA 0
+__device__ float g_chunk_dbg[40000 + 64 * 16];
+#endif
+
 size_t chunk_tc_workspace_bytes(long BH, int T) {
     const long nchunks = (T + 63) / 64;
     return (size_t)BH * nchunks * 64 * 64 * 2;     // the bf16 T of every chunk
@@ -608,8 +613,12 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const v
     static std::atomic<uint64_t> smem_set{0};
     e = set_smem_limit_once(chunk_tc_kernel, (int)SMEM_BYTES, smem_set);
     if (e != cudaSuccess) return e;
+    float* dbg = nullptr;
+#if EFLA_CHUNK_TRACE
+    if (cudaGetSymbolAddress((void**)&dbg, g_chunk_dbg) != cudaSuccess) dbg = nullptr;
+#endif
     chunk_tc_kernel<<<(unsigned)(BH * 2), kThreads, SMEM_BYTES, stream>>>(mq, mk, mv, mt, S0, (__nv_bfloat16*)o,
-                                                                          S_T, T, err, kWaitLimitNs, nullptr);
+                                                                          S_T, T, err, kWaitLimitNs, dbg);
     return cudaGetLastError();
 }
 
@@ -619,3 +628,11 @@ cudaError_t launch_wait_timeout_selftest(uint32_t* err, unsigned long long limit
 }
 
 }  // namespace efla
+
+#if EFLA_CHUNK_TRACE
+// tracing builds only: copy CTA 0's milestone cycles (16 per chunk, chunks 0-63) to the host
+extern "C" int efla_chunk_trace_copy(float* host, int n) {
+    return (int)cudaMemcpyFromSymbol(host, efla::g_chunk_dbg, sizeof(float) * (size_t)std::min(n, 64 * 16),
+                                     sizeof(float) * 40000);
+}
+#endif

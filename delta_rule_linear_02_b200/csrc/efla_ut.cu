@@ -17,12 +17,12 @@
 // Tokens past T are zero-filled by TMA (k = 0, beta = 0: alpha = 0, their rows and
 // columns of T are zero).
 //
-// A persistent grid of four CTAs per SM walks the tiles.  Each CTA holds kStages K tiles
-// (the next tile's TMA is in flight while the current one is solved); one stage and four
-// CTAs per SM measured faster than two stages and three CTAs, since the CTAs on an SM
-// overlap each other's latency.  Warp 0 (whole-warp control flow, elect.sync) issues the
-// TMA copies and the MMA;
-// warps 1-4 compute the gate, the solve and the bf16 store.  Every wait is bounded.
+// A persistent grid of six CTAs per SM walks the tiles; the CTAs on an SM overlap each
+// other's latency.  The K tile is dead once G has been formed, so A^T is written over it:
+// a CTA holds one fp32 64 x 68 tile for K / A^T and one for X (36 KB), and the next K tile
+// is loaded while the T of the current one is stored.  Warp 0 (whole-warp control flow,
+// elect.sync) issues the TMA copies and the MMA; warps 1-4 compute the gate, the solve and
+// the bf16 store.  Every wait is bounded.
 #include "efla_common.cuh"
 #include "efla_kernels.h"
 #include "efla_tma.cuh"
@@ -36,13 +36,13 @@ using namespace sm100;
 using ut::LDX;
 
 constexpr int kThreads = 160;
-constexpr int kCtasPerSm = 4;
-constexpr int kStages = 1;                             // K tiles in flight per CTA
+constexpr int kCtasPerSm = 6;
 constexpr uint32_t TILE = 8192;
-constexpr uint32_t OFF_K = 0;                          // kStages x [K a0 | K a1]
-constexpr uint32_t F32_TILE = 64 * LDX * 4;
-constexpr uint32_t OFF_AT = OFF_K + kStages * 2 * TILE;
+constexpr uint32_t F32_TILE = 64 * LDX * 4;            // 17,408 bytes (a multiple of 1024)
+constexpr uint32_t OFF_K = 0;                          // [K a0 | K a1], then A^T over it
+constexpr uint32_t OFF_AT = OFF_K;
 constexpr uint32_t OFF_X = OFF_AT + F32_TILE;
+static_assert(2 * TILE <= F32_TILE && F32_TILE % 1024 == 0, "K / A^T region");
 constexpr uint32_t OFF_ALPHA = OFF_X + F32_TILE;
 constexpr uint32_t OFF_BETA = OFF_ALPHA + 256;
 constexpr uint32_t OFF_BAR = OFF_BETA + 256;
@@ -52,8 +52,7 @@ constexpr uint32_t SMEM_USED = OFF_MISC + 16;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;
 static_assert(kCtasPerSm * SMEM_BYTES <= 232448, "UT kernel: shared memory for the target occupancy");
 
-enum : int { B_FULL = 0 /* [kStages] */, B_GP_FULL = 2, B_GP_FREE = 3, B_DRAIN = 4 };
-static_assert(kStages <= 2, "barrier map holds two stages");
+enum : int { B_FULL = 0, B_GP_FULL = 1, B_GP_FREE = 2, B_AT_FREE = 3, B_DRAIN = 4 };
 constexpr uint32_t TM_COLS = 64;
 constexpr uint32_t ID_G = idesc_bf16(64, 64, false, false);
 constexpr int NB_W = 1;                                // named barrier of the 128 worker threads
@@ -129,39 +128,32 @@ ut_kernel(const __grid_constant__ CUtensorMap tm_k, const __nv_bfloat16* __restr
             if (lane == 0) {
                 const long tile = first + (long)j * step;
                 const int bh = (int)(tile / nchunks), c = (int)(tile % nchunks);
-                uint8_t* st = sm + OFF_K + (j % kStages) * 2 * TILE;
-                mbar_arrive_expect_tx(bar + B_FULL + (j % kStages), 2 * TILE);
-                tma_load_3d(st, &tm_k, bar + B_FULL + (j % kStages), 0, c * 64, bh);
-                tma_load_3d(st + TILE, &tm_k, bar + B_FULL + (j % kStages), 64, c * 64, bh);
+                mbar_arrive_expect_tx(bar + B_FULL, 2 * TILE);
+                tma_load_3d(sm + OFF_K, &tm_k, bar + B_FULL, 0, c * 64, bh);
+                tma_load_3d(sm + OFF_K + TILE, &tm_k, bar + B_FULL, 64, c * 64, bh);
             }
             __syncwarp();
         };
-        for (int j = 0; j < min(kStages, ntile); ++j) load(j);
+        if (ntile > 0) load(0);
         bool ok = true;
         for (int j = 0; j < ntile && ok; ++j) {
-            const int s = j % kStages;
-            ok = wait(bar + B_FULL + s, (j / kStages) & 1) && (j == 0 || wait(bar + B_GP_FREE, (j - 1) & 1));
+            ok = wait(bar + B_FULL, j & 1) && (j == 0 || wait(bar + B_GP_FREE, (j - 1) & 1));
             if (!ok) break;
             tc_fence_after();
-            const uint32_t st = sb + OFF_K + s * 2 * TILE;
-            const uint64_t d0 = sdesc_sw128(st, 16, 1024);
+            const uint64_t d0 = sdesc_sw128(sb + OFF_K, 16, 1024);
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks) {
                 const uint64_t d = d0 + (((ks >> 2) * TILE + (ks & 3) * 32) >> 4);
                 mma_bf16_elect(tmem, d, d, ID_G, ks > 0);
             }
             mma_commit_elect(bar + B_GP_FULL);
-            if (j + kStages < ntile) {  // the stage is free once this MMA has read it
-                if (!(ok = wait(bar + B_GP_FULL, j & 1))) break;
-                load(j + kStages);
+            if (j + 1 < ntile) {  // the region is free once the solve no longer reads A^T
+                if (!(ok = wait(bar + B_AT_FREE, j & 1))) break;
+                load(j + 1);
             }
         }
         mma_commit_elect(bar + B_DRAIN);
-        if (lane == 0) {
-            mbar_wait(bar + B_DRAIN, 0, limit_ns);
-            for (int j = max(0, ntile - kStages); j < ntile; ++j)
-                mbar_wait(bar + B_FULL + j % kStages, (j / kStages) & 1, limit_ns);
-        }
+        if (lane == 0) mbar_wait(bar + B_DRAIN, 0, limit_ns);
         __syncwarp();
     } else {
         // ------------------------------------------------------------ workers (128 threads)
@@ -187,28 +179,44 @@ ut_kernel(const __grid_constant__ CUtensorMap tm_k, const __nv_bfloat16* __restr
             ok = bar_and(NB_W, 128, ok && wait_bounded(bar + B_GP_FULL, j & 1, abort, limit_ns));
             if (!ok) break;
             tc_fence_after();
-            float g[64];
-            tmem_ld64_wait(tmem + lane_off, g);
-            if (grow) {
-                float lam = 0.f;
+            {   // lambda_r = G_rr from the 32-column half that holds column r (warp-uniform)
+                float g[32];
+                tmem_ld32_wait(tmem + lane_off + 32 * (q >> 1), g);
+                if (grow) {
+                    // a masked sum, not a select chain: it keeps g in registers (the compiler
+                    // turns a select chain over g into an indexed local-memory load)
+                    const int d = r - 32 * (q >> 1);
+                    float lam = 0.f;
 #pragma unroll
-                for (int e = 0; e < 64; ++e) lam = (e == r) ? g[e] : lam;
-                al[r] = rule_alpha(rule, bt[r], lam);
-            }
-            tc_fence_before();
-            bar_sync(NB_W, 128);                     // alpha visible, G read
-            if (wt == 0) mbar_arrive(bar + B_GP_FREE);
-            if (grow) {
-                // A^T[r][i] = A[i][r] = alpha_i G[i][r] = alpha_i G[r][i]; only i > r is read
-#pragma unroll
-                for (int m = 0; m < 16; ++m) {
-                    const float4 a = *reinterpret_cast<const float4*>(al + 4 * m);
-                    *reinterpret_cast<float4*>(At + r * LDX + 4 * m) =
-                        make_float4(a.x * g[4 * m], a.y * g[4 * m + 1], a.z * g[4 * m + 2], a.w * g[4 * m + 3]);
+                    for (int e = 0; e < 32; ++e) lam = fmaf(g[e], e == d ? 1.f : 0.f, lam);
+                    al[r] = rule_alpha(rule, bt[r], lam);
                 }
             }
-            bar_sync(NB_W, 128);
+            bar_sync(NB_W, 128);                     // alpha visible
+            // A^T[r][i] = A[i][r] = alpha_i G[i][r] = alpha_i G[r][i]; only i > r is read.
+            // The K tile under A^T was read by the finished G MMA.
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                float g[32];
+                tmem_ld32_wait(tmem + lane_off + 32 * h, g);
+                if (grow) {
+#pragma unroll
+                    for (int m = 0; m < 8; ++m) {
+                        const float4 a = *reinterpret_cast<const float4*>(al + 32 * h + 4 * m);
+                        *reinterpret_cast<float4*>(At + r * LDX + 32 * h + 4 * m) =
+                            make_float4(a.x * g[4 * m], a.y * g[4 * m + 1], a.z * g[4 * m + 2], a.w * g[4 * m + 3]);
+                    }
+                }
+            }
+            tc_fence_before();
+            bar_sync(NB_W, 128);                     // G read, A^T written
+            if (wt == 0) mbar_arrive(bar + B_GP_FREE);
             ut::ut_solve<NB_W, 128>(At, X, wt);
+            // A^T is dead: the next K tile may land over it (the async-proxy TMA write is
+            // ordered after this tile's generic writes there)
+            fence_proxy_async_smem();
+            bar_sync(NB_W, 128);
+            if (wt == 0) mbar_arrive(bar + B_AT_FREE);
             {   // T = X diag(alpha) -> bf16, 64 bytes per thread (a warp reads 32 consecutive
                 // rows of one column half: conflict-free with the 68-float row stride)
                 const long tile = first + (long)j * step;
