@@ -314,38 +314,62 @@ def main():
                 "tensor_tflops": flops / (launch_ms * 1e-3) / 1e12,
                 "roofline_time_us": t_star * 1e6, "roofline_frac": t_star / (launch_ms * 1e-3)}
 
-    # ---- end to end through the public API with host buffers (pinned), copies timed
+    # ---- end to end through the public API with host buffers (pinned), copies timed.
+    # Every step copies its inputs from pinned host memory and reads its result (o and
+    # S_T) back; steps are pipelined two deep on three streams, as a serving loop would
+    # run them: the upload of step i+1 and the download of step i-1 overlap the forward of
+    # step i (PCIe is full duplex).
     host = {k: (None if v is None else v.cpu().pin_memory()) for k, v in sets[0].items()}
-    o_h = torch.empty(B, H, T, d, dtype=w.dtype).pin_memory()
-    ST_h = torch.empty(B, H, d, d, dtype=torch.float32).pin_memory()
-    dbuf = {k: (None if v is None else torch.empty_like(v, device=dev)) for k, v in host.items()}
-    o_d, ST_d = outs[0]
+    o_h = [torch.empty(B, H, T, d, dtype=w.dtype).pin_memory() for _ in range(2)]
+    ST_h = [torch.empty(B, H, d, d, dtype=torch.float32).pin_memory() for _ in range(2)]
+    dbuf = [{k: (None if v is None else torch.empty_like(v, device=dev)) for k, v in host.items()}
+            for _ in range(2)]
+    outd = [outs[0], outs[1]]
     h2d = sum(v.numel() * v.element_size() for v in host.values() if v is not None)
-    d2h = o_h.numel() * o_h.element_size() + ST_h.numel() * ST_h.element_size()
+    d2h = o_h[0].numel() * o_h[0].element_size() + ST_h[0].numel() * ST_h[0].element_size()
+    s_up, s_down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    up_done = [torch.cuda.Event() for _ in range(2)]
+    fw_done = [torch.cuda.Event() for _ in range(2)]
+    down_done = [torch.cuda.Event() for _ in range(2)]
 
-    def e2e_step():
-        for k, v in host.items():
-            if v is not None:
-                dbuf[k].copy_(v, non_blocking=True)
-        efla.efla_chunk_fwd(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["beta"], dbuf["S0"], o=o_d,
-                            S_T=ST_d, workspace=ws, stream=stream)
-        o_h.copy_(o_d, non_blocking=True)
-        ST_h.copy_(ST_d, non_blocking=True)
+    def e2e_step(i):
+        b = i % 2
+        with torch.cuda.stream(s_up):
+            if i >= 2:
+                s_up.wait_event(fw_done[b])             # the forward of step i-2 has read dbuf[b]
+            for k, v in host.items():
+                if v is not None:
+                    dbuf[b][k].copy_(v, non_blocking=True)
+            up_done[b].record(s_up)
+        stream.wait_event(up_done[b])
+        if i >= 2:
+            stream.wait_event(down_done[b])             # step i-2's results have left outd[b]
+        efla.efla_chunk_fwd(dbuf[b]["q"], dbuf[b]["k"], dbuf[b]["v"], dbuf[b]["beta"], dbuf[b]["S0"],
+                            o=outd[b][0], S_T=outd[b][1], workspace=ws, stream=stream)
+        fw_done[b].record(stream)
+        with torch.cuda.stream(s_down):
+            s_down.wait_event(fw_done[b])
+            o_h[b].copy_(outd[b][0], non_blocking=True)
+            ST_h[b].copy_(outd[b][1], non_blocking=True)
+            down_done[b].record(s_down)
 
-    e2e_steps = max(3, min(args.steps, 20))
-    for _ in range(3):
-        e2e_step()
+    e2e_steps = max(4, min(args.steps, 20))
+    for i in range(3):
+        e2e_step(i)
+    torch.cuda.synchronize(dev)
     barrier(world)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
-    e1.record(stream)
+    e0.record(s_up)
+    for i in range(e2e_steps):
+        e2e_step(i)
+    e1.record(s_down)                                   # after the last download
+    torch.cuda.synchronize(dev)
     barrier(world)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / e2e_steps
     e2e = {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-           "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
-    del sets, outs, dbuf
+           "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+           "pipeline": "2 steps in flight: upload, forward and download on three streams"}
+    del sets, outs, dbuf, o_h, ST_h
 
     # ---- decode step (N=256, H=16, d=128, fp32 state updated in place)
     dec = None

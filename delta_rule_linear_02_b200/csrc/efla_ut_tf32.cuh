@@ -44,28 +44,43 @@ __device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], 
 }
 
 // One warp: C(16 x 16) = sum over k-steps [k0, k1) of A(16 x 8) B(8 x 16).
-//   A(r, k) = a_base[k * a_ks + r * a_rs]      B(k, n) = b_base[k * LDX + n]
+//   A(r, k) = a_base[k * LDX + r]  (A_KROWS: k along rows)   or   a_base[r * LDX + k]
+//   B(k, n) = b_base[k * LDX + n]
 // Output fragment: rows g, g + 8 (g = lane / 4), columns 8 nt + 2 t, + 1 (t = lane % 4).
-__device__ __forceinline__ void warp_mm16x16(float (&c)[2][4], const float* __restrict__ a_base, int a_ks,
-                                             int a_rs, const float* __restrict__ b_base, int k0, int k1,
-                                             int lane) {
+// Within a k-step the MMA's k slots t and t + 4 take columns k = 2t and 2t + 1 of the
+// step (the same permutation for A and B leaves the sum unchanged).  With the row stride
+// of 68 floats (4 mod 32 banks) a k-along-rows load then hits bank 8t + g + const, all 32
+// lanes distinct, and a k-along-columns load reads the pair (2t, 2t + 1) as one float2,
+// two wavefronts for the warp: no bank conflicts either way.
+template <bool A_KROWS>
+__device__ __forceinline__ void warp_mm16x16(float (&c)[2][4], const float* __restrict__ a_base,
+                                             const float* __restrict__ b_base, int k0, int k1, int lane) {
     const int g = lane >> 2, t = lane & 3;
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
         for (int e = 0; e < 4; ++e) c[nt][e] = 0.f;
     for (int ks = k0; ks < k1; ++ks) {
-        const int k = 8 * ks + t;
+        const int k = 8 * ks + 2 * t;
         uint32_t a[4];
-        a[0] = to_tf32(a_base[k * a_ks + g * a_rs]);
-        a[1] = to_tf32(a_base[k * a_ks + (g + 8) * a_rs]);
-        a[2] = to_tf32(a_base[(k + 4) * a_ks + g * a_rs]);
-        a[3] = to_tf32(a_base[(k + 4) * a_ks + (g + 8) * a_rs]);
+        if (A_KROWS) {
+            a[0] = to_tf32(a_base[k * LDX + g]);
+            a[1] = to_tf32(a_base[k * LDX + g + 8]);
+            a[2] = to_tf32(a_base[(k + 1) * LDX + g]);
+            a[3] = to_tf32(a_base[(k + 1) * LDX + g + 8]);
+        } else {
+            const float2 lo = *reinterpret_cast<const float2*>(a_base + g * LDX + k);
+            const float2 hi = *reinterpret_cast<const float2*>(a_base + (g + 8) * LDX + k);
+            a[0] = to_tf32(lo.x);
+            a[1] = to_tf32(hi.x);
+            a[2] = to_tf32(lo.y);
+            a[3] = to_tf32(hi.y);
+        }
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) {
             uint32_t b[2];
             b[0] = to_tf32(b_base[k * LDX + 8 * nt + g]);
-            b[1] = to_tf32(b_base[(k + 4) * LDX + 8 * nt + g]);
+            b[1] = to_tf32(b_base[(k + 1) * LDX + 8 * nt + g]);
             mma_tf32(c[nt], a, b);
         }
     }
@@ -111,25 +126,25 @@ __device__ __forceinline__ void ut_solve(float* __restrict__ At, float* __restri
     float acc[2][4];
     if (pw < 2) {      // (2a) Y = A21 X11 for super-block pw (16 x 16 x 16; X11 lower: k >= n)
         const int r0 = 32 * pw + 16, c0 = 32 * pw;
-        warp_mm16x16(acc, At + c0 * LDX + r0, LDX, 1, X + c0 * LDX + c0, 0, 2, lane);
+        warp_mm16x16<true>(acc, At + c0 * LDX + r0, X + c0 * LDX + c0, 0, 2, lane);
         warp_st16x16(At + r0 * LDX + c0, acc, 1.f, lane);
     }
     bar_sync(NB, NT);
     if (pw < 2) {      // (2b) X21 = -X22 Y
         const int r0 = 32 * pw + 16, c0 = 32 * pw;
-        warp_mm16x16(acc, X + r0 * LDX + r0, 1, LDX, At + r0 * LDX + c0, 0, 2, lane);
+        warp_mm16x16<false>(acc, X + r0 * LDX + r0, At + r0 * LDX + c0, 0, 2, lane);
         warp_st16x16(X + r0 * LDX + c0, acc, -1.f, lane);
     }
     bar_sync(NB, NT);
     if (pw < 4) {      // (3a) Y = A21 X11 (32 x 32 x 32); tile (wr, wc), X11[k][n] = 0 for k < 16 wc
         const int wr = pw >> 1, wc = pw & 1;
-        warp_mm16x16(acc, At + 32 + 16 * wr, LDX, 1, X + 16 * wc, 2 * wc, 4, lane);
+        warp_mm16x16<true>(acc, At + 32 + 16 * wr, X + 16 * wc, 2 * wc, 4, lane);
         warp_st16x16(At + (32 + 16 * wr) * LDX + 16 * wc, acc, 1.f, lane);
     }
     bar_sync(NB, NT);
     if (pw < 4) {      // (3b) X21 = -X22 Y; X22[m][k] = 0 for k > 16 wr + 15
         const int wr = pw >> 1, wc = pw & 1;
-        warp_mm16x16(acc, X + (32 + 16 * wr) * LDX + 32, 1, LDX, At + 32 * LDX + 16 * wc, 0, 2 * wr + 2, lane);
+        warp_mm16x16<false>(acc, X + (32 + 16 * wr) * LDX + 32, At + 32 * LDX + 16 * wc, 0, 2 * wr + 2, lane);
         warp_st16x16(X + (32 + 16 * wr) * LDX + 16 * wc, acc, -1.f, lane);
     }
     bar_sync(NB, NT);
