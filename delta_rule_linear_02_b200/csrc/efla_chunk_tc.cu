@@ -44,13 +44,13 @@
 //   warps 6-13   chain, two per lane quarter (32-column halves).  Quarters 0-1 form Delta
 //                (U taken from its accumulator as soon as it lands); all eight rebuild the
 //                bf16 S and S_T.
+// A hand-off between roles is an mbarrier that counts warps: each warp of a role waits on
+// its own (every lane polls, the warp votes) and arrives once after its own fences, so no
+// hand-off passes a named barrier.
 // Every wait is bounded (2 s); a wait that runs out sets a CTA-wide abort flag, every
 // role winds down, and the caller's workspace records the timeout.
-// Built with EFLA_CHUNK_TRACE=2 (never in the library), `dbg` receives CTA 0's chunk-0
-// intermediates for diagnosis:
-// W [8256,16448) U [16448,20544) WS [20544,24640) S after the chunk [24640,32832); and
-// with EFLA_CHUNK_TRACE >= 1, per chunk c < 64 the cycle at which each role passed its
-// milestones, at
+// Built with EFLA_CHUNK_TRACE=1 (never in the library), `dbg` receives, per chunk c < 64,
+// the cycle at which each role of CTA 0 passed its milestones, at
 // [40000 + 16 c + k): k = 0 QK^T, 1 [W|U], 2 [W;Q]S, 3 K^T Delta issued; 4 P ready;
 // 5 Q ready; 6 W ready; 7 U taken; 8 Delta ready; 9 new S ready; 10 O stored; 11 TMA.
 #include <cudaTypedefs.h>
@@ -65,11 +65,9 @@ namespace efla {
 #ifndef EFLA_CHUNK_TRACE
 #define EFLA_CHUNK_TRACE 0
 #endif
-// diagnosis stores compiled in only for tracing builds (1: milestone cycles, 2: also
-// chunk-0 intermediates): they cost instruction-cache space in the role loops even when
-// never taken
+// diagnosis stores compiled in only for tracing builds (milestone cycles): they cost
+// instruction-cache space in the role loops even when never taken
 constexpr bool kTrace = EFLA_CHUNK_TRACE >= 1;
-constexpr bool kTraceDump = EFLA_CHUNK_TRACE >= 2;
 
 namespace {
 using namespace sm100;
@@ -106,7 +104,7 @@ enum : int {
     B_GP_FREE,          // P~ read
     B_P_READY,          // P in the A operand
     B_WU_FULL,          // [W | U] landed
-    B_WU_FREE,          // count 2: W and U both taken
+    B_WU_FREE,          // W and U both taken
     B_W_READY,          // W in the A operand
     B_Q_READY,          // Q in the A operand
     B_XS_FULL,          // [W;Q] S landed
@@ -117,6 +115,17 @@ enum : int {
     B_X_FREE,           // O stored
     B_DRAIN,
 };
+
+// arrivals per phase: one per arriving warp (W: warps 4-5; Q/P: warps 2-3; Delta: the four
+// chain warps of quarters 0-1; S: all eight chain warps); TMA and MMA commits arrive once
+__host__ __device__ constexpr uint32_t bar_count(int i) {
+    return i == B_WU_FREE                                                   ? 6u
+         : i == B_W_READY || i == B_Q_READY || i == B_GP_FREE || i == B_P_READY || i == B_X_FREE ||
+                   i == B_Q_FREE || i == B_Q_FREE + 1                       ? 2u
+         : i == B_D_READY                                                   ? 4u
+         : i == B_SB_READY                                                  ? 8u
+                                                                            : 1u;
+}
 
 // ---- TMEM columns
 constexpr uint32_t TM_S = 0;          // fp32 S (d_k x 64)
@@ -132,9 +141,6 @@ constexpr uint32_t ID_WU = idesc_bf16(128, 192, false, true);     // [T;*] [K | 
 constexpr uint32_t ID_GP = idesc_bf16(128, 64, false, false);     // [W;Q] K^T
 constexpr uint32_t ID_S = idesc_bf16(128, 64, true, true);        // K^T Delta
 
-// ---- named barriers
-constexpr int NB_CW = 1, NB_CQ = 2, NB_DELTA = 3, NB_CHAIN = 4;
-constexpr int kPair = 64, kHalfChain = 128, kChainThreads = 256;
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
     __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
@@ -175,6 +181,15 @@ struct Ctl {
             }
         }
         return true;
+    }
+    // whole-warp forms: every lane polls, the warp votes (warp-uniform control flow)
+    __device__ __forceinline__ bool wwait(int i, uint32_t parity) const {
+        return __all_sync(0xffffffffu, wait(i, parity));
+    }
+    // one arrival per warp once the whole warp got here (after its own fences)
+    __device__ __forceinline__ void warp_arrive(int i, int lane) const {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar + i);
     }
 };
 
@@ -227,7 +242,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     } while (0)
 
     if (tid == 0) {
-        for (int i = 0; i < (int)NBAR; ++i) mbar_init(ctl.bar + i, i == B_WU_FREE ? 2 : 1);
+        for (int i = 0; i < (int)NBAR; ++i) mbar_init(ctl.bar + i, bar_count(i));
         *ctl.abort = 0;
         fence_mbar_init();
         tma_prefetch_desc(&tm_q);
@@ -355,11 +370,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         __syncwarp();
     } else if (warp == 4 || warp == 5) {
         // ================================================================ W -> A operand (quarters 0-1)
-        const int r = 32 * q + lane;                  // W row in this lane
         bool ok = true;
         for (int c = 0; c < nchunks && ok; ++c) {
             // [W | U](c) landed, and [W;Q] S(c-1) no longer reads the A operand
-            ok = bar_and(NB_CW, kPair, ctl.wait(B_WU_FULL, c & 1) && (c == 0 || ctl.wait(B_XS_FULL, (c - 1) & 1)));
+            ok = ctl.wwait(B_WU_FULL, c & 1) && (c == 0 || ctl.wwait(B_XS_FULL, (c - 1) & 1));
             if (!ok) break;
             tc_fence_after();
 #pragma unroll
@@ -370,17 +384,12 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
                 for (int j = 0; j < 32; ++j) pk[j] = pack_bf16x2(w[2 * j], w[2 * j + 1]);
                 tmem_st32(tmem + lane_off + TM_AWQ + 32 * h, pk);
-                if (kTraceDump && dbg && blockIdx.x == 0 && c == 0)
-                    for (int j = 0; j < 64; ++j) dbg[8256 + r * 128 + 64 * h + j] = w[j];
             }
             tmem_wait_st();
             tc_fence_before();
-            bar_sync(NB_CW, kPair);
-            if (warp == 4 && lane == 0) {
-                mbar_arrive(ctl.b(B_W_READY));
-                mbar_arrive(ctl.b(B_WU_FREE));
-                EFLA_STAMP(c, 6);
-            }
+            ctl.warp_arrive(B_WU_FREE, lane);
+            ctl.warp_arrive(B_W_READY, lane);
+            if (warp == 4 && lane == 0) EFLA_STAMP(c, 6);
         }
     } else if (warp < 4) {
         // ================================================================ Q and P -> A operands (quarters 2-3)
@@ -397,29 +406,22 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 }
                 tmem_st32(tmem + lane_off + TM_AWQ + 32 * h, pk);
             }
+            ctl.warp_arrive(B_Q_FREE + c % kQStages, lane);
             tmem_wait_st();
             tc_fence_before();
-            bar_sync(NB_CQ, kPair);
-            if (warp == 2 && lane == 0) {
-                mbar_arrive(ctl.b(B_Q_READY));
-                mbar_arrive(ctl.b(B_Q_FREE + c % kQStages));
-                EFLA_STAMP(c, 5);
-            }
+            ctl.warp_arrive(B_Q_READY, lane);
+            if (warp == 2 && lane == 0) EFLA_STAMP(c, 5);
         };
         // O(c) = X rows 64-127 once P Delta(c) has landed: taken into registers, X released
         // at once for [W;Q] S(c+1), then stored to global as bf16 (rows past T skipped)
         auto store_o = [&](int c) {
-            bool fine = bar_and(NB_CQ, kPair, ctl.wait(B_O_FULL, c & 1));
-            if (!fine) return false;
+            if (!ctl.wwait(B_O_FULL, c & 1)) return false;
             tc_fence_after();
             float t[64];
             tmem_ld64_wait(tmem + lane_off + TM_X, t);
             tc_fence_before();
-            bar_sync(NB_CQ, kPair);
-            if (warp == 2 && lane == 0) {
-                mbar_arrive(ctl.b(B_X_FREE));
-                EFLA_STAMP(c, 10);
-            }
+            ctl.warp_arrive(B_X_FREE, lane);
+            if (warp == 2 && lane == 0) EFLA_STAMP(c, 10);
             const int t0 = c * 64;
             if (r < min(64, T - t0)) {
                 uint4* dst = reinterpret_cast<uint4*>(o + (tok0 + t0 + r) * kD + col0);
@@ -435,13 +437,12 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
             return true;
         };
-        bool ok = bar_and(NB_CQ, kPair, ctl.wait(B_Q_FULL, 0));
+        bool ok = ctl.wwait(B_Q_FULL, 0);
         if (ok) copy_q(0);
         for (int c = 0; c < nchunks && ok; ++c) {
             if (c > 0 && !(ok = store_o(c - 1))) break;
             // P = Q K^T masked causally (diagonal kept) -> A rows 64-127 (P Delta(c-1) is done)
-            ok = bar_and(NB_CQ, kPair, ctl.wait(B_GP_FULL, c & 1));
-            if (!ok) break;
+            if (!(ok = ctl.wwait(B_GP_FULL, c & 1))) break;
             tc_fence_after();
             {
                 float t[64];
@@ -454,17 +455,12 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
             tmem_wait_st();
             tc_fence_before();
-            bar_sync(NB_CQ, kPair);
-            if (warp == 2 && lane == 0) {
-                mbar_arrive(ctl.b(B_GP_FREE));
-                mbar_arrive(ctl.b(B_P_READY));
-                EFLA_STAMP(c, 4);
-            }
+            ctl.warp_arrive(B_GP_FREE, lane);
+            ctl.warp_arrive(B_P_READY, lane);
+            if (warp == 2 && lane == 0) EFLA_STAMP(c, 4);
             // Q(c+1) -> A rows 64-127, once [W;Q] S(c) no longer reads them
             if (c + 1 < nchunks) {
-                ok = bar_and(NB_CQ, kPair,
-                             ctl.wait(B_Q_FULL + (c + 1) % kQStages, ((c + 1) / kQStages) & 1) &&
-                             ctl.wait(B_XS_FULL, c & 1));
+                ok = ctl.wwait(B_Q_FULL + (c + 1) % kQStages, ((c + 1) / kQStages) & 1) && ctl.wwait(B_XS_FULL, c & 1);
                 if (!ok) break;
                 copy_q(c + 1);
             }
@@ -472,9 +468,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (ok) store_o(nchunks - 1);
     } else {
         // ================================================================ chain (two warps per lane quarter)
-        // Quarters 0-1 (X rows 0-63, W S) form Delta; all eight rebuild the bf16 S.  A group
-        // that gives up still reaches the next S-epilogue barrier with ok = false, so both
-        // stop together.
+        // Quarters 0-1 (X rows 0-63, W S) form Delta; all eight rebuild the bf16 S.  Each warp
+        // waits and arrives on its own (the barriers count warps): no group barrier in a
+        // hand-off.
         const int ch = (warp - 6) >> 2;               // column half: 32 of this CTA's 64 columns
         const int cc = 32 * ch;
         const int ct = 32 * q + lane;                 // d_k row of S, and row of X / [W | U]
@@ -496,59 +492,41 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             tmem_wait_st();
             fence_proxy_async_smem();
             tc_fence_before();
-            bar_sync(NB_CHAIN, kChainThreads);
-            if (warp == 6 && lane == 0) mbar_arrive(ctl.b(B_SB_READY));
+            ctl.warp_arrive(B_SB_READY, lane);
         }
         bool ok = true;
-        for (int c = 0; c < nchunks; ++c) {
-            if (delta_group && ok) {
+        for (int c = 0; c < nchunks && ok; ++c) {
+            if (delta_group) {
                 // take U(c) from its accumulator as soon as it lands ([W|U](c+1) reuses it)
                 float u[32];
-                ok = bar_and(NB_DELTA, kHalfChain, ctl.wait(B_WU_FULL, c & 1));
-                if (ok) {
-                    tc_fence_after();
-                    tmem_ld32_wait(tmem + lane_off + TM_WU + 128 + cc, u);
-                    tc_fence_before();
-                    bar_sync(NB_DELTA, kHalfChain);
-                    if (warp == 8 && lane == 0) {
-                        mbar_arrive(ctl.b(B_WU_FREE));
-                        EFLA_STAMP(c, 7);
-                    }
-                    if (kTraceDump && dbg && blockIdx.x == 0 && c == 0)
-                        for (int j = 0; j < 32; ++j) dbg[16448 + ct * 64 + cc + j] = u[j];
-                    // Delta = U - W S (X rows 0-63)
-                    ok = bar_and(NB_DELTA, kHalfChain, ctl.wait(B_XS_FULL, c & 1));
-                }
-                if (ok) {
-                    tc_fence_after();
-                    float t[32];
-                    tmem_ld32_wait(tmem + lane_off + TM_X + cc, t);
-                    if (kTraceDump && dbg && blockIdx.x == 0 && c == 0)
-                        for (int j = 0; j < 32; ++j) dbg[20544 + ct * 64 + cc + j] = t[j];
+                if (!(ok = ctl.wwait(B_WU_FULL, c & 1))) break;
+                tc_fence_after();
+                tmem_ld32_wait(tmem + lane_off + TM_WU + 128 + cc, u);
+                tc_fence_before();
+                ctl.warp_arrive(B_WU_FREE, lane);
+                if (warp == 8 && lane == 0) EFLA_STAMP(c, 7);
+                // Delta = U - W S (X rows 0-63)
+                if (!(ok = ctl.wwait(B_XS_FULL, c & 1))) break;
+                tc_fence_after();
+                float t[32];
+                tmem_ld32_wait(tmem + lane_off + TM_X + cc, t);
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) t[j] = u[j] - t[j];
+                for (int j = 0; j < 32; ++j) t[j] = u[j] - t[j];
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) st_chunk(sm + OFF_DL + sw128_off(ct, 4 * ch + j), t + 8 * j);
-                    fence_proxy_async_smem();
-                    tc_fence_before();
-                    bar_sync(NB_DELTA, kHalfChain);
-                    if (warp == 8 && lane == 0) {
-                        mbar_arrive(ctl.b(B_D_READY));
-                        EFLA_STAMP(c, 8);
-                    }
-                }
+                for (int j = 0; j < 4; ++j) st_chunk(sm + OFF_DL + sw128_off(ct, 4 * ch + j), t + 8 * j);
+                fence_proxy_async_smem();
+                tc_fence_before();
+                ctl.warp_arrive(B_D_READY, lane);
+                if (warp == 8 && lane == 0) EFLA_STAMP(c, 8);
             }
             // the new state: bf16 operand for the next chunk (and S_T after the last)
-            ok = bar_and(NB_CHAIN, kChainThreads, ok && ctl.wait(B_S_FULL, c & 1));
-            if (!ok) break;
+            if (!(ok = ctl.wwait(B_S_FULL, c & 1))) break;
             tc_fence_after();
             {
                 float t[32];
                 tmem_ld32_wait(tmem + lane_off + TM_S + cc, t);
 #pragma unroll
                 for (int j = 0; j < 4; ++j) st_chunk(sm + OFF_SB + sw128_off(ct, 4 * ch + j), t + 8 * j);
-                if (kTraceDump && dbg && blockIdx.x == 0 && c == 0)
-                    for (int j = 0; j < 32; ++j) dbg[24640 + ct * 64 + cc + j] = t[j];
                 if (c == nchunks - 1 && S_T) {
                     float* dst = S_T + ((size_t)bh * kD + ct) * kD + col0 + cc;
 #pragma unroll
@@ -558,11 +536,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
             fence_proxy_async_smem();
             tc_fence_before();
-            bar_sync(NB_CHAIN, kChainThreads);
-            if (warp == 6 && lane == 0) {
-                mbar_arrive(ctl.b(B_SB_READY));
-                EFLA_STAMP(c, 9);
-            }
+            ctl.warp_arrive(B_SB_READY, lane);
+            if (warp == 6 && lane == 0) EFLA_STAMP(c, 9);
         }
     }
 
