@@ -437,20 +437,38 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
             return true;
         };
+        if (q == 2) {       // bf16 P columns 32-63 of chunk rows 0-31: zero for good
+            const float z[16] = {};
+            tmem_st16(tmem + lane_off + TM_AP + 16, z);
+            tmem_wait_st();
+            tc_fence_before();
+        }
         bool ok = ctl.wwait(B_Q_FULL, 0);
         if (ok) copy_q(0);
         for (int c = 0; c < nchunks && ok; ++c) {
             if (c > 0 && !(ok = store_o(c - 1))) break;
-            // P = Q K^T masked causally (diagonal kept) -> A rows 64-127 (P Delta(c-1) is done)
+            // P = Q K^T masked causally (diagonal kept) -> A rows 64-127 (P Delta(c-1) is done).
+            // Chunk rows 0-31 have no entry past column 31 (those bf16 columns were zeroed
+            // once, above); rows 32-63 keep columns 0-31 whole.  Each warp masks 32 columns.
             if (!(ok = ctl.wwait(B_GP_FULL, c & 1))) break;
             tc_fence_after();
-            {
+            if (q == 2) {
+                float t[32], pk[16];
+                tmem_ld32_wait(tmem + lane_off + TM_GP, t);
+#pragma unroll
+                for (int j = 0; j < 16; ++j)
+                    pk[j] = __uint_as_float(
+                        pack_bf16x2(2 * j <= lane ? t[2 * j] : 0.f, 2 * j + 1 <= lane ? t[2 * j + 1] : 0.f));
+                tmem_st16(tmem + lane_off + TM_AP, pk);
+            } else {
                 float t[64];
                 uint32_t pk[32];
                 tmem_ld64_wait(tmem + lane_off + TM_GP, t);
 #pragma unroll
-                for (int j = 0; j < 32; ++j)
-                    pk[j] = pack_bf16x2(2 * j <= r ? t[2 * j] : 0.f, 2 * j + 1 <= r ? t[2 * j + 1] : 0.f);
+                for (int j = 0; j < 16; ++j) {
+                    pk[j] = pack_bf16x2(t[2 * j], t[2 * j + 1]);
+                    pk[16 + j] = pack_bf16x2(2 * j <= lane ? t[32 + 2 * j] : 0.f, 2 * j + 1 <= lane ? t[33 + 2 * j] : 0.f);
+                }
                 tmem_st32(tmem + lane_off + TM_AP, pk);
             }
             tmem_wait_st();
