@@ -53,6 +53,10 @@ def load(path: Optional[str] = None):
     lib.efla_oracle_fwd.restype = I
     lib.efla_oracle_step.argtypes = [dp, dp, dp, dp, dp, dp, L, L, L, L, I, I]
     lib.efla_oracle_step.restype = I
+    lib.efla_oracle_dalpha_dlambda.argtypes = [ctypes.c_double, ctypes.c_double]
+    lib.efla_oracle_dalpha_dlambda.restype = ctypes.c_double
+    lib.efla_oracle_bwd.argtypes = [dp] * 12 + [L, L, L, L, L, I, I]
+    lib.efla_oracle_bwd.restype = I
     if path is None:
         _lib = lib
     return lib
@@ -136,3 +140,30 @@ def step(q, k, v, beta, S, mode: int = EXACT, threads: Optional[int] = None, lib
     if rc != 0:
         raise MemoryError("oracle could not allocate its per-stream state")
     return o, S
+
+
+def dalpha_dlambda(beta: float, lam: float, lib=None) -> float:
+    return (lib or load()).efla_oracle_dalpha_dlambda(float(beta), float(lam))
+
+
+def bwd(q, k, v, beta, dO, S0=None, dS_T=None, mode: int = EXACT, threads: Optional[int] = None,
+        lib=None):
+    """Reverse-mode derivative of fwd for the loss sum(dO * o) + sum(dS_T * S_T).
+
+    Returns (dq, dk [B,H,T,dk], dv [B,H,T,dv], dbeta [B,H,T], dS0 [B,H,dk,dv]) as float64.
+    Keeps every state of a running stream: (T + 1) dk dv doubles per thread.
+    """
+    q, k, v, beta, dO, S0, dS_T = (_f64(x) for x in (q, k, v, beta, dO, S0, dS_T))
+    B, H, T, dk = k.shape
+    dv = v.shape[-1]
+    assert q.shape == k.shape and v.shape[:3] == (B, H, T) and dO.shape == v.shape
+    dq, dk_ = np.empty_like(q), np.empty_like(k)
+    dv_, dbeta = np.empty_like(v), np.empty((B, H, T), dtype=np.float64)
+    dS0 = np.empty((B, H, dk, dv), dtype=np.float64)
+    rc = (lib or load()).efla_oracle_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(S0), _ptr(dO),
+                                         _ptr(dS_T), _ptr(dq), _ptr(dk_), _ptr(dv_), _ptr(dbeta),
+                                         _ptr(dS0), B, H, T, dk, dv, mode,
+                                         threads or default_threads())
+    if rc != 0:
+        raise MemoryError("oracle could not allocate the states of a stream")
+    return dq, dk_, dv_, dbeta, dS0

@@ -30,6 +30,19 @@
  *
  * Mode EFLA_ORACLE_EULER (alpha_t = beta_t) is the plain delta rule of Section 2; the tests
  * use it for the small-step limit of Section 3.4.
+ *
+ * efla_oracle_bwd is the reverse-mode derivative of the same recurrence, the pass training
+ * needs (Section 4.6 reports training throughput on par with DeltaNet; the pages print no
+ * backward formulas, so this is the chain rule written out one step at a time in reverse
+ * order, from stored states).  With G = dL/dS_t and r_t = S_{t-1}^T k_t - v_t:
+ *   G     += q_t dO_t^T              dq_t = S_t dO_t
+ *   g      = G^T k_t                 dalpha_t = -g . r_t
+ *   dv_t   = alpha_t g               dk_t = -alpha_t (G r_t + S_{t-1} g) + dalpha_t dalpha/dlambda 2 k_t
+ *   dbeta_t = dalpha_t dalpha/dbeta  G <- G - alpha_t k_t g^T   (= dL/dS_{t-1})
+ * and dS0 = G at the end.  The gate derivatives, from alpha = (1 - e^{-beta lambda})/lambda:
+ *   dalpha/dbeta = e^{-beta lambda},   dalpha/dlambda = (beta e^{-beta lambda} - alpha)/lambda,
+ * the latter by its Taylor series in x = beta lambda when x is small (its limit at lambda = 0
+ * is -beta^2/2).  Euler mode: dalpha/dbeta = 1, dalpha/dlambda = 0.
  */
 #include <math.h>
 #include <stddef.h>
@@ -142,4 +155,140 @@ int efla_oracle_step(const double *q, const double *k, const double *v, const do
                      int nthreads)
 {
     return efla_oracle_fwd(q, k, v, beta, S, o, S, N, H, 1, dk, dv, mode, nthreads);
+}
+
+/* d alpha / d lambda of the exact gate.  For x = beta*lambda < 1e-3 the difference
+ * beta e^{-x} - alpha cancels, so the series beta^2 sum_{n>=1} (-1)^n n x^{n-1}/(n+1)! is used
+ * (five terms; the next is below 1e-18 relative). */
+double efla_oracle_dalpha_dlambda(double beta, double lambda)
+{
+    const double x = beta * lambda;
+    if (fabs(x) < 1e-3)
+        return beta * beta * (-0.5 + x / 3.0 - x * x / 8.0 + x * x * x / 30.0 - x * x * x * x / 144.0);
+    const double a = -expm1(-x) / lambda;
+    return (beta * exp(-x) - a) / lambda;
+}
+
+/* Reverse sweep of one stream.  Ss holds S_0 .. S_T ((T + 1) dk dv doubles); G, r, g are
+ * scratch.  Gradients are written (not accumulated). */
+static void bwd_stream(const double *q, const double *k, const double *v, const double *beta,
+                       const double *dO, const double *dST, double *Ss, double *G, double *r,
+                       double *g, double *dq, double *dk, double *dv, double *dbeta, double *dS0,
+                       long T, long dk_, long dv_, int mode)
+{
+    const long D = dk_ * dv_;
+    /* forward, keeping every state */
+    for (long t = 0; t < T; ++t) {
+        const double *kx = k + t * dk_, *vx = v + t * dv_;
+        const double *Sp = Ss + t * D;
+        double *Sn = Ss + (t + 1) * D;
+        double l2 = 0.0;
+        for (long i = 0; i < dk_; ++i)
+            l2 += kx[i] * kx[i];
+        const double at = (mode == EFLA_ORACLE_EULER) ? beta[t] : efla_oracle_alpha(beta[t], l2);
+        for (long j = 0; j < dv_; ++j)
+            r[j] = -vx[j];
+        for (long i = 0; i < dk_; ++i)
+            for (long j = 0; j < dv_; ++j)
+                r[j] += kx[i] * Sp[i * dv_ + j];
+        for (long i = 0; i < dk_; ++i)
+            for (long j = 0; j < dv_; ++j)
+                Sn[i * dv_ + j] = Sp[i * dv_ + j] - at * kx[i] * r[j];
+    }
+    /* reverse */
+    for (long x = 0; x < D; ++x)
+        G[x] = dST ? dST[x] : 0.0;
+    for (long t = T - 1; t >= 0; --t) {
+        const double *qx = q + t * dk_, *kx = k + t * dk_, *vx = v + t * dv_, *dox = dO + t * dv_;
+        const double *Sp = Ss + t * D, *Sc = Ss + (t + 1) * D;
+        double l2 = 0.0;
+        for (long i = 0; i < dk_; ++i)
+            l2 += kx[i] * kx[i];
+        const double at = (mode == EFLA_ORACLE_EULER) ? beta[t] : efla_oracle_alpha(beta[t], l2);
+        /* o_t = S_t^T q_t */
+        for (long i = 0; i < dk_; ++i) {
+            double acc = 0.0;
+            for (long j = 0; j < dv_; ++j) {
+                G[i * dv_ + j] += qx[i] * dox[j];
+                acc += Sc[i * dv_ + j] * dox[j];
+            }
+            dq[t * dk_ + i] = acc;
+        }
+        /* S_t = S_{t-1} - alpha k r^T with r = S_{t-1}^T k - v */
+        for (long j = 0; j < dv_; ++j) {
+            double rj = -vx[j], gj = 0.0;
+            for (long i = 0; i < dk_; ++i) {
+                rj += kx[i] * Sp[i * dv_ + j];
+                gj += G[i * dv_ + j] * kx[i];
+            }
+            r[j] = rj;
+            g[j] = gj;
+        }
+        double da = 0.0;
+        for (long j = 0; j < dv_; ++j) {
+            da -= g[j] * r[j];
+            dv[t * dv_ + j] = at * g[j];
+        }
+        double dadb, dadl;
+        if (mode == EFLA_ORACLE_EULER) {
+            dadb = 1.0;
+            dadl = 0.0;
+        } else if (l2 == 0.0) {
+            dadb = 1.0;
+            dadl = -0.5 * beta[t] * beta[t];
+        } else {
+            dadb = exp(-beta[t] * l2);
+            dadl = efla_oracle_dalpha_dlambda(beta[t], l2);
+        }
+        for (long i = 0; i < dk_; ++i) {
+            double gr = 0.0, sg = 0.0;
+            for (long j = 0; j < dv_; ++j) {
+                gr += G[i * dv_ + j] * r[j];
+                sg += Sp[i * dv_ + j] * g[j];
+            }
+            dk[t * dk_ + i] = -at * (gr + sg) + da * dadl * 2.0 * kx[i];
+        }
+        dbeta[t] = da * dadb;
+        for (long i = 0; i < dk_; ++i)
+            for (long j = 0; j < dv_; ++j)
+                G[i * dv_ + j] -= at * kx[i] * g[j];
+    }
+    if (dS0)
+        memcpy(dS0, G, (size_t)D * sizeof(double));
+}
+
+/*
+ * Backward over [B, H, T] streams: given dO [B, H, T, dv] and dS_T [B, H, dk, dv] (or NULL,
+ * zero), writes dq, dk [B, H, T, dk], dv [B, H, T, dv], dbeta [B, H, T] and dS0 [B, H, dk, dv]
+ * (dS0 may be NULL).  S0 as in efla_oracle_fwd.  Keeps all T + 1 states of a stream:
+ * (T + 1) dk dv doubles per running stream.  Returns 0, or -1 on allocation failure.
+ */
+int efla_oracle_bwd(const double *q, const double *k, const double *v, const double *beta,
+                    const double *S0, const double *dO, const double *dST, double *dq, double *dk,
+                    double *dv, double *dbeta, double *dS0, long B, long H, long T, long dk_,
+                    long dv_, int mode, int nthreads)
+{
+    const long BH = B * H, D = dk_ * dv_;
+    int failed = 0;
+    if (nthreads < 1)
+        nthreads = 1;
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads) reduction(| : failed)
+    for (long bh = 0; bh < BH; ++bh) {
+        double *Ss = (double *)malloc((size_t)((T + 2) * D + 2 * dv_) * sizeof(double));
+        if (!Ss) {
+            failed |= 1;
+            continue;
+        }
+        double *G = Ss + (T + 1) * D, *r = G + D, *g = r + dv_;
+        if (S0 != NULL)
+            memcpy(Ss, S0 + bh * D, (size_t)D * sizeof(double));
+        else
+            memset(Ss, 0, (size_t)D * sizeof(double));
+        bwd_stream(q + bh * T * dk_, k + bh * T * dk_, v + bh * T * dv_, beta + bh * T,
+                   dO + bh * T * dv_, dST ? dST + bh * D : NULL, Ss, G, r, g, dq + bh * T * dk_,
+                   dk + bh * T * dk_, dv + bh * T * dv_, dbeta + bh * T, dS0 ? dS0 + bh * D : NULL,
+                   T, dk_, dv_, mode);
+        free(Ss);
+    }
+    return failed ? -1 : 0;
 }
