@@ -7,8 +7,9 @@ d_k=d_v=128, chunk 64, bf16 in / fp32 state): the gate, the intra-chunk UT trans
 the inter-chunk state propagation, fused.  Multi-GPU (torchrun, one rank per GPU) is data
 parallel over independent (b, h) streams: every rank runs its own batch with no data-path
 collective (weak scaling); the timing is the max over ranks.  The single-token decode step
-(N=256, H=16, d=128, fp32 state, in place) is measured in the same run and reported under
-"decode".  Rank 0 prints one JSON line.
+(N=256, H=16, d=128, fp32 state, in place) and the backward pass on the forward's workload
+are measured in the same run and reported under "decode" and "backward".  Rank 0 prints
+one JSON line.
 """
 from __future__ import annotations
 
@@ -66,23 +67,52 @@ def decode_alg(w):
     return NH * (2 * d * d * 4 + (3 * d + 1 + d) * 4), NH * 6 * d * d
 
 
-def kernel_source_hash():
+# The sources each entry point's kernels are compiled from (the C-ABI glue and the other
+# entry points' files excluded): a traffic figure stays valid while these are unchanged.
+KERNEL_SOURCES = {
+    "efla_chunk_fwd": ["efla_chunk_tc.cu", "efla_ut.cu", "efla_ut_tf32.cuh", "efla_ut_solve.cuh",
+                       "efla_chunk_simt.cu", "efla_common.cuh", "efla_tma.cuh", "sm100.cuh"],
+    "efla_recurrent_step": ["efla_decode.cu", "efla_common.cuh"],
+    "efla_backward": ["efla_bwd.cu", "efla_common.cuh"],
+}
+
+
+def backward_alg(w):
+    """One backward call.  Bytes: read q, k, v, dO, beta (w.dtype) and write dq, dk, dv, dbeta
+    (fp32), plus dS0 (fp32).  Flops of the recurrent reverse pass as built (fp32 CUDA cores),
+    18 d^2 per token and head: the forward sweep's S^T k and rank-1 write, then G += q dO^T,
+    S dO, G^T k, the rebuilt S_{t-1}, G r, S_{t-1} g and G -= alpha k g^T (2 d^2 each)."""
+    es = 2 if w.dtype == torch.bfloat16 else 4
+    BH, T, d = w.B * w.H, w.T, w.dk
+    nbytes = BH * T * (4 * d * es + es + 3 * d * 4 + 4) + BH * d * d * 4
+    return nbytes, BH * T * 18 * d * d
+
+
+def fp32_alu_peak_tflops():
+    """FMA peak of the CUDA cores: 148 SMs x 128 fp32 lanes x 2 flops x 1.965 GHz."""
+    return 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def kernel_source_hash(entry=None):
+    """sha256 prefix over the kernel sources of one entry point (all of csrc/ for None)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "delta_rule_linear_02_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    names = sorted(os.listdir(csrc)) if entry is None else sorted(KERNEL_SOURCES[entry])
+    for name in names:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
 
 
 def ncu_traffic(kernel: str):
-    """dram bytes per launch recorded in profiles/traffic.md for the current kernel sources."""
+    """dram bytes per launch recorded in profiles/traffic.md for the entry point's current
+    kernel sources."""
     path = os.path.join(ROOT, "profiles", "traffic.md")
     try:
         lines = open(path).read().splitlines()
     except OSError:
         return None
-    src = kernel_source_hash()
+    src = kernel_source_hash(kernel)
     for ln in lines:
         if ln.startswith("traffic|"):
             _, name, nbytes, sha = ln.split("|")[:4]
@@ -251,6 +281,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="efla", choices=["efla", "reference"])
     ap.add_argument("--decode-steps", type=int, default=1000)
+    ap.add_argument("--bwd-steps", type=int, default=5,
+                    help="backward calls timed on the forward's workload (0: skip)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--other-steps", type=int, default=10,
                     help="forwards timed on each of the long-context and stiff workloads (0: skip)")
@@ -402,6 +434,43 @@ def main():
                "gpu_launches": nd}
         del S, st
 
+    # ---- backward (training) pass on the forward's workload: dq, dk, dv, dbeta, dS0 from dO
+    bwd = None
+    if args.bwd_steps > 0:
+        wb = w.replace(seed=w.seed + 500)
+        xb = {k_: v_.to(dev) for k_, v_ in workloads.make_chunk_inputs(wb).items() if v_ is not None}
+        cb = workloads.make_cotangents(wb, with_state_grad=False)
+        dOb = cb["dO"].to(dev)
+        f32 = dict(device=dev, dtype=torch.float32)
+        gb = (torch.empty(B, H, T, d, **f32), torch.empty(B, H, T, d, **f32), torch.empty(B, H, T, d, **f32),
+              torch.empty(B, H, T, **f32), torch.empty(B, H, d, d, **f32))
+        wsb = torch.empty(efla.efla_backward_workspace_bytes(B, H, T, d, d, wb.dtype), dtype=torch.uint8, device=dev)
+        callb = lambda: efla.efla_backward(xb["q"], xb["k"], xb["v"], xb["beta"], dOb, grads=gb, workspace=wsb,
+                                           stream=stream)
+        for _ in range(args.warmup):
+            callb()
+        barrier(world)
+        b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        b0.record(stream)
+        for _ in range(args.bwd_steps):
+            callb()
+        b1.record(stream)
+        barrier(world)
+        bms = max_over_ranks(b0.elapsed_time(b1), world) / args.bwd_steps
+        bbytes, bflops = backward_alg(wb)
+        alu = fp32_alu_peak_tflops()
+        bach = bflops / (bms * 1e-3) / 1e12
+        bwd = {"metric": "EFLA backward tokens/s (B4 H16 T2048 d128 bf16 in, fp32 state and gradients)",
+               "value": wb.tokens * world / (bms * 1e-3), "unit": "tokens/s", "ms_per_step": bms,
+               "steps": args.bwd_steps, "dtype": "f32",
+               "roofline": {"bound": "alu", "achieved": bach, "peak": alu, "unit": "TFLOP/s", "frac": bach / alu,
+                            "peak_source": "148 SMs x 128 fp32 FMA lanes x 2 x 1.965 GHz (recipe unit counts and clock)",
+                            "alg_flops_per_launch": bflops, "alg_bytes_per_launch": bbytes,
+                            "hbm_time_us": bbytes / (hbm * 1e9) * 1e6, "traffic": ncu_traffic("efla_backward")},
+               # three zero fills, the sweep kernel and the gate kernel per call
+               "gpu_launches": 5 * args.bwd_steps}
+        del xb, dOb, gb, wsb
+
     # ---- the other forward workloads (long context, stiff keys): tokens/s and roofline
     # fraction of a few forwards each, inputs resident in HBM, CUDA events around the calls
     others = {}
@@ -452,8 +521,8 @@ def main():
             "roofline": roofline, "e2e": e2e,
             # bf16, d = 128: each efla_chunk_fwd launches the UT kernel and the chain kernel
             "gpu_launches": 2 * args.steps,
-            "clocks": clk.summary(), "decode": dec, "other_workloads": others, "cpu_baseline": cpu,
-            "kernel_source": kernel_source_hash(),
+            "clocks": clk.summary(), "decode": dec, "backward": bwd, "other_workloads": others, "cpu_baseline": cpu,
+            "kernel_source": {e: kernel_source_hash(e) for e in KERNEL_SOURCES},
         }
         print(json.dumps(line), flush=True)
     if world > 1:

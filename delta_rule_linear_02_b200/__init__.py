@@ -56,6 +56,12 @@ def _load() -> ctypes.CDLL:
     lib.efla_recurrent_step.restype = I
     lib.efla_recurrent_step_ex.argtypes = [vp, vp, vp, vp, vp, vp, I, I, I, I, I, I, vp]
     lib.efla_recurrent_step_ex.restype = I
+    lib.efla_backward_workspace_bytes.argtypes = [I, I, I, I, I, I]
+    lib.efla_backward_workspace_bytes.restype = Z
+    lib.efla_backward.argtypes = [vp] * 12 + [I, I, I, I, I, I, vp, Z, vp]
+    lib.efla_backward.restype = I
+    lib.efla_backward_ex.argtypes = [vp] * 12 + [I, I, I, I, I, I, I, vp, Z, vp]
+    lib.efla_backward_ex.restype = I
     return lib
 
 
@@ -197,6 +203,45 @@ def efla_recurrent_step(q, k, v, beta, S, o=None, stream=None, rule: int = EFLA_
     return o
 
 
-__all__ = ["EFLA_RULE_EXACT", "EFLA_RULE_EULER", "efla_gate", "efla_chunk_fwd", "efla_chunk_fwd_noalloc", "efla_chunk_fwd_workspace_bytes", "efla_recurrent_step",
+def efla_backward_workspace_bytes(B, H, T, d_k, d_v, dtype=torch.bfloat16) -> int:
+    return int(lib.efla_backward_workspace_bytes(B, H, T, d_k, d_v, _DTYPES[dtype]))
+
+
+def efla_backward(q, k, v, beta, dO, S0=None, dS_T=None, want_dS0: bool = True, grads=None,
+                  workspace=None, stream=None, rule: int = EFLA_RULE_EXACT):
+    """Gradients of efla_chunk_fwd for the loss sum(dO * o) + sum(dS_T * S_T).
+
+    q, k [B,H,T,d_k], v, dO [B,H,T,d_v], beta [B,H,T] (one dtype); S0, dS_T [B,H,d_k,d_v]
+    float32 or None.  Returns (dq, dk, dv, dbeta, dS0 or None), all float32.  `grads` may
+    supply those five tensors preallocated (dS0 may be None)."""
+    dt = k.dtype
+    for t, nme in ((q, "q"), (k, "k"), (v, "v"), (beta, "beta"), (dO, "dO")):
+        _check(t, nme, dt)
+    B, H, T, d_k = k.shape
+    d_v = v.shape[-1]
+    for t, nme in ((S0, "S0"), (dS_T, "dS_T")):
+        if t is not None:
+            _check(t, nme, torch.float32)
+    f32 = dict(device=k.device, dtype=torch.float32)
+    if grads is None:
+        grads = (torch.empty((B, H, T, d_k), **f32), torch.empty((B, H, T, d_k), **f32),
+                 torch.empty((B, H, T, d_v), **f32), torch.empty((B, H, T), **f32),
+                 torch.empty((B, H, d_k, d_v), **f32) if want_dS0 else None)
+    for t, nme in zip(grads, ("dq", "dk", "dv", "dbeta", "dS0")):
+        if t is not None:
+            _check(t, nme, torch.float32)
+    if workspace is None:
+        n = efla_backward_workspace_bytes(B, H, T, d_k, d_v, dt)
+        if n == 0 and B * H * T > 0:
+            raise EflaError(EFLA_ERR_UNSUPPORTED, "efla_backward_workspace_bytes")
+        workspace = torch.empty(max(n, 16), dtype=torch.uint8, device=k.device)
+    st = lib.efla_backward_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(S0), _ptr(dO), _ptr(dS_T),
+                              *(_ptr(g) for g in grads), B, H, T, d_k, d_v, _DTYPES.get(dt, -1), int(rule),
+                              _ptr(workspace), workspace.numel(), _stream(stream))
+    _raise(st, "efla_backward")
+    return grads
+
+
+__all__ = ["efla_backward", "efla_backward_workspace_bytes", "EFLA_RULE_EXACT", "EFLA_RULE_EULER", "efla_gate", "efla_chunk_fwd", "efla_chunk_fwd_noalloc", "efla_chunk_fwd_workspace_bytes", "efla_recurrent_step",
            "efla_workspace_status", "efla_status_string", "efla_selftest_wait_timeout", "new_workspace", "EflaError", "lib",
            "LIB_PATH", "CHUNK"]

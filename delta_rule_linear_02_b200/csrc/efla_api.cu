@@ -202,4 +202,68 @@ int efla_recurrent_step(const void* q, const void* k, const void* v, const void*
     return efla_recurrent_step_ex(q, k, v, beta, S, o, N, H, d_k, d_v, dtype, EFLA_RULE_EXACT, stream);
 }
 
+// ---------------------------------------------------------------- backward
+static int check_bwd_shape(int B, int H, int T, int d_k, int d_v, int dtype) {
+    if (B < 0 || H < 0 || T < 0 || d_k <= 0 || d_v <= 0) return EFLA_ERR_INVALID_ARG;
+    if (dtype != EFLA_DTYPE_F32 && dtype != EFLA_DTYPE_BF16) return EFLA_ERR_UNSUPPORTED;
+    if (d_k != d_v || (d_k != 64 && d_k != 128)) return EFLA_ERR_UNSUPPORTED;
+    if ((long long)B * H * (d_k / 32) >= (1ll << 31)) return EFLA_ERR_UNSUPPORTED;
+    return EFLA_OK;
+}
+
+size_t efla_backward_workspace_bytes(int B, int H, int T, int d_k, int d_v, int dtype) {
+    if (check_bwd_shape(B, H, T, d_k, d_v, dtype) != EFLA_OK) return 0;
+    return efla::bwd_workspace_bytes((long)B * H, T, d_k);
+}
+
+int efla_backward_ex(const void* q, const void* k, const void* v, const void* beta, const float* S0,
+                     const void* dO, const float* dS_T, float* dq, float* dk, float* dv, float* dbeta,
+                     float* dS0, int B, int H, int T, int d_k, int d_v, int dtype, int rule, void* workspace,
+                     size_t workspace_bytes, efla_stream_t stream) {
+    int st = check_bwd_shape(B, H, T, d_k, d_v, dtype);
+    if (st != EFLA_OK) return st;
+    if (rule != EFLA_RULE_EXACT && rule != EFLA_RULE_EULER) return EFLA_ERR_INVALID_ARG;
+    const long BH = (long)B * H;
+    const size_t ns = (size_t)BH * d_k * d_v * sizeof(float);
+    cudaStream_t s = (cudaStream_t)stream;
+    if ((S0 && !aligned16(S0)) || (dS_T && !aligned16(dS_T)) || (dS0 && !aligned16(dS0)))
+        return EFLA_ERR_INVALID_ARG;
+    if (BH == 0) return EFLA_OK;
+    if (T == 0) {   // no token: the state gradient passes through
+        if (!dS0 || dS0 == dS_T) return EFLA_OK;
+        return from_cuda(dS_T ? cudaMemcpyAsync(dS0, dS_T, ns, cudaMemcpyDeviceToDevice, s)
+                              : cudaMemsetAsync(dS0, 0, ns, s));
+    }
+    const size_t need = efla_backward_workspace_bytes(B, H, T, d_k, d_v, dtype);
+    if (!workspace || !aligned16(workspace) || workspace_bytes < need) return EFLA_ERR_INVALID_ARG;
+    if (!q || !k || !v || !beta || !dO || !dq || !dk || !dv || !dbeta) return EFLA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(beta) || !aligned16(dO) ||
+        !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(dbeta))
+        return EFLA_ERR_INVALID_ARG;
+    const size_t es = elem_size(dtype);
+    const size_t nqk = (size_t)BH * T * d_k * es, nv = (size_t)BH * T * d_v * es, nb = (size_t)BH * T * es;
+    const size_t gqk = (size_t)BH * T * d_k * 4, gv = (size_t)BH * T * d_v * 4, gb = (size_t)BH * T * 4;
+    // every output must be disjoint from every input, from the workspace and from the others
+    const void* outs[5] = {dq, dk, dv, dbeta, dS0};
+    const size_t outn[5] = {gqk, gqk, gv, gb, ns};
+    const void* ins[8] = {q, k, v, beta, dO, S0, dS_T, workspace};
+    const size_t inn[8] = {nqk, nqk, nv, nb, nv, ns, ns, workspace_bytes};
+    for (int i = 0; i < 5; ++i) {
+        for (int j = 0; j < 8; ++j)
+            if (overlaps(outs[i], outn[i], ins[j], inn[j])) return EFLA_ERR_INVALID_ARG;
+        for (int j = i + 1; j < 5; ++j)
+            if (overlaps(outs[i], outn[i], outs[j], outn[j])) return EFLA_ERR_INVALID_ARG;
+    }
+    return from_cuda(efla::launch_bwd(q, k, v, beta, S0, dO, dS_T, dq, dk, dv, dbeta, dS0, BH, T, d_k,
+                                      dtype == EFLA_DTYPE_BF16, rule, workspace, s));
+}
+
+int efla_backward(const void* q, const void* k, const void* v, const void* beta, const float* S0,
+                  const void* dO, const float* dS_T, float* dq, float* dk, float* dv, float* dbeta,
+                  float* dS0, int B, int H, int T, int d_k, int d_v, int dtype, void* workspace,
+                  size_t workspace_bytes, efla_stream_t stream) {
+    return efla_backward_ex(q, k, v, beta, S0, dO, dS_T, dq, dk, dv, dbeta, dS0, B, H, T, d_k, d_v, dtype,
+                            EFLA_RULE_EXACT, workspace, workspace_bytes, stream);
+}
+
 }  // extern "C"

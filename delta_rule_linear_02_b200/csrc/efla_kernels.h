@@ -27,6 +27,12 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const v
 cudaError_t launch_ut(const void* k, const void* beta, void* Tout, long BH, int T, uint32_t* err,
                       unsigned long long limit_ns, int rule, cudaStream_t stream);
 
+// reverse-mode pass (efla_bwd.cu): fp32 gradients; workspace of bwd_workspace_bytes
+size_t bwd_workspace_bytes(long BH, int T, int D);
+cudaError_t launch_bwd(const void* q, const void* k, const void* v, const void* beta, const float* S0,
+                       const void* dO, const float* dST, float* dq, float* dk, float* dv, float* dbeta, float* dS0,
+                       long BH, int T, int D, bool bf16, int rule, void* workspace, cudaStream_t stream);
+
 cudaError_t launch_wait_timeout_selftest(uint32_t* err, unsigned long long limit_ns, cudaStream_t stream);
 
 }  // namespace efla

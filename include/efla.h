@@ -186,6 +186,49 @@ int efla_recurrent_step_ex(const void *q, const void *k, const void *v, const vo
                            float *S, void *o, int N, int H, int d_k, int d_v, int dtype,
                            int rule, efla_stream_t stream);
 
+/*
+ * efla_backward_workspace_bytes -- bytes of device workspace efla_backward needs:
+ * B*H*T*d_v + B*H*T floats (the residuals r_t = S_{t-1}^T k_t - v_t of a forward sweep,
+ * and the gate gradient).  0 for an unsupported shape or dtype.
+ */
+size_t efla_backward_workspace_bytes(int B, int H, int T, int d_k, int d_v, int dtype);
+
+/*
+ * efla_backward -- gradients of the forward pass (efla_chunk_fwd / the recurrence of
+ * Section 3.2 with o_t = S_t^T q_t) for the loss sum(dO * o) + sum(dS_T * S_T): the
+ * chain rule of the recurrence taken in reverse (training, Section 4.6; the pages print
+ * no backward formulas).  With G = dL/dS_t, r_t = S_{t-1}^T k_t - v_t:
+ *   dq_t = S_t dO_t, dv_t = alpha_t G^T k_t, dk_t = -alpha_t (G r_t + S_{t-1} G^T k_t)
+ *   + dalpha_t (d alpha / d lambda) 2 k_t, dbeta_t = dalpha_t (d alpha / d beta) with
+ *   dalpha_t = -(G^T k_t) . r_t, G <- G - alpha_t k_t (G^T k_t)^T; dS0 = G at t = 0.
+ *
+ *   q, k [B,H,T,d_k], v, dO [B,H,T,d_v], beta [B,H,T]   inputs, `dtype`
+ *   S0, dS_T [B,H,d_k,d_v] float32, or NULL (zero)
+ *   dq, dk [B,H,T,d_k], dv [B,H,T,d_v], dbeta [B,H,T]   float32 outputs
+ *   dS0 [B,H,d_k,d_v] float32 output, or NULL (not wanted)
+ *   workspace (>= efla_backward_workspace_bytes, 16-byte aligned), caller-owned
+ *
+ * Supported: d_k = d_v in {64, 128}; dtype f32 or bf16; any T >= 0 (T = 0 copies dS_T
+ * into dS0).  All pointers 16-byte aligned; no output may overlap an input, the
+ * workspace or another output; else EFLA_ERR_INVALID_ARG and nothing is launched.  The
+ * state is fp32 throughout; the outputs are accumulated in fp32 (the row sums over d_v
+ * columns with atomics, so their last bits depend on arrival order).  Asynchronous on
+ * `stream`; launch failures return EFLA_ERR_CUDA.
+ */
+int efla_backward(const void *q, const void *k, const void *v, const void *beta, const float *S0,
+                  const void *dO, const float *dS_T, float *dq, float *dk, float *dv, float *dbeta,
+                  float *dS0, int B, int H, int T, int d_k, int d_v, int dtype, void *workspace,
+                  size_t workspace_bytes, efla_stream_t stream);
+
+/*
+ * efla_backward_ex -- efla_backward with the step rule chosen (`rule` an efla_rule, else
+ * EFLA_ERR_INVALID_ARG).  EFLA_RULE_EULER differentiates the Euler step alpha = beta.
+ */
+int efla_backward_ex(const void *q, const void *k, const void *v, const void *beta, const float *S0,
+                     const void *dO, const float *dS_T, float *dq, float *dk, float *dv, float *dbeta,
+                     float *dS0, int B, int H, int T, int d_k, int d_v, int dtype, int rule,
+                     void *workspace, size_t workspace_bytes, efla_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

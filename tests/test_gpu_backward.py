@@ -1,0 +1,102 @@
+"""The backward pass (efla_backward, CUDA) against the oracle's fp64 reverse sweep.
+
+The oracle's backward is pinned by finite differences of the pinned forward oracle
+(tests/oracle_bwd_pins.py).  Both sides take the same dtype-cast inputs; the CUDA path
+keeps the state and every gradient in fp32, so the bound is the fp32 one, 1e-4 relative
+Frobenius per gradient, for bf16 inputs too (the inputs are exact in both).  At the full
+1.3B-layer shape (B4 H16 T2048 d128) two sampled streams are compared with the oracle run
+on those streams alone, at 1e-3 (2,048 steps of fp32 rounding in the rebuilt states).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from helpers import rel_frob
+
+pytestmark = pytest.mark.gpu
+
+W = workloads.CHUNK_WORKLOADS
+NAMES = ("dq", "dk", "dv", "dbeta", "dS0")
+
+
+def run_both(efla, cuda, w, with_state=True, rule=None, streams=None, unit_keys=False):
+    inp = workloads.make_chunk_inputs(w)
+    if unit_keys:   # beta ||k||^2 < 2: the explicit (Euler) step stays stable
+        k = inp["k"].float()
+        inp["k"] = (k / k.norm(dim=-1, keepdim=True).clamp_min(1e-30)).to(inp["k"].dtype)
+    cot = workloads.make_cotangents(w, with_state_grad=with_state)
+    S0 = inp["S0"]
+    if with_state and S0 is None:
+        S0 = 0.1 * torch.randn(w.B, w.H, w.dk, w.dv, generator=torch.Generator().manual_seed(w.seed + 7))
+    if not with_state:
+        S0 = None
+    d = {k: (None if v is None else v.to(cuda)) for k, v in dict(inp, S0=S0, **cot).items()}
+    kw = {} if rule is None else dict(rule=rule)
+    got = efla.efla_backward(d["q"], d["k"], d["v"], d["beta"], d["dO"], S0=d["S0"], dS_T=d["dS_T"], **kw)
+    torch.cuda.synchronize()
+    mode = oracle.EULER if rule == efla.EFLA_RULE_EULER else oracle.EXACT
+    if streams is None:
+        ref = oracle.bwd(inp["q"], inp["k"], inp["v"], inp["beta"], cot["dO"], S0=S0, dS_T=cot["dS_T"], mode=mode)
+        return [g.cpu() for g in got], ref
+    sel = lambda t: None if t is None else torch.stack([t[b, h] for b, h in streams])[None]
+    ref = oracle.bwd(sel(inp["q"]), sel(inp["k"]), sel(inp["v"]), sel(inp["beta"]), sel(cot["dO"]),
+                     S0=sel(S0), dS_T=sel(cot["dS_T"]), mode=mode, threads=len(streams))
+    got = [sel(g.cpu()) for g in got]
+    return got, ref
+
+
+CASES = [("tiny_fp32", dict(B=1, H=2, T=200)),                          # fp32, d = 64, ragged T
+         ("tiny_fp32", dict(B=2, H=1, T=97, dk=128, dv=128)),             # fp32, d = 128
+         ("lm1p3b_bf16", dict(B=1, H=2, T=150)),                          # bf16, d = 128
+         ("lm1p3b_bf16", dict(B=1, H=3, T=64, dk=64, dv=64)),             # bf16, d = 64
+         ("stiff_bf16", dict(B=1, H=2, T=300))]                           # stiff keys, corrupted tokens
+
+
+@pytest.mark.parametrize("name,over", CASES, ids=lambda x: str(x))
+def test_backward_matches_oracle(efla, cuda, name, over):
+    w = W[name].replace(**over)
+    got, ref = run_both(efla, cuda, w)
+    for nme, g, r in zip(NAMES, got, ref):
+        e = rel_frob(g, r)
+        assert e <= 1e-4, (nme, e)
+
+
+def test_backward_without_state_tensors(efla, cuda):
+    """No S0, no dS_T: the oracle's zero state and zero final gradient."""
+    w = W["tiny_fp32"].replace(B=1, H=2, T=77)
+    got, ref = run_both(efla, cuda, w, with_state=False)
+    for nme, g, r in zip(NAMES, got, ref):
+        assert rel_frob(g, r) <= 1e-4, nme
+
+
+def test_backward_euler_rule(efla, cuda):
+    """The Euler step alpha = beta differentiated (keys of unit norm, as for the forward's
+    Euler test: with beta ||k||^2 up to ~64 the explicit step diverges and overflows)."""
+    w = W["tiny_fp32"].replace(B=1, H=2, T=90)
+    got, ref = run_both(efla, cuda, w, rule=efla.EFLA_RULE_EULER, unit_keys=True)
+    for nme, g, r in zip(NAMES, got, ref):
+        assert rel_frob(g, r) <= 1e-4, nme
+
+
+def test_backward_single_token_and_empty(efla, cuda):
+    w = W["tiny_fp32"].replace(B=1, H=3, T=1)
+    got, ref = run_both(efla, cuda, w)
+    for nme, g, r in zip(NAMES, got, ref):
+        assert rel_frob(g, r) <= 1e-5, nme
+    # T = 0: the state gradient passes straight through
+    dST = torch.randn(1, 2, 64, 64, device=cuda)
+    e = torch.empty(1, 2, 0, 64, device=cuda)
+    out = efla.efla_backward(e, e, e, torch.empty(1, 2, 0, device=cuda), e, dS_T=dST)
+    torch.cuda.synchronize()
+    assert torch.equal(out[4], dST)
+
+
+def test_backward_full_shape_sampled_streams(efla, cuda):
+    """B4 H16 T2048 d128 bf16, the forward's benchmark shape: two streams against the oracle."""
+    w = W["lm1p3b_bf16"]
+    got, ref = run_both(efla, cuda, w, streams=[(0, 0), (3, 15)])
+    for nme, g, r in zip(NAMES, got, ref):
+        e = rel_frob(g, r)
+        assert e <= 1e-3, (nme, e)

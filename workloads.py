@@ -158,3 +158,12 @@ def make_decode_steps(w: DecodeWorkload, steps: Optional[int] = None, device="cp
     v = torch.randn(*shp, w.dv, generator=g, device=device, dtype=f32)
     beta = torch.sigmoid(torch.randn(*shp, generator=g, device=device, dtype=f32))
     return {"q": q, "k": k, "v": v, "beta": beta}
+
+
+def make_cotangents(w: ChunkWorkload, with_state_grad: bool = True) -> dict:
+    """The backward pass's seeded inputs: dO [B,H,T,dv] ~ N(0, 1) in w.dtype and
+    dS_T [B,H,dk,dv] ~ N(0, 1) float32 (or None), drawn on the CPU from seed w.seed + 1000."""
+    g = torch.Generator().manual_seed(w.seed + 1000)
+    dO = torch.randn(w.B, w.H, w.T, w.dv, generator=g, dtype=torch.float32).to(w.dtype).contiguous()
+    dST = torch.randn(w.B, w.H, w.dk, w.dv, generator=g, dtype=torch.float32) if with_state_grad else None
+    return {"dO": dO, "dS_T": dST}
