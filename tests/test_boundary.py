@@ -135,3 +135,47 @@ def test_binding_fails_loudly_without_the_library(tmp_path):
     r = subprocess.run([sys.executable, "-c", "import delta_rule_linear_02_b200"], cwd=tmp_path,
                        capture_output=True, text=True)
     assert r.returncode != 0 and "libefla.so is not built" in r.stderr
+
+
+def _bwd(L, ptrs, B=1, H=1, T=64, d=128, dtype=1, ws=1 << 20, rule=0):
+    q, k, v, b, s0, do, dst, dq, dk, dv, db, ds0, w = ptrs
+    return L.efla_backward_ex(q, k, v, b, s0, do, dst, dq, dk, dv, db, ds0, B, H, T, d, d, dtype, rule, w, ws,
+                              None)
+
+
+# 13 fake device addresses 16 MiB apart: no two ranges of the small problems below overlap
+GOOD_B = [ctypes.c_void_p(0x10000000 + 0x1000000 * i) for i in range(13)]
+
+
+def test_backward_workspace_bytes(efla):
+    L = efla.lib
+    assert L.efla_backward_workspace_bytes(4, 16, 2048, 128, 128, 1) == 4 * 16 * 2048 * (128 + 1) * 4
+    assert L.efla_backward_workspace_bytes(1, 1, 1, 96, 96, 0) == 0      # unsupported d
+    assert L.efla_backward_workspace_bytes(1, 1, 1, 128, 64, 1) == 0     # d_k != d_v
+    assert L.efla_backward_workspace_bytes(1, 1, 1, 64, 64, 5) == 0      # dtype
+    assert L.efla_backward_workspace_bytes(1, -1, 1, 64, 64, 0) == 0     # negative
+
+
+def test_backward_rejects_bad_arguments(efla):
+    L = efla.lib
+    assert _bwd(L, GOOD_B, d=96) == UNSUPPORTED
+    assert _bwd(L, GOOD_B, dtype=3) == UNSUPPORTED
+    assert _bwd(L, GOOD_B, rule=9) == INVALID
+    assert _bwd(L, GOOD_B, T=-1) == INVALID
+    for i in (0, 1, 2, 3, 5, 7, 8, 9, 10):        # inputs, dO and dq, dk, dv, dbeta are required
+        bad = list(GOOD_B); bad[i] = None
+        assert _bwd(L, bad) == INVALID, i
+    for i in range(13):                           # every pointer must be 16-byte aligned
+        bad = list(GOOD_B); bad[i] = ctypes.c_void_p(GOOD_B[i].value + 4)
+        assert _bwd(L, bad) == INVALID, i
+    bad = list(GOOD_B); bad[12] = None            # workspace required
+    assert _bwd(L, bad) == INVALID
+    assert _bwd(L, GOOD_B, ws=64) == INVALID      # workspace too small
+    bad = list(GOOD_B); bad[7] = GOOD_B[0]        # dq aliases q
+    assert _bwd(L, bad) == INVALID
+    bad = list(GOOD_B); bad[8] = GOOD_B[7]        # dk aliases dq
+    assert _bwd(L, bad) == INVALID
+    bad = list(GOOD_B); bad[11] = GOOD_B[4]       # dS0 aliases S0
+    assert _bwd(L, bad) == INVALID
+    assert _bwd(L, GOOD_B, B=0) == OK             # nothing to do, nothing launched
+    assert _bwd(L, GOOD_B, H=0) == OK
