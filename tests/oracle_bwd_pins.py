@@ -11,7 +11,9 @@ References, none of which re-types the reverse sweep:
     returned gradient;
   * the same finite differences, element by element, on a tiny case;
   * the gate's derivatives by finite differences of the gate itself, and the limit
-    d alpha / d lambda -> -beta^2 / 2 as lambda -> 0 (from alpha = beta - beta^2 lambda / 2 + ...).
+    d alpha / d lambda -> -beta^2 / 2 as lambda -> 0 (from alpha = beta - beta^2 lambda / 2 + ...);
+  * a second algorithm for the same numbers (tests/bwd_mirror.py: no stored states, each
+    earlier state rebuilt from the later one, column slices summed), to 1e-12.
 """
 from __future__ import annotations
 
@@ -113,5 +115,22 @@ def pin_gate_derivatives(lib):
         assert abs(oracle.dalpha_dlambda(beta, 1e-14, lib) + 0.5 * beta * beta) <= 1e-12 * beta * beta
 
 
+def pin_bwd_state_reversal(lib):
+    """The reverse sweep the CUDA kernel uses (residuals stored, earlier states rebuilt from
+    later ones, column slices summed; tests/bwd_mirror.py) gives the oracle's gradients to
+    1e-12, with and without slicing, in both modes."""
+    from bwd_mirror import stream_bwd
+    rng = np.random.default_rng(6)
+    for mode, cols in ((oracle.EXACT, None), (oracle.EXACT, 2), (oracle.EULER, 3)):
+        q, k, v, beta, S0, dO, dST = _problem(rng, B=1, H=2, T=9, dk=4, dv=6)
+        got = oracle.bwd(q, k, v, beta, dO, S0=S0, dS_T=dST, mode=mode, threads=1, lib=lib)
+        for h in range(2):
+            ref = stream_bwd(q[0, h], k[0, h], v[0, h], beta[0, h], dO[0, h], S0[0, h], dST[0, h],
+                             euler=(mode == oracle.EULER), slice_cols=cols)
+            for x, y in zip((g[0, h] for g in got), ref):
+                assert np.allclose(x, y, rtol=1e-12, atol=1e-12), (mode, cols, h)
+
+
 ALL_PINS = [pin_bwd_directional_exact, pin_bwd_directional_stiff, pin_bwd_directional_euler,
-            pin_bwd_elementwise, pin_bwd_zero_state_and_no_final_gradient, pin_gate_derivatives]
+            pin_bwd_elementwise, pin_bwd_zero_state_and_no_final_gradient, pin_gate_derivatives,
+            pin_bwd_state_reversal]
