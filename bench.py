@@ -78,19 +78,37 @@ KERNEL_SOURCES = {
 
 
 def backward_alg(w):
-    """One backward call.  Bytes: read q, k, v, dO, beta (w.dtype) and write dq, dk, dv, dbeta
-    (fp32), plus dS0 (fp32).  Flops of the recurrent reverse pass as built (fp32 CUDA cores),
-    18 d^2 per token and head: the forward sweep's S^T k and rank-1 write, then G += q dO^T,
-    S dO, G^T k, the rebuilt S_{t-1}, G r, S_{t-1} g and G -= alpha k g^T (2 d^2 each)."""
+    """One backward call, counted for the method's chunked form (not for the kernel as built).
+
+    Bytes: read q, k, v, dO, beta (w.dtype), write dq, dk, dv, dbeta (fp32) and dS0 (fp32).
+    Flops per (stream, chunk): the forward's chunk products recomputed (5 x 2 C^2 d +
+    3 x 2 C d^2) and their transposed products for the gradients, two per forward product
+    (dA = dC B^T, dB = A^T dC): 3 x the forward's count.
+    """
     es = 2 if w.dtype == torch.bfloat16 else 4
     BH, T, d = w.B * w.H, w.T, w.dk
     nbytes = BH * T * (4 * d * es + es + 3 * d * 4 + 4) + BH * d * d * 4
-    return nbytes, BH * T * 18 * d * d
+    chunks = (T + 63) // 64
+    flops = 3 * BH * chunks * (5 * 2 * 64 * 64 * d + 3 * 2 * 64 * d * d)
+    return nbytes, flops
 
 
-def fp32_alu_peak_tflops():
-    """FMA peak of the CUDA cores: 148 SMs x 128 fp32 lanes x 2 flops x 1.965 GHz."""
-    return 148 * 128 * 2 * 1.965e9 / 1e12
+def roofline_record(nbytes, flops, seconds, hbm, tc, peak_kind):
+    """Roofline of one call from its algorithmic bytes and flops and its measured time: the
+    bound is whichever of bytes / HBM bandwidth and flops / tensor peak takes longer, and
+    frac = that time / the measured time."""
+    t_hbm, t_tc = nbytes / (hbm * 1e9), flops / (tc * 1e12)
+    if t_hbm >= t_tc:
+        rec = {"bound": "hbm", "achieved": nbytes / seconds / 1e9, "peak": hbm, "unit": "GB/s",
+               "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"}
+    else:
+        rec = {"bound": "tensor", "achieved": flops / seconds / 1e12, "peak": tc, "unit": "TFLOP/s",
+               "peak_source": f"{peak_kind} cuBLAS bf16 burst (MEASURED_PEAKS.json bf16_tflops)"}
+    rec["frac"] = max(t_hbm, t_tc) / seconds
+    rec.update({"alg_bytes_per_launch": nbytes, "alg_flops_per_launch": flops,
+                "tensor_tflops": flops / seconds / 1e12, "hbm_gbs": nbytes / seconds / 1e9,
+                "roofline_time_us": max(t_hbm, t_tc) * 1e6})
+    return rec
 
 
 def kernel_source_hash(entry=None):
@@ -104,21 +122,64 @@ def kernel_source_hash(entry=None):
     return h.hexdigest()[:16]
 
 
-def ncu_traffic(kernel: str):
-    """dram bytes per launch recorded in profiles/traffic.md for the entry point's current
-    kernel sources."""
-    path = os.path.join(ROOT, "profiles", "traffic.md")
+TRAFFIC_JSON = os.path.join(ROOT, "profiles", "traffic.json")
+# the kernels each entry point launches (ncu kernel-name prefixes)
+ENTRY_KERNELS = {
+    "efla_chunk_fwd": ("ut_kernel", "chunk_tc_kernel"),
+    "efla_recurrent_step": ("decode_kernel",),
+    "efla_backward": ("bwd_kernel", "bwd_gate_kernel"),
+}
+
+
+def ncu_traffic(entry: str):
+    """DRAM bytes (read + write) per call of an entry point, from profiles/traffic.json as
+    written by --traffic-from; None unless it was recorded for the current kernel sources."""
     try:
-        lines = open(path).read().splitlines()
-    except OSError:
+        with open(TRAFFIC_JSON) as f:
+            rec = json.load(f).get(entry)
+    except (OSError, ValueError):
         return None
-    src = kernel_source_hash(kernel)
-    for ln in lines:
-        if ln.startswith("traffic|"):
-            _, name, nbytes, sha = ln.split("|")[:4]
-            if name == kernel and sha.strip() == src:
-                return int(nbytes)
-    return None
+    if not rec or rec.get("kernel_source") != kernel_source_hash(entry):
+        return None
+    return int(rec["bytes_per_call"])
+
+
+def traffic_from_csv(csv_path: str, entry: str, calls: int):
+    """Write profiles/traffic.json's record for `entry` from an ncu --csv log of
+    dram__bytes_read.sum and dram__bytes_write.sum: the last `calls` calls' launches of the
+    entry point's kernels, summed and divided by `calls`."""
+    import csv
+    rows = []
+    with open(csv_path) as f:
+        lines = [ln for ln in f if ln.startswith('"')]
+    def bare(name):      # "void (anonymous namespace)::decode_kernel<float, 128>(...)" -> "decode_kernel"
+        name = name.removeprefix("void ").replace("(anonymous namespace)::", "").replace("unnamed>::", "")
+        return name.split("(")[0].split("<")[0].split("::")[-1].strip()
+
+    for r in csv.DictReader(lines):
+        name = bare(r.get("Kernel Name", ""))
+        if name in ENTRY_KERNELS[entry] and r.get("Metric Name", "").startswith("dram__bytes_"):
+            unit = r.get("Metric Unit", "byte")
+            scale = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9, "KB": 1e3, "MB": 1e6, "GB": 1e9}.get(unit, 1)
+            rows.append((int(r["ID"]), name, r["Metric Name"], float(r["Metric Value"].replace(",", "")) * scale))
+    ids = sorted({i for i, _, _, _ in rows})
+    per_call = len(ENTRY_KERNELS[entry]) if entry != "efla_backward" else 2
+    keep = set(ids[-calls * per_call:])
+    total = sum(v for i, _, _, v in rows if i in keep)
+    rec = {"bytes_per_call": int(round(total / calls)), "calls": calls,
+           "launches": len(keep), "kernel_source": kernel_source_hash(entry),
+           "kernels": sorted({n for i, n, _, _ in rows if i in keep}),
+           "from": os.path.basename(csv_path)}
+    try:
+        with open(TRAFFIC_JSON) as f:
+            data = json.load(f)
+    except (OSError, ValueError):
+        data = {}
+    data[entry] = rec
+    with open(TRAFFIC_JSON, "w") as f:
+        json.dump(data, f, indent=1, sort_keys=True)
+        f.write("\n")
+    return rec
 
 
 class Clocks:
@@ -225,7 +286,8 @@ def rank_workload(rank: int, world: int):
 
 def cpu_baseline(w, cpu_seconds: float = 12.0):
     """The fp64 oracle, as it stands, on the workload's streams: whole passes over all
-    B*H streams, repeated until about `cpu_seconds` of CPU work (wall x threads) is done."""
+    B*H streams, repeated until about `cpu_seconds` of CPU work (wall x threads) is done;
+    and the same oracle on one thread over a sample of 4 streams."""
     import oracle
     inp = workloads.make_chunk_inputs(w)
     threads = oracle.default_threads()
@@ -237,9 +299,17 @@ def cpu_baseline(w, cpu_seconds: float = 12.0):
         if dt * threads >= cpu_seconds or dt >= 60.0:
             break
     tokens = passes * w.B * w.T                 # a token spans all H heads
+    n1 = 4
+    one = {k: (None if v is None else v[0, :n1].unsqueeze(0).contiguous()) for k, v in inp.items()}
+    t1 = time.perf_counter()
+    oracle.fwd(one["q"], one["k"], one["v"], one["beta"], one["S0"], threads=1)
+    dt1 = time.perf_counter() - t1
     return {"value": tokens / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
             "sample": f"{passes} full pass(es) over all {w.B * w.H} (b,h) streams of the workload "
-                      f"(T={w.T}), {dt:.1f} s wall on {threads} threads"}
+                      f"(T={w.T}), {dt:.1f} s wall on {threads} threads",
+            "single_thread": {"value": n1 * w.T / w.H / dt1, "unit": "tokens/s", "cores": 1,
+                              "sample": f"{n1} of {w.B * w.H} (b,h) streams at T={w.T} on 1 thread, "
+                                        f"{dt1:.2f} s; tokens counted as streams x T / H"}}
 
 
 def run_reference(args):
@@ -274,6 +344,45 @@ def run_reference(args):
     }), flush=True)
 
 
+def profile_call(args):
+    """warm-up + steps calls of one entry point on its bench workload and nothing else, so
+    that an ncu capture (-s warm-up launches, -c launches) sees only those launches."""
+    import delta_rule_linear_02_b200 as efla
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.current_stream(dev)
+    if args.profile_call == "decode":
+        S = workloads.make_decode_state(DECODE, device=dev)
+        n = args.warmup + args.steps
+        st = workloads.make_decode_steps(DECODE, steps=n, device=dev)
+        o = torch.empty(DECODE.N, DECODE.H, DECODE.dv, device=dev)
+        calls = [lambda i=i: efla.efla_recurrent_step(st["q"][i], st["k"][i], st["v"][i], st["beta"][i], S,
+                                                       o=o, stream=stream) for i in range(n)]
+    else:
+        w = WORKLOAD
+        x = {k: (None if v is None else v.to(dev)) for k, v in workloads.make_chunk_inputs(w).items()}
+        B, H, T, d = w.B, w.H, w.T, w.dk
+        if args.profile_call == "fwd":
+            ws = efla.new_workspace(B, H, T, d, d, 64, w.dtype, dev)
+            o = torch.empty(B, H, T, d, dtype=w.dtype, device=dev)
+            ST = torch.empty(B, H, d, d, dtype=torch.float32, device=dev)
+            one = lambda: efla.efla_chunk_fwd(x["q"], x["k"], x["v"], x["beta"], x["S0"], o=o, S_T=ST,
+                                              workspace=ws, stream=stream)
+        else:
+            dO = workloads.make_cotangents(w, with_state_grad=False)["dO"].to(dev)
+            f32 = dict(device=dev, dtype=torch.float32)
+            g = (torch.empty(B, H, T, d, **f32), torch.empty(B, H, T, d, **f32), torch.empty(B, H, T, d, **f32),
+                 torch.empty(B, H, T, **f32), torch.empty(B, H, d, d, **f32))
+            wsb = torch.empty(efla.efla_backward_workspace_bytes(B, H, T, d, d, w.dtype), dtype=torch.uint8,
+                              device=dev)
+            one = lambda: efla.efla_backward(x["q"], x["k"], x["v"], x["beta"], dO, grads=g, workspace=wsb,
+                                             stream=stream)
+        calls = [one] * (args.warmup + args.steps)
+    for c in calls:
+        c()
+    torch.cuda.synchronize(dev)
+    print(json.dumps({"profile_call": args.profile_call, "calls": len(calls)}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -286,10 +395,24 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--other-steps", type=int, default=10,
                     help="forwards timed on each of the long-context and stiff workloads (0: skip)")
+    ap.add_argument("--profile-call", choices=["fwd", "decode", "bwd"],
+                    help="only run warm-up + steps calls of one entry point (for an ncu capture)")
+    ap.add_argument("--traffic-from", metavar="CSV",
+                    help="write profiles/traffic.json's record from an ncu --csv log of "
+                         "dram__bytes_read.sum and dram__bytes_write.sum, then exit")
+    ap.add_argument("--traffic-entry", default="efla_chunk_fwd", choices=sorted(ENTRY_KERNELS))
+    ap.add_argument("--traffic-calls", type=int, default=1,
+                    help="calls of the entry point at the end of the CSV that the record averages")
     args = ap.parse_args()
+    if args.traffic_from:
+        print(json.dumps(traffic_from_csv(args.traffic_from, args.traffic_entry, args.traffic_calls)))
+        return
     args.warmup = max(args.warmup, 3)
     if args.impl == "reference":
         run_reference(args)
+        return
+    if args.profile_call:
+        profile_call(args)
         return
 
     import delta_rule_linear_02_b200 as efla
@@ -337,14 +460,10 @@ def main():
     value = tokens / (ms_per_step * 1e-3)
 
     nbytes, flops = chunk_alg(w)
-    achieved = nbytes / (launch_ms * 1e-3) / 1e9
-    t_star = max(nbytes / (hbm * 1e9), flops / (tc * 1e12))
-    roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                "frac": achieved / hbm, "traffic": ncu_traffic("efla_chunk_fwd"),
-                "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
-                "alg_bytes_per_launch": nbytes, "alg_flops_per_launch": flops,
-                "tensor_tflops": flops / (launch_ms * 1e-3) / 1e12,
-                "roofline_time_us": t_star * 1e6, "roofline_frac": t_star / (launch_ms * 1e-3)}
+    # the same timed region as `value`: whole-region time / steps
+    roofline = roofline_record(nbytes, flops, ms_per_step * 1e-3, hbm, tc, peak_kind)
+    roofline.update({"traffic": ncu_traffic("efla_chunk_fwd"), "timed": "whole timed region / steps",
+                     "call_events_mean_us": launch_ms * 1e3})
 
     # ---- end to end through the public API with host buffers (pinned), copies timed.
     # Every step copies its inputs from pinned host memory and reads its result (o and
@@ -430,7 +549,7 @@ def main():
                "steps": nd, "dtype": "f32",
                "roofline": {"bound": "hbm", "achieved": dach, "peak": hbm, "unit": "GB/s",
                             "frac": dach / hbm, "traffic": ncu_traffic("efla_recurrent_step"),
-                            "alg_bytes_per_launch": dbytes},
+                            "alg_bytes_per_launch": dbytes, "alg_flops_per_launch": dflops},
                "gpu_launches": nd}
         del S, st
 
@@ -458,15 +577,12 @@ def main():
         barrier(world)
         bms = max_over_ranks(b0.elapsed_time(b1), world) / args.bwd_steps
         bbytes, bflops = backward_alg(wb)
-        alu = fp32_alu_peak_tflops()
-        bach = bflops / (bms * 1e-3) / 1e12
+        brf = roofline_record(bbytes, bflops, bms * 1e-3, hbm, tc, peak_kind)
+        brf["traffic"] = ncu_traffic("efla_backward")
         bwd = {"metric": "EFLA backward tokens/s (B4 H16 T2048 d128 bf16 in, fp32 state and gradients)",
                "value": wb.tokens * world / (bms * 1e-3), "unit": "tokens/s", "ms_per_step": bms,
-               "steps": args.bwd_steps, "dtype": "f32",
-               "roofline": {"bound": "alu", "achieved": bach, "peak": alu, "unit": "TFLOP/s", "frac": bach / alu,
-                            "peak_source": "148 SMs x 128 fp32 FMA lanes x 2 x 1.965 GHz (recipe unit counts and clock)",
-                            "alg_flops_per_launch": bflops, "alg_bytes_per_launch": bbytes,
-                            "hbm_time_us": bbytes / (hbm * 1e9) * 1e6, "traffic": ncu_traffic("efla_backward")},
+               "steps": args.bwd_steps, "dtype": "bf16", "grad_dtype": "f32",
+               "roofline": brf, "roofline_basis": "the method's chunked form: bytes at HBM, 3x forward flops at tensor peak",
                # three zero fills, the sweep kernel and the gate kernel per call
                "gpu_launches": 5 * args.bwd_steps}
         del xb, dOb, gb, wsb
@@ -496,12 +612,10 @@ def main():
         if efla.efla_workspace_status(wso, clear=True, stream=stream) != efla.EFLA_OK:
             raise SystemExit(f"device reported a timeout on {name}")
         ob, of = chunk_alg(wo)
-        ot = max(ob / (hbm * 1e9), of / (tc * 1e12))
         others[name] = {"value": wo.tokens * world / (oms * 1e-3), "unit": "tokens/s", "ms_per_step": oms,
                         "steps": args.other_steps,
                         "config": {"B": wo.B, "H": wo.H, "T": wo.T, "d_k": wo.dk, "d_v": wo.dv, "chunk": 64},
-                        "roofline": {"bound": "hbm", "achieved": ob / (oms * 1e-3) / 1e9, "peak": hbm,
-                                     "unit": "GB/s", "frac": ot / (oms * 1e-3), "roofline_time_us": ot * 1e6},
+                        "roofline": roofline_record(ob, of, oms * 1e-3, hbm, tc, peak_kind),
                         "gpu_launches": 2 * args.other_steps}
         del xo, wso, oo, So
 

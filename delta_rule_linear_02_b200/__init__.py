@@ -50,6 +50,8 @@ def _load() -> ctypes.CDLL:
     lib.efla_chunk_fwd_noalloc.restype = I
     lib.efla_workspace_status.argtypes = [vp, I, vp]
     lib.efla_workspace_status.restype = I
+    lib.efla_noalloc_status.argtypes = [I, vp]
+    lib.efla_noalloc_status.restype = I
     lib.efla_selftest_wait_timeout.argtypes = [vp, ctypes.c_longlong, vp]
     lib.efla_selftest_wait_timeout.restype = I
     lib.efla_recurrent_step.argtypes = [vp, vp, vp, vp, vp, vp, I, I, I, I, I, vp]
@@ -180,6 +182,11 @@ def efla_workspace_status(workspace: torch.Tensor, clear: bool = False, stream=N
     return int(lib.efla_workspace_status(_ptr(workspace), int(clear), _stream(stream)))
 
 
+def efla_noalloc_status(clear: bool = False, stream=None) -> int:
+    """Device error word of efla_chunk_fwd_noalloc's static scratch (current device)."""
+    return int(lib.efla_noalloc_status(int(clear), _stream(stream)))
+
+
 def efla_selftest_wait_timeout(workspace: torch.Tensor, limit_ns: int = 1_000_000, stream=None) -> None:
     _raise(lib.efla_selftest_wait_timeout(_ptr(workspace), int(limit_ns), _stream(stream)),
            "efla_selftest_wait_timeout")
@@ -243,5 +250,5 @@ def efla_backward(q, k, v, beta, dO, S0=None, dS_T=None, want_dS0: bool = True, 
 
 
 __all__ = ["efla_backward", "efla_backward_workspace_bytes", "EFLA_RULE_EXACT", "EFLA_RULE_EULER", "efla_gate", "efla_chunk_fwd", "efla_chunk_fwd_noalloc", "efla_chunk_fwd_workspace_bytes", "efla_recurrent_step",
-           "efla_workspace_status", "efla_status_string", "efla_selftest_wait_timeout", "new_workspace", "EflaError", "lib",
+           "efla_workspace_status", "efla_noalloc_status", "efla_status_string", "efla_selftest_wait_timeout", "new_workspace", "EflaError", "lib",
            "LIB_PATH", "CHUNK"]

@@ -2,6 +2,8 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <atomic>
+
 #include "../../include/efla.h"
 #include "efla_common.cuh"
 #include "efla_kernels.h"
@@ -96,6 +98,12 @@ int efla_chunk_fwd_ex(const void* q, const void* k, const void* v, const void* b
         (overlaps(S_T, ns, q, nqk) || overlaps(S_T, ns, k, nqk) || overlaps(S_T, ns, v, nv) ||
          overlaps(S_T, ns, beta, nb) || overlaps(S_T, ns, S0, ns)))
         return EFLA_ERR_INVALID_ARG;
+    // the kernels write the workspace (error word, UT transforms) while the inputs are
+    // still being read, and S_T last: neither may share bytes with it
+    if (overlaps(workspace, workspace_bytes, q, nqk) || overlaps(workspace, workspace_bytes, k, nqk) ||
+        overlaps(workspace, workspace_bytes, v, nv) || overlaps(workspace, workspace_bytes, beta, nb) ||
+        overlaps(workspace, workspace_bytes, S0, ns) || overlaps(workspace, workspace_bytes, S_T, ns))
+        return EFLA_ERR_INVALID_ARG;
     if (dtype == EFLA_DTYPE_BF16 && d_k == 128)
         return from_cuda(efla::launch_chunk_tc(q, k, v, beta, S0, o, S_T, BH, T,
                                                static_cast<uint32_t*>(workspace),
@@ -119,23 +127,27 @@ int efla_chunk_fwd(const void* q, const void* k, const void* v, const void* beta
 static constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;   // 32 MiB
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
+// The address is cached per device in an atomic slot (host threads may race on the first
+// call; each writes the same value).  A cudaDeviceReset invalidates the module and with it
+// the address: a process that resets a device must not call the no-alloc entry points on
+// it afterwards.
 static void* noalloc_scratch(int* status) {
     constexpr int kMaxDevices = 64;
-    static void* addr[kMaxDevices] = {};
+    static std::atomic<void*> addr[kMaxDevices];
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
         *status = EFLA_ERR_CUDA;
         return nullptr;
     }
-    if (!addr[dev]) {   // first call on this device (with it current): resolve the address
-        void* p = nullptr;
+    void* p = addr[dev].load(std::memory_order_acquire);
+    if (!p) {   // first call on this device (with it current): resolve the address
         if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
             *status = EFLA_ERR_CUDA;
             return nullptr;
         }
-        addr[dev] = p;
+        addr[dev].store(p, std::memory_order_release);
     }
-    return addr[dev];
+    return p;
 }
 
 int efla_chunk_fwd_noalloc(const void* q, const void* k, const void* v, const void* beta,
@@ -150,6 +162,13 @@ int efla_chunk_fwd_noalloc(const void* q, const void* k, const void* v, const vo
     // the scratch keeps the previous call's contents: the device error word starts at zero
     if (cudaMemsetAsync(ws, 0, 16, (cudaStream_t)stream) != cudaSuccess) return EFLA_ERR_CUDA;
     return efla_chunk_fwd(q, k, v, beta, S0, o, S_T, B, H, T, d_k, d_v, chunk, dtype, ws, need, stream);
+}
+
+int efla_noalloc_status(int clear, efla_stream_t stream) {
+    int st = EFLA_OK;
+    void* ws = noalloc_scratch(&st);
+    if (!ws) return st;
+    return efla_workspace_status(ws, clear, stream);
 }
 
 int efla_workspace_status(void* workspace, int clear, efla_stream_t stream) {
@@ -254,6 +273,10 @@ int efla_backward_ex(const void* q, const void* k, const void* v, const void* be
         for (int j = i + 1; j < 5; ++j)
             if (overlaps(outs[i], outn[i], outs[j], outn[j])) return EFLA_ERR_INVALID_ARG;
     }
+    // the forward sweep writes its residuals into the workspace before the reverse sweep
+    // reads the inputs: no input may share bytes with it
+    for (int j = 0; j < 7; ++j)
+        if (overlaps(workspace, workspace_bytes, ins[j], inn[j])) return EFLA_ERR_INVALID_ARG;
     return from_cuda(efla::launch_bwd(q, k, v, beta, S0, dO, dS_T, dq, dk, dv, dbeta, dS0, BH, T, d_k,
                                       dtype == EFLA_DTYPE_BF16, rule, workspace, s));
 }

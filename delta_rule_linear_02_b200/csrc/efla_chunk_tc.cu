@@ -49,10 +49,6 @@
 // hand-off passes a named barrier.
 // Every wait is bounded (2 s); a wait that runs out sets a CTA-wide abort flag, every
 // role winds down, and the caller's workspace records the timeout.
-// Built with EFLA_CHUNK_TRACE=1 (never in the library), `dbg` receives, per chunk c < 64,
-// the cycle at which each role of CTA 0 passed its milestones, at
-// [40000 + 16 c + k): k = 0 QK^T, 1 [W|U], 2 [W;Q]S, 3 K^T Delta issued; 4 P ready;
-// 5 Q ready; 6 W ready; 7 U taken; 8 Delta ready; 9 new S ready; 10 O stored; 11 TMA.
 #include <cudaTypedefs.h>
 
 #include "efla_common.cuh"
@@ -61,13 +57,6 @@
 #include "sm100.cuh"
 
 namespace efla {
-
-#ifndef EFLA_CHUNK_TRACE
-#define EFLA_CHUNK_TRACE 0
-#endif
-// diagnosis stores compiled in only for tracing builds (milestone cycles): they cost
-// instruction-cache space in the role loops even when never taken
-constexpr bool kTrace = EFLA_CHUNK_TRACE >= 1;
 
 namespace {
 using namespace sm100;
@@ -221,7 +210,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_t,
                 const float* __restrict__ S0, __nv_bfloat16* __restrict__ o, float* __restrict__ S_T,
-                int T, uint32_t* __restrict__ err, unsigned long long limit_ns, float* __restrict__ dbg) {
+                int T, uint32_t* __restrict__ err, unsigned long long limit_ns) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sb = smem_u32(sm);
@@ -235,11 +224,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const int col0 = (blockIdx.x & 1) * 64;
     const int nchunks = (T + 63) / 64;
     const size_t tok0 = (size_t)bh * T;
-    const long long t_start = clock64();
-#define EFLA_STAMP(c, k)                                                                  \
-    do {                                                                                  \
-        if (kTrace && dbg && blockIdx.x == 0 && (c) < 64) dbg[40000 + 16 * (c) + (k)] = (float)(clock64() - t_start); \
-    } while (0)
 
     if (tid == 0) {
         for (int i = 0; i < (int)NBAR; ++i) mbar_init(ctl.bar + i, bar_count(i));
@@ -290,7 +274,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     tma_load_3d(st + TILE, &tm_q, full, 64, t0, bh);
                     q_issued = c + 1;
                 }
-                EFLA_STAMP(c, 11);
                 if (c + 3 < nchunks) {      // warm L2 for the chunk three ahead
                     const int t3 = t0 + 192;
                     tma_prefetch_l2_3d(&tm_k, 0, t3, bh);
@@ -320,7 +303,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                                   ID_GP, ks > 0);
             if (k1 == 8) {
                 mma_commit_elect(ctl.b(B_GP_FULL));
-                EFLA_STAMP(c, 0);
             }
         };
         auto issue_wu = [&](int c) {      // [W | U] = [T; *] [K | V]
@@ -328,7 +310,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             const uint32_t st = sb + kvt(c);
             mma_ss(tmem + TM_WU, st + KVT_T, TILE, 32, 16, st + KVT_K, 4 * 2048, 2048, TILE, ID_WU, 4, 0);
             mma_commit_elect(ctl.b(B_WU_FULL));
-            EFLA_STAMP(c, 1);
         };
         bool ok = wait(B_KVT_FULL, 0);
         if (ok) issue_wu(0);
@@ -340,7 +321,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             tc_fence_after();
             mma_ts(tmem + TM_X, tmem + TM_AWQ, sb + OFF_SB, 4 * 2048, 2048, TILE, ID_N64, 8, 0);
             mma_commit_elect(ctl.b(B_XS_FULL));
-            EFLA_STAMP(c, 2);
             // this chunk's Q K^T (its Q has been in place since the last chunk) and the next
             // chunk's [W | U] fill the pipe while Delta is formed; after K^T Delta only
             // P Delta remains ahead of the next [W;Q] S
@@ -358,7 +338,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                    4, 1);
             mma_commit_elect(ctl.b(B_S_FULL));
             mma_commit_elect(ctl.b(B_KVT_FREE + c % kKvtStages));
-            EFLA_STAMP(c, 3);
             // X += [*; P] Delta: rows 64-127 become O = Q S + P Delta
             if (!(ok = wait(B_P_READY, c & 1))) break;
             tc_fence_after();
@@ -389,7 +368,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             tc_fence_before();
             ctl.warp_arrive(B_WU_FREE, lane);
             ctl.warp_arrive(B_W_READY, lane);
-            if (warp == 4 && lane == 0) EFLA_STAMP(c, 6);
         }
     } else if (warp < 4) {
         // ================================================================ Q and P -> A operands (quarters 2-3)
@@ -410,7 +388,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             tmem_wait_st();
             tc_fence_before();
             ctl.warp_arrive(B_Q_READY, lane);
-            if (warp == 2 && lane == 0) EFLA_STAMP(c, 5);
         };
         // O(c) = X rows 64-127 once P Delta(c) has landed: taken into registers, X released
         // at once for [W;Q] S(c+1), then stored to global as bf16 (rows past T skipped)
@@ -421,7 +398,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             tmem_ld64_wait(tmem + lane_off + TM_X, t);
             tc_fence_before();
             ctl.warp_arrive(B_X_FREE, lane);
-            if (warp == 2 && lane == 0) EFLA_STAMP(c, 10);
             const int t0 = c * 64;
             if (r < min(64, T - t0)) {
                 uint4* dst = reinterpret_cast<uint4*>(o + (tok0 + t0 + r) * kD + col0);
@@ -475,7 +451,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             tc_fence_before();
             ctl.warp_arrive(B_GP_FREE, lane);
             ctl.warp_arrive(B_P_READY, lane);
-            if (warp == 2 && lane == 0) EFLA_STAMP(c, 4);
             // Q(c+1) -> A rows 64-127, once [W;Q] S(c) no longer reads them
             if (c + 1 < nchunks) {
                 ok = ctl.wwait(B_Q_FULL + (c + 1) % kQStages, ((c + 1) / kQStages) & 1) && ctl.wwait(B_XS_FULL, c & 1);
@@ -522,7 +497,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 tmem_ld32_wait(tmem + lane_off + TM_WU + 128 + cc, u);
                 tc_fence_before();
                 ctl.warp_arrive(B_WU_FREE, lane);
-                if (warp == 8 && lane == 0) EFLA_STAMP(c, 7);
                 // Delta = U - W S (X rows 0-63)
                 if (!(ok = ctl.wwait(B_XS_FULL, c & 1))) break;
                 tc_fence_after();
@@ -535,7 +509,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 fence_proxy_async_smem();
                 tc_fence_before();
                 ctl.warp_arrive(B_D_READY, lane);
-                if (warp == 8 && lane == 0) EFLA_STAMP(c, 8);
             }
             // the new state: bf16 operand for the next chunk (and S_T after the last)
             if (!(ok = ctl.wwait(B_S_FULL, c & 1))) break;
@@ -555,7 +528,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             fence_proxy_async_smem();
             tc_fence_before();
             ctl.warp_arrive(B_SB_READY, lane);
-            if (warp == 6 && lane == 0) EFLA_STAMP(c, 9);
         }
     }
 
@@ -564,7 +536,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     __syncthreads();
     if (tid == 0 && *ctl.abort) atomicOr(err, kDevTimeout);
     if (warp == 0) tmem_dealloc(tmem, TM_COLS);
-#undef EFLA_STAMP
 }
 
 // A wait on an mbarrier that nothing arrives on: exercises the bounded wait and the
@@ -582,11 +553,6 @@ __global__ void wait_timeout_selftest_kernel(uint32_t* err, unsigned long long l
 }  // namespace
 
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;   // 2 s per wait
-
-#if EFLA_CHUNK_TRACE
-// tracing builds only: the diagnosis record of CTA 0
-__device__ float g_chunk_dbg[40000 + 64 * 16];
-#endif
 
 size_t chunk_tc_workspace_bytes(long BH, int T) {
     const long nchunks = (T + 63) / 64;
@@ -606,12 +572,8 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const v
     static std::atomic<uint64_t> smem_set{0};
     e = set_smem_limit_once(chunk_tc_kernel, (int)SMEM_BYTES, smem_set);
     if (e != cudaSuccess) return e;
-    float* dbg = nullptr;
-#if EFLA_CHUNK_TRACE
-    if (cudaGetSymbolAddress((void**)&dbg, g_chunk_dbg) != cudaSuccess) dbg = nullptr;
-#endif
     chunk_tc_kernel<<<(unsigned)(BH * 2), kThreads, SMEM_BYTES, stream>>>(mq, mk, mv, mt, S0, (__nv_bfloat16*)o,
-                                                                          S_T, T, err, kWaitLimitNs, dbg);
+                                                                          S_T, T, err, kWaitLimitNs);
     return cudaGetLastError();
 }
 
@@ -621,11 +583,3 @@ cudaError_t launch_wait_timeout_selftest(uint32_t* err, unsigned long long limit
 }
 
 }  // namespace efla
-
-#if EFLA_CHUNK_TRACE
-// tracing builds only: copy CTA 0's milestone cycles (16 per chunk, chunks 0-63) to the host
-extern "C" int efla_chunk_trace_copy(float* host, int n) {
-    return (int)cudaMemcpyFromSymbol(host, efla::g_chunk_dbg, sizeof(float) * (size_t)std::min(n, 64 * 16),
-                                     sizeof(float) * 40000);
-}
-#endif

@@ -17,9 +17,13 @@
  *   - Tensors are contiguous, row-major, head-major: q, k [B, H, T, d_k]; v, o [B, H, T, d_v];
  *     beta [B, H, T]; states [B, H, d_k, d_v] float32.
  *   - q, k, v, beta and o share one element type (efla_dtype); states are always float32.
- *   - All data pointers are DEVICE pointers owned by the caller.  The library keeps no
- *     global state and never allocates: calls on different streams may run concurrently
- *     as long as their buffers do not overlap.
+ *   - All data pointers are DEVICE pointers owned by the caller.  The library calls no
+ *     allocator.  Its only global state is per-device host-side caches (SM count, kernel
+ *     attributes, the scratch address below) and one 32 MiB static device array, the
+ *     scratch of efla_chunk_fwd_noalloc, shared by every call of that entry point (calls
+ *     that overlap on the GPU race on it).  Every other entry point works only on the
+ *     caller's buffers: calls on different streams may run concurrently as long as their
+ *     buffers (workspaces included) do not overlap.
  *   - Every pointer must be 16-byte aligned.
  *   - Calls are asynchronous on `stream` (NULL: the legacy default stream) and never
  *     synchronise the host.  A non-OK status from argument checking means nothing was
@@ -92,7 +96,7 @@ size_t efla_chunk_fwd_workspace_bytes(int B, int H, int T, int d_k, int d_v, int
  *   S0   [B,H,d_k,d_v] float32 or NULL (zero initial state)
  *   o    [B,H,T,d_v]  output, `dtype`
  *   S_T  [B,H,d_k,d_v] float32 final state, or NULL (not written).  S_T may alias S0.
- *   o must not overlap any input.
+ *   o must not overlap any input.  No input, output or state may overlap the workspace.
  *   workspace: device memory of at least efla_chunk_fwd_workspace_bytes(...) bytes,
  *   16-byte aligned, owned by the caller; its first bytes hold a sticky device error word
  *   (zero it once before first use, e.g. with cudaMemset).  For bf16 with d = 128 it also
@@ -137,12 +141,21 @@ int efla_chunk_fwd_ex(const void *q, const void *k, const void *v, const void *b
  * current); make that first call before any stream capture.  Every call shares the one
  * array and each call clears its error word first, so calls that overlap on the GPU
  * (different streams, or different host threads) race on it and must be serialised by
- * the caller.  A device-side wait timeout in this variant is recorded only in the
- * internal scratch and is not reported to the caller.
+ * the caller.  A device-side wait timeout in this variant is recorded in the scratch's
+ * error word; efla_noalloc_status reads it back (each call clears it first).
  */
 int efla_chunk_fwd_noalloc(const void *q, const void *k, const void *v, const void *beta,
                            const float *S0, void *o, float *S_T, int B, int H, int T, int d_k,
                            int d_v, int chunk, int dtype, efla_stream_t stream);
+
+/*
+ * efla_noalloc_status -- efla_workspace_status for the static scratch of
+ * efla_chunk_fwd_noalloc on the current device: waits for `stream`, then returns
+ * EFLA_ERR_TIMEOUT if the last efla_chunk_fwd_noalloc call on this device gave up on a
+ * device wait (its outputs are then invalid), else EFLA_OK.  clear != 0 resets the word.
+ * Like efla_chunk_fwd_noalloc, it has no counterpart in the paper.
+ */
+int efla_noalloc_status(int clear, efla_stream_t stream);
 
 /*
  * efla_workspace_status -- waits for `stream`, then returns EFLA_ERR_TIMEOUT if any
@@ -210,7 +223,8 @@ size_t efla_backward_workspace_bytes(int B, int H, int T, int d_k, int d_v, int 
  *
  * Supported: d_k = d_v in {64, 128}; dtype f32 or bf16; any T >= 0 (T = 0 copies dS_T
  * into dS0).  All pointers 16-byte aligned; no output may overlap an input, the
- * workspace or another output; else EFLA_ERR_INVALID_ARG and nothing is launched.  The
+ * workspace or another output, and no input may overlap the workspace; else
+ * EFLA_ERR_INVALID_ARG and nothing is launched.  The
  * state is fp32 throughout; the outputs are accumulated in fp32 (the row sums over d_v
  * columns with atomics, so their last bits depend on arrival order).  Asynchronous on
  * `stream`; launch failures return EFLA_ERR_CUDA.

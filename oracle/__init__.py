@@ -47,8 +47,6 @@ def load(path: Optional[str] = None):
     L, I = ctypes.c_long, ctypes.c_int
     lib.efla_oracle_alpha.argtypes = [ctypes.c_double, ctypes.c_double]
     lib.efla_oracle_alpha.restype = ctypes.c_double
-    lib.efla_oracle_gate.argtypes = [dp, dp, dp, L, L, I]
-    lib.efla_oracle_gate.restype = None
     lib.efla_oracle_fwd.argtypes = [dp, dp, dp, dp, dp, dp, dp, L, L, L, L, L, I, I]
     lib.efla_oracle_fwd.restype = I
     lib.efla_oracle_step.argtypes = [dp, dp, dp, dp, dp, dp, L, L, L, L, I, I]
@@ -87,17 +85,6 @@ def default_threads() -> int:
 
 def alpha(beta: float, lam: float, lib=None) -> float:
     return (lib or load()).efla_oracle_alpha(float(beta), float(lam))
-
-
-def gate(k, beta, mode: int = EXACT, lib=None) -> np.ndarray:
-    """alpha_t for keys k [..., dk] and gates beta [...]."""
-    k, beta = _f64(k), _f64(beta)
-    dk = k.shape[-1]
-    n = int(np.prod(k.shape[:-1]))
-    assert beta.size == n
-    out = np.empty(beta.shape, dtype=np.float64)
-    (lib or load()).efla_oracle_gate(_ptr(k), _ptr(beta), _ptr(out), n, dk, mode)
-    return out
 
 
 def fwd(q, k, v, beta, S0=None, mode: int = EXACT, threads: Optional[int] = None, lib=None,

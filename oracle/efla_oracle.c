@@ -61,18 +61,6 @@ double efla_oracle_alpha(double beta, double lambda)
     return -expm1(-beta * lambda) / lambda;
 }
 
-/* alpha_t for n tokens: k is [n, dk], beta is [n]. */
-void efla_oracle_gate(const double *k, const double *beta, double *alpha, long n, long dk,
-                      int mode)
-{
-    for (long t = 0; t < n; ++t) {
-        double lam = 0.0;
-        for (long i = 0; i < dk; ++i)
-            lam += k[t * dk + i] * k[t * dk + i];
-        alpha[t] = (mode == EFLA_ORACLE_EULER) ? beta[t] : efla_oracle_alpha(beta[t], lam);
-    }
-}
-
 /* One recurrence over T tokens of one (b, h) stream.  S (dk x dv) is updated in place;
  * r is scratch of dv doubles.  o may be NULL. */
 static void run_stream(const double *q, const double *k, const double *v, const double *beta,

@@ -1,6 +1,7 @@
 """bench.py's host-side arithmetic (CPU only): the algorithmic bytes and flops the roofline
-fractions divide by, the fp32 ALU peak, and the traffic lookup keyed on kernel sources."""
-import os
+fractions divide by, the bound each record picks, and the traffic record written from an
+ncu CSV and keyed on kernel sources."""
+import json
 
 import bench
 import workloads
@@ -28,27 +29,52 @@ def test_decode_and_backward_algorithmic_counts():
     token_heads = 4 * 16 * 2048
     # read q, k, v, dO (bf16) and beta; write dq, dk, dv (fp32) and dbeta; dS0 per head
     assert bbytes == token_heads * (4 * 128 * 2 + 2 + 3 * 128 * 4 + 4) + 64 * 128 * 128 * 4
-    assert bflops == token_heads * 18 * 128 * 128
+    # the chunked form: three times the forward's chunk products
+    assert bflops == 3 * bench.chunk_alg(W["lm1p3b_bf16"])[1]
 
 
-def test_fp32_alu_peak():
-    assert abs(bench.fp32_alu_peak_tflops() - 148 * 128 * 2 * 1.965e9 / 1e12) < 1e-9
+def test_roofline_record_picks_the_slower_bound():
+    hbm, tc = 6545.9, 1646.8
+    r = bench.roofline_record(138_674_176, 23_622_320_128, 100e-6, hbm, tc, "measured")
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s"
+    assert abs(r["frac"] - 138_674_176 / (hbm * 1e9) / 100e-6) < 1e-12
+    assert abs(r["achieved"] / r["peak"] - r["frac"]) < 1e-12
+    r = bench.roofline_record(1_000, 1e12, 1e-3, hbm, tc, "measured")
+    assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
+    assert abs(r["achieved"] / r["peak"] - r["frac"]) < 1e-12
 
 
-def test_traffic_lookup_follows_the_entry_points_sources(tmp_path, monkeypatch):
+CSV = """==PROF== Connected to process 1
+"ID","Process ID","Process Name","Host Name","Kernel Name","Context","Stream","Block Size","Grid Size","Device","CC","Section Name","Metric Name","Metric Unit","Metric Value"
+"0","1","python","h","(anonymous namespace)::ut_kernel(CUtensorMap_st, bf16)","1","7","(160, 1, 1)","(888, 1, 1)","0","10.0","Command line profiler metrics","dram__bytes_read.sum","byte","1,000"
+"0","1","python","h","(anonymous namespace)::ut_kernel(CUtensorMap_st, bf16)","1","7","(160, 1, 1)","(888, 1, 1)","0","10.0","Command line profiler metrics","dram__bytes_write.sum","byte","10"
+"1","1","python","h","unnamed>::chunk_tc_kernel(CUtensorMap_st)","1","7","(448, 1, 1)","(128, 1, 1)","0","10.0","Command line profiler metrics","dram__bytes_read.sum","Kbyte","2"
+"1","1","python","h","unnamed>::chunk_tc_kernel(CUtensorMap_st)","1","7","(448, 1, 1)","(128, 1, 1)","0","10.0","Command line profiler metrics","dram__bytes_write.sum","byte","300"
+"2","1","python","h","(anonymous namespace)::ut_kernel(CUtensorMap_st, bf16)","1","7","(160, 1, 1)","(888, 1, 1)","0","10.0","Command line profiler metrics","dram__bytes_read.sum","byte","5,000"
+"2","1","python","h","(anonymous namespace)::ut_kernel(CUtensorMap_st, bf16)","1","7","(160, 1, 1)","(888, 1, 1)","0","10.0","Command line profiler metrics","dram__bytes_write.sum","byte","50"
+"3","1","python","h","unnamed>::chunk_tc_kernel(CUtensorMap_st)","1","7","(448, 1, 1)","(128, 1, 1)","0","10.0","Command line profiler metrics","dram__bytes_read.sum","byte","7,000"
+"3","1","python","h","unnamed>::chunk_tc_kernel(CUtensorMap_st)","1","7","(448, 1, 1)","(128, 1, 1)","0","10.0","Command line profiler metrics","dram__bytes_write.sum","byte","700"
+"""
+
+
+def test_traffic_record_is_written_from_the_ncu_csv_and_follows_the_sources(tmp_path, monkeypatch):
     h_fwd = bench.kernel_source_hash("efla_chunk_fwd")
     h_dec = bench.kernel_source_hash("efla_recurrent_step")
     assert h_fwd != h_dec and len(h_fwd) == 16
-    prof = tmp_path / "profiles"
-    prof.mkdir()
-    (prof / "traffic.md").write_text(
-        f"traffic|efla_chunk_fwd|111|{h_fwd}\ntraffic|efla_recurrent_step|222|0000000000000000\n")
-    csrc = os.path.join(bench.ROOT, "delta_rule_linear_02_b200")
-    os.symlink(csrc, tmp_path / "delta_rule_linear_02_b200")
-    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
-    assert bench.ncu_traffic("efla_chunk_fwd") == 111
-    assert bench.ncu_traffic("efla_recurrent_step") is None      # recorded for other sources
-    assert bench.ncu_traffic("efla_backward") is None            # not recorded
+    csv = tmp_path / "dram.csv"
+    csv.write_text(CSV)
+    monkeypatch.setattr(bench, "TRAFFIC_JSON", str(tmp_path / "traffic.json"))
+    rec = bench.traffic_from_csv(str(csv), "efla_chunk_fwd", calls=1)     # the last call only
+    assert rec["bytes_per_call"] == 5_000 + 50 + 7_000 + 700 and rec["launches"] == 2
+    rec = bench.traffic_from_csv(str(csv), "efla_chunk_fwd", calls=2)     # both calls, averaged
+    assert rec["bytes_per_call"] == (1_010 + 2_300 + 5_050 + 7_700) // 2
+    assert bench.ncu_traffic("efla_chunk_fwd") == rec["bytes_per_call"]
+    assert bench.ncu_traffic("efla_backward") is None                    # not recorded
+    assert rec["kernels"] == ["chunk_tc_kernel", "ut_kernel"]
+    data = json.loads((tmp_path / "traffic.json").read_text())
+    data["efla_recurrent_step"] = dict(rec, kernel_source="0000000000000000")
+    (tmp_path / "traffic.json").write_text(json.dumps(data))
+    assert bench.ncu_traffic("efla_recurrent_step") is None              # recorded for other sources
 
 
 def test_cotangents_are_seeded():

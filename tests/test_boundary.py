@@ -75,6 +75,9 @@ def test_chunk_fwd_rejects_bad_arguments(efla):
     assert _fwd(L, GOOD, ws=8) == INVALID         # workspace too small
     bad = list(GOOD); bad[5] = GOOD[0]            # o aliases q
     assert _fwd(L, bad) == INVALID
+    for i in (0, 1, 2, 3, 4, 6):                  # no input or state may lie inside the workspace
+        bad = list(GOOD); bad[i] = ctypes.c_void_p(GOOD[7].value + 1024)
+        assert _fwd(L, bad, ws=1 << 20) == INVALID, i
     assert _fwd(L, GOOD, B=0) == OK               # nothing to do, nothing launched
     assert _fwd(L, GOOD, H=0) == OK
 
@@ -177,5 +180,8 @@ def test_backward_rejects_bad_arguments(efla):
     assert _bwd(L, bad) == INVALID
     bad = list(GOOD_B); bad[11] = GOOD_B[4]       # dS0 aliases S0
     assert _bwd(L, bad) == INVALID
+    for i in range(7):                            # no input may lie inside the workspace
+        bad = list(GOOD_B); bad[i] = ctypes.c_void_p(GOOD_B[12].value + 4096)
+        assert _bwd(L, bad) == INVALID, i
     assert _bwd(L, GOOD_B, B=0) == OK             # nothing to do, nothing launched
     assert _bwd(L, GOOD_B, H=0) == OK

@@ -11,7 +11,7 @@ import torch
 
 import oracle
 import workloads
-from helpers import TOL, oracle_streams, rel_frob
+from helpers import TOL, rel_frob
 
 pytestmark = pytest.mark.gpu
 
@@ -79,27 +79,45 @@ def test_chunk_fwd_small(efla, cuda, name, over):
     assert rel_frob(ST, ST_ref) <= tol, rel_frob(ST, ST_ref)
 
 
-FULL = [("tiny_fp32", None), ("lm1p3b_bf16", [(0, 0), (1, 7), (2, 3), (3, 15)]),
-        ("longctx_bf16", [(0, 0), (0, 11)]), ("stiff_bf16", [(0, 2), (1, 9), (1, 15)])]
+FULL = ["tiny_fp32", "lm1p3b_bf16", "longctx_bf16", "stiff_bf16"]
 
 
-@pytest.mark.parametrize("name,streams", FULL, ids=[f[0] for f in FULL])
-def test_chunk_fwd_full_size(efla, cuda, name, streams):
-    """The full workload in the bench's launch configuration; the oracle checks sampled streams."""
+def per_stream_errors(x, ref):
+    """Relative Frobenius error of every (b, h) stream: [B, H] float64."""
+    x = x.detach().double().cpu().numpy() if hasattr(x, "detach") else np.asarray(x, np.float64)
+    ref = np.asarray(ref, np.float64)
+    axes = tuple(range(2, ref.ndim))
+    num = np.sqrt(((x - ref) ** 2).sum(axis=axes))
+    den = np.sqrt((ref ** 2).sum(axis=axes))
+    return num / np.where(den > 0, den, 1.0)
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_chunk_fwd_full_size(efla, cuda, name):
+    """The full workload in the bench's launch configuration, every stream against the oracle:
+    whole-tensor error on o and S_T, and the worst single (b, h) stream."""
     w = W[name]
-    inp = workloads.make_chunk_inputs(w)
+    inp = workloads.make_chunk_inputs(w, with_mask=True)
     o, ST = run_fwd(efla, to_dev(inp, cuda))
     torch.cuda.synchronize()
     assert torch.isfinite(o.float()).all() and torch.isfinite(ST).all()
     tol = TOL[w.dtype]
-    if streams is None:
-        o_ref, ST_ref = oracle.fwd(inp["q"], inp["k"], inp["v"], inp["beta"], inp["S0"])
-        assert rel_frob(o, o_ref) <= tol and rel_frob(ST, ST_ref) <= tol
-        return
-    o_ref, ST_ref = oracle_streams(inp, streams)
-    for i, (b, h) in enumerate(streams):
-        eo, es = rel_frob(o[b, h], o_ref[i]), rel_frob(ST[b, h], ST_ref[i])
-        assert eo <= tol and es <= tol, ((b, h), eo, es)
+    o_ref, ST_ref = oracle.fwd(inp["q"], inp["k"], inp["v"], inp["beta"], inp["S0"])
+    eo, es = rel_frob(o, o_ref), rel_frob(ST, ST_ref)
+    po, ps = per_stream_errors(o, o_ref), per_stream_errors(ST, ST_ref)
+    print(f"{name}: o {eo:.3e} (worst stream {po.max():.3e}), S_T {es:.3e} (worst stream {ps.max():.3e})")
+    assert eo <= tol and es <= tol, (eo, es)
+    assert po.max() <= tol and ps.max() <= tol, (np.unravel_index(po.argmax(), po.shape), po.max(),
+                                                 np.unravel_index(ps.argmax(), ps.shape), ps.max())
+    bad = inp["corrupt"]
+    if bad.any():
+        # the high-energy tokens dominate ||o||_F: the clean tokens must also agree on their own
+        clean = ~bad.numpy()                                         # [B, T]
+        og = o.double().cpu().numpy().transpose(0, 2, 1, 3)[clean]   # [n_clean, H, dv]
+        orf = o_ref.transpose(0, 2, 1, 3)[clean]
+        ec = rel_frob(og, orf)
+        print(f"{name}: o over the {int(clean.sum())} clean (b, t) tokens {ec:.3e}")
+        assert ec <= tol, ec
 
 
 def test_state_carry_split_equals_single_run(efla, cuda):
@@ -196,31 +214,29 @@ def test_decode_small(efla, cuda, dtype, D):
     assert rel_frob(Sd, So) <= tol
 
 
-def test_decode_full_size_sampled(efla, cuda):
-    """1000 in-place steps at N=256, H=16, d=128; the oracle follows 24 sampled heads."""
+def test_decode_full_size(efla, cuda):
+    """1000 in-place steps at N=256, H=16, d=128; the oracle follows every head: o over all
+    1000 steps and the final state, whole-tensor relative Frobenius error."""
     w = workloads.DECODE_WORKLOAD
     S = workloads.make_decode_state(w, device=cuda)
+    S_o = S.double().cpu().numpy()                                  # oracle state, updated in place
     steps = workloads.make_decode_steps(w, device=cuda)
-    rng = np.random.default_rng(5)
-    heads = sorted({(int(a), int(b)) for a, b in zip(rng.integers(0, w.N, 24), rng.integers(0, w.H, 24))})
-    ni = torch.tensor([a for a, _ in heads], device=cuda)
-    hi = torch.tensor([b for _, b in heads], device=cuda)
-    S_ref = S[ni, hi].double().cpu().numpy()[None]                 # [1, n, dk, dv]
-    outs = []
+    outs = torch.empty((w.steps, w.N, w.H, w.dv), device=cuda, dtype=torch.float32)
     for s in range(w.steps):
-        o = efla.efla_recurrent_step(steps["q"][s], steps["k"][s], steps["v"][s], steps["beta"][s], S)
-        outs.append(o[ni, hi])
-    o_gpu = torch.stack(outs).cpu()                                  # [steps, n, dv]
-    sel = {k: v[:, ni, hi].cpu() for k, v in steps.items()}         # [steps, n, ...]
-    S_o = S_ref[0].copy()
-    orefs = []
+        efla.efla_recurrent_step(steps["q"][s], steps["k"][s], steps["v"][s], steps["beta"][s], S,
+                                 o=outs[s])
+    torch.cuda.synchronize()
+    err2 = ref2 = 0.0
     for s in range(w.steps):
-        oref, S_o = oracle.step(sel["q"][s][None], sel["k"][s][None], sel["v"][s][None],
-                                sel["beta"][s][None], S_o[None])
-        S_o = S_o[0]
-        orefs.append(oref[0])
-    assert rel_frob(o_gpu, np.stack(orefs)) <= 1e-4
-    assert rel_frob(S[ni, hi], S_o) <= 1e-4
+        oref, S_o = oracle.step(steps["q"][s].cpu(), steps["k"][s].cpu(), steps["v"][s].cpu(),
+                                steps["beta"][s].cpu(), S_o)
+        d = outs[s].double().cpu().numpy() - oref
+        err2 += float((d * d).sum())
+        ref2 += float((oref * oref).sum())
+    eo = math.sqrt(err2 / ref2)
+    es = rel_frob(S, S_o)
+    print(f"decode: o {eo:.3e}, S {es:.3e}")
+    assert eo <= 1e-4 and es <= 1e-4, (eo, es)
 
 
 # ------------------------------------------------------------------------------ failure detection

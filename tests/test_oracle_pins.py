@@ -11,21 +11,6 @@ def test_pin(pin, oracle_lib):
     pin(oracle_lib)
 
 
-def test_gate_vectorised_matches_scalar(oracle_lib):
-    rng = np.random.default_rng(7)
-    k = rng.standard_normal((33, 16)) * rng.uniform(0, 50, (33, 1))
-    k[3] = 0.0
-    beta = rng.uniform(0, 2, 33)
-    a = oracle.gate(k, beta, lib=oracle_lib)
-    for t in range(33):
-        lam = 0.0
-        for x in k[t]:          # same summation order as the oracle's loop
-            lam += x * x
-        assert a[t] == oracle.alpha(beta[t], lam, lib=oracle_lib)
-    assert a[3] == beta[3]
-    assert np.array_equal(oracle.gate(k, beta, mode=oracle.EULER, lib=oracle_lib), beta)
-
-
 def test_threads_do_not_change_results(oracle_lib):
     rng = np.random.default_rng(8)
     q, k = rng.standard_normal((2, 2, 2, 11, 6))

@@ -11,6 +11,7 @@ import ctypes
 import pytest
 import torch
 
+import oracle
 import workloads
 from helpers import TOL, rel_frob
 
@@ -24,8 +25,10 @@ CASES = [("lm1p3b_bf16", {"B": 1, "H": 3, "T": 333}),
 @pytest.mark.parametrize("name,over", CASES, ids=[c[0] for c in CASES])
 def test_noalloc_matches_workspace_entry_point_twice(efla, cuda, name, over):
     w = workloads.CHUNK_WORKLOADS[name].replace(**over)
-    d = {k: (None if v is None else v.to(cuda)) for k, v in workloads.make_chunk_inputs(w).items()}
+    inp = workloads.make_chunk_inputs(w)
+    d = {k: (None if v is None else v.to(cuda)) for k, v in inp.items()}
     o_ref, S_ref = efla.efla_chunk_fwd(d["q"], d["k"], d["v"], d["beta"], d["S0"])
+    o_orc, S_orc = oracle.fwd(inp["q"], inp["k"], inp["v"], inp["beta"], inp["S0"])
     tol = TOL[w.dtype]
     o = torch.empty_like(o_ref)
     S = torch.empty_like(S_ref)
@@ -34,7 +37,10 @@ def test_noalloc_matches_workspace_entry_point_twice(efla, cuda, name, over):
         S.fill_(float("nan"))
         efla.efla_chunk_fwd_noalloc(d["q"], d["k"], d["v"], d["beta"], d["S0"], o=o, S_T=S)
         torch.cuda.synchronize()
+        assert efla.efla_noalloc_status() == efla.EFLA_OK
         assert rel_frob(o, o_ref) <= tol and rel_frob(S, S_ref) <= tol
+        # and against the fp64 oracle directly, not only against the other CUDA entry point
+        assert rel_frob(o, o_orc) <= tol and rel_frob(S, S_orc) <= tol
 
 
 def test_noalloc_rejects_bad_arguments(efla, cuda):

@@ -84,10 +84,12 @@ def _unit_rows(x: torch.Tensor) -> torch.Tensor:
     return x / x.norm(dim=-1, keepdim=True)
 
 
-def make_chunk_inputs(w: ChunkWorkload) -> dict:
+def make_chunk_inputs(w: ChunkWorkload, with_mask: bool = False) -> dict:
     """Draw q, k, v, beta (in w.dtype) and S0 (float32 or None) on the CPU.
 
-    The draw order is fixed, so the same workload always gives the same tensors.
+    The draw order is fixed, so the same workload always gives the same tensors.  With
+    with_mask, the dict also holds "corrupt" [B, T] bool: the (b, t) tokens replaced by
+    high-energy noise (the "stiff" distribution; all False for the others).
     """
     g = torch.Generator().manual_seed(w.seed)
     B, H, T, dk, dv = w.B, w.H, w.T, w.dk, w.dv
@@ -121,16 +123,21 @@ def make_chunk_inputs(w: ChunkWorkload) -> dict:
         v = torch.where(corrupt, cv, v)
     else:
         raise ValueError(f"unknown distribution {w.dist!r}")
+    if w.dist != "stiff":
+        corrupt = torch.zeros(B, 1, T, 1, dtype=torch.bool)
     S0 = None
     if w.s0_std is not None:
         S0 = w.s0_std * torch.randn(B, H, dk, dv, generator=g, dtype=f32)
-    return {
+    out = {
         "q": q.to(w.dtype).contiguous(),
         "k": k.to(w.dtype).contiguous(),
         "v": v.to(w.dtype).contiguous(),
         "beta": beta.to(w.dtype).contiguous(),
         "S0": S0,
     }
+    if with_mask:
+        out["corrupt"] = corrupt[:, 0, :, 0].clone()
+    return out
 
 
 def make_decode_state(w: DecodeWorkload, device="cpu") -> torch.Tensor:
