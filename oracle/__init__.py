@@ -51,6 +51,10 @@ def load(path: Optional[str] = None):
     lib.efla_oracle_fwd.restype = I
     lib.efla_oracle_step.argtypes = [dp, dp, dp, dp, dp, dp, L, L, L, L, I, I]
     lib.efla_oracle_step.restype = I
+    lib.efla_oracle_fwd_gated.argtypes = [dp] * 8 + [L, L, L, L, L, I, I]
+    lib.efla_oracle_fwd_gated.restype = I
+    lib.efla_oracle_step_gated.argtypes = [dp] * 7 + [L, L, L, L, I, I]
+    lib.efla_oracle_step_gated.restype = I
     lib.efla_oracle_dalpha_dlambda.argtypes = [ctypes.c_double, ctypes.c_double]
     lib.efla_oracle_dalpha_dlambda.restype = ctypes.c_double
     lib.efla_oracle_bwd.argtypes = [dp] * 12 + [L, L, L, L, L, I, I]
@@ -124,6 +128,40 @@ def step(q, k, v, beta, S, mode: int = EXACT, threads: Optional[int] = None, lib
     rc = (lib or load()).efla_oracle_step(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(S),
                                           _ptr(o), N, H, dk, dv, mode,
                                           threads or default_threads())
+    if rc != 0:
+        raise MemoryError("oracle could not allocate its per-stream state")
+    return o, S
+
+
+def fwd_gated(q, k, v, beta, g, S0=None, mode: int = EXACT, threads: Optional[int] = None, lib=None,
+              want_o: bool = True):
+    """Gated forward (per-token log-decay g [B,H,T]); otherwise as fwd."""
+    q, k, v, beta, g, S0 = _f64(q), _f64(k), _f64(v), _f64(beta), _f64(g), _f64(S0)
+    B, H, T, dk = k.shape
+    dv = v.shape[-1]
+    assert q.shape == k.shape and v.shape[:3] == (B, H, T) and beta.shape == (B, H, T) and g.shape == (B, H, T)
+    if S0 is not None:
+        assert S0.shape == (B, H, dk, dv)
+    o = np.empty((B, H, T, dv), dtype=np.float64) if want_o else None
+    ST = np.empty((B, H, dk, dv), dtype=np.float64)
+    rc = (lib or load()).efla_oracle_fwd_gated(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), _ptr(S0),
+                                               _ptr(o), _ptr(ST), B, H, T, dk, dv, mode,
+                                               threads or default_threads())
+    if rc != 0:
+        raise MemoryError("oracle could not allocate its per-stream state")
+    return o, ST
+
+
+def step_gated(q, k, v, beta, g, S, mode: int = EXACT, threads: Optional[int] = None, lib=None):
+    """One gated decode step (g [N,H]); otherwise as step."""
+    q, k, v, beta, g = _f64(q), _f64(k), _f64(v), _f64(beta), _f64(g)
+    if not (isinstance(S, np.ndarray) and S.dtype == np.float64 and S.flags.c_contiguous):
+        S = _f64(S).copy()
+    N, H, dk = k.shape
+    dv = v.shape[-1]
+    o = np.empty((N, H, dv), dtype=np.float64)
+    rc = (lib or load()).efla_oracle_step_gated(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), _ptr(S),
+                                                _ptr(o), N, H, dk, dv, mode, threads or default_threads())
     if rc != 0:
         raise MemoryError("oracle could not allocate its per-stream state")
     return o, S

@@ -43,6 +43,22 @@
  *   dalpha/dbeta = e^{-beta lambda},   dalpha/dlambda = (beta e^{-beta lambda} - alpha)/lambda,
  * the latter by its Taylor series in x = beta lambda when x is small (its limit at lambda = 0
  * is -beta^2/2).  Euler mode: dalpha/dbeta = 1, dalpha/dlambda = 0.
+ *
+ * efla_oracle_fwd_gated is the gated variant (Section 3.4 says the method carries over to
+ * gated recurrences as "Gated EFLA"; App. F, the exact-flow form of Gated DeltaNet, survives
+ * only as a title, so the formula below is this oracle's own reading).  Each token adds a
+ * forget gate, a per-token log-decay g_t (g <= 0 decays), to the same zero-order-hold ODE,
+ * held constant over the token's unit interval together with the write rate beta_t:
+ *   dS/dtau = g S - beta (k k^T S - k v^T),   tau in [0, 1].
+ * Its generator g I - beta k k^T has the eigenvalue g - beta*lambda along k and g on the
+ * orthogonal complement, so e^{g I - beta k k^T} = e^g (I - alpha k k^T) with the same alpha
+ * as above, and the input integral int_0^1 e^{(1-tau)(g - beta lambda)} d tau * beta k v^T
+ * collapses to abar k v^T.  With phi1(x) = (1 - e^{-x}) / x (phi1(0) = 1):
+ *   alpha_t = beta_t phi1(beta_t lambda_t),   abar_t = beta_t phi1(beta_t lambda_t - g_t),
+ *   S_t = e^{g_t} (S_{t-1} - alpha_t k_t (k_t^T S_{t-1})) + abar_t k_t v_t^T,   o_t = S_t^T q_t.
+ * g = 0 gives the exact flow above.  Euler mode here is the gated delta rule (Gated
+ * DeltaNet): alpha = abar = beta, i.e. the exact decay followed by one Euler step of the
+ * delta-rule write.
  */
 #include <math.h>
 #include <stddef.h>
@@ -133,6 +149,81 @@ int efla_oracle_fwd(const double *q, const double *k, const double *v, const dou
     return failed ? -1 : 0;
 }
 
+/* phi1(x) = (1 - e^{-x}) / x, exact to rounding for small |x| through expm1; phi1(0) = 1. */
+static double phi1(double x)
+{
+    if (x == 0.0)
+        return 1.0;
+    return -expm1(-x) / x;
+}
+
+/* The gated recurrence over T tokens of one stream; g is the per-token log-decay. */
+static void run_stream_gated(const double *q, const double *k, const double *v, const double *beta,
+                             const double *g, double *S, double *o, double *m, long T, long dk,
+                             long dv, int mode)
+{
+    for (long t = 0; t < T; ++t) {
+        const double *key = k + t * dk, *query = q + t * dk, *value = v + t * dv;
+        double lambda = 0.0;
+        for (long i = 0; i < dk; ++i)
+            lambda += key[i] * key[i];
+        double a = beta[t], ab = beta[t];
+        if (mode != EFLA_ORACLE_EULER) {
+            a = efla_oracle_alpha(beta[t], lambda);
+            ab = beta[t] * phi1(beta[t] * lambda - g[t]);
+        }
+        const double dec = exp(g[t]);
+        /* m = S^T k : what the memory returns for this key */
+        for (long j = 0; j < dv; ++j)
+            m[j] = 0.0;
+        for (long i = 0; i < dk; ++i)
+            for (long j = 0; j < dv; ++j)
+                m[j] += S[i * dv + j] * key[i];
+        /* S <- e^g (S - a k m^T) + ab k v^T */
+        for (long i = 0; i < dk; ++i)
+            for (long j = 0; j < dv; ++j)
+                S[i * dv + j] = dec * (S[i * dv + j] - a * key[i] * m[j]) + ab * key[i] * value[j];
+        if (o) {
+            double *out = o + t * dv;
+            for (long j = 0; j < dv; ++j)
+                out[j] = 0.0;
+            for (long i = 0; i < dk; ++i)
+                for (long j = 0; j < dv; ++j)
+                    out[j] += S[i * dv + j] * query[i];
+        }
+    }
+}
+
+/* Gated forward: as efla_oracle_fwd, plus g [B, H, T], the per-token log-decay. */
+int efla_oracle_fwd_gated(const double *q, const double *k, const double *v, const double *beta,
+                          const double *g, const double *S0, double *o, double *S_T, long B, long H,
+                          long T, long dk, long dv, int mode, int nthreads)
+{
+    const long BH = B * H;
+    int failed = 0;
+    if (nthreads < 1)
+        nthreads = 1;
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads) reduction(| : failed)
+    for (long bh = 0; bh < BH; ++bh) {
+        double *S = (double *)malloc((size_t)(dk * dv + dv) * sizeof(double));
+        if (!S) {
+            failed |= 1;
+            continue;
+        }
+        double *r = S + dk * dv;
+        if (S0 == NULL)
+            memset(S, 0, (size_t)(dk * dv) * sizeof(double));
+        else
+            memcpy(S, S0 + bh * dk * dv, (size_t)(dk * dv) * sizeof(double));
+        run_stream_gated(q + bh * T * dk, k + bh * T * dk, v + bh * T * dv, beta + bh * T, g + bh * T, S,
+                         o ? o + bh * T * dv : NULL, r, T, dk, dv, mode);
+        if (S_T)
+            memcpy(S_T + bh * dk * dv, S, (size_t)(dk * dv) * sizeof(double));
+        free(S);
+    }
+    return failed ? -1 : 0;
+}
+
 /*
  * One decode step for N*H streams: the recurrence of efla_oracle_fwd with T = 1.
  *   q, k : [N, H, dk]   v : [N, H, dv]   beta : [N, H]   S : [N, H, dk, dv] in/out
@@ -143,6 +234,14 @@ int efla_oracle_step(const double *q, const double *k, const double *v, const do
                      int nthreads)
 {
     return efla_oracle_fwd(q, k, v, beta, S, o, S, N, H, 1, dk, dv, mode, nthreads);
+}
+
+/* One gated decode step (efla_oracle_fwd_gated with T = 1); g is [N, H]. */
+int efla_oracle_step_gated(const double *q, const double *k, const double *v, const double *beta,
+                           const double *g, double *S, double *o, long N, long H, long dk, long dv,
+                           int mode, int nthreads)
+{
+    return efla_oracle_fwd_gated(q, k, v, beta, g, S, o, S, N, H, 1, dk, dv, mode, nthreads);
 }
 
 /* d alpha / d lambda of the exact gate.  For x = beta*lambda < 1e-3 the difference
