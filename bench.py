@@ -590,15 +590,23 @@ def main():
     # ---- the other forward workloads (long context, stiff keys): tokens/s and roofline
     # fraction of a few forwards each, inputs resident in HBM, CUDA events around the calls
     others = {}
-    for name in ([] if args.other_steps <= 0 else ["longctx_bf16", "stiff_bf16"]):
-        wo = workloads.CHUNK_WORKLOADS[name]
+    for name in ([] if args.other_steps <= 0 else ["longctx_bf16", "stiff_bf16", "lm1p3b_bf16_gated"]):
+        gated = name.endswith("_gated")
+        wo = workloads.CHUNK_WORKLOADS[name.removesuffix("_gated")]
         wo = wo.replace(seed=wo.seed + 1000 * rank)
         xo = {k_: (None if v_ is None else v_.to(dev)) for k_, v_ in workloads.make_chunk_inputs(wo).items()}
-        wso = efla.new_workspace(wo.B, wo.H, wo.T, wo.dk, wo.dv, 64, wo.dtype, dev)
         oo = torch.empty(wo.B, wo.H, wo.T, wo.dv, dtype=wo.dtype, device=dev)
         So = torch.empty(wo.B, wo.H, wo.dk, wo.dv, dtype=torch.float32, device=dev)
-        call = lambda: efla.efla_chunk_fwd(xo["q"], xo["k"], xo["v"], xo["beta"], xo["S0"], o=oo, S_T=So,
-                                           workspace=wso, stream=stream)
+        if gated:   # Gated EFLA: the same shape with a per-token log-decay
+            go = workloads.make_log_decay((wo.B, wo.H, wo.T), wo.seed + 7).to(dev)
+            wso = torch.zeros(efla.lib.efla_chunk_fwd_gated_workspace_bytes(wo.B, wo.H, wo.T, wo.dk, wo.dv, 64, 1),
+                              dtype=torch.uint8, device=dev)
+            call = lambda: efla.efla_chunk_fwd_gated(xo["q"], xo["k"], xo["v"], xo["beta"], go, xo["S0"], o=oo,
+                                                     S_T=So, workspace=wso, stream=stream)
+        else:
+            wso = efla.new_workspace(wo.B, wo.H, wo.T, wo.dk, wo.dv, 64, wo.dtype, dev)
+            call = lambda: efla.efla_chunk_fwd(xo["q"], xo["k"], xo["v"], xo["beta"], xo["S0"], o=oo, S_T=So,
+                                               workspace=wso, stream=stream)
         for _ in range(args.warmup):
             call()
         barrier(world)
@@ -612,6 +620,8 @@ def main():
         if efla.efla_workspace_status(wso, clear=True, stream=stream) != efla.EFLA_OK:
             raise SystemExit(f"device reported a timeout on {name}")
         ob, of = chunk_alg(wo)
+        if gated:
+            ob += wo.B * wo.H * wo.T * 4          # the fp32 log-decay is read too
         others[name] = {"value": wo.tokens * world / (oms * 1e-3), "unit": "tokens/s", "ms_per_step": oms,
                         "steps": args.other_steps,
                         "config": {"B": wo.B, "H": wo.H, "T": wo.T, "d_k": wo.dk, "d_v": wo.dv, "chunk": 64},

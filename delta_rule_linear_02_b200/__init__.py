@@ -52,6 +52,12 @@ def _load() -> ctypes.CDLL:
     lib.efla_workspace_status.restype = I
     lib.efla_noalloc_status.argtypes = [I, vp]
     lib.efla_noalloc_status.restype = I
+    lib.efla_chunk_fwd_gated_workspace_bytes.argtypes = [I, I, I, I, I, I, I]
+    lib.efla_chunk_fwd_gated_workspace_bytes.restype = Z
+    lib.efla_chunk_fwd_gated.argtypes = [vp] * 8 + [I, I, I, I, I, I, I, I, vp, Z, vp]
+    lib.efla_chunk_fwd_gated.restype = I
+    lib.efla_recurrent_step_gated.argtypes = [vp] * 7 + [I, I, I, I, I, I, vp]
+    lib.efla_recurrent_step_gated.restype = I
     lib.efla_selftest_wait_timeout.argtypes = [vp, ctypes.c_longlong, vp]
     lib.efla_selftest_wait_timeout.restype = I
     lib.efla_recurrent_step.argtypes = [vp, vp, vp, vp, vp, vp, I, I, I, I, I, vp]
@@ -152,6 +158,55 @@ def efla_chunk_fwd(q, k, v, beta, S0=None, chunk: int = CHUNK, o=None, S_T=None,
     return o, S_T
 
 
+def efla_chunk_fwd_gated(q, k, v, beta, g, S0=None, chunk: int = CHUNK, o=None, S_T=None,
+                         workspace=None, want_state: bool = True, stream=None, rule: int = EFLA_RULE_EXACT
+                         ) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Gated EFLA forward: efla_chunk_fwd plus g [B,H,T] float32, the per-token log-decay."""
+    dt = k.dtype
+    for t, nme in ((q, "q"), (k, "k"), (v, "v"), (beta, "beta")):
+        _check(t, nme, dt)
+    _check(g, "g", torch.float32)
+    B, H, T, d_k = k.shape
+    d_v = v.shape[-1]
+    if S0 is not None:
+        _check(S0, "S0", torch.float32)
+    if o is None:
+        o = torch.empty((B, H, T, d_v), device=k.device, dtype=dt)
+    _check(o, "o", dt)
+    if S_T is None and want_state:
+        S_T = torch.empty((B, H, d_k, d_v), device=k.device, dtype=torch.float32)
+    if S_T is not None:
+        _check(S_T, "S_T", torch.float32)
+    if workspace is None:
+        n = int(lib.efla_chunk_fwd_gated_workspace_bytes(B, H, T, d_k, d_v, chunk, _DTYPES.get(dt, -1)))
+        if n == 0:
+            raise EflaError(EFLA_ERR_UNSUPPORTED, "efla_chunk_fwd_gated_workspace_bytes")
+        workspace = torch.zeros(n, dtype=torch.uint8, device=k.device)
+    st = lib.efla_chunk_fwd_gated(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), _ptr(S0), _ptr(o), _ptr(S_T),
+                                  B, H, T, d_k, d_v, chunk, _DTYPES.get(dt, -1), int(rule), _ptr(workspace),
+                                  workspace.numel(), _stream(stream))
+    _raise(st, "efla_chunk_fwd_gated")
+    return o, S_T
+
+
+def efla_recurrent_step_gated(q, k, v, beta, g, S, o=None, stream=None, rule: int = EFLA_RULE_EXACT):
+    """One gated decode token: efla_recurrent_step plus g [N,H] float32, the log-decay."""
+    dt = k.dtype
+    for t, nme in ((q, "q"), (k, "k"), (v, "v"), (beta, "beta")):
+        _check(t, nme, dt)
+    _check(g, "g", torch.float32)
+    _check(S, "S", torch.float32)
+    N, H, d_k = k.shape
+    d_v = v.shape[-1]
+    if o is None:
+        o = torch.empty((N, H, d_v), device=k.device, dtype=dt)
+    _check(o, "o", dt)
+    _raise(lib.efla_recurrent_step_gated(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), _ptr(S), _ptr(o),
+                                         N, H, d_k, d_v, _DTYPES.get(dt, -1), int(rule), _stream(stream)),
+           "efla_recurrent_step_gated")
+    return o
+
+
 def efla_chunk_fwd_noalloc(q, k, v, beta, S0=None, chunk: int = CHUNK, o=None, S_T=None,
                            want_state: bool = True, stream=None
                            ) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
@@ -249,6 +304,6 @@ def efla_backward(q, k, v, beta, dO, S0=None, dS_T=None, want_dS0: bool = True, 
     return grads
 
 
-__all__ = ["efla_backward", "efla_backward_workspace_bytes", "EFLA_RULE_EXACT", "EFLA_RULE_EULER", "efla_gate", "efla_chunk_fwd", "efla_chunk_fwd_noalloc", "efla_chunk_fwd_workspace_bytes", "efla_recurrent_step",
+__all__ = ["efla_chunk_fwd_gated", "efla_recurrent_step_gated", "efla_backward", "efla_backward_workspace_bytes", "EFLA_RULE_EXACT", "EFLA_RULE_EULER", "efla_gate", "efla_chunk_fwd", "efla_chunk_fwd_noalloc", "efla_chunk_fwd_workspace_bytes", "efla_recurrent_step",
            "efla_workspace_status", "efla_noalloc_status", "efla_status_string", "efla_selftest_wait_timeout", "new_workspace", "EflaError", "lib",
            "LIB_PATH", "CHUNK"]

@@ -66,15 +66,24 @@ size_t efla_chunk_fwd_workspace_bytes(int B, int H, int T, int d_k, int d_v, int
     return kWorkspaceHeader;
 }
 
-int efla_chunk_fwd_ex(const void* q, const void* k, const void* v, const void* beta, const float* S0,
-                      void* o, float* S_T, int B, int H, int T, int d_k, int d_v, int chunk, int dtype,
-                      int rule, void* workspace, size_t workspace_bytes, efla_stream_t stream) {
+size_t efla_chunk_fwd_gated_workspace_bytes(int B, int H, int T, int d_k, int d_v, int chunk, int dtype) {
+    if (check_chunk_shape(B, H, T, d_k, d_v, chunk, dtype) != EFLA_OK) return 0;
+    if (dtype == EFLA_DTYPE_BF16 && d_k == 128)   // + two transforms and the log-decays per chunk
+        return kWorkspaceHeader + efla::chunk_tc_gated_workspace_bytes((long)B * H, T);
+    return kWorkspaceHeader;
+}
+
+// The forward with or without the gated flow's log-decay g (null: ungated).
+static int chunk_fwd_impl(const void* q, const void* k, const void* v, const void* beta, const float* g,
+                          const float* S0, void* o, float* S_T, int B, int H, int T, int d_k, int d_v,
+                          int chunk, int dtype, int rule, void* workspace, size_t workspace_bytes,
+                          efla_stream_t stream) {
     int st = check_chunk_shape(B, H, T, d_k, d_v, chunk, dtype);
     if (st != EFLA_OK) return st;
     if (rule != EFLA_RULE_EXACT && rule != EFLA_RULE_EULER) return EFLA_ERR_INVALID_ARG;
-    if (!workspace || !aligned16(workspace) ||
-        workspace_bytes < efla_chunk_fwd_workspace_bytes(B, H, T, d_k, d_v, chunk, dtype))
-        return EFLA_ERR_INVALID_ARG;
+    const size_t need = g ? efla_chunk_fwd_gated_workspace_bytes(B, H, T, d_k, d_v, chunk, dtype)
+                          : efla_chunk_fwd_workspace_bytes(B, H, T, d_k, d_v, chunk, dtype);
+    if (!workspace || !aligned16(workspace) || workspace_bytes < need) return EFLA_ERR_INVALID_ARG;
     const long BH = (long)B * H;
     if (BH == 0) return EFLA_OK;
     const size_t es = elem_size(dtype);
@@ -90,26 +99,44 @@ int efla_chunk_fwd_ex(const void* q, const void* k, const void* v, const void* b
     if (!q || !k || !v || !beta || !o) return EFLA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(beta) || !aligned16(o))
         return EFLA_ERR_INVALID_ARG;
+    const size_t ng = g ? (size_t)BH * T * sizeof(float) : 0;
+    if (g && !aligned16(g)) return EFLA_ERR_INVALID_ARG;
     if (overlaps(o, nv, q, nqk) || overlaps(o, nv, k, nqk) || overlaps(o, nv, v, nv) ||
         overlaps(o, nv, beta, nb) || overlaps(o, nv, S0, ns) || overlaps(o, nv, S_T, ns) ||
-        overlaps(o, nv, workspace, workspace_bytes))
+        overlaps(o, nv, g, ng) || overlaps(o, nv, workspace, workspace_bytes))
         return EFLA_ERR_INVALID_ARG;
     if (S_T && S_T != S0 &&
         (overlaps(S_T, ns, q, nqk) || overlaps(S_T, ns, k, nqk) || overlaps(S_T, ns, v, nv) ||
-         overlaps(S_T, ns, beta, nb) || overlaps(S_T, ns, S0, ns)))
+         overlaps(S_T, ns, beta, nb) || overlaps(S_T, ns, S0, ns) || overlaps(S_T, ns, g, ng)))
         return EFLA_ERR_INVALID_ARG;
     // the kernels write the workspace (error word, UT transforms) while the inputs are
     // still being read, and S_T last: neither may share bytes with it
     if (overlaps(workspace, workspace_bytes, q, nqk) || overlaps(workspace, workspace_bytes, k, nqk) ||
         overlaps(workspace, workspace_bytes, v, nv) || overlaps(workspace, workspace_bytes, beta, nb) ||
-        overlaps(workspace, workspace_bytes, S0, ns) || overlaps(workspace, workspace_bytes, S_T, ns))
+        overlaps(workspace, workspace_bytes, S0, ns) || overlaps(workspace, workspace_bytes, S_T, ns) ||
+        overlaps(workspace, workspace_bytes, g, ng))
         return EFLA_ERR_INVALID_ARG;
     if (dtype == EFLA_DTYPE_BF16 && d_k == 128)
         return from_cuda(efla::launch_chunk_tc(q, k, v, beta, S0, o, S_T, BH, T,
                                                static_cast<uint32_t*>(workspace),
-                                               static_cast<char*>(workspace) + kWorkspaceHeader, rule, s));
+                                               static_cast<char*>(workspace) + kWorkspaceHeader, rule, s, g));
     return from_cuda(efla::launch_chunk_simt(q, k, v, beta, S0, o, S_T, BH, T, d_k,
-                                             dtype == EFLA_DTYPE_BF16, rule, s));
+                                             dtype == EFLA_DTYPE_BF16, rule, s, g));
+}
+
+int efla_chunk_fwd_ex(const void* q, const void* k, const void* v, const void* beta, const float* S0,
+                      void* o, float* S_T, int B, int H, int T, int d_k, int d_v, int chunk, int dtype,
+                      int rule, void* workspace, size_t workspace_bytes, efla_stream_t stream) {
+    return chunk_fwd_impl(q, k, v, beta, nullptr, S0, o, S_T, B, H, T, d_k, d_v, chunk, dtype, rule, workspace,
+                          workspace_bytes, stream);
+}
+
+int efla_chunk_fwd_gated(const void* q, const void* k, const void* v, const void* beta, const float* g,
+                         const float* S0, void* o, float* S_T, int B, int H, int T, int d_k, int d_v, int chunk,
+                         int dtype, int rule, void* workspace, size_t workspace_bytes, efla_stream_t stream) {
+    if (!g && B > 0 && H > 0 && T > 0) return EFLA_ERR_INVALID_ARG;
+    return chunk_fwd_impl(q, k, v, beta, g, S0, o, S_T, B, H, T, d_k, d_v, chunk, dtype, rule, workspace,
+                          workspace_bytes, stream);
 }
 
 int efla_chunk_fwd(const void* q, const void* k, const void* v, const void* beta, const float* S0,
@@ -192,8 +219,25 @@ int efla_selftest_wait_timeout(void* workspace, long long limit_ns, efla_stream_
                                                         (cudaStream_t)stream));
 }
 
+static int recurrent_step_impl(const void* q, const void* k, const void* v, const void* beta, const float* g,
+                               float* S, void* o, int N, int H, int d_k, int d_v, int dtype, int rule,
+                               efla_stream_t stream);
+
 int efla_recurrent_step_ex(const void* q, const void* k, const void* v, const void* beta, float* S,
                            void* o, int N, int H, int d_k, int d_v, int dtype, int rule, efla_stream_t stream) {
+    return recurrent_step_impl(q, k, v, beta, nullptr, S, o, N, H, d_k, d_v, dtype, rule, stream);
+}
+
+int efla_recurrent_step_gated(const void* q, const void* k, const void* v, const void* beta, const float* g,
+                              float* S, void* o, int N, int H, int d_k, int d_v, int dtype, int rule,
+                              efla_stream_t stream) {
+    if (!g && N > 0 && H > 0) return EFLA_ERR_INVALID_ARG;
+    return recurrent_step_impl(q, k, v, beta, g, S, o, N, H, d_k, d_v, dtype, rule, stream);
+}
+
+static int recurrent_step_impl(const void* q, const void* k, const void* v, const void* beta, const float* g,
+                               float* S, void* o, int N, int H, int d_k, int d_v, int dtype, int rule,
+                               efla_stream_t stream) {
     if (N < 0 || H < 0 || d_k <= 0 || d_v <= 0) return EFLA_ERR_INVALID_ARG;
     if (rule != EFLA_RULE_EXACT && rule != EFLA_RULE_EULER) return EFLA_ERR_INVALID_ARG;
     if (dtype != EFLA_DTYPE_F32 && dtype != EFLA_DTYPE_BF16) return EFLA_ERR_UNSUPPORTED;
@@ -208,12 +252,15 @@ int efla_recurrent_step_ex(const void* q, const void* k, const void* v, const vo
     const size_t es = elem_size(dtype);
     const size_t nq = (size_t)NH * d_k * es, nv = (size_t)NH * d_v * es, nb = (size_t)NH * es;
     const size_t ns = (size_t)NH * d_k * d_v * sizeof(float);
+    const size_t ng = g ? (size_t)NH * sizeof(float) : 0;
+    if (g && !aligned16(g)) return EFLA_ERR_INVALID_ARG;
     if (overlaps(o, nv, S, ns) || overlaps(o, nv, q, nq) || overlaps(o, nv, k, nq) ||
         overlaps(o, nv, v, nv) || overlaps(o, nv, beta, nb) || overlaps(S, ns, q, nq) ||
-        overlaps(S, ns, k, nq) || overlaps(S, ns, v, nv) || overlaps(S, ns, beta, nb))
+        overlaps(S, ns, k, nq) || overlaps(S, ns, v, nv) || overlaps(S, ns, beta, nb) ||
+        overlaps(o, nv, g, ng) || overlaps(S, ns, g, ng))
         return EFLA_ERR_INVALID_ARG;
     return from_cuda(efla::launch_decode(q, k, v, beta, S, o, NH, d_k, dtype == EFLA_DTYPE_BF16, rule,
-                                         (cudaStream_t)stream));
+                                         (cudaStream_t)stream, g));
 }
 
 int efla_recurrent_step(const void* q, const void* k, const void* v, const void* beta, float* S,

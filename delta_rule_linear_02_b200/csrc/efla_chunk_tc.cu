@@ -67,21 +67,30 @@ constexpr int kKvtStages = 3, kQStages = 2;
 
 // ---- shared-memory map (bytes from a 1024-aligned base); tiles are 64 x 64 bf16, SW128
 constexpr uint32_t TILE = 8192;
-constexpr uint32_t KVT_K = 0, KVT_V = 2 * TILE, KVT_T = 3 * TILE, KVT_BYTES = 4 * TILE;
 constexpr uint32_t Q_BYTES = 2 * TILE;                         // [Q a0 | Q a1]
-constexpr uint32_t OFF_KVT = 0;
-constexpr uint32_t OFF_Q = OFF_KVT + kKvtStages * KVT_BYTES;
-constexpr uint32_t OFF_DL = OFF_Q + kQStages * Q_BYTES;        // Delta, MN-major 64 x 64
-constexpr uint32_t OFF_SB = OFF_DL + TILE;                     // S bf16, MN-major 128 x 64
-constexpr uint32_t OFF_BAR = OFF_SB + 2 * TILE;
+// A stage holds K (two tiles), the V half and T; the gated flow adds T_U and the chunk's
+// cumulative log-decay (64 fp32, log2 units).  Gated Delta has a second, decay-scaled copy.
+template <bool G>
+struct Lay {
+    static constexpr uint32_t KVT_K = 0, KVT_V = 2 * TILE, KVT_T = 3 * TILE, KVT_TU = 4 * TILE, KVT_GL = 5 * TILE;
+    static constexpr uint32_t KVT_BYTES = G ? 5 * TILE + 1024 : 4 * TILE;
+    static constexpr uint32_t KVT_TX = G ? 5 * TILE + 256 : 4 * TILE;    // transaction bytes per stage
+    static constexpr uint32_t OFF_KVT = 0;
+    static constexpr uint32_t OFF_Q = OFF_KVT + kKvtStages * KVT_BYTES;
+    static constexpr uint32_t OFF_DL = OFF_Q + kQStages * Q_BYTES;       // Delta, MN-major 64 x 64
+    static constexpr uint32_t OFF_DL2 = G ? OFF_DL + TILE : OFF_DL;     // gated: Delta scaled by Gam_last / Gam_r
+    static constexpr uint32_t OFF_SB = OFF_DL2 + TILE;                  // S bf16, MN-major 128 x 64
+    static constexpr uint32_t OFF_BAR = OFF_SB + 2 * TILE;
+    static constexpr uint32_t OFF_MISC = OFF_BAR + 32 * 8;
+    static constexpr uint32_t SMEM_USED = OFF_MISC + 16;
+    static constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;           // + alignment slack
+    static_assert(SMEM_BYTES <= 232448, "shared-memory map exceeds 227 KB");
+    // A [T; *] operand reads the 8 KiB after its T as (unused) rows 64-127: that stays inside
+    // the map for every stage (the last stage is followed by the Q ring).
+    static_assert(OFF_KVT + (kKvtStages - 1) * KVT_BYTES + (G ? KVT_TU : KVT_T) + 2 * TILE <= OFF_BAR,
+                  "[T; *] reads past the map");
+};
 constexpr uint32_t NBAR = 32;
-constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
-constexpr uint32_t SMEM_USED = OFF_MISC + 16;
-constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;          // + alignment slack
-static_assert(SMEM_BYTES <= 232448, "shared-memory map exceeds 227 KB");
-// The [T; *] operand reads the 8 KiB after T as its (unused) rows 64-127: that stays
-// inside the map for every stage (the last stage is followed by the Q ring).
-static_assert(OFF_KVT + (kKvtStages - 1) * KVT_BYTES + KVT_T + 2 * TILE <= OFF_BAR, "[T; *] reads past the map");
 
 // ---- mbarriers (count 1 unless noted)
 enum : int {
@@ -129,6 +138,7 @@ constexpr uint32_t ID_N64 = idesc_bf16(128, 64, false, true);     // [W;Q] S, [*
 constexpr uint32_t ID_WU = idesc_bf16(128, 192, false, true);     // [T;*] [K | V]
 constexpr uint32_t ID_GP = idesc_bf16(128, 64, false, false);     // [W;Q] K^T
 constexpr uint32_t ID_S = idesc_bf16(128, 64, true, true);        // K^T Delta
+constexpr uint32_t ID_W = idesc_bf16(128, 128, false, true);      // gated: [T_W;*] K
 
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
@@ -206,11 +216,17 @@ __device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a_tmem, uint32_t b, 
                           (acc | ks) != 0);
 }
 
+template <bool kGated>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_t,
                 const float* __restrict__ S0, __nv_bfloat16* __restrict__ o, float* __restrict__ S_T,
-                int T, uint32_t* __restrict__ err, unsigned long long limit_ns) {
+                int T, uint32_t* __restrict__ err, unsigned long long limit_ns,
+                const float* __restrict__ gl_all, long ntiles) {
+    using L = Lay<kGated>;
+    constexpr uint32_t KVT_K = L::KVT_K, KVT_V = L::KVT_V, KVT_T = L::KVT_T, KVT_BYTES = L::KVT_BYTES;
+    constexpr uint32_t OFF_KVT = L::OFF_KVT, OFF_Q = L::OFF_Q, OFF_DL = L::OFF_DL, OFF_SB = L::OFF_SB;
+    constexpr uint32_t OFF_BAR = L::OFF_BAR, OFF_MISC = L::OFF_MISC;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sb = smem_u32(sm);
@@ -257,11 +273,15 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     if (c >= kKvtStages && !(ok = ctl.wait(B_KVT_FREE + s, ((c - kKvtStages) / kKvtStages) & 1))) break;
                     uint8_t* st = sm + kvt(c);
                     uint64_t* full = ctl.b(B_KVT_FULL + s);
-                    mbar_arrive_expect_tx(full, 4 * TILE);
+                    mbar_arrive_expect_tx(full, L::KVT_TX);
                     tma_load_3d(st + KVT_K, &tm_k, full, 0, t0, bh);
                     tma_load_3d(st + KVT_K + TILE, &tm_k, full, 64, t0, bh);
                     tma_load_3d(st + KVT_V, &tm_v, full, col0, t0, bh);
                     tma_load_2d(st + KVT_T, &tm_t, full, 0, (bh * nchunks + c) * 64);
+                    if constexpr (kGated) {
+                        tma_load_2d(st + L::KVT_TU, &tm_t, full, 0, (int)((ntiles + (long)bh * nchunks + c) * 64));
+                        bulk_load(st + L::KVT_GL, gl_all + ((long)bh * nchunks + c) * 64, 256, full);
+                    }
                     kvt_issued = c + 1;
                 }
                 {   // Q of chunk c
@@ -305,10 +325,15 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 mma_commit_elect(ctl.b(B_GP_FULL));
             }
         };
-        auto issue_wu = [&](int c) {      // [W | U] = [T; *] [K | V]
+        auto issue_wu = [&](int c) {      // [W | U] = [T; *] [K | V]   (gated: [T_W;*] K | [T_U;*] V)
             tc_fence_after();
             const uint32_t st = sb + kvt(c);
-            mma_ss(tmem + TM_WU, st + KVT_T, TILE, 32, 16, st + KVT_K, 4 * 2048, 2048, TILE, ID_WU, 4, 0);
+            if constexpr (kGated) {
+                mma_ss(tmem + TM_WU, st + KVT_T, TILE, 32, 16, st + KVT_K, 4 * 2048, 2048, TILE, ID_W, 4, 0);
+                mma_ss(tmem + TM_WU + 128, st + L::KVT_TU, TILE, 32, 16, st + KVT_V, 4 * 2048, 2048, TILE, ID_N64, 4, 0);
+            } else {
+                mma_ss(tmem + TM_WU, st + KVT_T, TILE, 32, 16, st + KVT_K, 4 * 2048, 2048, TILE, ID_WU, 4, 0);
+            }
             mma_commit_elect(ctl.b(B_WU_FULL));
         };
         bool ok = wait(B_KVT_FULL, 0);
@@ -334,15 +359,17 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             // S += K^T Delta (state chain)
             if (!(ok = wait(B_D_READY, c & 1))) break;
             tc_fence_after();
-            mma_ss(tmem + TM_S, sb + kvt(c) + KVT_K, 4 * 2048, 2048, TILE, sb + OFF_DL, 4 * 2048, 2048, TILE, ID_S,
-                   4, 1);
+            mma_ss(tmem + TM_S, sb + kvt(c) + KVT_K, 4 * 2048, 2048, TILE, sb + L::OFF_DL2, 4 * 2048, 2048, TILE,
+                   ID_S, 4, 1);
             mma_commit_elect(ctl.b(B_S_FULL));
-            mma_commit_elect(ctl.b(B_KVT_FREE + c % kKvtStages));
+            // gated: the P warps still read the stage's log-decays until P is ready
+            if constexpr (!kGated) mma_commit_elect(ctl.b(B_KVT_FREE + c % kKvtStages));
             // X += [*; P] Delta: rows 64-127 become O = Q S + P Delta
             if (!(ok = wait(B_P_READY, c & 1))) break;
             tc_fence_after();
             mma_ts(tmem + TM_X, tmem + TM_AP, sb + OFF_DL, 4 * 2048, 2048, TILE, ID_N64, 4, 1);
             mma_commit_elect(ctl.b(B_O_FULL));
+            if constexpr (kGated) mma_commit_elect(ctl.b(B_KVT_FREE + c % kKvtStages));
         }
         mma_commit_elect(ctl.b(B_DRAIN));
         if (lane == 0) mbar_wait(ctl.b(B_DRAIN), 0, limit_ns);
@@ -428,7 +455,48 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             // once, above); rows 32-63 keep columns 0-31 whole.  Each warp masks 32 columns.
             if (!(ok = ctl.wwait(B_GP_FULL, c & 1))) break;
             tc_fence_after();
-            if (q == 2) {
+            if constexpr (kGated) {
+                // P~[r][s] = (Q K^T)[r][s] Gam_r / Gam_s (s <= r), and the Q S rows of X scaled by
+                // Gam_r before P Delta accumulates onto them: O = diag(Gam) Q S + P~ Delta
+                const float* glc = reinterpret_cast<const float*>(sm + kvt(c) + L::KVT_GL);
+                const float glr = glc[r];
+                if (q == 2) {
+                    float t[32], pk[16];
+                    tmem_ld32_wait(tmem + lane_off + TM_GP, t);
+#pragma unroll
+                    for (int j = 0; j < 16; ++j)
+                        pk[j] = __uint_as_float(pack_bf16x2(2 * j <= lane ? t[2 * j] * exp2f(glr - glc[2 * j]) : 0.f,
+                                                            2 * j + 1 <= lane ? t[2 * j + 1] * exp2f(glr - glc[2 * j + 1]) : 0.f));
+                    tmem_st16(tmem + lane_off + TM_AP, pk);
+                } else {
+                    float t[64];
+                    uint32_t pk[32];
+                    tmem_ld64_wait(tmem + lane_off + TM_GP, t);
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        pk[j] = pack_bf16x2(t[2 * j] * exp2f(glr - glc[2 * j]), t[2 * j + 1] * exp2f(glr - glc[2 * j + 1]));
+                        pk[16 + j] = pack_bf16x2(2 * j <= lane ? t[32 + 2 * j] * exp2f(glr - glc[32 + 2 * j]) : 0.f,
+                                                 2 * j + 1 <= lane ? t[33 + 2 * j] * exp2f(glr - glc[33 + 2 * j]) : 0.f);
+                    }
+                    tmem_st32(tmem + lane_off + TM_AP, pk);
+                }
+                {
+                    const float gm = exp2f(glr);
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        float x[32];
+                        tmem_ld32_wait(tmem + lane_off + TM_X + 32 * h, x);
+                        float y0[16], y1[16];
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            y0[j] = x[j] * gm;
+                            y1[j] = x[16 + j] * gm;
+                        }
+                        tmem_st16(tmem + lane_off + TM_X + 32 * h, y0);
+                        tmem_st16(tmem + lane_off + TM_X + 32 * h + 16, y1);
+                    }
+                }
+            } else if (q == 2) {
                 float t[32], pk[16];
                 tmem_ld32_wait(tmem + lane_off + TM_GP, t);
 #pragma unroll
@@ -468,8 +536,17 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const int cc = 32 * ch;
         const int ct = 32 * q + lane;                 // d_k row of S, and row of X / [W | U]
         const bool delta_group = q < 2;
+        // gated: the accumulator carries Gam_last(c) S_c into the write of chunk c
+        auto decay_of = [&](int c) -> float {
+            if constexpr (kGated) {
+                if (!ctl.wwait(B_KVT_FULL + c % kKvtStages, (c / kKvtStages) & 1)) return 1.f;
+                return exp2f(reinterpret_cast<const float*>(sm + kvt(c) + L::KVT_GL)[63]);
+            }
+            return 1.f;
+        };
         {   // initial state
             const float* src = S0 ? S0 + ((size_t)bh * kD + ct) * kD + col0 + cc : nullptr;
+            const float dec0 = decay_of(0);
 #pragma unroll
             for (int qd = 0; qd < 2; ++qd) {
                 float s16[16];
@@ -478,9 +555,13 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     float4 x = src ? *reinterpret_cast<const float4*>(src + 16 * qd + j) : make_float4(0.f, 0.f, 0.f, 0.f);
                     s16[j] = x.x; s16[j + 1] = x.y; s16[j + 2] = x.z; s16[j + 3] = x.w;
                 }
-                tmem_st16(tmem + lane_off + TM_S + cc + 16 * qd, s16);
                 st_chunk(sm + OFF_SB + sw128_off(ct, 4 * ch + 2 * qd), s16);
                 st_chunk(sm + OFF_SB + sw128_off(ct, 4 * ch + 2 * qd + 1), s16 + 8);
+                if constexpr (kGated) {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) s16[j] *= dec0;
+                }
+                tmem_st16(tmem + lane_off + TM_S + cc + 16 * qd, s16);
             }
             tmem_wait_st();
             fence_proxy_async_smem();
@@ -506,6 +587,14 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 for (int j = 0; j < 32; ++j) t[j] = u[j] - t[j];
 #pragma unroll
                 for (int j = 0; j < 4; ++j) st_chunk(sm + OFF_DL + sw128_off(ct, 4 * ch + j), t + 8 * j);
+                if constexpr (kGated) {   // the state's copy: row r scaled by Gam_last / Gam_r
+                    const float* glc = reinterpret_cast<const float*>(sm + kvt(c) + L::KVT_GL);
+                    const float sc = exp2f(glc[63] - glc[ct]);
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) t[j] *= sc;
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) st_chunk(sm + L::OFF_DL2 + sw128_off(ct, 4 * ch + j), t + 8 * j);
+                }
                 fence_proxy_async_smem();
                 tc_fence_before();
                 ctl.warp_arrive(B_D_READY, lane);
@@ -523,6 +612,20 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
                     for (int j = 0; j < 32; j += 4)
                         *reinterpret_cast<float4*>(dst + j) = make_float4(t[j], t[j + 1], t[j + 2], t[j + 3]);
+                }
+                if constexpr (kGated) {
+                    if (c + 1 < nchunks) {
+                        const float dec = decay_of(c + 1);
+                        float y0[16], y1[16];
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            y0[j] = t[j] * dec;
+                            y1[j] = t[16 + j] * dec;
+                        }
+                        tmem_st16(tmem + lane_off + TM_S + cc, y0);
+                        tmem_st16(tmem + lane_off + TM_S + cc + 16, y1);
+                        tmem_wait_st();
+                    }
                 }
             }
             fence_proxy_async_smem();
@@ -559,21 +662,36 @@ size_t chunk_tc_workspace_bytes(long BH, int T) {
     return (size_t)BH * nchunks * 64 * 64 * 2;     // the bf16 T of every chunk
 }
 
+size_t chunk_tc_gated_workspace_bytes(long BH, int T) {
+    const long ntiles = BH * ((T + 63) / 64);
+    return (size_t)ntiles * (2 * 64 * 64 * 2 + 64 * 4);   // T_W, T_U (bf16) and G log2(e) (fp32) per tile
+}
+
 cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const void* beta, const float* S0,
                             void* o, float* S_T, long BH, int T, uint32_t* err, void* scratch,
-                            int rule, cudaStream_t stream) {
+                            int rule, cudaStream_t stream, const float* g) {
     const int nchunks = (T + 63) / 64;
-    cudaError_t e = launch_ut(k, beta, scratch, BH, T, err, kWaitLimitNs, rule, stream);
+    const long ntiles = BH * nchunks;
+    cudaError_t e = launch_ut(k, beta, scratch, BH, T, err, kWaitLimitNs, rule, stream, g);
     if (e != cudaSuccess) return e;
     CUtensorMap mq, mk, mv, mt;
     if (!tma_map_tokens(&mq, q, kD, T, BH) || !tma_map_tokens(&mk, k, kD, T, BH) ||
-        !tma_map_tokens(&mv, v, kD, T, BH) || !tma_map_rows64(&mt, scratch, BH * nchunks * 64))
+        !tma_map_tokens(&mv, v, kD, T, BH) || !tma_map_rows64(&mt, scratch, (g ? 2 : 1) * ntiles * 64))
         return cudaErrorInvalidValue;
+    if (g) {
+        const float* gl = reinterpret_cast<const float*>(static_cast<const char*>(scratch) + ntiles * 8192 * 2);
+        static std::atomic<uint64_t> smem_set_g{0};
+        e = set_smem_limit_once(chunk_tc_kernel<true>, (int)Lay<true>::SMEM_BYTES, smem_set_g);
+        if (e != cudaSuccess) return e;
+        chunk_tc_kernel<true><<<(unsigned)(BH * 2), kThreads, Lay<true>::SMEM_BYTES, stream>>>(
+            mq, mk, mv, mt, S0, (__nv_bfloat16*)o, S_T, T, err, kWaitLimitNs, gl, ntiles);
+        return cudaGetLastError();
+    }
     static std::atomic<uint64_t> smem_set{0};
-    e = set_smem_limit_once(chunk_tc_kernel, (int)SMEM_BYTES, smem_set);
+    e = set_smem_limit_once(chunk_tc_kernel<false>, (int)Lay<false>::SMEM_BYTES, smem_set);
     if (e != cudaSuccess) return e;
-    chunk_tc_kernel<<<(unsigned)(BH * 2), kThreads, SMEM_BYTES, stream>>>(mq, mk, mv, mt, S0, (__nv_bfloat16*)o,
-                                                                          S_T, T, err, kWaitLimitNs);
+    chunk_tc_kernel<false><<<(unsigned)(BH * 2), kThreads, Lay<false>::SMEM_BYTES, stream>>>(
+        mq, mk, mv, mt, S0, (__nv_bfloat16*)o, S_T, T, err, kWaitLimitNs, nullptr, ntiles);
     return cudaGetLastError();
 }
 

@@ -64,6 +64,63 @@ __device__ __forceinline__ float gate_alpha(float beta, float lambda) {
     return -expm1f(-x) / lambda;
 }
 
+// The gated flow (Gated EFLA, Section 3.4): a per-token log-decay g joins the ODE over the
+// token's unit interval, dS/dtau = g S - beta (k k^T S - k v^T).  The flow keeps alpha for the
+// rank-1 contraction, decays the state by e^g, and writes with
+//     abar = beta phi1(beta lambda - g),   phi1(x) = (1 - e^{-x}) / x,
+// which equals alpha at g = 0.  phi1 uses the same short series as gate_alpha near x = 0.
+// Under the Euler rule (the gated delta rule) the write uses beta.
+__device__ __forceinline__ float phi1(float x) {
+    if (fabsf(x) < 0.0009765625f) return 1.0f - x * (0.5f - x * (1.0f / 6.0f));
+    return -expm1f(-x) / x;
+}
+__device__ __forceinline__ float rule_write_gate(int rule, float beta, float lambda, float g) {
+    return rule == kRuleEuler ? beta : beta * phi1(beta * lambda - g);
+}
+
+// ---------------------------------------------------------------- streams and tiles
+// One recurrence ("stream") per (sequence, head).  Dense batches: stream bh of B*H, each T
+// tokens, tensors [B*H][T][d].  Packed variable-length batches (Section 3.3's chunking per
+// sequence): N sequences of one head-major stream per head, tensors [H][total_T][d], sequence
+// n at tokens cu[n] .. cu[n+1] of every head; stream n*H + h; chunks restart at each
+// sequence start, so a sequence's tail chunk is padded with alpha = 0 (its rows past the
+// sequence end belong to the next sequence and are never written).
+struct StreamJob {
+    int z;          // index along the outer tensor dimension: bh (dense) or h (packed)
+    int y0;         // first token of the stream within that row
+    int len;        // tokens
+    long tile0;     // UT tile of the stream's chunk 0
+};
+struct Seqs {
+    const int* cu;        // packed: N+1 offsets (device); null for dense batches
+    const int* tileoff;   // packed: N+1 prefix sums of the sequences' chunk counts
+    int N, H;             // packed: sequences, heads
+    int T;                // dense: tokens per stream
+    long total_tiles;     // packed: tileoff[N] (per head)
+    __device__ __forceinline__ StreamJob job(long s) const {
+        if (!cu) return StreamJob{(int)s, 0, T, s * (long)((T + 63) / 64)};
+        const int n = (int)(s / H), h = (int)(s % H);
+        return StreamJob{h, cu[n], cu[n + 1] - cu[n], (long)h * total_tiles + tileoff[n]};
+    }
+    // UT tile i -> its stream's job and chunk
+    __device__ __forceinline__ StreamJob tile(long i, int* chunk) const {
+        if (!cu) {
+            const int nc = (T + 63) / 64;
+            *chunk = (int)(i % nc);
+            return StreamJob{(int)(i / nc), 0, T, i - *chunk};
+        }
+        const int h = (int)(i / total_tiles);
+        const int j = (int)(i % total_tiles);
+        int lo = 0, hi = N;                   // largest n with tileoff[n] <= j (sequences with chunks)
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (tileoff[mid] <= j) lo = mid; else hi = mid;
+        }
+        *chunk = j - tileoff[lo];
+        return StreamJob{h, cu[lo], cu[lo + 1] - cu[lo], (long)h * total_tiles + tileoff[lo]};
+    }
+};
+
 // Device error word values (kept in the caller's workspace).
 enum : uint32_t { kDevOk = 0u, kDevTimeout = 1u };
 

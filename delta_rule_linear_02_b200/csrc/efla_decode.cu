@@ -4,6 +4,9 @@
 // recurrent form; the read-out o_t = S_t^T q_t is taken after the write.  With
 // r = k^T S, p = q^T S, c = q.k and e = r - v (row convention, S is d_k x d_v):
 //     S_new = S - alpha k e^T,      o = S_new^T q = p - alpha c e.
+// The gated flow (Section 3.4, Gated EFLA) with decay d = e^g and write gate abar:
+//     S_new = d S - k w^T,  w = d alpha r - abar v,   o = d p - c w
+// (d = 1 and abar = alpha give the line above).
 // Column j of S_new depends only on column j of S, so each CTA owns a 32-column slice
 // of one head's state and streams it exactly once through registers: one HBM read and
 // one HBM write of the 4*d_k*d_v-byte state per token, the bound for this step.
@@ -16,13 +19,14 @@ namespace {
 constexpr int kCols = 32;      // state columns per CTA
 constexpr int kThreads = 256;  // 8 column-quads x 32 row groups
 
-template <typename Tin, int D>
+template <typename Tin, int D, bool kGated = false>
 __global__ void __launch_bounds__(kThreads) decode_kernel(const Tin* __restrict__ q,
                                                           const Tin* __restrict__ k,
                                                           const Tin* __restrict__ v,
                                                           const Tin* __restrict__ beta,
                                                           float* __restrict__ S,
-                                                          Tin* __restrict__ o, int rule) {
+                                                          Tin* __restrict__ o, int rule,
+                                                          const float* __restrict__ gdec = nullptr) {
     constexpr int RPT = D / 32;                 // rows per thread
     constexpr int SLICES = D / kCols;
     const int t = threadIdx.x;
@@ -50,7 +54,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const Tin* __restrict_
 
     __shared__ float4 red_r[8][8];
     __shared__ float4 red_p[8][8];
-    __shared__ float sh_alpha, sh_c;
+    __shared__ float sh_alpha, sh_c, sh_abar, sh_dec;
 
     // 2. lambda = ||k||^2 and c = q.k over the full key, by warp 0
     if (warp == 0) {
@@ -67,8 +71,14 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const Tin* __restrict_
             c += __shfl_xor_sync(0xffffffffu, c, off);
         }
         if (lane == 0) {
-            sh_alpha = rule_alpha(rule, Elem<Tin>::to_f(beta[head]), lam);
+            const float bt = Elem<Tin>::to_f(beta[head]);
+            sh_alpha = rule_alpha(rule, bt, lam);
             sh_c = c;
+            if constexpr (kGated) {
+                const float gh = gdec[head];
+                sh_abar = rule_write_gate(rule, bt, lam, gh);
+                sh_dec = expf(gh);
+            }
         }
     }
 
@@ -104,6 +114,24 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const Tin* __restrict_
         p.x += b.x; p.y += b.y; p.z += b.z; p.w += b.w;
     }
     const float alpha = sh_alpha, c = sh_c;
+    if constexpr (kGated) {
+        // w = d alpha r - abar v;  S_new = d S - k w^T;  o = d p - c w
+        const float dec = sh_dec, da = sh_dec * sh_alpha, ab = sh_abar;
+        const float4 w = make_float4(fmaf(da, r.x, -ab * vv.x), fmaf(da, r.y, -ab * vv.y),
+                                     fmaf(da, r.z, -ab * vv.z), fmaf(da, r.w, -ab * vv.w));
+#pragma unroll
+        for (int m = 0; m < RPT; ++m) {
+            const float km = kr[m];
+            float4 u = s[m];
+            u.x = fmaf(-km, w.x, dec * u.x); u.y = fmaf(-km, w.y, dec * u.y);
+            u.z = fmaf(-km, w.z, dec * u.z); u.w = fmaf(-km, w.w, dec * u.w);
+            __stcs(reinterpret_cast<float4*>(Sh + (long)(rg + 32 * m) * D + j0), u);
+        }
+        if (rg == 0)
+            store4(o + head * D + j0, make_float4(fmaf(-c, w.x, dec * p.x), fmaf(-c, w.y, dec * p.y),
+                                                  fmaf(-c, w.z, dec * p.z), fmaf(-c, w.w, dec * p.w)));
+        return;
+    }
     const float4 e = make_float4(r.x - vv.x, r.y - vv.y, r.z - vv.z, r.w - vv.w);
 
     // 5. rank-1 write S -= alpha k e^T, streamed back
@@ -125,22 +153,26 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const Tin* __restrict_
 
 template <typename Tin, int D>
 cudaError_t launch_decode_t(const void* q, const void* k, const void* v, const void* beta,
-                            float* S, void* o, long NH, int rule, cudaStream_t stream) {
+                            float* S, void* o, long NH, int rule, const float* g, cudaStream_t stream) {
     const long blocks = NH * (D / kCols);
-    decode_kernel<Tin, D><<<(unsigned)blocks, kThreads, 0, stream>>>(
-        (const Tin*)q, (const Tin*)k, (const Tin*)v, (const Tin*)beta, S, (Tin*)o, rule);
+    if (g)
+        decode_kernel<Tin, D, true><<<(unsigned)blocks, kThreads, 0, stream>>>(
+            (const Tin*)q, (const Tin*)k, (const Tin*)v, (const Tin*)beta, S, (Tin*)o, rule, g);
+    else
+        decode_kernel<Tin, D><<<(unsigned)blocks, kThreads, 0, stream>>>(
+            (const Tin*)q, (const Tin*)k, (const Tin*)v, (const Tin*)beta, S, (Tin*)o, rule);
     return cudaGetLastError();
 }
 }  // namespace
 
 cudaError_t launch_decode(const void* q, const void* k, const void* v, const void* beta, float* S,
-                          void* o, long NH, int D, bool bf16, int rule, cudaStream_t stream) {
+                          void* o, long NH, int D, bool bf16, int rule, cudaStream_t stream, const float* g) {
     if (bf16) {
-        return D == 128 ? launch_decode_t<__nv_bfloat16, 128>(q, k, v, beta, S, o, NH, rule, stream)
-                        : launch_decode_t<__nv_bfloat16, 64>(q, k, v, beta, S, o, NH, rule, stream);
+        return D == 128 ? launch_decode_t<__nv_bfloat16, 128>(q, k, v, beta, S, o, NH, rule, g, stream)
+                        : launch_decode_t<__nv_bfloat16, 64>(q, k, v, beta, S, o, NH, rule, g, stream);
     }
-    return D == 128 ? launch_decode_t<float, 128>(q, k, v, beta, S, o, NH, rule, stream)
-                    : launch_decode_t<float, 64>(q, k, v, beta, S, o, NH, rule, stream);
+    return D == 128 ? launch_decode_t<float, 128>(q, k, v, beta, S, o, NH, rule, g, stream)
+                    : launch_decode_t<float, 64>(q, k, v, beta, S, o, NH, rule, g, stream);
 }
 
 }  // namespace efla

@@ -10,22 +10,28 @@ namespace efla {
 cudaError_t launch_gate(const void* k, const void* beta, float* alpha, long n, int dk, bool bf16,
                         cudaStream_t stream);
 
-// rule: kRuleExact (the exact-flow gate) or kRuleEuler (alpha = beta, the delta rule)
+// rule: kRuleExact (the exact-flow gate) or kRuleEuler (alpha = beta, the delta rule).
+// g: per-token log-decay (float32, one per stream and token) for the gated flow, or null.
 cudaError_t launch_decode(const void* q, const void* k, const void* v, const void* beta, float* S,
-                          void* o, long NH, int D, bool bf16, int rule, cudaStream_t stream);
+                          void* o, long NH, int D, bool bf16, int rule, cudaStream_t stream,
+                          const float* g = nullptr);
 
 cudaError_t launch_chunk_simt(const void* q, const void* k, const void* v, const void* beta,
                               const float* S0, void* o, float* S_T, long BH, int T, int D, bool bf16,
-                              int rule, cudaStream_t stream);
+                              int rule, cudaStream_t stream, const float* g = nullptr);
 
 // bf16, d_k = d_v = 128: the UT kernel (efla_ut.cu) writes every chunk's T into `scratch`
 // (chunk_tc_workspace_bytes bytes, 16-byte aligned), then the chain kernel runs.
 size_t chunk_tc_workspace_bytes(long BH, int T);
+// the gated flow (g != null): two transforms and the cumulative log-decay per chunk
+size_t chunk_tc_gated_workspace_bytes(long BH, int T);
 cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const void* beta, const float* S0,
                             void* o, float* S_T, long BH, int T, uint32_t* err, void* scratch,
-                            int rule, cudaStream_t stream);
+                            int rule, cudaStream_t stream, const float* g = nullptr);
+// g != null: the gated flow's transforms (two per tile plus the cumulative log-decay, see
+// efla_ut.cu) into Tout, which then holds chunk_tc_gated_workspace_bytes.
 cudaError_t launch_ut(const void* k, const void* beta, void* Tout, long BH, int T, uint32_t* err,
-                      unsigned long long limit_ns, int rule, cudaStream_t stream);
+                      unsigned long long limit_ns, int rule, cudaStream_t stream, const float* g = nullptr);
 
 // reverse-mode pass (efla_bwd.cu): fp32 gradients; workspace of bwd_workspace_bytes
 size_t bwd_workspace_bytes(long BH, int T, int D);

@@ -17,6 +17,13 @@
 // Tokens past T are zero-filled by TMA (k = 0, beta = 0: alpha = 0, their rows and
 // columns of T are zero).
 //
+// Gated flow (Section 3.4, Gated EFLA; per-token log-decay g): with the cumulative
+// log-decay G_r = g_0 + ... + g_r of the tile and Gam_r = e^{G_r},
+//   A[r][s] = alpha_r (Gam_r / Gam_s) G[r][s]  (s < r),  X = (I + A)^{-1},
+// and two transforms are stored, T_W = X diag(alpha Gam) (at Tout, as above) and
+// T_U = X diag(abar) (ntiles tiles further on), plus G_r log2(e) of every row (fp32, 64 per
+// tile, after both transform regions) for the chain kernel's decay factors.
+//
 // A persistent grid of six CTAs per SM walks the tiles; the CTAs on an SM overlap each
 // other's latency.  The K tile is dead once G has been formed, so A^T is written over it:
 // a CTA holds one fp32 64 x 68 tile for K / A^T and one for X (36 KB), and the next K tile
@@ -51,6 +58,13 @@ constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
 constexpr uint32_t SMEM_USED = OFF_MISC + 16;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;
 static_assert(kCtasPerSm * SMEM_BYTES <= 232448, "UT kernel: shared memory for the target occupancy");
+// gated flow only: raw log-decay, its cumulative sum (log2 units), abar, alpha * Gam
+constexpr uint32_t OFF_GRAW = SMEM_USED;
+constexpr uint32_t OFF_GL = OFF_GRAW + 256;
+constexpr uint32_t OFF_ABAR = OFF_GL + 256;
+constexpr uint32_t OFF_MW = OFF_ABAR + 256;
+constexpr uint32_t SMEM_BYTES_G = OFF_MW + 256 + 1024;
+static_assert(kCtasPerSm * (SMEM_BYTES_G + 1024) <= 233472, "gated UT kernel: shared memory per SM");
 
 enum : int { B_FULL = 0, B_GP_FULL = 1, B_GP_FREE = 2, B_AT_FREE = 3, B_DRAIN = 4 };
 constexpr uint32_t TM_COLS = 64;
@@ -76,10 +90,11 @@ __device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, vol
     return true;
 }
 
+template <bool kGated>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 ut_kernel(const __grid_constant__ CUtensorMap tm_k, const __nv_bfloat16* __restrict__ beta,
           __nv_bfloat16* __restrict__ Tout, int T, int nchunks, long ntiles, uint32_t* __restrict__ err,
-          unsigned long long limit_ns, int rule) {
+          unsigned long long limit_ns, int rule, const float* __restrict__ gdec) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sb = smem_u32(sm);
@@ -87,6 +102,10 @@ ut_kernel(const __grid_constant__ CUtensorMap tm_k, const __nv_bfloat16* __restr
     float* X = reinterpret_cast<float*>(sm + OFF_X);
     float* al = reinterpret_cast<float*>(sm + OFF_ALPHA);
     float* bt = reinterpret_cast<float*>(sm + OFF_BETA);
+    float* graw = reinterpret_cast<float*>(sm + OFF_GRAW);    // gated flow only
+    float* gl = reinterpret_cast<float*>(sm + OFF_GL);
+    float* abar = reinterpret_cast<float*>(sm + OFF_ABAR);
+    float* mw = reinterpret_cast<float*>(sm + OFF_MW);
     uint64_t* bar = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + OFF_MISC);
     volatile int* abort = reinterpret_cast<volatile int*>(sm + OFF_MISC + 4);
@@ -169,12 +188,42 @@ ut_kernel(const __grid_constant__ CUtensorMap tm_k, const __nv_bfloat16* __restr
             const int t = (int)(tile % nchunks) * 64 + wt;
             return t < T ? __bfloat162float(beta[bh * T + t]) : 0.f;
         };
+        auto g_of = [&](int j) -> float {
+            if (j >= ntile || wt >= 64) return 0.f;
+            const long tile = first + (long)j * step;
+            const long bh = tile / nchunks;
+            const int t = (int)(tile % nchunks) * 64 + wt;
+            return t < T ? gdec[bh * T + t] : 0.f;
+        };
         float beta_next = beta_of(0);
+        float g_next = 0.f;
+        if constexpr (kGated) g_next = g_of(0);
         bool ok = true;
         for (int j = 0; j < ntile; ++j) {
             if (wt < 64) {
                 bt[wt] = beta_next;
                 beta_next = beta_of(j + 1);
+                if constexpr (kGated) {
+                    graw[wt] = g_next;
+                    g_next = g_of(j + 1);
+                }
+            }
+            if constexpr (kGated) {   // cumulative log-decay (log2 units) by worker warp 0, a shuffle scan
+                bar_sync(NB_W, 128);
+                if (wt < 32) {
+                    const float a0 = graw[2 * wt], a1 = graw[2 * wt + 1];
+                    float run = a0 + a1;
+#pragma unroll
+                    for (int off = 1; off < 32; off <<= 1) {
+                        const float y = __shfl_up_sync(0xffffffffu, run, off);
+                        if (wt >= off) run += y;
+                    }
+                    float before = __shfl_up_sync(0xffffffffu, run, 1);
+                    if (wt == 0) before = 0.f;
+                    constexpr float kLog2e = 1.4426950408889634f;
+                    gl[2 * wt] = (before + a0) * kLog2e;
+                    gl[2 * wt + 1] = ((before + a0) + a1) * kLog2e;
+                }
             }
             ok = bar_and(NB_W, 128, ok && wait_bounded(bar + B_GP_FULL, j & 1, abort, limit_ns));
             if (!ok) break;
@@ -189,7 +238,12 @@ ut_kernel(const __grid_constant__ CUtensorMap tm_k, const __nv_bfloat16* __restr
                     float lam = 0.f;
 #pragma unroll
                     for (int e = 0; e < 32; ++e) lam = fmaf(g[e], e == d ? 1.f : 0.f, lam);
-                    al[r] = rule_alpha(rule, bt[r], lam);
+                    const float a = rule_alpha(rule, bt[r], lam);
+                    al[r] = a;
+                    if constexpr (kGated) {
+                        abar[r] = rule_write_gate(rule, bt[r], lam, graw[r]);
+                        mw[r] = a * exp2f(gl[r]);
+                    }
                 }
             }
             bar_sync(NB_W, 128);                     // alpha visible
@@ -200,11 +254,25 @@ ut_kernel(const __grid_constant__ CUtensorMap tm_k, const __nv_bfloat16* __restr
                 float g[32];
                 tmem_ld32_wait(tmem + lane_off + 32 * h, g);
                 if (grow) {
+                    if constexpr (kGated) {
+                        // A^T[r][i] = alpha_i (Gam_i / Gam_r) G[r][i]; only i > r is read, where the
+                        // ratio is <= 1 for decays
+                        const float glr = gl[r];
 #pragma unroll
-                    for (int m = 0; m < 8; ++m) {
-                        const float4 a = *reinterpret_cast<const float4*>(al + 32 * h + 4 * m);
-                        *reinterpret_cast<float4*>(At + r * LDX + 32 * h + 4 * m) =
-                            make_float4(a.x * g[4 * m], a.y * g[4 * m + 1], a.z * g[4 * m + 2], a.w * g[4 * m + 3]);
+                        for (int m = 0; m < 8; ++m) {
+                            const float4 a = *reinterpret_cast<const float4*>(al + 32 * h + 4 * m);
+                            const float4 l = *reinterpret_cast<const float4*>(gl + 32 * h + 4 * m);
+                            *reinterpret_cast<float4*>(At + r * LDX + 32 * h + 4 * m) =
+                                make_float4(a.x * exp2f(l.x - glr) * g[4 * m], a.y * exp2f(l.y - glr) * g[4 * m + 1],
+                                            a.z * exp2f(l.z - glr) * g[4 * m + 2], a.w * exp2f(l.w - glr) * g[4 * m + 3]);
+                        }
+                    } else {
+#pragma unroll
+                        for (int m = 0; m < 8; ++m) {
+                            const float4 a = *reinterpret_cast<const float4*>(al + 32 * h + 4 * m);
+                            *reinterpret_cast<float4*>(At + r * LDX + 32 * h + 4 * m) =
+                                make_float4(a.x * g[4 * m], a.y * g[4 * m + 1], a.z * g[4 * m + 2], a.w * g[4 * m + 3]);
+                        }
                     }
                 }
             }
@@ -218,22 +286,32 @@ ut_kernel(const __grid_constant__ CUtensorMap tm_k, const __nv_bfloat16* __restr
             bar_sync(NB_W, 128);
             if (wt == 0) mbar_arrive(bar + B_AT_FREE);
             {   // T = X diag(alpha) -> bf16, 64 bytes per thread (a warp reads 32 consecutive
-                // rows of one column half: conflict-free with the 68-float row stride)
+                // rows of one column half: conflict-free with the 68-float row stride).
+                // Gated: T_W = X diag(alpha Gam), T_U = X diag(abar), and the row's G log2(e).
                 const long tile = first + (long)j * step;
                 const int rr = wt & 63, h = wt >> 6;
-                uint4* dst = reinterpret_cast<uint4*>(Tout + (tile * 64 + rr) * 64 + 32 * h);
+                auto store = [&](const float* mult, long tile_at) {
+                    uint4* dst = reinterpret_cast<uint4*>(Tout + (tile_at * 64 + rr) * 64 + 32 * h);
 #pragma unroll
-                for (int m = 0; m < 4; ++m) {
-                    const float4 x0 = *reinterpret_cast<const float4*>(X + rr * LDX + 32 * h + 8 * m);
-                    const float4 x1 = *reinterpret_cast<const float4*>(X + rr * LDX + 32 * h + 8 * m + 4);
-                    const float4 a0 = *reinterpret_cast<const float4*>(al + 32 * h + 8 * m);
-                    const float4 a1 = *reinterpret_cast<const float4*>(al + 32 * h + 8 * m + 4);
-                    uint4 u;
-                    u.x = pack_bf16x2(x0.x * a0.x, x0.y * a0.y);
-                    u.y = pack_bf16x2(x0.z * a0.z, x0.w * a0.w);
-                    u.z = pack_bf16x2(x1.x * a1.x, x1.y * a1.y);
-                    u.w = pack_bf16x2(x1.z * a1.z, x1.w * a1.w);
-                    dst[m] = u;
+                    for (int m = 0; m < 4; ++m) {
+                        const float4 x0 = *reinterpret_cast<const float4*>(X + rr * LDX + 32 * h + 8 * m);
+                        const float4 x1 = *reinterpret_cast<const float4*>(X + rr * LDX + 32 * h + 8 * m + 4);
+                        const float4 a0 = *reinterpret_cast<const float4*>(mult + 32 * h + 8 * m);
+                        const float4 a1 = *reinterpret_cast<const float4*>(mult + 32 * h + 8 * m + 4);
+                        uint4 u;
+                        u.x = pack_bf16x2(x0.x * a0.x, x0.y * a0.y);
+                        u.y = pack_bf16x2(x0.z * a0.z, x0.w * a0.w);
+                        u.z = pack_bf16x2(x1.x * a1.x, x1.y * a1.y);
+                        u.w = pack_bf16x2(x1.z * a1.z, x1.w * a1.w);
+                        dst[m] = u;
+                    }
+                };
+                if constexpr (kGated) {
+                    store(mw, tile);
+                    store(abar, ntiles + tile);
+                    if (wt < 64) reinterpret_cast<float*>(Tout + 2 * ntiles * 4096)[tile * 64 + wt] = gl[wt];
+                } else {
+                    store(al, tile);
                 }
             }
         }
@@ -255,18 +333,26 @@ int sm_count() {
 }  // namespace
 
 cudaError_t launch_ut(const void* k, const void* beta, void* Tout, long BH, int T, uint32_t* err,
-                      unsigned long long limit_ns, int rule, cudaStream_t stream) {
+                      unsigned long long limit_ns, int rule, cudaStream_t stream, const float* g) {
     CUtensorMap mk;
     if (!tma_map_tokens(&mk, k, 128, T, BH)) return cudaErrorInvalidValue;
     const int nchunks = (T + 63) / 64;
     const long ntiles = BH * nchunks;
     const long grid = std::min<long>(ntiles, (long)sm_count() * kCtasPerSm);
-    static std::atomic<uint64_t> smem_set{0};
-    cudaError_t e = set_smem_limit_once(ut_kernel, (int)SMEM_BYTES, smem_set);
-    if (e != cudaSuccess) return e;
-    ut_kernel<<<(unsigned)grid, kThreads, SMEM_BYTES, stream>>>(mk, (const __nv_bfloat16*)beta,
-                                                                (__nv_bfloat16*)Tout, T, nchunks, ntiles, err,
-                                                                limit_ns, rule);
+    cudaError_t e;
+    if (g) {
+        static std::atomic<uint64_t> smem_set_g{0};
+        e = set_smem_limit_once(ut_kernel<true>, (int)SMEM_BYTES_G, smem_set_g);
+        if (e != cudaSuccess) return e;
+        ut_kernel<true><<<(unsigned)grid, kThreads, SMEM_BYTES_G, stream>>>(
+            mk, (const __nv_bfloat16*)beta, (__nv_bfloat16*)Tout, T, nchunks, ntiles, err, limit_ns, rule, g);
+    } else {
+        static std::atomic<uint64_t> smem_set{0};
+        e = set_smem_limit_once(ut_kernel<false>, (int)SMEM_BYTES, smem_set);
+        if (e != cudaSuccess) return e;
+        ut_kernel<false><<<(unsigned)grid, kThreads, SMEM_BYTES, stream>>>(
+            mk, (const __nv_bfloat16*)beta, (__nv_bfloat16*)Tout, T, nchunks, ntiles, err, limit_ns, rule, nullptr);
+    }
     return cudaGetLastError();
 }
 

@@ -126,6 +126,48 @@ int efla_chunk_fwd_ex(const void *q, const void *k, const void *v, const void *b
                       size_t workspace_bytes, efla_stream_t stream);
 
 /*
+ * Gated EFLA (Section 3.4 names the method's gated variant; App. F, "exact-flow
+ * formulation of Gated DeltaNet", survives on the pages only as a title, so the update
+ * below is this library's reading).  Each token carries a log-decay g_t (a forget gate
+ * e^{g_t}; g <= 0 decays) that joins the zero-order-hold ODE over the token's unit
+ * interval together with the write rate beta_t:
+ *     dS/dtau = g S - beta (k k^T S - k v^T),   tau in [0, 1].
+ * Its exact flow is
+ *     S_t = e^{g_t} (S_{t-1} - alpha_t k_t (k_t^T S_{t-1})) + abar_t k_t v_t^T,   o_t = S_t^T q_t,
+ *     alpha_t = beta_t phi1(beta_t lambda_t),  abar_t = beta_t phi1(beta_t lambda_t - g_t),
+ *     phi1(x) = (1 - e^{-x}) / x,
+ * which is efla_chunk_fwd's update at g = 0.  EFLA_RULE_EULER gives the gated delta rule
+ * (Gated DeltaNet), alpha = abar = beta.
+ *
+ * efla_chunk_fwd_gated_workspace_bytes -- workspace of efla_chunk_fwd_gated (0 for
+ * arguments it would reject).
+ */
+size_t efla_chunk_fwd_gated_workspace_bytes(int B, int H, int T, int d_k, int d_v, int chunk,
+                                            int dtype);
+
+/*
+ * efla_chunk_fwd_gated -- efla_chunk_fwd_ex with the gated flow above.
+ *   g [B,H,T] float32, the per-token log-decay (16-byte aligned, must not overlap o, S_T
+ *   or the workspace).  Every other argument, layout, supported shape and error is that of
+ *   efla_chunk_fwd_ex; the workspace must hold efla_chunk_fwd_gated_workspace_bytes.
+ *   g == NULL with B*H*T > 0 is EFLA_ERR_INVALID_ARG.
+ */
+int efla_chunk_fwd_gated(const void *q, const void *k, const void *v, const void *beta,
+                         const float *g, const float *S0, void *o, float *S_T, int B, int H, int T,
+                         int d_k, int d_v, int chunk, int dtype, int rule, void *workspace,
+                         size_t workspace_bytes, efla_stream_t stream);
+
+/*
+ * efla_recurrent_step_gated -- efla_recurrent_step_ex with the gated flow above:
+ *   g [N,H] float32, this token's log-decay per stream (16-byte aligned, must not overlap o
+ *   or S).  One pass over S: with r = k^T S, p = q^T S, c = q.k, d = e^g,
+ *   w = d alpha r - abar v:  S <- d S - k w^T,  o = d p - c w.
+ */
+int efla_recurrent_step_gated(const void *q, const void *k, const void *v, const void *beta,
+                              const float *g, float *S, void *o, int N, int H, int d_k, int d_v,
+                              int dtype, int rule, efla_stream_t stream);
+
+/*
  * efla_chunk_fwd_noalloc -- efla_chunk_fwd without a caller-provided workspace.
  * The paper has no counterpart: this is an integration variant for callers that cannot
  * allocate device memory, e.g. code embedded in a host runtime that owns every device

@@ -185,3 +185,31 @@ def test_backward_rejects_bad_arguments(efla):
         assert _bwd(L, bad) == INVALID, i
     assert _bwd(L, GOOD_B, B=0) == OK             # nothing to do, nothing launched
     assert _bwd(L, GOOD_B, H=0) == OK
+
+
+def test_gated_entry_points_validate_arguments(efla):
+    """efla_chunk_fwd_gated / efla_recurrent_step_gated: g is required, aligned and disjoint
+    from the outputs and the workspace; the rest is validated as for the ungated calls."""
+    L = efla.lib
+    q, k, v, b, s0, o, st, w = GOOD
+    gp = ctypes.c_void_p(0x90000000)
+    B, H, T, d = 1, 2, 128, 128
+    ws = L.efla_chunk_fwd_gated_workspace_bytes(B, H, T, d, d, 64, 1)
+    assert ws >= L.efla_chunk_fwd_workspace_bytes(B, H, T, d, d, 64, 1)
+    assert L.efla_chunk_fwd_gated_workspace_bytes(B, H, T, 96, 96, 64, 1) == 0
+    fwd = lambda g=gp, o_=o, **kw: L.efla_chunk_fwd_gated(q, k, v, b, g, s0, o_, st, kw.get("B", B), H, T, d, d,
+                                                          64, 1, kw.get("rule", 0), w, kw.get("ws", ws), None)
+    assert fwd(g=None) == INVALID                              # g required
+    assert fwd(g=ctypes.c_void_p(gp.value + 4)) == INVALID     # misaligned
+    assert fwd(o_=gp) == INVALID                               # o overlaps g
+    assert fwd(g=ctypes.c_void_p(w.value + 512), ws=1 << 24) == INVALID   # g inside the workspace
+    assert fwd(rule=5) == INVALID
+    assert fwd(ws=8) == INVALID
+    assert fwd(B=0) == OK and fwd(g=None, B=0) == OK
+    step = lambda g=gp, N=4, rule=0: L.efla_recurrent_step_gated(q, k, v, b, g, s0, o, N, 2, 128, 128, 0, rule,
+                                                                   None)
+    assert step(g=None) == INVALID
+    assert step(g=ctypes.c_void_p(gp.value + 8)) == INVALID
+    assert step(g=s0) == INVALID                               # g overlaps S
+    assert step(rule=-1) == INVALID
+    assert step(N=0) == OK

@@ -20,7 +20,7 @@ from typing import Optional
 import torch
 
 __all__ = ["ChunkWorkload", "DecodeWorkload", "CHUNK_WORKLOADS", "DECODE_WORKLOAD",
-           "make_chunk_inputs", "make_decode_state", "make_decode_steps"]
+           "make_chunk_inputs", "make_decode_state", "make_decode_steps", "make_log_decay"]
 
 
 @dataclasses.dataclass(frozen=True)
@@ -138,6 +138,18 @@ def make_chunk_inputs(w: ChunkWorkload, with_mask: bool = False) -> dict:
     if with_mask:
         out["corrupt"] = corrupt[:, 0, :, 0].clone()
     return out
+
+
+def make_log_decay(shape, seed: int, device="cpu") -> torch.Tensor:
+    """Per-token log-decay g of the gated flow, float32: g = -softplus(N(-3, 1.5)).
+
+    The pages give no gated workload; this draw makes most per-token decays e^g lie in
+    (0.9, 1) with a tail down to about 0.3, so a 64-token chunk decays its entry state by
+    e^-3 on average and the within-chunk ratios Gam_r / Gam_s span several orders.
+    """
+    g = torch.Generator(device=device).manual_seed(seed)
+    x = -3.0 + 1.5 * torch.randn(*shape, generator=g, device=device, dtype=torch.float32)
+    return -torch.nn.functional.softplus(x)
 
 
 def make_decode_state(w: DecodeWorkload, device="cpu") -> torch.Tensor:
