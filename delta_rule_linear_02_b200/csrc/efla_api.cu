@@ -116,11 +116,94 @@ static int chunk_fwd_impl(const void* q, const void* k, const void* v, const voi
         overlaps(workspace, workspace_bytes, S0, ns) || overlaps(workspace, workspace_bytes, S_T, ns) ||
         overlaps(workspace, workspace_bytes, g, ng))
         return EFLA_ERR_INVALID_ARG;
+    efla::Seqs seqs{nullptr, nullptr, 0, 0, T, 0};
     if (dtype == EFLA_DTYPE_BF16 && d_k == 128)
-        return from_cuda(efla::launch_chunk_tc(q, k, v, beta, S0, o, S_T, BH, T,
+        return from_cuda(efla::launch_chunk_tc(q, k, v, beta, S0, o, S_T, seqs, BH, BH, T, BH * ((T + 63) / 64),
                                                static_cast<uint32_t*>(workspace),
                                                static_cast<char*>(workspace) + kWorkspaceHeader, rule, s, g));
-    return from_cuda(efla::launch_chunk_simt(q, k, v, beta, S0, o, S_T, BH, T, d_k,
+    return from_cuda(efla::launch_chunk_simt(q, k, v, beta, S0, o, S_T, seqs, BH, T, d_k,
+                                             dtype == EFLA_DTYPE_BF16, rule, s, g));
+}
+
+// ---------------------------------------------------------------- packed variable-length batches
+// Workspace: [header 256 B][cu: N+1 int32][tileoff: N+1 int32][pad to 256 B][UT tiles].
+static size_t varlen_meta_bytes(int N) { return (((size_t)2 * (N + 1) * sizeof(int)) + 255) & ~(size_t)255; }
+
+// Checks the host offsets; returns the chunks per head (sum of ceil(len / 64)) or -1.
+static long varlen_chunks(const int* cu, int N) {
+    if (!cu || N < 0 || cu[0] != 0) return -1;
+    long chunks = 0;
+    for (int n = 0; n < N; ++n) {
+        if (cu[n + 1] < cu[n]) return -1;
+        chunks += (cu[n + 1] - cu[n] + 63) / 64;
+    }
+    return chunks;
+}
+
+size_t efla_chunk_fwd_varlen_workspace_bytes(const int* cu_seqlens, int N, int H, int d_k, int d_v, int chunk,
+                                             int dtype, int gated) {
+    if (check_chunk_shape(1, H, 0, d_k, d_v, chunk, dtype) != EFLA_OK || N < 1) return 0;
+    const long chunks = varlen_chunks(cu_seqlens, N);
+    if (chunks < 0 || (long long)N * H * 2 >= (1ll << 31)) return 0;
+    size_t tiles = 0;
+    if (dtype == EFLA_DTYPE_BF16 && d_k == 128) {
+        const long ntiles = chunks * H;
+        tiles = gated ? (size_t)ntiles * (2 * 8192 + 256) : (size_t)ntiles * 8192;
+    }
+    return kWorkspaceHeader + varlen_meta_bytes(N) + tiles;
+}
+
+int efla_chunk_fwd_varlen(const void* q, const void* k, const void* v, const void* beta, const float* g,
+                          const int* cu_seqlens, const float* S0, void* o, float* S_T, int N, int H, int d_k,
+                          int d_v, int chunk, int dtype, int rule, void* workspace, size_t workspace_bytes,
+                          efla_stream_t stream) {
+    int st = check_chunk_shape(1, H, 0, d_k, d_v, chunk, dtype);
+    if (st != EFLA_OK) return st;
+    if (rule != EFLA_RULE_EXACT && rule != EFLA_RULE_EULER) return EFLA_ERR_INVALID_ARG;
+    if (N < 1 || H < 1) return N == 0 || H == 0 ? EFLA_OK : EFLA_ERR_INVALID_ARG;
+    const long chunks = varlen_chunks(cu_seqlens, N);
+    if (chunks < 0) return EFLA_ERR_INVALID_ARG;
+    const size_t need = efla_chunk_fwd_varlen_workspace_bytes(cu_seqlens, N, H, d_k, d_v, chunk, dtype, g != nullptr);
+    if (need == 0) return EFLA_ERR_UNSUPPORTED;
+    if (!workspace || !aligned16(workspace) || workspace_bytes < need) return EFLA_ERR_INVALID_ARG;
+    const int total_T = cu_seqlens[N];
+    const size_t es = elem_size(dtype);
+    const size_t nqk = (size_t)H * total_T * d_k * es, nv = (size_t)H * total_T * d_v * es;
+    const size_t nb = (size_t)H * total_T * es, ns = (size_t)N * H * d_k * d_v * sizeof(float);
+    const size_t ng = g ? (size_t)H * total_T * sizeof(float) : 0;
+    if ((S0 && !aligned16(S0)) || (S_T && !aligned16(S_T)) || (g && !aligned16(g))) return EFLA_ERR_INVALID_ARG;
+    if (total_T > 0) {
+        if (!q || !k || !v || !beta || !o) return EFLA_ERR_INVALID_ARG;
+        if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(beta) || !aligned16(o))
+            return EFLA_ERR_INVALID_ARG;
+    }
+    const void* ins[6] = {q, k, v, beta, S0, g};
+    const size_t inn[6] = {nqk, nqk, nv, nb, ns, ng};
+    for (int j = 0; j < 6; ++j)
+        if (overlaps(o, nv, ins[j], inn[j]) || overlaps(workspace, workspace_bytes, ins[j], inn[j]) ||
+            (S_T != S0 && overlaps(S_T, ns, ins[j], inn[j])))
+            return EFLA_ERR_INVALID_ARG;
+    if (overlaps(o, nv, S_T, ns) || overlaps(o, nv, workspace, workspace_bytes) ||
+        overlaps(S_T, ns, workspace, workspace_bytes))
+        return EFLA_ERR_INVALID_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (total_T == 0) {   // every sequence empty: the states pass through unchanged
+        if (!S_T || S_T == S0) return EFLA_OK;
+        return from_cuda(S0 ? cudaMemcpyAsync(S_T, S0, ns, cudaMemcpyDeviceToDevice, s) : cudaMemsetAsync(S_T, 0, ns, s));
+    }
+    char* ws = static_cast<char*>(workspace);
+    int* cu_dev = reinterpret_cast<int*>(ws + kWorkspaceHeader);
+    int* tileoff_dev = cu_dev + (N + 1);
+    if (cudaMemcpyAsync(cu_dev, cu_seqlens, (size_t)(N + 1) * sizeof(int), cudaMemcpyHostToDevice, s) != cudaSuccess)
+        return EFLA_ERR_CUDA;
+    if (efla::launch_seq_prep(cu_dev, tileoff_dev, N, s) != cudaSuccess) return EFLA_ERR_CUDA;
+    efla::Seqs seqs{cu_dev, tileoff_dev, N, H, 0, chunks};
+    const long nstreams = (long)N * H;
+    char* scratch = ws + kWorkspaceHeader + varlen_meta_bytes(N);
+    if (dtype == EFLA_DTYPE_BF16 && d_k == 128)
+        return from_cuda(efla::launch_chunk_tc(q, k, v, beta, S0, o, S_T, seqs, nstreams, H, total_T, chunks * H,
+                                               static_cast<uint32_t*>(workspace), scratch, rule, s, g));
+    return from_cuda(efla::launch_chunk_simt(q, k, v, beta, S0, o, S_T, seqs, nstreams, total_T, d_k,
                                              dtype == EFLA_DTYPE_BF16, rule, s, g));
 }
 

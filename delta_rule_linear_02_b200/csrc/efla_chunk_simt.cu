@@ -84,8 +84,8 @@ __global__ void __launch_bounds__(kNT, 1) chunk_simt_kernel(const Tin* __restric
                                                             const Tin* __restrict__ beta,
                                                             const float* __restrict__ S0,
                                                             Tin* __restrict__ o,
-                                                            float* __restrict__ S_T, int T, int rule,
-                                                            const float* __restrict__ gdec = nullptr) {
+                                                            float* __restrict__ S_T, Seqs seqs, int Tdim,
+                                                            int rule, const float* __restrict__ gdec = nullptr) {
     using L = SimtSmem<D>;
     constexpr int NSL = D / 64;                 // d_v slices per stream
     extern __shared__ float smem[];
@@ -107,8 +107,10 @@ __global__ void __launch_bounds__(kNT, 1) chunk_simt_kernel(const Tin* __restric
     if constexpr (kGated) {
         if (tid < kC) ones[tid] = 1.f;
     }
-    const long bh = blockIdx.x / NSL;
+    const long bh = blockIdx.x / NSL;           // stream (state index)
     const int col0 = (blockIdx.x % NSL) * 64;   // first d_v column of this slice
+    const StreamJob jb = seqs.job(bh);
+    const int T = jb.len;
 
     // initial state slice
     for (int e = tid; e < D * 64; e += kNT) {
@@ -116,7 +118,7 @@ __global__ void __launch_bounds__(kNT, 1) chunk_simt_kernel(const Tin* __restric
         Ss[i * kLD + j] = S0 ? S0[(bh * D + i) * D + col0 + j] : 0.f;
     }
 
-    const long base = bh * (long)T;             // first token row of this stream
+    const long base = (long)jb.z * Tdim + jb.y0;  // first token row of this stream
     for (int r0 = 0; r0 < T; r0 += kC) {
         const int n = min(kC, T - r0);
         __syncthreads();                        // previous chunk is done with K, Q, V
@@ -299,33 +301,35 @@ __global__ void __launch_bounds__(kNT, 1) chunk_simt_kernel(const Tin* __restric
 
 template <typename Tin, int D, bool kGated>
 cudaError_t launch_t(const void* q, const void* k, const void* v, const void* beta, const float* S0,
-                     void* o, float* S_T, long BH, int T, int rule, const float* g, cudaStream_t stream) {
+                     void* o, float* S_T, const Seqs& seqs, long nstreams, int Tdim, int rule, const float* g,
+                     cudaStream_t stream) {
     using L = SimtSmem<D>;
     auto kern = chunk_simt_kernel<Tin, D, kGated>;
     static std::atomic<uint64_t> smem_set{0};
     cudaError_t err = set_smem_limit_once(kern, (int)L::kBytes, smem_set);
     if (err != cudaSuccess) return err;
-    kern<<<(unsigned)(BH * (D / 64)), kNT, L::kBytes, stream>>>((const Tin*)q, (const Tin*)k, (const Tin*)v,
-                                                                 (const Tin*)beta, S0, (Tin*)o, S_T, T, rule, g);
+    kern<<<(unsigned)(nstreams * (D / 64)), kNT, L::kBytes, stream>>>(
+        (const Tin*)q, (const Tin*)k, (const Tin*)v, (const Tin*)beta, S0, (Tin*)o, S_T, seqs, Tdim, rule, g);
     return cudaGetLastError();
 }
 
 template <typename Tin, int D>
 cudaError_t launch_g(const void* q, const void* k, const void* v, const void* beta, const float* S0,
-                     void* o, float* S_T, long BH, int T, int rule, const float* g, cudaStream_t stream) {
-    return g ? launch_t<Tin, D, true>(q, k, v, beta, S0, o, S_T, BH, T, rule, g, stream)
-             : launch_t<Tin, D, false>(q, k, v, beta, S0, o, S_T, BH, T, rule, nullptr, stream);
+                     void* o, float* S_T, const Seqs& seqs, long nstreams, int Tdim, int rule, const float* g,
+                     cudaStream_t stream) {
+    return g ? launch_t<Tin, D, true>(q, k, v, beta, S0, o, S_T, seqs, nstreams, Tdim, rule, g, stream)
+             : launch_t<Tin, D, false>(q, k, v, beta, S0, o, S_T, seqs, nstreams, Tdim, rule, nullptr, stream);
 }
 }  // namespace
 
 cudaError_t launch_chunk_simt(const void* q, const void* k, const void* v, const void* beta,
-                              const float* S0, void* o, float* S_T, long BH, int T, int D, bool bf16,
-                              int rule, cudaStream_t stream, const float* g) {
+                              const float* S0, void* o, float* S_T, const Seqs& seqs, long nstreams, int Tdim,
+                              int D, bool bf16, int rule, cudaStream_t stream, const float* g) {
     if (bf16)
-        return D == 128 ? launch_g<__nv_bfloat16, 128>(q, k, v, beta, S0, o, S_T, BH, T, rule, g, stream)
-                        : launch_g<__nv_bfloat16, 64>(q, k, v, beta, S0, o, S_T, BH, T, rule, g, stream);
-    return D == 128 ? launch_g<float, 128>(q, k, v, beta, S0, o, S_T, BH, T, rule, g, stream)
-                    : launch_g<float, 64>(q, k, v, beta, S0, o, S_T, BH, T, rule, g, stream);
+        return D == 128 ? launch_g<__nv_bfloat16, 128>(q, k, v, beta, S0, o, S_T, seqs, nstreams, Tdim, rule, g, stream)
+                        : launch_g<__nv_bfloat16, 64>(q, k, v, beta, S0, o, S_T, seqs, nstreams, Tdim, rule, g, stream);
+    return D == 128 ? launch_g<float, 128>(q, k, v, beta, S0, o, S_T, seqs, nstreams, Tdim, rule, g, stream)
+                    : launch_g<float, 64>(q, k, v, beta, S0, o, S_T, seqs, nstreams, Tdim, rule, g, stream);
 }
 
 }  // namespace efla

@@ -221,7 +221,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_t,
                 const float* __restrict__ S0, __nv_bfloat16* __restrict__ o, float* __restrict__ S_T,
-                int T, uint32_t* __restrict__ err, unsigned long long limit_ns,
+                Seqs seqs, int Tdim, uint32_t* __restrict__ err, unsigned long long limit_ns,
                 const float* __restrict__ gl_all, long ntiles) {
     using L = Lay<kGated>;
     constexpr uint32_t KVT_K = L::KVT_K, KVT_V = L::KVT_V, KVT_T = L::KVT_T, KVT_BYTES = L::KVT_BYTES;
@@ -236,10 +236,22 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int q = warp & 3;                                                  // TMEM lane quarter
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
-    const int bh = blockIdx.x >> 1;
+    const long sidx = blockIdx.x >> 1;                                     // stream (state index)
+    const StreamJob jb = seqs.job(sidx);
     const int col0 = (blockIdx.x & 1) * 64;
+    const int T = jb.len, zc = jb.z, y0 = jb.y0;
     const int nchunks = (T + 63) / 64;
-    const size_t tok0 = (size_t)bh * T;
+    const size_t tok0 = (size_t)zc * Tdim + y0;
+    if (nchunks == 0) {   // an empty sequence: the state passes through (nothing else runs)
+        if (S_T) {
+            for (int e = tid; e < kD * 64; e += kThreads) {
+                const int i = e >> 6, j = e & 63;
+                const size_t at = ((size_t)sidx * kD + i) * kD + col0 + j;
+                S_T[at] = S0 ? S0[at] : 0.f;
+            }
+        }
+        return;
+    }
 
     if (tid == 0) {
         for (int i = 0; i < (int)NBAR; ++i) mbar_init(ctl.bar + i, bar_count(i));
@@ -274,13 +286,13 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     uint8_t* st = sm + kvt(c);
                     uint64_t* full = ctl.b(B_KVT_FULL + s);
                     mbar_arrive_expect_tx(full, L::KVT_TX);
-                    tma_load_3d(st + KVT_K, &tm_k, full, 0, t0, bh);
-                    tma_load_3d(st + KVT_K + TILE, &tm_k, full, 64, t0, bh);
-                    tma_load_3d(st + KVT_V, &tm_v, full, col0, t0, bh);
-                    tma_load_2d(st + KVT_T, &tm_t, full, 0, (bh * nchunks + c) * 64);
+                    tma_load_3d(st + KVT_K, &tm_k, full, 0, y0 + t0, zc);
+                    tma_load_3d(st + KVT_K + TILE, &tm_k, full, 64, y0 + t0, zc);
+                    tma_load_3d(st + KVT_V, &tm_v, full, col0, y0 + t0, zc);
+                    tma_load_2d(st + KVT_T, &tm_t, full, 0, (int)((jb.tile0 + c) * 64));
                     if constexpr (kGated) {
-                        tma_load_2d(st + L::KVT_TU, &tm_t, full, 0, (int)((ntiles + (long)bh * nchunks + c) * 64));
-                        bulk_load(st + L::KVT_GL, gl_all + ((long)bh * nchunks + c) * 64, 256, full);
+                        tma_load_2d(st + L::KVT_TU, &tm_t, full, 0, (int)((ntiles + jb.tile0 + c) * 64));
+                        bulk_load(st + L::KVT_GL, gl_all + (jb.tile0 + c) * 64, 256, full);
                     }
                     kvt_issued = c + 1;
                 }
@@ -290,18 +302,18 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     uint8_t* st = sm + qst(c);
                     uint64_t* full = ctl.b(B_Q_FULL + s);
                     mbar_arrive_expect_tx(full, 2 * TILE);
-                    tma_load_3d(st, &tm_q, full, 0, t0, bh);
-                    tma_load_3d(st + TILE, &tm_q, full, 64, t0, bh);
+                    tma_load_3d(st, &tm_q, full, 0, y0 + t0, zc);
+                    tma_load_3d(st + TILE, &tm_q, full, 64, y0 + t0, zc);
                     q_issued = c + 1;
                 }
                 if (c + 3 < nchunks) {      // warm L2 for the chunk three ahead
-                    const int t3 = t0 + 192;
-                    tma_prefetch_l2_3d(&tm_k, 0, t3, bh);
-                    tma_prefetch_l2_3d(&tm_k, 64, t3, bh);
-                    tma_prefetch_l2_3d(&tm_v, col0, t3, bh);
-                    tma_prefetch_l2_3d(&tm_q, 0, t3, bh);
-                    tma_prefetch_l2_3d(&tm_q, 64, t3, bh);
-                    tma_prefetch_l2_2d(&tm_t, 0, (bh * nchunks + c + 3) * 64);
+                    const int t3 = y0 + t0 + 192;
+                    tma_prefetch_l2_3d(&tm_k, 0, t3, zc);
+                    tma_prefetch_l2_3d(&tm_k, 64, t3, zc);
+                    tma_prefetch_l2_3d(&tm_v, col0, t3, zc);
+                    tma_prefetch_l2_3d(&tm_q, 0, t3, zc);
+                    tma_prefetch_l2_3d(&tm_q, 64, t3, zc);
+                    tma_prefetch_l2_2d(&tm_t, 0, (int)((jb.tile0 + c + 3) * 64));
                 }
             }
             // no copy may land after exit
@@ -545,7 +557,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             return 1.f;
         };
         {   // initial state
-            const float* src = S0 ? S0 + ((size_t)bh * kD + ct) * kD + col0 + cc : nullptr;
+            const float* src = S0 ? S0 + ((size_t)sidx * kD + ct) * kD + col0 + cc : nullptr;
             const float dec0 = decay_of(0);
 #pragma unroll
             for (int qd = 0; qd < 2; ++qd) {
@@ -608,7 +620,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
                 for (int j = 0; j < 4; ++j) st_chunk(sm + OFF_SB + sw128_off(ct, 4 * ch + j), t + 8 * j);
                 if (c == nchunks - 1 && S_T) {
-                    float* dst = S_T + ((size_t)bh * kD + ct) * kD + col0 + cc;
+                    float* dst = S_T + ((size_t)sidx * kD + ct) * kD + col0 + cc;
 #pragma unroll
                     for (int j = 0; j < 32; j += 4)
                         *reinterpret_cast<float4*>(dst + j) = make_float4(t[j], t[j + 1], t[j + 2], t[j + 3]);
@@ -668,30 +680,28 @@ size_t chunk_tc_gated_workspace_bytes(long BH, int T) {
 }
 
 cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const void* beta, const float* S0,
-                            void* o, float* S_T, long BH, int T, uint32_t* err, void* scratch,
-                            int rule, cudaStream_t stream, const float* g) {
-    const int nchunks = (T + 63) / 64;
-    const long ntiles = BH * nchunks;
-    cudaError_t e = launch_ut(k, beta, scratch, BH, T, err, kWaitLimitNs, rule, stream, g);
+                            void* o, float* S_T, const Seqs& seqs, long nstreams, long Z, int Tdim, long ntiles,
+                            uint32_t* err, void* scratch, int rule, cudaStream_t stream, const float* g) {
+    cudaError_t e = launch_ut(k, beta, scratch, seqs, Z, Tdim, ntiles, err, kWaitLimitNs, rule, stream, g);
     if (e != cudaSuccess) return e;
     CUtensorMap mq, mk, mv, mt;
-    if (!tma_map_tokens(&mq, q, kD, T, BH) || !tma_map_tokens(&mk, k, kD, T, BH) ||
-        !tma_map_tokens(&mv, v, kD, T, BH) || !tma_map_rows64(&mt, scratch, (g ? 2 : 1) * ntiles * 64))
+    if (!tma_map_tokens(&mq, q, kD, Tdim, Z) || !tma_map_tokens(&mk, k, kD, Tdim, Z) ||
+        !tma_map_tokens(&mv, v, kD, Tdim, Z) || !tma_map_rows64(&mt, scratch, std::max<long>(1, (g ? 2 : 1) * ntiles) * 64))
         return cudaErrorInvalidValue;
     if (g) {
         const float* gl = reinterpret_cast<const float*>(static_cast<const char*>(scratch) + ntiles * 8192 * 2);
         static std::atomic<uint64_t> smem_set_g{0};
         e = set_smem_limit_once(chunk_tc_kernel<true>, (int)Lay<true>::SMEM_BYTES, smem_set_g);
         if (e != cudaSuccess) return e;
-        chunk_tc_kernel<true><<<(unsigned)(BH * 2), kThreads, Lay<true>::SMEM_BYTES, stream>>>(
-            mq, mk, mv, mt, S0, (__nv_bfloat16*)o, S_T, T, err, kWaitLimitNs, gl, ntiles);
+        chunk_tc_kernel<true><<<(unsigned)(nstreams * 2), kThreads, Lay<true>::SMEM_BYTES, stream>>>(
+            mq, mk, mv, mt, S0, (__nv_bfloat16*)o, S_T, seqs, Tdim, err, kWaitLimitNs, gl, ntiles);
         return cudaGetLastError();
     }
     static std::atomic<uint64_t> smem_set{0};
     e = set_smem_limit_once(chunk_tc_kernel<false>, (int)Lay<false>::SMEM_BYTES, smem_set);
     if (e != cudaSuccess) return e;
-    chunk_tc_kernel<false><<<(unsigned)(BH * 2), kThreads, Lay<false>::SMEM_BYTES, stream>>>(
-        mq, mk, mv, mt, S0, (__nv_bfloat16*)o, S_T, T, err, kWaitLimitNs, nullptr, ntiles);
+    chunk_tc_kernel<false><<<(unsigned)(nstreams * 2), kThreads, Lay<false>::SMEM_BYTES, stream>>>(
+        mq, mk, mv, mt, S0, (__nv_bfloat16*)o, S_T, seqs, Tdim, err, kWaitLimitNs, nullptr, ntiles);
     return cudaGetLastError();
 }
 

@@ -93,7 +93,7 @@ __device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, vol
 template <bool kGated>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 ut_kernel(const __grid_constant__ CUtensorMap tm_k, const __nv_bfloat16* __restrict__ beta,
-          __nv_bfloat16* __restrict__ Tout, int T, int nchunks, long ntiles, uint32_t* __restrict__ err,
+          __nv_bfloat16* __restrict__ Tout, Seqs seqs, int Tdim, long ntiles, uint32_t* __restrict__ err,
           unsigned long long limit_ns, int rule, const float* __restrict__ gdec) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -146,10 +146,11 @@ ut_kernel(const __grid_constant__ CUtensorMap tm_k, const __nv_bfloat16* __restr
         auto load = [&](int j) {
             if (lane == 0) {
                 const long tile = first + (long)j * step;
-                const int bh = (int)(tile / nchunks), c = (int)(tile % nchunks);
+                int c;
+                const StreamJob jb = seqs.tile(tile, &c);
                 mbar_arrive_expect_tx(bar + B_FULL, 2 * TILE);
-                tma_load_3d(sm + OFF_K, &tm_k, bar + B_FULL, 0, c * 64, bh);
-                tma_load_3d(sm + OFF_K + TILE, &tm_k, bar + B_FULL, 64, c * 64, bh);
+                tma_load_3d(sm + OFF_K, &tm_k, bar + B_FULL, 0, jb.y0 + c * 64, jb.z);
+                tma_load_3d(sm + OFF_K + TILE, &tm_k, bar + B_FULL, 64, jb.y0 + c * 64, jb.z);
             }
             __syncwarp();
         };
@@ -184,16 +185,18 @@ ut_kernel(const __grid_constant__ CUtensorMap tm_k, const __nv_bfloat16* __restr
         auto beta_of = [&](int j) -> float {
             if (j >= ntile || wt >= 64) return 0.f;
             const long tile = first + (long)j * step;
-            const long bh = tile / nchunks;
-            const int t = (int)(tile % nchunks) * 64 + wt;
-            return t < T ? __bfloat162float(beta[bh * T + t]) : 0.f;
+            int c;
+            const StreamJob jb = seqs.tile(tile, &c);
+            const int t = c * 64 + wt;
+            return t < jb.len ? __bfloat162float(beta[(long)jb.z * Tdim + jb.y0 + t]) : 0.f;
         };
         auto g_of = [&](int j) -> float {
             if (j >= ntile || wt >= 64) return 0.f;
             const long tile = first + (long)j * step;
-            const long bh = tile / nchunks;
-            const int t = (int)(tile % nchunks) * 64 + wt;
-            return t < T ? gdec[bh * T + t] : 0.f;
+            int c;
+            const StreamJob jb = seqs.tile(tile, &c);
+            const int t = c * 64 + wt;
+            return t < jb.len ? gdec[(long)jb.z * Tdim + jb.y0 + t] : 0.f;
         };
         float beta_next = beta_of(0);
         float g_next = 0.f;
@@ -332,12 +335,12 @@ int sm_count() {
 }
 }  // namespace
 
-cudaError_t launch_ut(const void* k, const void* beta, void* Tout, long BH, int T, uint32_t* err,
-                      unsigned long long limit_ns, int rule, cudaStream_t stream, const float* g) {
+cudaError_t launch_ut(const void* k, const void* beta, void* Tout, const Seqs& seqs, long Z, int Tdim,
+                      long ntiles, uint32_t* err, unsigned long long limit_ns, int rule, cudaStream_t stream,
+                      const float* g) {
+    if (ntiles == 0) return cudaSuccess;
     CUtensorMap mk;
-    if (!tma_map_tokens(&mk, k, 128, T, BH)) return cudaErrorInvalidValue;
-    const int nchunks = (T + 63) / 64;
-    const long ntiles = BH * nchunks;
+    if (!tma_map_tokens(&mk, k, 128, Tdim, Z)) return cudaErrorInvalidValue;
     const long grid = std::min<long>(ntiles, (long)sm_count() * kCtasPerSm);
     cudaError_t e;
     if (g) {
@@ -345,13 +348,13 @@ cudaError_t launch_ut(const void* k, const void* beta, void* Tout, long BH, int 
         e = set_smem_limit_once(ut_kernel<true>, (int)SMEM_BYTES_G, smem_set_g);
         if (e != cudaSuccess) return e;
         ut_kernel<true><<<(unsigned)grid, kThreads, SMEM_BYTES_G, stream>>>(
-            mk, (const __nv_bfloat16*)beta, (__nv_bfloat16*)Tout, T, nchunks, ntiles, err, limit_ns, rule, g);
+            mk, (const __nv_bfloat16*)beta, (__nv_bfloat16*)Tout, seqs, Tdim, ntiles, err, limit_ns, rule, g);
     } else {
         static std::atomic<uint64_t> smem_set{0};
         e = set_smem_limit_once(ut_kernel<false>, (int)SMEM_BYTES, smem_set);
         if (e != cudaSuccess) return e;
         ut_kernel<false><<<(unsigned)grid, kThreads, SMEM_BYTES, stream>>>(
-            mk, (const __nv_bfloat16*)beta, (__nv_bfloat16*)Tout, T, nchunks, ntiles, err, limit_ns, rule, nullptr);
+            mk, (const __nv_bfloat16*)beta, (__nv_bfloat16*)Tout, seqs, Tdim, ntiles, err, limit_ns, rule, nullptr);
     }
     return cudaGetLastError();
 }

@@ -168,6 +168,38 @@ int efla_recurrent_step_gated(const void *q, const void *k, const void *v, const
                               int dtype, int rule, efla_stream_t stream);
 
 /*
+ * Packed variable-length batches (Section 3.3's chunkwise form, applied to each sequence
+ * on its own; the pages note that long and mixed contexts are where recurrent memories are
+ * used, App. A).  N sequences of different lengths are packed head-major along the token
+ * axis, with no padding between them:
+ *   q, k [H, total_T, d_k], v, o [H, total_T, d_v], beta [H, total_T]   (dtype)
+ *   g    [H, total_T] float32 log-decay for the gated flow, or NULL (ungated)
+ *   S0, S_T [N, H, d_k, d_v] float32 (each may be NULL; S_T may alias S0)
+ *   cu_seqlens: HOST array of N + 1 int32 offsets, cu_seqlens[0] = 0, non-decreasing,
+ *   total_T = cu_seqlens[N]; sequence n is tokens cu_seqlens[n] .. cu_seqlens[n+1] - 1 of every
+ *   head.  Each (sequence, head) is an independent recurrence from its own S0 slice; its
+ *   chunks start at its first token, and an empty sequence passes its state through.
+ * The call copies cu_seqlens into the workspace (cudaMemcpyAsync; from pageable host memory
+ * that copy may synchronise the host with `stream`, and it cannot be captured in a graph).
+ *
+ * efla_chunk_fwd_varlen_workspace_bytes -- workspace bytes for these offsets (gated != 0 for
+ * the gated flow), or 0 for arguments efla_chunk_fwd_varlen would reject.
+ */
+size_t efla_chunk_fwd_varlen_workspace_bytes(const int *cu_seqlens, int N, int H, int d_k, int d_v,
+                                             int chunk, int dtype, int gated);
+
+/*
+ * efla_chunk_fwd_varlen -- the chunked forward (or, with g, the gated forward) over a packed
+ * variable-length batch, layouts above.  Supported shapes, dtypes, rules, alignment and
+ * errors are those of efla_chunk_fwd_ex; cu_seqlens that are not valid offsets are
+ * EFLA_ERR_INVALID_ARG.  No input may overlap o, S_T or the workspace.
+ */
+int efla_chunk_fwd_varlen(const void *q, const void *k, const void *v, const void *beta,
+                          const float *g, const int *cu_seqlens, const float *S0, void *o, float *S_T,
+                          int N, int H, int d_k, int d_v, int chunk, int dtype, int rule,
+                          void *workspace, size_t workspace_bytes, efla_stream_t stream);
+
+/*
  * efla_chunk_fwd_noalloc -- efla_chunk_fwd without a caller-provided workspace.
  * The paper has no counterpart: this is an integration variant for callers that cannot
  * allocate device memory, e.g. code embedded in a host runtime that owns every device

@@ -213,3 +213,24 @@ def test_gated_entry_points_validate_arguments(efla):
     assert step(g=s0) == INVALID                               # g overlaps S
     assert step(rule=-1) == INVALID
     assert step(N=0) == OK
+
+
+def test_varlen_entry_point_validates_offsets(efla):
+    L = efla.lib
+    import ctypes as C
+    arr = lambda xs: (C.c_int * len(xs))(*xs)
+    q, k, v, b, s0, o, st, w = GOOD
+    ok_cu = arr([0, 64, 64, 200])
+    ws = L.efla_chunk_fwd_varlen_workspace_bytes(ok_cu, 3, 2, 128, 128, 64, 1, 0)
+    assert ws > 0 and L.efla_chunk_fwd_varlen_workspace_bytes(ok_cu, 3, 2, 128, 128, 64, 1, 1) > ws
+    for bad in ([1, 64, 64, 200], [0, 64, 63, 200]):          # cu[0] != 0, decreasing
+        assert L.efla_chunk_fwd_varlen_workspace_bytes(arr(bad), 3, 2, 128, 128, 64, 1, 0) == 0
+        assert L.efla_chunk_fwd_varlen(q, k, v, b, None, arr(bad), s0, o, st, 3, 2, 128, 128, 64, 1, 0, w, 1 << 26,
+                                       None) == INVALID
+    call = lambda cu=ok_cu, N=3, ws_=ws, rule=0, d=128: L.efla_chunk_fwd_varlen(
+        q, k, v, b, None, cu, s0, o, st, N, 2, d, d, 64, 1, rule, w, ws_, None)
+    assert call(d=96) == UNSUPPORTED
+    assert call(rule=4) == INVALID
+    assert call(ws_=16) == INVALID
+    assert call(cu=None) == INVALID
+    assert call(N=0) == OK

@@ -20,7 +20,8 @@ from typing import Optional
 import torch
 
 __all__ = ["ChunkWorkload", "DecodeWorkload", "CHUNK_WORKLOADS", "DECODE_WORKLOAD",
-           "make_chunk_inputs", "make_decode_state", "make_decode_steps", "make_log_decay"]
+           "make_chunk_inputs", "make_decode_state", "make_decode_steps", "make_log_decay",
+           "make_varlen_inputs", "varlen_lengths"]
 
 
 @dataclasses.dataclass(frozen=True)
@@ -137,6 +138,37 @@ def make_chunk_inputs(w: ChunkWorkload, with_mask: bool = False) -> dict:
     }
     if with_mask:
         out["corrupt"] = corrupt[:, 0, :, 0].clone()
+    return out
+
+
+def varlen_lengths(n: int, total: int, seed: int, min_len: int = 1) -> list:
+    """n sequence lengths summing to `total`, a log-uniform mix (short and long sequences
+    together, as in packed training batches); at least min_len each."""
+    g = torch.Generator().manual_seed(seed)
+    w = torch.exp(torch.rand(n, generator=g) * 4.0)            # weights spread over e^0 .. e^4
+    raw = (w / w.sum() * (total - n * min_len)).floor().to(torch.int64) + min_len
+    raw[-1] += total - int(raw.sum())
+    return [int(x) for x in raw]
+
+
+def make_varlen_inputs(w: ChunkWorkload, lengths, with_g: bool = False) -> dict:
+    """A packed batch: sequence n drawn as a one-stream workload of w's distribution with
+    length lengths[n], all heads, packed head-major along the token axis.
+
+    Returns q, k [H, total_T, d_k], v [H, total_T, d_v], beta [H, total_T] (w.dtype),
+    S0 [N, H, d_k, d_v] float32 or None, cu (list of N + 1 offsets) and, with with_g,
+    g [H, total_T] float32 (make_log_decay).
+    """
+    parts = [make_chunk_inputs(w.replace(B=1, T=int(L), seed=w.seed + 31 * n)) for n, L in enumerate(lengths)]
+    cat = lambda key: torch.cat([p[key][0] for p in parts], dim=1).contiguous()
+    out = {"q": cat("q"), "k": cat("k"), "v": cat("v"), "beta": cat("beta")}
+    out["S0"] = None if w.s0_std is None else torch.cat([p["S0"] for p in parts], dim=0).contiguous()
+    cu = [0]
+    for L in lengths:
+        cu.append(cu[-1] + int(L))
+    out["cu"] = cu
+    if with_g:
+        out["g"] = make_log_decay((w.H, cu[-1]), w.seed + 7)
     return out
 
 
