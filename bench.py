@@ -590,9 +590,11 @@ def main():
     # ---- the other forward workloads (long context, stiff keys): tokens/s and roofline
     # fraction of a few forwards each, inputs resident in HBM, CUDA events around the calls
     others = {}
-    for name in ([] if args.other_steps <= 0 else ["longctx_bf16", "stiff_bf16", "lm1p3b_bf16_gated"]):
+    for name in ([] if args.other_steps <= 0 else ["longctx_bf16", "longctx_bf16_segmented", "stiff_bf16",
+                                                    "lm1p3b_bf16_gated"]):
         gated = name.endswith("_gated")
-        wo = workloads.CHUNK_WORKLOADS[name.removesuffix("_gated")]
+        segmented = name.endswith("_segmented")
+        wo = workloads.CHUNK_WORKLOADS[name.removesuffix("_gated").removesuffix("_segmented")]
         wo = wo.replace(seed=wo.seed + 1000 * rank)
         xo = {k_: (None if v_ is None else v_.to(dev)) for k_, v_ in workloads.make_chunk_inputs(wo).items()}
         oo = torch.empty(wo.B, wo.H, wo.T, wo.dv, dtype=wo.dtype, device=dev)
@@ -603,6 +605,11 @@ def main():
                               dtype=torch.uint8, device=dev)
             call = lambda: efla.efla_chunk_fwd_gated(xo["q"], xo["k"], xo["v"], xo["beta"], go, xo["S0"], o=oo,
                                                      S_T=So, workspace=wso, stream=stream)
+        elif segmented:   # long streams as a segmented scan, the library's segment count
+            wso = torch.zeros(efla.lib.efla_chunk_fwd_segmented_workspace_bytes(wo.B, wo.H, wo.T, wo.dk, wo.dv, 64, 1,
+                                                                                 0, 0), dtype=torch.uint8, device=dev)
+            call = lambda: efla.efla_chunk_fwd_segmented(xo["q"], xo["k"], xo["v"], xo["beta"], xo["S0"], o=oo,
+                                                         S_T=So, workspace=wso, stream=stream)
         else:
             wso = efla.new_workspace(wo.B, wo.H, wo.T, wo.dk, wo.dv, 64, wo.dtype, dev)
             call = lambda: efla.efla_chunk_fwd(xo["q"], xo["k"], xo["v"], xo["beta"], xo["S0"], o=oo, S_T=So,
@@ -626,7 +633,7 @@ def main():
                         "steps": args.other_steps,
                         "config": {"B": wo.B, "H": wo.H, "T": wo.T, "d_k": wo.dk, "d_v": wo.dv, "chunk": 64},
                         "roofline": roofline_record(ob, of, oms * 1e-3, hbm, tc, peak_kind),
-                        "gpu_launches": 2 * args.other_steps}
+                        "gpu_launches": (4 if segmented else 2) * args.other_steps}
         del xo, wso, oo, So
 
     cpu = None

@@ -2,6 +2,7 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <algorithm>
 #include <atomic>
 
 #include "../../include/efla.h"
@@ -123,6 +124,94 @@ static int chunk_fwd_impl(const void* q, const void* k, const void* v, const voi
                                                static_cast<char*>(workspace) + kWorkspaceHeader, rule, s, g));
     return from_cuda(efla::launch_chunk_simt(q, k, v, beta, S0, o, S_T, seqs, BH, T, d_k,
                                              dtype == EFLA_DTYPE_BF16, rule, s, g));
+}
+
+// ---------------------------------------------------------------- segmented scan of long streams
+static int device_sms() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return 148;
+    return n;
+}
+
+// Segments per stream: the request, or (0) the most whose chain CTAs still fit one wave
+// (B*H*(4G - 2) <= SMs), each segment at least 8 chunks long.
+static int seg_count(long BH, int T, int segments) {
+    const int nchunks = (T + 63) / 64;
+    int G = segments;
+    if (G <= 0) {
+        G = 1;
+        while (BH * (4L * (G + 1) - 2) <= device_sms()) ++G;
+    }
+    G = std::min(G, std::max(1, nchunks / 8));
+    return std::max(1, G);
+}
+
+static size_t seg_workspace(long BH, int T, int G, bool gated) {
+    const size_t tiles = gated ? efla::chunk_tc_gated_workspace_bytes(BH, T) : efla::chunk_tc_workspace_bytes(BH, T);
+    const size_t mats = (size_t)BH * G * 128 * 128 * sizeof(float);
+    return kWorkspaceHeader + tiles + 3 * mats + (size_t)BH * T * 128 * 2;
+}
+
+size_t efla_chunk_fwd_segmented_workspace_bytes(int B, int H, int T, int d_k, int d_v, int chunk, int dtype, int gated,
+                                                int segments) {
+    if (check_chunk_shape(B, H, T, d_k, d_v, chunk, dtype) != EFLA_OK || segments < 0) return 0;
+    const long BH = (long)B * H;
+    if (!(dtype == EFLA_DTYPE_BF16 && d_k == 128) || BH == 0 || seg_count(BH, T, segments) == 1)
+        return gated ? efla_chunk_fwd_gated_workspace_bytes(B, H, T, d_k, d_v, chunk, dtype)
+                     : efla_chunk_fwd_workspace_bytes(B, H, T, d_k, d_v, chunk, dtype);
+    return seg_workspace(BH, T, seg_count(BH, T, segments), gated);
+}
+
+int efla_chunk_fwd_segmented(const void* q, const void* k, const void* v, const void* beta, const float* g,
+                             const float* S0, void* o, float* S_T, int B, int H, int T, int d_k, int d_v, int chunk,
+                             int dtype, int rule, int segments, void* workspace, size_t workspace_bytes,
+                             efla_stream_t stream) {
+    int st = check_chunk_shape(B, H, T, d_k, d_v, chunk, dtype);
+    if (st != EFLA_OK) return st;
+    if (segments < 0) return EFLA_ERR_INVALID_ARG;
+    const long BH = (long)B * H;
+    const int G = BH > 0 ? seg_count(BH, T, segments) : 1;
+    if (!(dtype == EFLA_DTYPE_BF16 && d_k == 128) || BH == 0 || T == 0 || G == 1)
+        return chunk_fwd_impl(q, k, v, beta, g, S0, o, S_T, B, H, T, d_k, d_v, chunk, dtype, rule, workspace,
+                              workspace_bytes, stream);
+    // the argument checks of the plain forward (nothing is launched by them)
+    if (rule != EFLA_RULE_EXACT && rule != EFLA_RULE_EULER) return EFLA_ERR_INVALID_ARG;
+    const size_t need = seg_workspace(BH, T, G, g != nullptr);
+    if (!workspace || !aligned16(workspace) || workspace_bytes < need) return EFLA_ERR_INVALID_ARG;
+    if (!q || !k || !v || !beta || !o) return EFLA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(beta) || !aligned16(o) ||
+        (S0 && !aligned16(S0)) || (S_T && !aligned16(S_T)) || (g && !aligned16(g)))
+        return EFLA_ERR_INVALID_ARG;
+    const size_t nx = (size_t)BH * T * d_k * 2, nb = (size_t)BH * T * 2, ns = (size_t)BH * d_k * d_v * 4;
+    const size_t ng = g ? (size_t)BH * T * 4 : 0;
+    const void* ins[6] = {q, k, v, beta, S0, g};
+    const size_t inn[6] = {nx, nx, nx, nb, ns, ng};
+    for (int j = 0; j < 6; ++j)
+        if (overlaps(o, nx, ins[j], inn[j]) || overlaps(workspace, workspace_bytes, ins[j], inn[j]) ||
+            (S_T != S0 && overlaps(S_T, ns, ins[j], inn[j])))
+            return EFLA_ERR_INVALID_ARG;
+    if (overlaps(o, nx, S_T, ns) || overlaps(o, nx, workspace, workspace_bytes) ||
+        overlaps(S_T, ns, workspace, workspace_bytes))
+        return EFLA_ERR_INVALID_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+    char* ws = static_cast<char*>(workspace);
+    char* scratch = ws + kWorkspaceHeader;
+    const size_t tiles = g ? efla::chunk_tc_gated_workspace_bytes(BH, T) : efla::chunk_tc_workspace_bytes(BH, T);
+    const size_t mats = (size_t)BH * G * 128 * 128 * sizeof(float);
+    efla::SegPlan plan;
+    plan.G = G;
+    plan.seg_chunks = ((T + 63) / 64 + G - 1) / G;
+    plan.Sloc = reinterpret_cast<float*>(scratch + tiles);
+    plan.Phi = reinterpret_cast<float*>(scratch + tiles + mats);
+    float* Sin = reinterpret_cast<float*>(scratch + tiles + 2 * mats);
+    plan.R = reinterpret_cast<__nv_bfloat16*>(scratch + tiles + 3 * mats);
+    efla::Seqs seqs{nullptr, nullptr, 0, 0, T, 0};
+    cudaError_t e = efla::launch_chunk_tc(q, k, v, beta, S0, o, S_T, seqs, BH, BH, T, BH * ((T + 63) / 64),
+                                          static_cast<uint32_t*>(workspace), scratch, rule, s, g, plan);
+    if (e == cudaSuccess) e = efla::launch_seg_combine(plan, S0, S_T, Sin, BH, s);
+    if (e == cudaSuccess) e = efla::launch_seg_correct(plan, Sin, static_cast<__nv_bfloat16*>(o), BH, T, s);
+    return from_cuda(e);
 }
 
 // ---------------------------------------------------------------- packed variable-length batches

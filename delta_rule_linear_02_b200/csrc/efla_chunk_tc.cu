@@ -222,7 +222,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_t,
                 const float* __restrict__ S0, __nv_bfloat16* __restrict__ o, float* __restrict__ S_T,
                 Seqs seqs, int Tdim, uint32_t* __restrict__ err, unsigned long long limit_ns,
-                const float* __restrict__ gl_all, long ntiles) {
+                const float* __restrict__ gl_all, long ntiles, SegPlan seg) {
     using L = Lay<kGated>;
     constexpr uint32_t KVT_K = L::KVT_K, KVT_V = L::KVT_V, KVT_T = L::KVT_T, KVT_BYTES = L::KVT_BYTES;
     constexpr uint32_t OFF_KVT = L::OFF_KVT, OFF_Q = L::OFF_Q, OFF_DL = L::OFF_DL, OFF_SB = L::OFF_SB;
@@ -236,21 +236,66 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int q = warp & 3;                                                  // TMEM lane quarter
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
-    const long sidx = blockIdx.x >> 1;                                     // stream (state index)
-    const StreamJob jb = seqs.job(sidx);
-    const int col0 = (blockIdx.x & 1) * 64;
+    // This CTA's recurrence: a stream's 64-column half of d_v, or with a segmented scan one
+    // segment of it (see SegPlan): its tokens, entering state, final state and outputs.
+    long sidx;
+    StreamJob jb;
+    int col0;
+    const float* s0p;             // entering state (128 x 128, row stride 128) or null (zero)
+    bool s0_identity = false;     // transition product: the entering state is I
+    float* stp;                   // final state (128 x 128) or null
+    __nv_bfloat16* op = o;        // outputs [.., Tdim, 128]
+    bool vzero = false;           // transition product: V = 0
+    if (seg.G <= 1) {
+        sidx = blockIdx.x >> 1;
+        jb = seqs.job(sidx);
+        col0 = (blockIdx.x & 1) * 64;
+        s0p = S0 ? S0 + (size_t)sidx * kD * kD : nullptr;
+        stp = S_T ? S_T + (size_t)sidx * kD * kD : nullptr;
+    } else {
+        const int per = 2 + 4 * (seg.G - 1);
+        sidx = blockIdx.x / per;
+        const int kk = (int)(blockIdx.x % per);
+        const int g = kk < 2 ? 0 : 1 + (kk - 2) / 4;
+        const int role = kk < 2 ? kk : (kk - 2) % 4;          // 0, 1: the state's halves; 2, 3: transition
+        jb = seqs.job(sidx);
+        const int first = g * seg.seg_chunks * 64;
+        const int last = g == seg.G - 1 ? jb.len : min(jb.len, first + seg.seg_chunks * 64);
+        jb.y0 += first;
+        jb.len = max(0, last - first);
+        jb.tile0 += (long)g * seg.seg_chunks;
+        col0 = (role & 1) * 64;
+        const size_t slot = ((size_t)sidx * seg.G + g) * kD * kD;
+        if (role < 2) {
+            s0p = g == 0 && S0 ? S0 + (size_t)sidx * kD * kD : nullptr;
+            stp = seg.Sloc + slot;
+        } else {
+            s0p = nullptr;
+            s0_identity = true;
+            stp = seg.Phi + slot;
+            op = seg.R;
+            vzero = true;
+        }
+    }
     const int T = jb.len, zc = jb.z, y0 = jb.y0;
     const int nchunks = (T + 63) / 64;
     const size_t tok0 = (size_t)zc * Tdim + y0;
     if (nchunks == 0) {   // an empty sequence: the state passes through (nothing else runs)
-        if (S_T) {
+        if (stp) {
             for (int e = tid; e < kD * 64; e += kThreads) {
                 const int i = e >> 6, j = e & 63;
-                const size_t at = ((size_t)sidx * kD + i) * kD + col0 + j;
-                S_T[at] = S0 ? S0[at] : 0.f;
+                const size_t at = (size_t)i * kD + col0 + j;
+                stp[at] = s0_identity ? (i == col0 + j ? 1.f : 0.f) : (s0p ? s0p[at] : 0.f);
             }
         }
         return;
+    }
+    if (vzero) {   // the transition product's V tiles stay zero (never loaded)
+        for (int e = tid; e < kKvtStages * (int)(TILE / 16); e += kThreads) {
+            const int stg = e / (int)(TILE / 16), off = e % (int)(TILE / 16);
+            reinterpret_cast<uint4*>(sm + OFF_KVT + stg * KVT_BYTES + KVT_V)[off] = make_uint4(0u, 0u, 0u, 0u);
+        }
+        fence_proxy_async_smem();
     }
 
     if (tid == 0) {
@@ -285,10 +330,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     if (c >= kKvtStages && !(ok = ctl.wait(B_KVT_FREE + s, ((c - kKvtStages) / kKvtStages) & 1))) break;
                     uint8_t* st = sm + kvt(c);
                     uint64_t* full = ctl.b(B_KVT_FULL + s);
-                    mbar_arrive_expect_tx(full, L::KVT_TX);
+                    mbar_arrive_expect_tx(full, L::KVT_TX - (vzero ? TILE : 0));
                     tma_load_3d(st + KVT_K, &tm_k, full, 0, y0 + t0, zc);
                     tma_load_3d(st + KVT_K + TILE, &tm_k, full, 64, y0 + t0, zc);
-                    tma_load_3d(st + KVT_V, &tm_v, full, col0, y0 + t0, zc);
+                    if (!vzero) tma_load_3d(st + KVT_V, &tm_v, full, col0, y0 + t0, zc);
                     tma_load_2d(st + KVT_T, &tm_t, full, 0, (int)((jb.tile0 + c) * 64));
                     if constexpr (kGated) {
                         tma_load_2d(st + L::KVT_TU, &tm_t, full, 0, (int)((ntiles + jb.tile0 + c) * 64));
@@ -310,7 +355,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     const int t3 = y0 + t0 + 192;
                     tma_prefetch_l2_3d(&tm_k, 0, t3, zc);
                     tma_prefetch_l2_3d(&tm_k, 64, t3, zc);
-                    tma_prefetch_l2_3d(&tm_v, col0, t3, zc);
+                    if (!vzero) tma_prefetch_l2_3d(&tm_v, col0, t3, zc);
                     tma_prefetch_l2_3d(&tm_q, 0, t3, zc);
                     tma_prefetch_l2_3d(&tm_q, 64, t3, zc);
                     tma_prefetch_l2_2d(&tm_t, 0, (int)((jb.tile0 + c + 3) * 64));
@@ -439,7 +484,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             ctl.warp_arrive(B_X_FREE, lane);
             const int t0 = c * 64;
             if (r < min(64, T - t0)) {
-                uint4* dst = reinterpret_cast<uint4*>(o + (tok0 + t0 + r) * kD + col0);
+                uint4* dst = reinterpret_cast<uint4*>(op + (tok0 + t0 + r) * kD + col0);
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
                     uint4 y;
@@ -557,7 +602,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             return 1.f;
         };
         {   // initial state
-            const float* src = S0 ? S0 + ((size_t)sidx * kD + ct) * kD + col0 + cc : nullptr;
+            const float* src = s0p ? s0p + (size_t)ct * kD + col0 + cc : nullptr;
             const float dec0 = decay_of(0);
 #pragma unroll
             for (int qd = 0; qd < 2; ++qd) {
@@ -565,6 +610,11 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
                 for (int j = 0; j < 16; j += 4) {
                     float4 x = src ? *reinterpret_cast<const float4*>(src + 16 * qd + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+                    if (s0_identity) {
+                        const int c0 = col0 + cc + 16 * qd + j;    // this row's 1 sits in column ct
+                        x = make_float4(ct == c0 ? 1.f : 0.f, ct == c0 + 1 ? 1.f : 0.f, ct == c0 + 2 ? 1.f : 0.f,
+                                        ct == c0 + 3 ? 1.f : 0.f);
+                    }
                     s16[j] = x.x; s16[j + 1] = x.y; s16[j + 2] = x.z; s16[j + 3] = x.w;
                 }
                 st_chunk(sm + OFF_SB + sw128_off(ct, 4 * ch + 2 * qd), s16);
@@ -619,8 +669,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 tmem_ld32_wait(tmem + lane_off + TM_S + cc, t);
 #pragma unroll
                 for (int j = 0; j < 4; ++j) st_chunk(sm + OFF_SB + sw128_off(ct, 4 * ch + j), t + 8 * j);
-                if (c == nchunks - 1 && S_T) {
-                    float* dst = S_T + ((size_t)sidx * kD + ct) * kD + col0 + cc;
+                if (c == nchunks - 1 && stp) {
+                    float* dst = stp + (size_t)ct * kD + col0 + cc;
 #pragma unroll
                     for (int j = 0; j < 32; j += 4)
                         *reinterpret_cast<float4*>(dst + j) = make_float4(t[j], t[j + 1], t[j + 2], t[j + 3]);
@@ -681,9 +731,11 @@ size_t chunk_tc_gated_workspace_bytes(long BH, int T) {
 
 cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const void* beta, const float* S0,
                             void* o, float* S_T, const Seqs& seqs, long nstreams, long Z, int Tdim, long ntiles,
-                            uint32_t* err, void* scratch, int rule, cudaStream_t stream, const float* g) {
+                            uint32_t* err, void* scratch, int rule, cudaStream_t stream, const float* g,
+                            const SegPlan& seg) {
     cudaError_t e = launch_ut(k, beta, scratch, seqs, Z, Tdim, ntiles, err, kWaitLimitNs, rule, stream, g);
     if (e != cudaSuccess) return e;
+    const long ctas = seg.G > 1 ? nstreams * (2 + 4 * (seg.G - 1)) : nstreams * 2;
     CUtensorMap mq, mk, mv, mt;
     if (!tma_map_tokens(&mq, q, kD, Tdim, Z) || !tma_map_tokens(&mk, k, kD, Tdim, Z) ||
         !tma_map_tokens(&mv, v, kD, Tdim, Z) || !tma_map_rows64(&mt, scratch, std::max<long>(1, (g ? 2 : 1) * ntiles) * 64))
@@ -693,15 +745,15 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const v
         static std::atomic<uint64_t> smem_set_g{0};
         e = set_smem_limit_once(chunk_tc_kernel<true>, (int)Lay<true>::SMEM_BYTES, smem_set_g);
         if (e != cudaSuccess) return e;
-        chunk_tc_kernel<true><<<(unsigned)(nstreams * 2), kThreads, Lay<true>::SMEM_BYTES, stream>>>(
-            mq, mk, mv, mt, S0, (__nv_bfloat16*)o, S_T, seqs, Tdim, err, kWaitLimitNs, gl, ntiles);
+        chunk_tc_kernel<true><<<(unsigned)ctas, kThreads, Lay<true>::SMEM_BYTES, stream>>>(
+            mq, mk, mv, mt, S0, (__nv_bfloat16*)o, S_T, seqs, Tdim, err, kWaitLimitNs, gl, ntiles, seg);
         return cudaGetLastError();
     }
     static std::atomic<uint64_t> smem_set{0};
     e = set_smem_limit_once(chunk_tc_kernel<false>, (int)Lay<false>::SMEM_BYTES, smem_set);
     if (e != cudaSuccess) return e;
-    chunk_tc_kernel<false><<<(unsigned)(nstreams * 2), kThreads, Lay<false>::SMEM_BYTES, stream>>>(
-        mq, mk, mv, mt, S0, (__nv_bfloat16*)o, S_T, seqs, Tdim, err, kWaitLimitNs, nullptr, ntiles);
+    chunk_tc_kernel<false><<<(unsigned)ctas, kThreads, Lay<false>::SMEM_BYTES, stream>>>(
+        mq, mk, mv, mt, S0, (__nv_bfloat16*)o, S_T, seqs, Tdim, err, kWaitLimitNs, nullptr, ntiles, seg);
     return cudaGetLastError();
 }
 

@@ -5,6 +5,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <cuda_bf16.h>
+
 #include "efla_common.cuh"
 
 namespace efla {
@@ -27,10 +29,31 @@ cudaError_t launch_chunk_simt(const void* q, const void* k, const void* v, const
 size_t chunk_tc_workspace_bytes(long BH, int T);
 // the gated flow (g != null): two transforms and the cumulative log-decay per chunk
 size_t chunk_tc_gated_workspace_bytes(long BH, int T);
+// Segmented scan of long streams (d = 128, bf16).  With G > 1 every stream is split into G
+// segments of seg_chunks chunks (the last takes the rest).  The chain launch then runs per
+// stream 2 CTAs for segment 0 (from S0, exact outputs, final state into Sloc[.][0]) and 4 per
+// later segment g: 2 from a zero state (outputs O_loc into o, final state into Sloc[.][g]) and
+// 2 for the segment's transition product (V = 0 from S = I: final state Phi[.][g], outputs
+// R into R).  The chunk map S -> (I - K^T W) S + K^T U is affine, so the true entering state
+// of segment g is S_in(g) = Phi[g-1] S_in(g-1) + Sloc[g-1] and its outputs O_loc + R S_in(g).
+struct SegPlan {
+    int G = 1;                     // 1: no segmentation
+    int seg_chunks = 0;
+    float* Sloc = nullptr;         // [nstreams][G][128][128]
+    float* Phi = nullptr;          // [nstreams][G][128][128]
+    __nv_bfloat16* R = nullptr;    // [Z][Tdim][128] (rows of segments >= 1)
+};
+
 // nstreams recurrences described by `seqs` over tensors [Z][Tdim][d]; ntiles UT tiles
 cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const void* beta, const float* S0,
                             void* o, float* S_T, const Seqs& seqs, long nstreams, long Z, int Tdim, long ntiles,
-                            uint32_t* err, void* scratch, int rule, cudaStream_t stream, const float* g = nullptr);
+                            uint32_t* err, void* scratch, int rule, cudaStream_t stream, const float* g = nullptr,
+                            const SegPlan& seg = SegPlan());
+// the segmented scan's combine (S_in of every segment, S_T) and output correction o += R S_in
+cudaError_t launch_seg_combine(const SegPlan& seg, const float* S0, float* S_T, float* Sin, long nstreams,
+                               cudaStream_t stream);
+cudaError_t launch_seg_correct(const SegPlan& seg, const float* Sin, __nv_bfloat16* o, long nstreams, int T,
+                               cudaStream_t stream);
 // g != null: the gated flow's transforms (two per tile plus the cumulative log-decay, see
 // efla_ut.cu) into Tout, which then holds chunk_tc_gated_workspace_bytes.
 // tiles: ntiles of `seqs` (dense: BH * ceil(T / 64); packed: H * tileoff[N]); tensors [Z][Tdim][d]

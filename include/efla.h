@@ -200,6 +200,40 @@ int efla_chunk_fwd_varlen(const void *q, const void *k, const void *v, const voi
                           void *workspace, size_t workspace_bytes, efla_stream_t stream);
 
 /*
+ * Segmented scan for long streams (Section 3.3's chunk recurrence is affine in the state,
+ * S -> (I - K^T W) S + K^T U; App. A notes long contexts as the open case).  With few streams
+ * and many chunks the chain of chunks, not the hardware, sets the time; splitting each
+ * stream into G segments runs them side by side:
+ *   - segment 0 runs from S0 as usual;
+ *   - every later segment g runs from a zero state (final state S_loc(g), outputs O_loc) and,
+ *     beside it, with V = 0 from S = I (final state Phi(g), the segment's transition
+ *     product, and outputs R(g), each token's linear dependence on the entering state);
+ *   - S_in(g+1) = Phi(g) S_in(g) + S_loc(g) in order (S_in(1) = segment 0's final state),
+ *     S_T = S_in(G), and every token of segment g >= 1 gets o += R S_in(g).
+ * The results equal efla_chunk_fwd's up to rounding (the transition product and R pass
+ * through the same bf16-operand, fp32-accumulate products as the state).
+ *
+ * efla_chunk_fwd_segmented_workspace_bytes -- workspace for `segments` (0: chosen by the
+ * library) and gated != 0 for the gated flow; 0 for arguments the call would reject.
+ */
+size_t efla_chunk_fwd_segmented_workspace_bytes(int B, int H, int T, int d_k, int d_v, int chunk,
+                                                int dtype, int gated, int segments);
+
+/*
+ * efla_chunk_fwd_segmented -- efla_chunk_fwd_ex (g == NULL) or efla_chunk_fwd_gated (g given)
+ * as a segmented scan.  segments >= 2 splits every stream into that many segments of equal
+ * chunk counts (fewer if the stream has under 8 chunks per segment); 0 lets the library
+ * choose the most segments whose chain CTAs fit one wave on the device (B*H*(4G - 2) <= SMs);
+ * 1 is the plain forward.  Only bf16 with d = 128 segments; other shapes run the plain
+ * forward.  Arguments, layouts and errors otherwise as efla_chunk_fwd_ex;
+ * segments < 0 is EFLA_ERR_INVALID_ARG.
+ */
+int efla_chunk_fwd_segmented(const void *q, const void *k, const void *v, const void *beta,
+                             const float *g, const float *S0, void *o, float *S_T, int B, int H,
+                             int T, int d_k, int d_v, int chunk, int dtype, int rule, int segments,
+                             void *workspace, size_t workspace_bytes, efla_stream_t stream);
+
+/*
  * efla_chunk_fwd_noalloc -- efla_chunk_fwd without a caller-provided workspace.
  * The paper has no counterpart: this is an integration variant for callers that cannot
  * allocate device memory, e.g. code embedded in a host runtime that owns every device

@@ -131,6 +131,22 @@ def pin_bwd_state_reversal(lib):
                 assert np.allclose(x, y, rtol=1e-12, atol=1e-12), (mode, cols, h)
 
 
+def pin_bwd_chunkwise_form(lib):
+    """The chunkwise (UT-form) reverse mode, derived independently (tests/chunk_bwd_mirror.py),
+    equals the oracle's token-by-token reverse sweep to 1e-10, for several chunk lengths
+    including ragged tails, stiff keys and the Euler rule."""
+    from chunk_bwd_mirror import chunk_bwd_mirror
+    for (mode, stiff, C, T, seed) in ((oracle.EXACT, False, 4, 11, 31), (oracle.EXACT, True, 8, 20, 32),
+                                      (oracle.EULER, False, 5, 13, 33), (oracle.EXACT, False, 64, 70, 34)):
+        rng = np.random.default_rng(seed)
+        q, k, v, beta, S0, dO, dST = _problem(rng, B=1, H=2, T=T, dk=4, dv=3, stiff=stiff)
+        ref = oracle.bwd(q, k, v, beta, dO, S0, dST, mode=mode, threads=1, lib=lib)
+        got = chunk_bwd_mirror(q, k, v, beta, dO, S0, dST, C=C, euler=(mode == oracle.EULER))
+        for name, a, b in zip(("dq", "dk", "dv", "dbeta", "dS0"), got, ref):
+            e = np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300)
+            assert e <= 1e-10, (mode, stiff, C, name, e)
+
+
 ALL_PINS = [pin_bwd_directional_exact, pin_bwd_directional_stiff, pin_bwd_directional_euler,
             pin_bwd_elementwise, pin_bwd_zero_state_and_no_final_gradient, pin_gate_derivatives,
-            pin_bwd_state_reversal]
+            pin_bwd_state_reversal, pin_bwd_chunkwise_form]

@@ -234,3 +234,20 @@ def test_varlen_entry_point_validates_offsets(efla):
     assert call(ws_=16) == INVALID
     assert call(cu=None) == INVALID
     assert call(N=0) == OK
+
+
+def test_segmented_entry_point_validates_arguments(efla):
+    L = efla.lib
+    q, k, v, b, s0, o, st, w = GOOD
+    plain = L.efla_chunk_fwd_workspace_bytes(1, 2, 4096, 128, 128, 64, 1)
+    seg = L.efla_chunk_fwd_segmented_workspace_bytes(1, 2, 4096, 128, 128, 64, 1, 0, 2)
+    assert seg > plain                                            # + states, transition products, R
+    assert L.efla_chunk_fwd_segmented_workspace_bytes(1, 2, 4096, 128, 128, 64, 1, 0, 1) == plain
+    assert L.efla_chunk_fwd_segmented_workspace_bytes(1, 2, 4096, 128, 128, 64, 1, 0, -1) == 0
+    assert L.efla_chunk_fwd_segmented_workspace_bytes(1, 2, 4096, 96, 96, 64, 1, 0, 2) == 0
+    call = lambda segments=2, ws=seg, rule=0, B=1: L.efla_chunk_fwd_segmented(
+        q, k, v, b, None, s0, o, st, B, 2, 4096, 128, 128, 64, 1, rule, segments, w, ws, None)
+    assert call(segments=-1) == INVALID
+    assert call(ws=plain) == INVALID                              # too small for two segments
+    assert call(rule=3) == INVALID
+    assert call(B=0) == OK
