@@ -73,7 +73,8 @@ KERNEL_SOURCES = {
     "efla_chunk_fwd": ["efla_chunk_tc.cu", "efla_ut.cu", "efla_ut_tf32.cuh", "efla_ut_solve.cuh",
                        "efla_chunk_simt.cu", "efla_common.cuh", "efla_tma.cuh", "sm100.cuh"],
     "efla_recurrent_step": ["efla_decode.cu", "efla_common.cuh"],
-    "efla_backward": ["efla_bwd.cu", "efla_common.cuh"],
+    "efla_backward": ["efla_bwd.cu", "efla_bwd_chunk.cu", "efla_mma_sync.cuh", "efla_chunk_tc.cu", "efla_ut.cu",
+                      "efla_ut_tf32.cuh", "efla_ut_solve.cuh", "efla_common.cuh", "efla_tma.cuh", "sm100.cuh"],
 }
 
 
@@ -127,7 +128,7 @@ TRAFFIC_JSON = os.path.join(ROOT, "profiles", "traffic.json")
 ENTRY_KERNELS = {
     "efla_chunk_fwd": ("ut_kernel", "chunk_tc_kernel"),
     "efla_recurrent_step": ("decode_kernel",),
-    "efla_backward": ("bwd_kernel", "bwd_gate_kernel"),
+    "efla_backward": ("ut_kernel", "chunk_tc_kernel", "bwd_chain_kernel", "bwd_tile_kernel"),
 }
 
 
@@ -163,7 +164,7 @@ def traffic_from_csv(csv_path: str, entry: str, calls: int):
             scale = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9, "KB": 1e3, "MB": 1e6, "GB": 1e9}.get(unit, 1)
             rows.append((int(r["ID"]), name, r["Metric Name"], float(r["Metric Value"].replace(",", "")) * scale))
     ids = sorted({i for i, _, _, _ in rows})
-    per_call = len(ENTRY_KERNELS[entry]) if entry != "efla_backward" else 2
+    per_call = len(ENTRY_KERNELS[entry])
     keep = set(ids[-calls * per_call:])
     total = sum(v for i, _, _, v in rows if i in keep)
     rec = {"bytes_per_call": int(round(total / calls)), "calls": calls,
@@ -358,10 +359,18 @@ def profile_call(args):
         calls = [lambda i=i: efla.efla_recurrent_step(st["q"][i], st["k"][i], st["v"][i], st["beta"][i], S,
                                                        o=o, stream=stream) for i in range(n)]
     else:
-        w = WORKLOAD
+        w = workloads.CHUNK_WORKLOADS["longctx_bf16"] if args.profile_call.startswith("long") else WORKLOAD
         x = {k: (None if v is None else v.to(dev)) for k, v in workloads.make_chunk_inputs(w).items()}
         B, H, T, d = w.B, w.H, w.T, w.dk
-        if args.profile_call == "fwd":
+        if args.profile_call == "longseg":
+            n = efla.lib.efla_chunk_fwd_segmented_workspace_bytes(B, H, T, d, d, 64, 1, 0, 0)
+            ws = torch.zeros(n, dtype=torch.uint8, device=dev)
+            one = lambda: efla.efla_chunk_fwd_segmented(x["q"], x["k"], x["v"], x["beta"], x["S0"], workspace=ws,
+                                                        stream=stream)
+        elif args.profile_call == "gated":
+            gd = workloads.make_log_decay((B, H, T), w.seed + 7).to(dev)
+            one = lambda: efla.efla_chunk_fwd_gated(x["q"], x["k"], x["v"], x["beta"], gd, x["S0"], stream=stream)
+        elif args.profile_call in ("fwd", "long"):
             ws = efla.new_workspace(B, H, T, d, d, 64, w.dtype, dev)
             o = torch.empty(B, H, T, d, dtype=w.dtype, device=dev)
             ST = torch.empty(B, H, d, d, dtype=torch.float32, device=dev)
@@ -372,7 +381,7 @@ def profile_call(args):
             f32 = dict(device=dev, dtype=torch.float32)
             g = (torch.empty(B, H, T, d, **f32), torch.empty(B, H, T, d, **f32), torch.empty(B, H, T, d, **f32),
                  torch.empty(B, H, T, **f32), torch.empty(B, H, d, d, **f32))
-            wsb = torch.empty(efla.efla_backward_workspace_bytes(B, H, T, d, d, w.dtype), dtype=torch.uint8,
+            wsb = torch.zeros(efla.efla_backward_workspace_bytes(B, H, T, d, d, w.dtype), dtype=torch.uint8,
                               device=dev)
             one = lambda: efla.efla_backward(x["q"], x["k"], x["v"], x["beta"], dO, grads=g, workspace=wsb,
                                              stream=stream)
@@ -395,7 +404,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--other-steps", type=int, default=10,
                     help="forwards timed on each of the long-context and stiff workloads (0: skip)")
-    ap.add_argument("--profile-call", choices=["fwd", "decode", "bwd"],
+    ap.add_argument("--profile-call", choices=["fwd", "decode", "bwd", "long", "longseg", "gated"],
                     help="only run warm-up + steps calls of one entry point (for an ncu capture)")
     ap.add_argument("--traffic-from", metavar="CSV",
                     help="write profiles/traffic.json's record from an ncu --csv log of "
@@ -563,7 +572,7 @@ def main():
         f32 = dict(device=dev, dtype=torch.float32)
         gb = (torch.empty(B, H, T, d, **f32), torch.empty(B, H, T, d, **f32), torch.empty(B, H, T, d, **f32),
               torch.empty(B, H, T, **f32), torch.empty(B, H, d, d, **f32))
-        wsb = torch.empty(efla.efla_backward_workspace_bytes(B, H, T, d, d, wb.dtype), dtype=torch.uint8, device=dev)
+        wsb = torch.zeros(efla.efla_backward_workspace_bytes(B, H, T, d, d, wb.dtype), dtype=torch.uint8, device=dev)
         callb = lambda: efla.efla_backward(xb["q"], xb["k"], xb["v"], xb["beta"], dOb, grads=gb, workspace=wsb,
                                            stream=stream)
         for _ in range(args.warmup):
@@ -583,8 +592,9 @@ def main():
                "value": wb.tokens * world / (bms * 1e-3), "unit": "tokens/s", "ms_per_step": bms,
                "steps": args.bwd_steps, "dtype": "bf16", "grad_dtype": "f32",
                "roofline": brf, "roofline_basis": "the method's chunked form: bytes at HBM, 3x forward flops at tensor peak",
-               # three zero fills, the sweep kernel and the gate kernel per call
-               "gpu_launches": 5 * args.bwd_steps}
+               # bf16, d = 128: the UT kernel, the forward chain storing states, the reverse chain and
+               # the per-chunk gradient kernel per call
+               "gpu_launches": 4 * args.bwd_steps}
         del xb, dOb, gb, wsb
 
     # ---- the other forward workloads (long context, stiff keys): tokens/s and roofline

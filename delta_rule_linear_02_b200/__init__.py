@@ -376,7 +376,7 @@ def efla_backward(q, k, v, beta, dO, S0=None, dS_T=None, want_dS0: bool = True, 
         n = efla_backward_workspace_bytes(B, H, T, d_k, d_v, dt)
         if n == 0 and B * H * T > 0:
             raise EflaError(EFLA_ERR_UNSUPPORTED, "efla_backward_workspace_bytes")
-        workspace = torch.empty(max(n, 16), dtype=torch.uint8, device=k.device)
+        workspace = torch.zeros(max(n, 16), dtype=torch.uint8, device=k.device)
     st = lib.efla_backward_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(S0), _ptr(dO), _ptr(dS_T),
                               *(_ptr(g) for g in grads), B, H, T, d_k, d_v, _DTYPES.get(dt, -1), int(rule),
                               _ptr(workspace), workspace.numel(), _stream(stream))

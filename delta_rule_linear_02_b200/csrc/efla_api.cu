@@ -449,8 +449,13 @@ static int check_bwd_shape(int B, int H, int T, int d_k, int d_v, int dtype) {
     return EFLA_OK;
 }
 
+// bf16 with d = 128 takes the backward through the chunkwise form (tensor cores); the rest
+// the token-by-token reverse sweep (fp32 CUDA cores).
+static bool bwd_chunked(int d_k, int dtype) { return dtype == EFLA_DTYPE_BF16 && d_k == 128; }
+
 size_t efla_backward_workspace_bytes(int B, int H, int T, int d_k, int d_v, int dtype) {
     if (check_bwd_shape(B, H, T, d_k, d_v, dtype) != EFLA_OK) return 0;
+    if (bwd_chunked(d_k, dtype)) return kWorkspaceHeader + efla::bwd_chunk_workspace_bytes((long)B * H, T);
     return efla::bwd_workspace_bytes((long)B * H, T, d_k);
 }
 
@@ -496,6 +501,10 @@ int efla_backward_ex(const void* q, const void* k, const void* v, const void* be
     // reads the inputs: no input may share bytes with it
     for (int j = 0; j < 7; ++j)
         if (overlaps(workspace, workspace_bytes, ins[j], inn[j])) return EFLA_ERR_INVALID_ARG;
+    if (bwd_chunked(d_k, dtype))
+        return from_cuda(efla::launch_bwd_chunk(q, k, v, beta, S0, dO, dS_T, dq, dk, dv, dbeta, dS0, BH, T, rule,
+                                                static_cast<uint32_t*>(workspace),
+                                                static_cast<char*>(workspace) + kWorkspaceHeader, s));
     return from_cuda(efla::launch_bwd(q, k, v, beta, S0, dO, dS_T, dq, dk, dv, dbeta, dS0, BH, T, d_k,
                                       dtype == EFLA_DTYPE_BF16, rule, workspace, s));
 }

@@ -180,17 +180,6 @@ __global__ void __launch_bounds__(kThreads) bwd_kernel(const Tin* __restrict__ q
     }
 }
 
-// d alpha / d lambda of the exact gate in fp32: (beta e^{-x} - alpha) / lambda, x = beta*lambda,
-// by its series beta^2 sum_{n>=1} (-1)^n n x^{n-1} / (n+1)! for |x| < 1/16 (where the
-// difference cancels; truncation below x^6 / 840 relative), limit -beta^2/2 at lambda = 0.
-__device__ __forceinline__ float gate_dalpha_dlambda(float beta, float lambda) {
-    const float x = beta * lambda;
-    if (fabsf(x) < 0.0625f)
-        return beta * beta *
-               (-0.5f + x * (1.0f / 3.0f - x * (1.0f / 8.0f - x * (1.0f / 30.0f - x * (1.0f / 144.0f - x * (1.0f / 840.0f))))));
-    return (beta * expf(-x) + expm1f(-x) / lambda) / lambda;
-}
-
 // the gate's share: dbeta_t = dalpha_t dalpha/dbeta, dk_t += dalpha_t dalpha/dlambda 2 k_t
 // (one warp per token)
 template <typename Tin, int D>

@@ -483,7 +483,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             tc_fence_before();
             ctl.warp_arrive(B_X_FREE, lane);
             const int t0 = c * 64;
-            if (r < min(64, T - t0)) {
+            if (op && r < min(64, T - t0)) {
                 uint4* dst = reinterpret_cast<uint4*>(op + (tok0 + t0 + r) * kD + col0);
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
@@ -619,6 +619,11 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 }
                 st_chunk(sm + OFF_SB + sw128_off(ct, 4 * ch + 2 * qd), s16);
                 st_chunk(sm + OFF_SB + sw128_off(ct, 4 * ch + 2 * qd + 1), s16 + 8);
+                if (seg.states) {   // chunk 0's entering state, for the backward
+                    uint8_t* dst = reinterpret_cast<uint8_t*>(seg.states + ((size_t)jb.tile0 * kD + ct) * kD + col0 + cc + 16 * qd);
+                    st_chunk(dst, s16);
+                    st_chunk(dst + 16, s16 + 8);
+                }
                 if constexpr (kGated) {
 #pragma unroll
                     for (int j = 0; j < 16; ++j) s16[j] *= dec0;
@@ -669,6 +674,11 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 tmem_ld32_wait(tmem + lane_off + TM_S + cc, t);
 #pragma unroll
                 for (int j = 0; j < 4; ++j) st_chunk(sm + OFF_SB + sw128_off(ct, 4 * ch + j), t + 8 * j);
+                if (seg.states && c + 1 < nchunks) {   // chunk c+1's entering state, for the backward
+                    uint8_t* dst = reinterpret_cast<uint8_t*>(seg.states + ((size_t)(jb.tile0 + c + 1) * kD + ct) * kD + col0 + cc);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) st_chunk(dst + 16 * j, t + 8 * j);
+                }
                 if (c == nchunks - 1 && stp) {
                     float* dst = stp + (size_t)ct * kD + col0 + cc;
 #pragma unroll

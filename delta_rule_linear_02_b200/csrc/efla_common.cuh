@@ -64,6 +64,31 @@ __device__ __forceinline__ float gate_alpha(float beta, float lambda) {
     return -expm1f(-x) / lambda;
 }
 
+// d alpha / d lambda of the exact gate in fp32: (beta e^{-x} - alpha) / lambda, x = beta*lambda,
+// by its series beta^2 sum_{n>=1} (-1)^n n x^{n-1} / (n+1)! for |x| < 1/16 (where the
+// difference cancels; truncation below x^6 / 840 relative), limit -beta^2/2 at lambda = 0.
+__device__ __forceinline__ float gate_dalpha_dlambda(float beta, float lambda) {
+    const float x = beta * lambda;
+    if (fabsf(x) < 0.0625f)
+        return beta * beta *
+               (-0.5f + x * (1.0f / 3.0f - x * (1.0f / 8.0f - x * (1.0f / 30.0f - x * (1.0f / 144.0f - x * (1.0f / 840.0f))))));
+    return (beta * expf(-x) + expm1f(-x) / lambda) / lambda;
+}
+
+// The gate's derivatives for the backward pass: dalpha/dbeta = e^{-beta lambda} and
+// dalpha/dlambda above (the Euler rule: 1 and 0).
+__device__ __forceinline__ void gate_derivatives(int rule, float beta, float lambda, float alpha, float* dadb,
+                                                 float* dadl) {
+    (void)alpha;
+    if (rule == kRuleEuler) {
+        *dadb = 1.f;
+        *dadl = 0.f;
+        return;
+    }
+    *dadb = expf(-beta * lambda);
+    *dadl = gate_dalpha_dlambda(beta, lambda);
+}
+
 // The gated flow (Gated EFLA, Section 3.4): a per-token log-decay g joins the ODE over the
 // token's unit interval, dS/dtau = g S - beta (k k^T S - k v^T).  The flow keeps alpha for the
 // rank-1 contraction, decays the state by e^g, and writes with

@@ -37,6 +37,7 @@ size_t chunk_tc_gated_workspace_bytes(long BH, int T);
 // R into R).  The chunk map S -> (I - K^T W) S + K^T U is affine, so the true entering state
 // of segment g is S_in(g) = Phi[g-1] S_in(g-1) + Sloc[g-1] and its outputs O_loc + R S_in(g).
 struct SegPlan {
+    __nv_bfloat16* states = nullptr;   // if set: the entering state of every chunk, bf16 [tiles][128][128]
     int G = 1;                     // 1: no segmentation
     int seg_chunks = 0;
     float* Sloc = nullptr;         // [nstreams][G][128][128]
@@ -50,9 +51,10 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const v
                             uint32_t* err, void* scratch, int rule, cudaStream_t stream, const float* g = nullptr,
                             const SegPlan& seg = SegPlan());
 // the segmented scan's combine (S_in of every segment, S_T) and output correction o += R S_in
-cudaError_t launch_seg_combine(const SegPlan& seg, const float* S0, float* S_T, float* Sin, long nstreams,
+// (SinT: bf16 [nstreams][G][128][128], S_in of every segment transposed, written by the combine)
+cudaError_t launch_seg_combine(const SegPlan& seg, const float* S0, float* S_T, void* SinT, long nstreams,
                                cudaStream_t stream);
-cudaError_t launch_seg_correct(const SegPlan& seg, const float* Sin, __nv_bfloat16* o, long nstreams, int T,
+cudaError_t launch_seg_correct(const SegPlan& seg, const void* SinT, __nv_bfloat16* o, long nstreams, int T,
                                cudaStream_t stream);
 // g != null: the gated flow's transforms (two per tile plus the cumulative log-decay, see
 // efla_ut.cu) into Tout, which then holds chunk_tc_gated_workspace_bytes.
@@ -69,6 +71,14 @@ cudaError_t launch_bwd(const void* q, const void* k, const void* v, const void* 
 
 // packed batches: tileoff[n] = sum over m < n of ceil((cu[m+1] - cu[m]) / 64), n = 0..N
 cudaError_t launch_seq_prep(const int* cu, int* tileoff, int N, cudaStream_t stream);
+
+// the backward through the chunkwise form (bf16, d = 128): UT transforms, the forward chain
+// storing each chunk's entering state, the reverse chain (dS' per chunk), per-chunk gradients.
+// scratch: bwd_chunk_workspace_bytes bytes (16-byte aligned); err: the device error word.
+size_t bwd_chunk_workspace_bytes(long BH, int T);
+cudaError_t launch_bwd_chunk(const void* q, const void* k, const void* v, const void* beta, const float* S0,
+                             const void* dO, const float* dST, float* dq, float* dk, float* dv, float* dbeta,
+                             float* dS0, long BH, int T, int rule, uint32_t* err, void* scratch, cudaStream_t stream);
 
 cudaError_t launch_wait_timeout_selftest(uint32_t* err, unsigned long long limit_ns, cudaStream_t stream);
 

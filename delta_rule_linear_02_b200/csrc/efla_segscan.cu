@@ -8,9 +8,11 @@
 // for every segment at once (SegPlan in efla_kernels.h); here
 //   combine:  S_in(1) = S_loc(0), S_in(g+1) = Phi(g) S_in(g) + S_loc(g), S_T = S_in(G)   (fp32)
 //   correct:  o[t] += R[t] S_in(g) for the tokens t of every segment g >= 1   (bf16 MMA,
-//             fp32 accumulation: R and S_in as bf16 operands, like every chunk product)
+//             fp32 accumulation: R and S_in as bf16 operands, like every chunk product;
+//             the combine hands S_in(g) over transposed in bf16)
 #include "efla_common.cuh"
 #include "efla_kernels.h"
+#include "efla_mma_sync.cuh"
 
 namespace efla {
 
@@ -19,20 +21,22 @@ constexpr int kD = 128;
 
 // One CTA per (stream, 32-column block): the column block of S_in(g) evolves on its own.
 __global__ void __launch_bounds__(256) seg_combine_kernel(SegPlan seg, float* __restrict__ S_T,
-                                                          float* __restrict__ Sin) {
+                                                          __nv_bfloat16* __restrict__ SinT) {
     __shared__ float cur[kD][33];                   // S_in(g)[:, block], padded
+    __shared__ float pk[kD][33];                    // a 32-column slab of Phi(g)
     const long s = blockIdx.x >> 2;
     const int j0 = (blockIdx.x & 3) * 32;
     const int t = threadIdx.x;
     const size_t mat = (size_t)kD * kD;
     const float* sloc = seg.Sloc + (size_t)s * seg.G * mat;
     const float* phi = seg.Phi + (size_t)s * seg.G * mat;
-    float* sin_ = Sin + (size_t)s * seg.G * mat;
+    // S_in(g) for the correction: bf16, transposed (SinT[g][n][k] = S_in(g)[k][n])
+    __nv_bfloat16* sint = SinT + (size_t)s * seg.G * mat;
     for (int e = t; e < kD * 32; e += 256) {         // S_in(1) = S_loc(0)
         const int i = e >> 5, j = e & 31;
         const float x = sloc[(size_t)i * kD + j0 + j];
         cur[i][j] = x;
-        if (seg.G > 1) sin_[mat + (size_t)i * kD + j0 + j] = x;
+        if (seg.G > 1) sint[mat + (size_t)(j0 + j) * kD + i] = __float2bfloat16_rn(x);
     }
     __syncthreads();
     for (int g = 1; g < seg.G; ++g) {
@@ -44,15 +48,24 @@ __global__ void __launch_bounds__(256) seg_combine_kernel(SegPlan seg, float* __
 #pragma unroll
             for (int c = 0; c < 4; ++c) acc[r][c] = sloc[g * mat + (size_t)(rb + 32 * r) * kD + j0 + cb + c];
         const float* P = phi + g * mat;
-        for (int k = 0; k < kD; ++k) {
-            float b[4];
+        for (int k0 = 0; k0 < kD; k0 += 32) {        // Phi[:, k0 .. k0 + 31] through shared memory
+            __syncthreads();
+            for (int e = t; e < kD * 32; e += 256) {
+                const int i = e >> 5, kk = e & 31;
+                pk[i][kk] = P[(size_t)i * kD + k0 + kk];
+            }
+            __syncthreads();
+#pragma unroll 4
+            for (int kk = 0; kk < 32; ++kk) {
+                float b[4];
 #pragma unroll
-            for (int c = 0; c < 4; ++c) b[c] = cur[k][cb + c];
+                for (int c = 0; c < 4; ++c) b[c] = cur[k0 + kk][cb + c];
 #pragma unroll
-            for (int r = 0; r < 4; ++r) {
-                const float a = P[(size_t)(rb + 32 * r) * kD + k];
+                for (int r = 0; r < 4; ++r) {
+                    const float a = pk[rb + 32 * r][kk];
 #pragma unroll
-                for (int c = 0; c < 4; ++c) acc[r][c] = fmaf(a, b[c], acc[r][c]);
+                    for (int c = 0; c < 4; ++c) acc[r][c] = fmaf(a, b[c], acc[r][c]);
+                }
             }
         }
         __syncthreads();                             // every read of cur is done
@@ -62,7 +75,7 @@ __global__ void __launch_bounds__(256) seg_combine_kernel(SegPlan seg, float* __
             for (int c = 0; c < 4; ++c) {
                 const int i = rb + 32 * r, j = cb + c;
                 cur[i][j] = acc[r][c];
-                if (g + 1 < seg.G) sin_[(g + 1) * mat + (size_t)i * kD + j0 + j] = acc[r][c];
+                if (g + 1 < seg.G) sint[(g + 1) * mat + (size_t)(j0 + j) * kD + i] = __float2bfloat16_rn(acc[r][c]);
             }
         __syncthreads();
     }
@@ -79,101 +92,85 @@ __device__ __forceinline__ uint32_t pack2(float a, float b) {
     return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// D (16x8, fp32) += A (16x16, bf16, row) B (16x8, bf16, col)
-__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
+constexpr int LW = kD + 8;     // bf16 row stride of the 128-wide tiles (conflict-free ldmatrix rows)
+constexpr int kTilesPerCta = 4;
 
-constexpr int kLdA = kD + 8;    // bf16 row stride of the R tile and of S_in^T (conflict-free fragments)
-
-// One CTA per (stream, 64-token tile of segments >= 1): o_tile += R_tile S_in(g).  Four warps,
-// 16 rows each, all 128 columns.
-__global__ void __launch_bounds__(128) seg_correct_kernel(SegPlan seg, const float* __restrict__ Sin,
-                                                          __nv_bfloat16* __restrict__ o, int T, int tiles_per) {
+// One CTA (8 warps) per (stream, run of 4 64-token tiles of segments >= 1): S_in^T of the
+// tiles' segment once, then o_tile += R_tile S_in for each tile.  Warp w: rows 16 (w % 4),
+// columns 64 (w / 4).  A run never straddles segments (segments are whole multiples of 4
+// tiles, or the run ends where its segment ends).
+__global__ void __launch_bounds__(256) seg_correct_kernel(SegPlan seg, const __nv_bfloat16* __restrict__ SinT,
+                                                          __nv_bfloat16* __restrict__ o, int T, int runs_per) {
+    using namespace mmas;
     extern __shared__ __align__(16) uint8_t seg_smem[];
-    __nv_bfloat16* Rt = reinterpret_cast<__nv_bfloat16*>(seg_smem);                  // 64 x kLdA
-    __nv_bfloat16* St = Rt + 64 * kLdA;        // S_in(g)^T: St[n][k] = S_in[k][n], kD x kLdA
-    const long s = blockIdx.x / tiles_per;
-    const int tile = (int)(blockIdx.x % tiles_per);
+    bf16* St = reinterpret_cast<bf16*>(seg_smem);    // kD x LW: S_in^T
+    bf16* Rt = St + kD * LW;                          // 2 x (64 x LW): R tiles, double-buffered
+    const long s = blockIdx.x / runs_per;
+    const int run = (int)(blockIdx.x % runs_per);
     const int L = seg.seg_chunks * 64;
-    const int t0 = L + tile * 64;                                // first token of the tile
-    const int g = min(seg.G - 1, t0 / L);
-    const int n_rows = min(64, T - t0);
+    const int runs_seg = (seg.seg_chunks + kTilesPerCta - 1) / kTilesPerCta;   // runs per segment
+    const int g = 1 + run / runs_seg;
+    const int t_first = g * L + (run % runs_seg) * kTilesPerCta * 64;
+    const int t_end = min(T, min((g + 1) * L, t_first + kTilesPerCta * 64));
+    if (g >= seg.G || t_first >= t_end) return;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const float* S = Sin + ((size_t)s * seg.G + g) * kD * kD;
-    for (int e = tid; e < kD * kD / 2; e += 128) {               // S_in -> bf16, transposed
-        const int k = e / (kD / 2), n = (e % (kD / 2)) * 2;
-        const float2 x = *reinterpret_cast<const float2*>(S + (size_t)k * kD + n);
-        St[n * kLdA + k] = __float2bfloat16_rn(x.x);
-        St[(n + 1) * kLdA + k] = __float2bfloat16_rn(x.y);
-    }
-    const __nv_bfloat16* Rg = seg.R + ((size_t)s * T + t0) * kD;
-    for (int e = tid; e < 64 * (kD / 8); e += 128) {              // R rows (zero past T)
-        const int r = e / (kD / 8), c = (e % (kD / 8)) * 8;
-        uint4 x = make_uint4(0u, 0u, 0u, 0u);
-        if (r < n_rows) x = *reinterpret_cast<const uint4*>(Rg + (size_t)r * kD + c);
-        *reinterpret_cast<uint4*>(Rt + r * kLdA + c) = x;
-    }
-    __syncthreads();
-    const int gq = lane >> 2, tq = lane & 3;
-    float acc[16][4];
-#pragma unroll
-    for (int j = 0; j < 16; ++j)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) acc[j][e] = 0.f;
-    const __nv_bfloat16* Aw = Rt + (16 * warp) * kLdA;
-#pragma unroll
-    for (int kk = 0; kk < kD / 16; ++kk) {
-        const int k = 16 * kk + 2 * tq;
-        uint32_t a[4];
-        a[0] = *reinterpret_cast<const uint32_t*>(Aw + gq * kLdA + k);
-        a[1] = *reinterpret_cast<const uint32_t*>(Aw + (gq + 8) * kLdA + k);
-        a[2] = *reinterpret_cast<const uint32_t*>(Aw + gq * kLdA + k + 8);
-        a[3] = *reinterpret_cast<const uint32_t*>(Aw + (gq + 8) * kLdA + k + 8);
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-            const __nv_bfloat16* Bn = St + (8 * j + gq) * kLdA + k;
-            mma16816(acc[j], a, *reinterpret_cast<const uint32_t*>(Bn), *reinterpret_cast<const uint32_t*>(Bn + 8));
+    const int wm = 16 * (warp & 3), wn = 64 * (warp >> 2);
+    load_tile(St, LW, SinT + ((size_t)s * seg.G + g) * kD * kD, kD, kD, kD, kD, tid, 256);
+    const bf16* Rg = seg.R + (size_t)s * T * kD;
+    auto issue = [&](int t0, bf16* dst) { load_tile(dst, LW, Rg + (size_t)t0 * kD, kD, 64, kD, min(64, t_end - t0), tid, 256); };
+    issue(t_first, Rt);
+    cp_async_commit();
+    int buf = 0;
+    for (int t0 = t_first; t0 < t_end; t0 += 64, buf ^= 1) {
+        if (t0 + 64 < t_end) {
+            issue(t0 + 64, Rt + (buf ^ 1) * 64 * LW);
+            cp_async_commit();
+            cp_async_wait<1>();
+        } else {
+            cp_async_wait<0>();
         }
-    }
-    __nv_bfloat16* Og = o + ((size_t)s * T + t0) * kD;
+        __syncthreads();
+        float acc[8][4];
+        zero_acc(acc);
+        warp_mma<8, false, false>(acc, Rt + buf * 64 * LW, LW, St, LW, wm, wn, kD, lane);
+        const int nrow = min(64, t_end - t0);
+        bf16* Og = o + ((size_t)s * T + t0) * kD;
+        const int gq = lane >> 2, tq = lane & 3;
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-        const int c = 8 * j + 2 * tq;
+        for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const int r = 16 * warp + gq + 8 * h;
-            if (r < n_rows) {
-                uint32_t* p = reinterpret_cast<uint32_t*>(Og + (size_t)r * kD + c);
-                const __nv_bfloat162 cur = *reinterpret_cast<const __nv_bfloat162*>(p);
-                const float2 f = __bfloat1622float2(cur);
-                *p = pack2(f.x + acc[j][2 * h], f.y + acc[j][2 * h + 1]);
+            for (int h = 0; h < 2; ++h) {
+                const int r = wm + gq + 8 * h, c = wn + 8 * nt + 2 * tq;
+                if (r < nrow) {
+                    uint32_t* p = reinterpret_cast<uint32_t*>(Og + (size_t)r * kD + c);
+                    const __nv_bfloat162 cur = *reinterpret_cast<const __nv_bfloat162*>(p);
+                    const float2 f = __bfloat1622float2(cur);
+                    *p = pack2(f.x + acc[nt][2 * h], f.y + acc[nt][2 * h + 1]);
+                }
             }
-        }
+        __syncthreads();                              // this buffer is reloaded two tiles later
     }
 }
 }  // namespace
 
-cudaError_t launch_seg_combine(const SegPlan& seg, const float* S0, float* S_T, float* Sin, long nstreams,
+cudaError_t launch_seg_combine(const SegPlan& seg, const float* S0, float* S_T, void* SinT, long nstreams,
                                cudaStream_t stream) {
     (void)S0;   // segment 0 starts from S0 inside the chain kernel; its final state is S_loc(0)
-    seg_combine_kernel<<<(unsigned)(nstreams * 4), 256, 0, stream>>>(seg, S_T, Sin);
+    seg_combine_kernel<<<(unsigned)(nstreams * 4), 256, 0, stream>>>(seg, S_T, static_cast<__nv_bfloat16*>(SinT));
     return cudaGetLastError();
 }
 
-cudaError_t launch_seg_correct(const SegPlan& seg, const float* Sin, __nv_bfloat16* o, long nstreams, int T,
+cudaError_t launch_seg_correct(const SegPlan& seg, const void* SinT, __nv_bfloat16* o, long nstreams, int T,
                                cudaStream_t stream) {
-    const int L = seg.seg_chunks * 64;
-    const int tiles_per = (T - L + 63) / 64;
-    if (tiles_per <= 0) return cudaSuccess;
-    constexpr int smem = (64 + kD) * kLdA * 2;
+    const int runs_seg = (seg.seg_chunks + kTilesPerCta - 1) / kTilesPerCta;
+    const int runs_per = runs_seg * (seg.G - 1);
+    if (runs_per <= 0) return cudaSuccess;
+    constexpr int smem = (kD + 2 * 64) * LW * 2;
     static std::atomic<uint64_t> smem_set{0};
     cudaError_t e = set_smem_limit_once(seg_correct_kernel, smem, smem_set);
     if (e != cudaSuccess) return e;
-    seg_correct_kernel<<<(unsigned)(nstreams * tiles_per), 128, smem, stream>>>(seg, Sin, o, T, tiles_per);
+    seg_correct_kernel<<<(unsigned)(nstreams * runs_per), 256, smem, stream>>>(
+        seg, static_cast<const __nv_bfloat16*>(SinT), o, T, runs_per);
     return cudaGetLastError();
 }
 

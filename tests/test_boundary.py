@@ -152,7 +152,10 @@ GOOD_B = [ctypes.c_void_p(0x10000000 + 0x1000000 * i) for i in range(13)]
 
 def test_backward_workspace_bytes(efla):
     L = efla.lib
-    assert L.efla_backward_workspace_bytes(4, 16, 2048, 128, 128, 1) == 4 * 16 * 2048 * (128 + 1) * 4
+    # bf16, d = 128 (the chunkwise path): error word + per tile T (64 x 64), S and dS' (128 x 128), bf16
+    assert L.efla_backward_workspace_bytes(4, 16, 2048, 128, 128, 1) == 256 + 64 * 32 * (64 * 64 + 2 * 128 * 128) * 2
+    # the reverse sweep: residuals and the gate gradient, fp32
+    assert L.efla_backward_workspace_bytes(4, 16, 2048, 128, 128, 0) == 4 * 16 * 2048 * (128 + 1) * 4
     assert L.efla_backward_workspace_bytes(1, 1, 1, 96, 96, 0) == 0      # unsupported d
     assert L.efla_backward_workspace_bytes(1, 1, 1, 128, 64, 1) == 0     # d_k != d_v
     assert L.efla_backward_workspace_bytes(1, 1, 1, 64, 64, 5) == 0      # dtype

@@ -1,11 +1,12 @@
 """The backward pass (efla_backward, CUDA) against the oracle's fp64 reverse sweep.
 
 The oracle's backward is pinned by finite differences of the pinned forward oracle
-(tests/oracle_bwd_pins.py).  Both sides take the same dtype-cast inputs; the CUDA path
-keeps the state and every gradient in fp32, so the bound is the fp32 one, 1e-4 relative
-Frobenius per gradient, for bf16 inputs too (the inputs are exact in both).  At the full
-1.3B-layer shape (B4 H16 T2048 d128) two sampled streams are compared with the oracle run
-on those streams alone, at 1e-3 (2,048 steps of fp32 rounding in the rebuilt states).
+(tests/oracle_bwd_pins.py).  Both sides take the same dtype-cast inputs.  Two CUDA paths:
+  * bf16 with d = 128 runs the backward through the chunkwise form on tensor cores, whose
+    products take bf16 operands (as the forward's do): 2e-2 relative Frobenius per gradient,
+    the bf16 bound of the forward; at the full 1.3B-layer shape (B4 H16 T2048) every stream;
+  * fp32 inputs and d = 64 run the token-by-token reverse sweep with the state and every
+    gradient in fp32: 1e-4.
 """
 import numpy as np
 import pytest
@@ -54,13 +55,31 @@ CASES = [("tiny_fp32", dict(B=1, H=2, T=200)),                          # fp32, 
          ("stiff_bf16", dict(B=1, H=2, T=300))]                           # stiff keys, corrupted tokens
 
 
+def tol_for(w):
+    return 2e-2 if (w.dtype == torch.bfloat16 and w.dk == 128) else 1e-4
+
+
 @pytest.mark.parametrize("name,over", CASES, ids=lambda x: str(x))
 def test_backward_matches_oracle(efla, cuda, name, over):
     w = W[name].replace(**over)
     got, ref = run_both(efla, cuda, w)
     for nme, g, r in zip(NAMES, got, ref):
         e = rel_frob(g, r)
-        assert e <= 1e-4, (nme, e)
+        print(f"{name} {over} {nme}: {e:.3e}")
+        assert e <= tol_for(w), (nme, e)
+
+
+@pytest.mark.parametrize("with_state,rule,T", [(False, None, 130), (True, "euler", 200), (True, None, 1),
+                                               (True, None, 64), (True, None, 65)])
+def test_chunked_backward_cases(efla, cuda, with_state, rule, T):
+    """bf16 d = 128 (the chunkwise path): no state tensors, the Euler rule, T = 1, one chunk, a
+    ragged second chunk."""
+    w = W["lm1p3b_bf16"].replace(B=1, H=2, T=T)
+    r = efla.EFLA_RULE_EULER if rule == "euler" else None
+    got, ref = run_both(efla, cuda, w, with_state=with_state, rule=r, unit_keys=rule == "euler")
+    for nme, g, rr in zip(NAMES, got, ref):
+        e = rel_frob(g, rr)
+        assert e <= 2e-2, (nme, e)
 
 
 def test_backward_without_state_tensors(efla, cuda):
@@ -93,10 +112,11 @@ def test_backward_single_token_and_empty(efla, cuda):
     assert torch.equal(out[4], dST)
 
 
-def test_backward_full_shape_sampled_streams(efla, cuda):
-    """B4 H16 T2048 d128 bf16, the forward's benchmark shape: two streams against the oracle."""
+def test_backward_full_shape_every_stream(efla, cuda):
+    """B4 H16 T2048 d128 bf16, the forward's benchmark shape: every stream against the oracle."""
     w = W["lm1p3b_bf16"]
-    got, ref = run_both(efla, cuda, w, streams=[(0, 0), (3, 15)])
+    got, ref = run_both(efla, cuda, w)
     for nme, g, r in zip(NAMES, got, ref):
         e = rel_frob(g, r)
-        assert e <= 1e-3, (nme, e)
+        print(f"full shape {nme}: {e:.3e}")
+        assert e <= 2e-2, (nme, e)
