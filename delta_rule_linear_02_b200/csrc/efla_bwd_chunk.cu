@@ -311,42 +311,64 @@ bwd_tile_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
         fA[r * LF + s2] *= al[s2];
     }
     __syncthreads();
-    {   // W = dX X^T into fY (thread: row r = tid / 4, 16 columns)
-        const int r = tid >> 2, cb = (tid & 3) * 16;
-        float w[16];
-#pragma unroll
-        for (int jj = 0; jj < 16; ++jj) w[jj] = 0.f;
+    // 64 x 64 x 64 fp32 products on CUDA cores, 4 x 4 outputs per thread (rows 4 (tid / 16),
+    // columns 4 (tid % 16)): per k, 4 + 4 shared loads for 16 FMAs
+    const int r4 = 4 * (tid >> 4), c4 = 4 * (tid & 15);
+    {   // W = dX X^T into fY:  W[r][c] = sum_m dX[r][m] X[c][m]
+        float w[4][4] = {};
         for (int m = 0; m < kC; ++m) {
-            const float a = fA[r * LF + m];
+            float a[4], b[4];
 #pragma unroll
-            for (int jj = 0; jj < 16; ++jj) w[jj] = fmaf(a, fX[(cb + jj) * LF + m], w[jj]);
+            for (int i = 0; i < 4; ++i) a[i] = fA[(r4 + i) * LF + m];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) b[j] = fX[(c4 + j) * LF + m];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) w[i][j] = fmaf(a[i], b[j], w[i][j]);
         }
 #pragma unroll
-        for (int jj = 0; jj < 16; ++jj) fY[r * LF + cb + jj] = w[jj];
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) fY[(r4 + i) * LF + c4 + j] = w[i][j];
     }
     __syncthreads();
-    {   // dA = strict_tril(-X^T W) over fA; dalpha_r += sum_{s<r} dA_rs G_rs
-        const int r = tid >> 2, cb = (tid & 3) * 16;
-        float w[16];
-#pragma unroll
-        for (int jj = 0; jj < 16; ++jj) w[jj] = 0.f;
+    {   // dA = strict_tril(-X^T W) over fA:  dA[r][c] = -sum_m X[m][r] W[m][c];  dalpha_r += sum_{s<r} dA_rs G_rs
+        float w[4][4] = {};
         for (int m = 0; m < kC; ++m) {
-            const float a = fX[m * LF + r];
+            float a[4], b[4];
 #pragma unroll
-            for (int jj = 0; jj < 16; ++jj) w[jj] = fmaf(a, fY[m * LF + cb + jj], w[jj]);
-        }
-        __syncthreads();                             // every read of dX (fA) is done
-        float part = 0.f;
+            for (int i = 0; i < 4; ++i) a[i] = fX[m * LF + r4 + i];
 #pragma unroll
-        for (int jj = 0; jj < 16; ++jj) {
-            const int s2 = cb + jj;
-            const float da = s2 < r ? -w[jj] : 0.f;
-            fA[r * LF + s2] = da;
-            part = fmaf(da, __bfloat162float(sh[L::GB + r * LH + s2]), part);
+            for (int j = 0; j < 4; ++j) b[j] = fY[m * LF + c4 + j];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) w[i][j] = fmaf(a[i], b[j], w[i][j]);
         }
-        part += __shfl_xor_sync(0xffffffffu, part, 1);
-        part += __shfl_xor_sync(0xffffffffu, part, 2);
-        if ((tid & 3) == 0) dal[r] += part;
+        // (fA, the dX tile, is not read here: it is overwritten at once)
+        float part[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            part[i] = 0.f;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int r = r4 + i, s2 = c4 + j;
+                const float da = s2 < r ? -w[i][j] : 0.f;
+                fA[r * LF + s2] = da;
+                part[i] = fmaf(da, __bfloat162float(sh[L::GB + r * LH + s2]), part[i]);
+            }
+        }
+        // the 16 column blocks of a row block sit in 16 consecutive lanes: sum over them
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+#pragma unroll
+            for (int off = 1; off < 16; off <<= 1) part[i] += __shfl_xor_sync(0xffffffffu, part[i], off);
+        }
+        if ((tid & 15) == 0) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) dal[r4 + i] += part[i];
+        }
     }
     __syncthreads();
     for (int e = tid; e < kC * kC; e += 256) {       // dG + dG^T with dG = diag(alpha) dA, bf16 over G

@@ -29,8 +29,10 @@
 // [W;Q] S -> Delta -> K^T Delta -> bf16 S -> the next [W;Q] S between roles.
 //
 // One warp issues every MMA, in a fixed order per chunk c:
-//   [W;Q] S(c), Q K^T(c), [W|U](c+1), K^T Delta(c) (after Delta), P Delta(c)
-// so that only P Delta(c) is in the pipe ahead of the next [W;Q] S.
+//   [W;Q] S(c), Q K^T(c), K^T Delta(c) (after Delta), P Delta(c), [W|U](c+2)
+// so that only Q K^T(c) is ahead of K^T Delta(c) in the in-order pipe, and [W|U] fills the
+// state-rebuild window two chunks ahead (the Delta warps take U(c+1) into registers right
+// after forming Delta(c), which frees its accumulator early).
 // Issue is by a converged warp with elect.sync (warp-uniform control flow keeps the
 // descriptors in uniform registers; a one-lane issuer in a data-dependent loop issues
 // several times slower).
@@ -395,6 +397,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         };
         bool ok = wait(B_KVT_FULL, 0);
         if (ok) issue_wu(0);
+        if (ok && nchunks > 1) {
+            ok = wait(B_KVT_FULL + 1, 0) && wait(B_WU_FREE, 0);
+            if (ok) issue_wu(1);
+        }
         for (int c = 0; c < nchunks && ok; ++c) {
             // X = [W; Q] S (state chain)
             if (!(ok = wait(B_W_READY, c & 1) && wait(B_Q_READY, c & 1) && wait(B_SB_READY, c & 1) &&
@@ -403,16 +409,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             tc_fence_after();
             mma_ts(tmem + TM_X, tmem + TM_AWQ, sb + OFF_SB, 4 * 2048, 2048, TILE, ID_N64, 8, 0);
             mma_commit_elect(ctl.b(B_XS_FULL));
-            // this chunk's Q K^T (its Q has been in place since the last chunk) and the next
-            // chunk's [W | U] fill the pipe while Delta is formed; after K^T Delta only
-            // P Delta remains ahead of the next [W;Q] S
+            // this chunk's Q K^T (its Q has been in place since the last chunk) runs while
+            // Delta is formed
             if (!(ok = c == 0 || wait(B_GP_FREE, (c - 1) & 1))) break;
             issue_qk(c, 0, 8);
-            if (c + 1 < nchunks) {
-                if (!(ok = wait(B_KVT_FULL + (c + 1) % kKvtStages, ((c + 1) / kKvtStages) & 1) &&
-                           wait(B_WU_FREE, c & 1))) break;
-                issue_wu(c + 1);
-            }
             // S += K^T Delta (state chain)
             if (!(ok = wait(B_D_READY, c & 1))) break;
             tc_fence_after();
@@ -427,6 +427,11 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             mma_ts(tmem + TM_X, tmem + TM_AP, sb + OFF_DL, 4 * 2048, 2048, TILE, ID_N64, 4, 1);
             mma_commit_elect(ctl.b(B_O_FULL));
             if constexpr (kGated) mma_commit_elect(ctl.b(B_KVT_FREE + c % kKvtStages));
+            if (c + 2 < nchunks) {   // [W|U] two chunks ahead, in this chunk's state-rebuild window
+                if (!(ok = wait(B_KVT_FULL + (c + 2) % kKvtStages, ((c + 2) / kKvtStages) & 1) &&
+                           wait(B_WU_FREE, (c + 1) & 1))) break;
+                issue_wu(c + 2);
+            }
         }
         mma_commit_elect(ctl.b(B_DRAIN));
         if (lane == 0) mbar_wait(ctl.b(B_DRAIN), 0, limit_ns);
@@ -636,15 +641,18 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             ctl.warp_arrive(B_SB_READY, lane);
         }
         bool ok = true;
+        float u[32];
+        auto take_u = [&](int cu) {
+            if (!ctl.wwait(B_WU_FULL, cu & 1)) return false;
+            tc_fence_after();
+            tmem_ld32_wait(tmem + lane_off + TM_WU + 128 + cc, u);
+            tc_fence_before();
+            ctl.warp_arrive(B_WU_FREE, lane);
+            return true;
+        };
+        if (delta_group) ok = take_u(0);
         for (int c = 0; c < nchunks && ok; ++c) {
             if (delta_group) {
-                // take U(c) from its accumulator as soon as it lands ([W|U](c+1) reuses it)
-                float u[32];
-                if (!(ok = ctl.wwait(B_WU_FULL, c & 1))) break;
-                tc_fence_after();
-                tmem_ld32_wait(tmem + lane_off + TM_WU + 128 + cc, u);
-                tc_fence_before();
-                ctl.warp_arrive(B_WU_FREE, lane);
                 // Delta = U - W S (X rows 0-63)
                 if (!(ok = ctl.wwait(B_XS_FULL, c & 1))) break;
                 tc_fence_after();
@@ -665,6 +673,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 fence_proxy_async_smem();
                 tc_fence_before();
                 ctl.warp_arrive(B_D_READY, lane);
+                if (c + 1 < nchunks && !(ok = take_u(c + 1))) break;   // U(c+1) before [W|U](c+2)
             }
             // the new state: bf16 operand for the next chunk (and S_T after the last)
             if (!(ok = ctl.wwait(B_S_FULL, c & 1))) break;
