@@ -153,9 +153,17 @@ def traffic_from_csv(csv_path: str, entry: str, calls: int):
     rows = []
     with open(csv_path) as f:
         lines = [ln for ln in f if ln.startswith('"')]
-    def bare(name):      # "void (anonymous namespace)::decode_kernel<float, 128>(...)" -> "decode_kernel"
-        name = name.removeprefix("void ").replace("(anonymous namespace)::", "").replace("unnamed>::", "")
-        return name.split("(")[0].split("<")[0].split("::")[-1].strip()
+    def bare(name):      # "void efla::<unnamed>::decode_kernel<float, 128, 0>(...)" -> "decode_kernel"
+        head = name.replace("(anonymous namespace)", "anon").split("(")[0].strip()
+        if head.endswith(">"):                       # drop the trailing template arguments
+            depth, i = 0, len(head) - 1
+            while i >= 0:
+                depth += {">": 1, "<": -1}.get(head[i], 0)
+                if depth == 0:
+                    break
+                i -= 1
+            head = head[:i]
+        return head.split("::")[-1].split(" ")[-1].strip()
 
     for r in csv.DictReader(lines):
         name = bare(r.get("Kernel Name", ""))

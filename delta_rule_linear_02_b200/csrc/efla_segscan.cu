@@ -105,6 +105,7 @@ __global__ void __launch_bounds__(256) seg_correct_kernel(SegPlan seg, const __n
     extern __shared__ __align__(16) uint8_t seg_smem[];
     bf16* St = reinterpret_cast<bf16*>(seg_smem);    // kD x LW: S_in^T
     bf16* Rt = St + kD * LW;                          // 2 x (64 x LW): R tiles, double-buffered
+    float* Ct = reinterpret_cast<float*>(Rt + 2 * 64 * LW);   // 64 x (kD + 4): R S_in of a tile, fp32
     const long s = blockIdx.x / runs_per;
     const int run = (int)(blockIdx.x % runs_per);
     const int L = seg.seg_chunks * 64;
@@ -133,22 +134,27 @@ __global__ void __launch_bounds__(256) seg_correct_kernel(SegPlan seg, const __n
         float acc[8][4];
         zero_acc(acc);
         warp_mma<8, false, false>(acc, Rt + buf * 64 * LW, LW, St, LW, wm, wn, kD, lane);
+        for_acc(acc, wm, wn, lane, [&](int r, int c, float& x) { Ct[r * (kD + 4) + c] = x; });
+        __syncthreads();                              // the tile's R S_in is staged; this R buffer is free
+        // o += R S_in with 16-byte accesses: 8 consecutive bf16 of a row per thread and step
         const int nrow = min(64, t_end - t0);
         bf16* Og = o + ((size_t)s * T + t0) * kD;
-        const int gq = lane >> 2, tq = lane & 3;
+        for (int e = tid; e < 64 * (kD / 8); e += 256) {
+            const int r = e / (kD / 8), c = (e % (kD / 8)) * 8;
+            if (r < nrow) {
+                uint4* p = reinterpret_cast<uint4*>(Og + (size_t)r * kD + c);
+                uint4 cur = *p;
+                const float* add = Ct + r * (kD + 4) + c;
+                uint32_t* w = reinterpret_cast<uint32_t*>(&cur);
 #pragma unroll
-        for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int r = wm + gq + 8 * h, c = wn + 8 * nt + 2 * tq;
-                if (r < nrow) {
-                    uint32_t* p = reinterpret_cast<uint32_t*>(Og + (size_t)r * kD + c);
-                    const __nv_bfloat162 cur = *reinterpret_cast<const __nv_bfloat162*>(p);
-                    const float2 f = __bfloat1622float2(cur);
-                    *p = pack2(f.x + acc[nt][2 * h], f.y + acc[nt][2 * h + 1]);
+                for (int m = 0; m < 4; ++m) {
+                    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(w + m));
+                    w[m] = pack2(f.x + add[2 * m], f.y + add[2 * m + 1]);
                 }
+                *p = cur;
             }
-        __syncthreads();                              // this buffer is reloaded two tiles later
+        }
+        __syncthreads();                              // Ct is rewritten by the next tile
     }
 }
 }  // namespace
@@ -165,7 +171,7 @@ cudaError_t launch_seg_correct(const SegPlan& seg, const void* SinT, __nv_bfloat
     const int runs_seg = (seg.seg_chunks + kTilesPerCta - 1) / kTilesPerCta;
     const int runs_per = runs_seg * (seg.G - 1);
     if (runs_per <= 0) return cudaSuccess;
-    constexpr int smem = (kD + 2 * 64) * LW * 2;
+    constexpr int smem = (kD + 2 * 64) * LW * 2 + 64 * (kD + 4) * 4;
     static std::atomic<uint64_t> smem_set{0};
     cudaError_t e = set_smem_limit_once(seg_correct_kernel, smem, smem_set);
     if (e != cudaSuccess) return e;

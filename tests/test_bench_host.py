@@ -48,12 +48,12 @@ CSV = """==PROF== Connected to process 1
 "ID","Process ID","Process Name","Host Name","Kernel Name","Context","Stream","Block Size","Grid Size","Device","CC","Section Name","Metric Name","Metric Unit","Metric Value"
 "0","1","python","h","(anonymous namespace)::ut_kernel(CUtensorMap_st, bf16)","1","7","(160, 1, 1)","(888, 1, 1)","0","10.0","Command line profiler metrics","dram__bytes_read.sum","byte","1,000"
 "0","1","python","h","(anonymous namespace)::ut_kernel(CUtensorMap_st, bf16)","1","7","(160, 1, 1)","(888, 1, 1)","0","10.0","Command line profiler metrics","dram__bytes_write.sum","byte","10"
-"1","1","python","h","unnamed>::chunk_tc_kernel(CUtensorMap_st)","1","7","(448, 1, 1)","(128, 1, 1)","0","10.0","Command line profiler metrics","dram__bytes_read.sum","Kbyte","2"
-"1","1","python","h","unnamed>::chunk_tc_kernel(CUtensorMap_st)","1","7","(448, 1, 1)","(128, 1, 1)","0","10.0","Command line profiler metrics","dram__bytes_write.sum","byte","300"
+"1","1","python","h","void efla::<unnamed>::chunk_tc_kernel<0>(CUtensorMap_st)","1","7","(448, 1, 1)","(128, 1, 1)","0","10.0","Command line profiler metrics","dram__bytes_read.sum","Kbyte","2"
+"1","1","python","h","void efla::<unnamed>::chunk_tc_kernel<0>(CUtensorMap_st)","1","7","(448, 1, 1)","(128, 1, 1)","0","10.0","Command line profiler metrics","dram__bytes_write.sum","byte","300"
 "2","1","python","h","(anonymous namespace)::ut_kernel(CUtensorMap_st, bf16)","1","7","(160, 1, 1)","(888, 1, 1)","0","10.0","Command line profiler metrics","dram__bytes_read.sum","byte","5,000"
 "2","1","python","h","(anonymous namespace)::ut_kernel(CUtensorMap_st, bf16)","1","7","(160, 1, 1)","(888, 1, 1)","0","10.0","Command line profiler metrics","dram__bytes_write.sum","byte","50"
-"3","1","python","h","unnamed>::chunk_tc_kernel(CUtensorMap_st)","1","7","(448, 1, 1)","(128, 1, 1)","0","10.0","Command line profiler metrics","dram__bytes_read.sum","byte","7,000"
-"3","1","python","h","unnamed>::chunk_tc_kernel(CUtensorMap_st)","1","7","(448, 1, 1)","(128, 1, 1)","0","10.0","Command line profiler metrics","dram__bytes_write.sum","byte","700"
+"3","1","python","h","void efla::<unnamed>::chunk_tc_kernel<0>(CUtensorMap_st)","1","7","(448, 1, 1)","(128, 1, 1)","0","10.0","Command line profiler metrics","dram__bytes_read.sum","byte","7,000"
+"3","1","python","h","void efla::<unnamed>::chunk_tc_kernel<0>(CUtensorMap_st)","1","7","(448, 1, 1)","(128, 1, 1)","0","10.0","Command line profiler metrics","dram__bytes_write.sum","byte","700"
 """
 
 
