@@ -15,8 +15,12 @@ import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libefla.so")
+# the same entry points built with EFLA_CHECKED=1: the tensor-core forward's kernels test
+# every direct global access against its buffer and report EFLA_ERR_BOUNDS through the
+# workspace status instead of touching memory out of range (build.py --checked)
+LIB_CHECKED_PATH = os.path.join(_PKG, "libefla_checked.so")
 
-EFLA_OK, EFLA_ERR_INVALID_ARG, EFLA_ERR_UNSUPPORTED, EFLA_ERR_CUDA, EFLA_ERR_TIMEOUT = range(5)
+EFLA_OK, EFLA_ERR_INVALID_ARG, EFLA_ERR_UNSUPPORTED, EFLA_ERR_CUDA, EFLA_ERR_TIMEOUT, EFLA_ERR_BOUNDS = range(6)
 EFLA_DTYPE_F32, EFLA_DTYPE_BF16 = 0, 1
 EFLA_RULE_EXACT, EFLA_RULE_EULER = 0, 1     # exact-flow gate, or alpha = beta (the delta rule)
 CHUNK = 64
@@ -30,11 +34,11 @@ class EflaError(RuntimeError):
         super().__init__(f"{where}: {efla_status_string(status)} ({status})")
 
 
-def _load() -> ctypes.CDLL:
-    if not os.path.exists(LIB_PATH):
-        raise ImportError(f"libefla.so is not built at {LIB_PATH}; run "
+def _load(path: str = LIB_PATH) -> ctypes.CDLL:
+    if not os.path.exists(path):
+        raise ImportError(f"{os.path.basename(path)} is not built at {path}; run "
                           "`python delta_rule_linear_02_b200/build.py` (nvcc, sm_100a)")
-    lib = ctypes.CDLL(LIB_PATH)
+    lib = ctypes.CDLL(path)
     vp, I, L, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_long, ctypes.c_size_t
     lib.efla_status_string.argtypes = [I]
     lib.efla_status_string.restype = ctypes.c_char_p
@@ -82,6 +86,12 @@ def _load() -> ctypes.CDLL:
 
 
 lib = _load()
+
+
+def load_checked() -> ctypes.CDLL:
+    """The checked build (libefla_checked.so) with the same argument types as `lib`; the
+    wrappers below call whichever library the module attribute `lib` holds."""
+    return _load(LIB_CHECKED_PATH)
 
 
 def efla_status_string(status: int) -> str:
@@ -385,5 +395,5 @@ def efla_backward(q, k, v, beta, dO, S0=None, dS_T=None, want_dS0: bool = True, 
 
 
 __all__ = ["efla_chunk_fwd_segmented", "efla_chunk_fwd_varlen", "efla_chunk_fwd_gated", "efla_recurrent_step_gated", "efla_backward", "efla_backward_workspace_bytes", "EFLA_RULE_EXACT", "EFLA_RULE_EULER", "efla_gate", "efla_chunk_fwd", "efla_chunk_fwd_noalloc", "efla_chunk_fwd_workspace_bytes", "efla_recurrent_step",
-           "efla_workspace_status", "efla_noalloc_status", "efla_status_string", "efla_selftest_wait_timeout", "new_workspace", "EflaError", "lib",
+           "efla_workspace_status", "efla_noalloc_status", "efla_status_string", "load_checked", "efla_selftest_wait_timeout", "new_workspace", "EflaError", "lib",
            "LIB_PATH", "CHUNK"]

@@ -36,6 +36,7 @@ const char* efla_status_string(int status) {
         case EFLA_ERR_UNSUPPORTED: return "EFLA_ERR_UNSUPPORTED";
         case EFLA_ERR_CUDA: return "EFLA_ERR_CUDA";
         case EFLA_ERR_TIMEOUT: return "EFLA_ERR_TIMEOUT";
+        case EFLA_ERR_BOUNDS: return "EFLA_ERR_BOUNDS";
         default: return "EFLA_ERR_UNKNOWN";
     }
 }
@@ -381,7 +382,8 @@ int efla_workspace_status(void* workspace, int clear, efla_stream_t stream) {
         if (cudaMemsetAsync(workspace, 0, sizeof(word), s) != cudaSuccess) return EFLA_ERR_CUDA;
         if (cudaStreamSynchronize(s) != cudaSuccess) return EFLA_ERR_CUDA;
     }
-    return word == efla::kDevOk ? EFLA_OK : EFLA_ERR_TIMEOUT;
+    if (word == efla::kDevOk) return EFLA_OK;
+    return (word & efla::kDevBounds) ? EFLA_ERR_BOUNDS : EFLA_ERR_TIMEOUT;
 }
 
 int efla_selftest_wait_timeout(void* workspace, long long limit_ns, efla_stream_t stream) {

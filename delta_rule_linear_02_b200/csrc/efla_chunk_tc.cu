@@ -224,7 +224,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_t,
                 const float* __restrict__ S0, __nv_bfloat16* __restrict__ o, float* __restrict__ S_T,
                 Seqs seqs, int Tdim, uint32_t* __restrict__ err, unsigned long long limit_ns,
-                const float* __restrict__ gl_all, long ntiles, SegPlan seg) {
+                const float* __restrict__ gl_all, long ntiles, SegPlan seg, ChainSpans spans) {
     using L = Lay<kGated>;
     constexpr uint32_t KVT_K = L::KVT_K, KVT_V = L::KVT_V, KVT_T = L::KVT_T, KVT_BYTES = L::KVT_BYTES;
     constexpr uint32_t OFF_KVT = L::OFF_KVT, OFF_Q = L::OFF_Q, OFF_DL = L::OFF_DL, OFF_SB = L::OFF_SB;
@@ -282,12 +282,19 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const int T = jb.len, zc = jb.z, y0 = jb.y0;
     const int nchunks = (T + 63) / 64;
     const size_t tok0 = (size_t)zc * Tdim + y0;
+    // the extents this CTA's pointers must stay inside (checked builds)
+    const Span op_span = op == o ? spans.o : spans.r;
+    const bool st_in_phi = seg.Phi && stp >= seg.Phi && stp < seg.Phi + spans.phi.bytes / sizeof(float);
+    const Span st_span = seg.G <= 1 ? spans.st : (st_in_phi ? spans.phi : spans.sloc);
+    const Span s0_span = spans.s0;
     if (nchunks == 0) {   // an empty sequence: the state passes through (nothing else runs)
         if (stp) {
             for (int e = tid; e < kD * 64; e += kThreads) {
                 const int i = e >> 6, j = e & 63;
                 const size_t at = (size_t)i * kD + col0 + j;
-                stp[at] = s0_identity ? (i == col0 + j ? 1.f : 0.f) : (s0p ? s0p[at] : 0.f);
+                float x = s0_identity ? (i == col0 + j ? 1.f : 0.f) : 0.f;
+                if (!s0_identity && s0p && span_ok(err, s0_span, s0p + at, 4)) x = s0p[at];
+                if (span_ok(err, st_span, stp + at, 4)) stp[at] = x;
             }
         }
         return;
@@ -336,10 +343,13 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     tma_load_3d(st + KVT_K, &tm_k, full, 0, y0 + t0, zc);
                     tma_load_3d(st + KVT_K + TILE, &tm_k, full, 64, y0 + t0, zc);
                     if (!vzero) tma_load_3d(st + KVT_V, &tm_v, full, col0, y0 + t0, zc);
+                    if (EFLA_CHECKED && (jb.tile0 + c + 1) * 64 > spans.t_rows) atomicOr(err, kDevBounds);
                     tma_load_2d(st + KVT_T, &tm_t, full, 0, (int)((jb.tile0 + c) * 64));
                     if constexpr (kGated) {
                         tma_load_2d(st + L::KVT_TU, &tm_t, full, 0, (int)((ntiles + jb.tile0 + c) * 64));
-                        bulk_load(st + L::KVT_GL, gl_all + (jb.tile0 + c) * 64, 256, full);
+                        const float* src = gl_all + (jb.tile0 + c) * 64;
+                        if (!span_ok(err, spans.gl, src, 256)) src = gl_all;   // keep the transaction count
+                        bulk_load(st + L::KVT_GL, src, 256, full);
                     }
                     kvt_issued = c + 1;
                 }
@@ -488,7 +498,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             tc_fence_before();
             ctl.warp_arrive(B_X_FREE, lane);
             const int t0 = c * 64;
-            if (op && r < min(64, T - t0)) {
+            if (op && r < min(64, T - t0) && span_ok(err, op_span, op + (tok0 + t0 + r) * kD + col0, 128)) {
                 uint4* dst = reinterpret_cast<uint4*>(op + (tok0 + t0 + r) * kD + col0);
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
@@ -614,7 +624,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 float s16[16];
 #pragma unroll
                 for (int j = 0; j < 16; j += 4) {
-                    float4 x = src ? *reinterpret_cast<const float4*>(src + 16 * qd + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+                    float4 x = src && span_ok(err, s0_span, src + 16 * qd + j, 16)
+                                   ? *reinterpret_cast<const float4*>(src + 16 * qd + j) : make_float4(0.f, 0.f, 0.f, 0.f);
                     if (s0_identity) {
                         const int c0 = col0 + cc + 16 * qd + j;    // this row's 1 sits in column ct
                         x = make_float4(ct == c0 ? 1.f : 0.f, ct == c0 + 1 ? 1.f : 0.f, ct == c0 + 2 ? 1.f : 0.f,
@@ -622,12 +633,16 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     }
                     s16[j] = x.x; s16[j + 1] = x.y; s16[j + 2] = x.z; s16[j + 3] = x.w;
                 }
-                st_chunk(sm + OFF_SB + sw128_off(ct, 4 * ch + 2 * qd), s16);
-                st_chunk(sm + OFF_SB + sw128_off(ct, 4 * ch + 2 * qd + 1), s16 + 8);
+                if (smem_ok(err, OFF_SB + sw128_off(ct, 4 * ch + 2 * qd + 1), 16, OFF_SB + 2 * TILE)) {
+                    st_chunk(sm + OFF_SB + sw128_off(ct, 4 * ch + 2 * qd), s16);
+                    st_chunk(sm + OFF_SB + sw128_off(ct, 4 * ch + 2 * qd + 1), s16 + 8);
+                }
                 if (seg.states) {   // chunk 0's entering state, for the backward
                     uint8_t* dst = reinterpret_cast<uint8_t*>(seg.states + ((size_t)jb.tile0 * kD + ct) * kD + col0 + cc + 16 * qd);
-                    st_chunk(dst, s16);
-                    st_chunk(dst + 16, s16 + 8);
+                    if (span_ok(err, spans.states, dst, 32)) {
+                        st_chunk(dst, s16);
+                        st_chunk(dst + 16, s16 + 8);
+                    }
                 }
                 if constexpr (kGated) {
 #pragma unroll
@@ -661,7 +676,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
                 for (int j = 0; j < 32; ++j) t[j] = u[j] - t[j];
 #pragma unroll
-                for (int j = 0; j < 4; ++j) st_chunk(sm + OFF_DL + sw128_off(ct, 4 * ch + j), t + 8 * j);
+                for (int j = 0; j < 4; ++j)
+                    if (smem_ok(err, OFF_DL + sw128_off(ct, 4 * ch + j), 16, OFF_DL + TILE))
+                        st_chunk(sm + OFF_DL + sw128_off(ct, 4 * ch + j), t + 8 * j);
                 if constexpr (kGated) {   // the state's copy: row r scaled by Gam_last / Gam_r
                     const float* glc = reinterpret_cast<const float*>(sm + kvt(c) + L::KVT_GL);
                     const float sc = exp2f(glc[63] - glc[ct]);
@@ -682,13 +699,17 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 float t[32];
                 tmem_ld32_wait(tmem + lane_off + TM_S + cc, t);
 #pragma unroll
-                for (int j = 0; j < 4; ++j) st_chunk(sm + OFF_SB + sw128_off(ct, 4 * ch + j), t + 8 * j);
+                for (int j = 0; j < 4; ++j)
+                    if (smem_ok(err, OFF_SB + sw128_off(ct, 4 * ch + j), 16, OFF_SB + 2 * TILE))
+                        st_chunk(sm + OFF_SB + sw128_off(ct, 4 * ch + j), t + 8 * j);
                 if (seg.states && c + 1 < nchunks) {   // chunk c+1's entering state, for the backward
                     uint8_t* dst = reinterpret_cast<uint8_t*>(seg.states + ((size_t)(jb.tile0 + c + 1) * kD + ct) * kD + col0 + cc);
+                    if (span_ok(err, spans.states, dst, 64)) {
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) st_chunk(dst + 16 * j, t + 8 * j);
+                        for (int j = 0; j < 4; ++j) st_chunk(dst + 16 * j, t + 8 * j);
+                    }
                 }
-                if (c == nchunks - 1 && stp) {
+                if (c == nchunks - 1 && stp && span_ok(err, st_span, stp + (size_t)ct * kD + col0 + cc, 128)) {
                     float* dst = stp + (size_t)ct * kD + col0 + cc;
 #pragma unroll
                     for (int j = 0; j < 32; j += 4)
@@ -755,6 +776,17 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const v
     cudaError_t e = launch_ut(k, beta, scratch, seqs, Z, Tdim, ntiles, err, kWaitLimitNs, rule, stream, g);
     if (e != cudaSuccess) return e;
     const long ctas = seg.G > 1 ? nstreams * (2 + 4 * (seg.G - 1)) : nstreams * 2;
+    ChainSpans sp;
+    const size_t obytes = (size_t)Z * Tdim * kD * 2, sbytes = (size_t)nstreams * kD * kD * 4;
+    sp.o = Span{o, obytes};
+    sp.r = Span{seg.R, obytes};
+    sp.s0 = Span{S0, sbytes};
+    sp.st = Span{S_T, sbytes};
+    sp.sloc = Span{seg.Sloc, sbytes * std::max(1, seg.G)};
+    sp.phi = Span{seg.Phi, sbytes * std::max(1, seg.G)};
+    sp.states = Span{seg.states, (size_t)ntiles * kD * kD * 2};
+    sp.gl = Span{g ? static_cast<const char*>(scratch) + ntiles * 8192 * 2 : nullptr, (size_t)ntiles * 256};
+    sp.t_rows = (g ? 2 : 1) * ntiles * 64;
     CUtensorMap mq, mk, mv, mt;
     if (!tma_map_tokens(&mq, q, kD, Tdim, Z) || !tma_map_tokens(&mk, k, kD, Tdim, Z) ||
         !tma_map_tokens(&mv, v, kD, Tdim, Z) || !tma_map_rows64(&mt, scratch, std::max<long>(1, (g ? 2 : 1) * ntiles) * 64))
@@ -765,14 +797,14 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const v
         e = set_smem_limit_once(chunk_tc_kernel<true>, (int)Lay<true>::SMEM_BYTES, smem_set_g);
         if (e != cudaSuccess) return e;
         chunk_tc_kernel<true><<<(unsigned)ctas, kThreads, Lay<true>::SMEM_BYTES, stream>>>(
-            mq, mk, mv, mt, S0, (__nv_bfloat16*)o, S_T, seqs, Tdim, err, kWaitLimitNs, gl, ntiles, seg);
+            mq, mk, mv, mt, S0, (__nv_bfloat16*)o, S_T, seqs, Tdim, err, kWaitLimitNs, gl, ntiles, seg, sp);
         return cudaGetLastError();
     }
     static std::atomic<uint64_t> smem_set{0};
     e = set_smem_limit_once(chunk_tc_kernel<false>, (int)Lay<false>::SMEM_BYTES, smem_set);
     if (e != cudaSuccess) return e;
     chunk_tc_kernel<false><<<(unsigned)ctas, kThreads, Lay<false>::SMEM_BYTES, stream>>>(
-        mq, mk, mv, mt, S0, (__nv_bfloat16*)o, S_T, seqs, Tdim, err, kWaitLimitNs, nullptr, ntiles, seg);
+        mq, mk, mv, mt, S0, (__nv_bfloat16*)o, S_T, seqs, Tdim, err, kWaitLimitNs, nullptr, ntiles, seg, sp);
     return cudaGetLastError();
 }
 

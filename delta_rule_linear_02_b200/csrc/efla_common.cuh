@@ -147,7 +147,43 @@ struct Seqs {
 };
 
 // Device error word values (kept in the caller's workspace).
-enum : uint32_t { kDevOk = 0u, kDevTimeout = 1u };
+enum : uint32_t { kDevOk = 0u, kDevTimeout = 1u, kDevBounds = 2u };
+
+// ---------------------------------------------------------------- checked builds
+// Built with -DEFLA_CHECKED=1 (delta_rule_linear_02_b200/build.py --checked, a separate
+// library), the tensor-core forward's kernels test every generic global access and every
+// computed shared-memory store against the extent of its buffer; a violation sets
+// kDevBounds in the error word and the access is skipped (no trap, no assert).  In the
+// normal build the tests compile away.
+#ifndef EFLA_CHECKED
+#define EFLA_CHECKED 0
+#endif
+struct Span {
+    const void* p = nullptr;
+    size_t bytes = 0;
+};
+__device__ __forceinline__ bool span_ok(uint32_t* err, Span s, const void* q, size_t n) {
+#if EFLA_CHECKED
+    const uintptr_t a = reinterpret_cast<uintptr_t>(s.p), b = reinterpret_cast<uintptr_t>(q);
+    if (s.p && b >= a && b + n <= a + s.bytes) return true;
+    atomicOr(err, kDevBounds);
+    return false;
+#else
+    (void)err; (void)s; (void)q; (void)n;
+    return true;
+#endif
+}
+// an offset into a CTA's shared-memory map of `limit` bytes
+__device__ __forceinline__ bool smem_ok(uint32_t* err, uint32_t off, uint32_t n, uint32_t limit) {
+#if EFLA_CHECKED
+    if (off + n <= limit) return true;
+    atomicOr(err, kDevBounds);
+    return false;
+#else
+    (void)err; (void)off; (void)n; (void)limit;
+    return true;
+#endif
+}
 
 // A kernel's dynamic shared-memory limit is a per-device attribute that persists, so it
 // is set once per device (bit `dev` of `done`); setting it on every launch would add a

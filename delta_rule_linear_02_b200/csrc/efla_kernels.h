@@ -45,6 +45,13 @@ struct SegPlan {
     __nv_bfloat16* R = nullptr;    // [Z][Tdim][128] (rows of segments >= 1)
 };
 
+// The extents of every buffer the chain kernel addresses directly (checked builds test each
+// access against them; see efla_common.cuh).
+struct ChainSpans {
+    Span o, r, s0, st, sloc, phi, states, gl;
+    long t_rows = 0;               // rows of the tensor map over the UT transforms
+};
+
 // nstreams recurrences described by `seqs` over tensors [Z][Tdim][d]; ntiles UT tiles
 cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const void* beta, const float* S0,
                             void* o, float* S_T, const Seqs& seqs, long nstreams, long Z, int Tdim, long ntiles,

@@ -94,7 +94,8 @@ template <bool kGated>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 ut_kernel(const __grid_constant__ CUtensorMap tm_k, const __nv_bfloat16* __restrict__ beta,
           __nv_bfloat16* __restrict__ Tout, Seqs seqs, int Tdim, long ntiles, uint32_t* __restrict__ err,
-          unsigned long long limit_ns, int rule, const float* __restrict__ gdec) {
+          unsigned long long limit_ns, int rule, const float* __restrict__ gdec, Span t_span, Span b_span,
+          Span g_span) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sb = smem_u32(sm);
@@ -188,7 +189,8 @@ ut_kernel(const __grid_constant__ CUtensorMap tm_k, const __nv_bfloat16* __restr
             int c;
             const StreamJob jb = seqs.tile(tile, &c);
             const int t = c * 64 + wt;
-            return t < jb.len ? __bfloat162float(beta[(long)jb.z * Tdim + jb.y0 + t]) : 0.f;
+            const __nv_bfloat16* p = beta + (long)jb.z * Tdim + jb.y0 + t;
+            return t < jb.len && span_ok(err, b_span, p, 2) ? __bfloat162float(*p) : 0.f;
         };
         auto g_of = [&](int j) -> float {
             if (j >= ntile || wt >= 64) return 0.f;
@@ -196,7 +198,8 @@ ut_kernel(const __grid_constant__ CUtensorMap tm_k, const __nv_bfloat16* __restr
             int c;
             const StreamJob jb = seqs.tile(tile, &c);
             const int t = c * 64 + wt;
-            return t < jb.len ? gdec[(long)jb.z * Tdim + jb.y0 + t] : 0.f;
+            const float* p = gdec + (long)jb.z * Tdim + jb.y0 + t;
+            return t < jb.len && span_ok(err, g_span, p, 4) ? *p : 0.f;
         };
         float beta_next = beta_of(0);
         float g_next = 0.f;
@@ -295,6 +298,7 @@ ut_kernel(const __grid_constant__ CUtensorMap tm_k, const __nv_bfloat16* __restr
                 const int rr = wt & 63, h = wt >> 6;
                 auto store = [&](const float* mult, long tile_at) {
                     uint4* dst = reinterpret_cast<uint4*>(Tout + (tile_at * 64 + rr) * 64 + 32 * h);
+                    if (!span_ok(err, t_span, dst, 64)) return;
 #pragma unroll
                     for (int m = 0; m < 4; ++m) {
                         const float4 x0 = *reinterpret_cast<const float4*>(X + rr * LDX + 32 * h + 8 * m);
@@ -312,7 +316,8 @@ ut_kernel(const __grid_constant__ CUtensorMap tm_k, const __nv_bfloat16* __restr
                 if constexpr (kGated) {
                     store(mw, tile);
                     store(abar, ntiles + tile);
-                    if (wt < 64) reinterpret_cast<float*>(Tout + 2 * ntiles * 4096)[tile * 64 + wt] = gl[wt];
+                    float* gdst = reinterpret_cast<float*>(Tout + 2 * ntiles * 4096) + tile * 64 + wt;
+                    if (wt < 64 && span_ok(err, t_span, gdst, 4)) *gdst = gl[wt];
                 } else {
                     store(al, tile);
                 }
@@ -342,19 +347,23 @@ cudaError_t launch_ut(const void* k, const void* beta, void* Tout, const Seqs& s
     CUtensorMap mk;
     if (!tma_map_tokens(&mk, k, 128, Tdim, Z)) return cudaErrorInvalidValue;
     const long grid = std::min<long>(ntiles, (long)sm_count() * kCtasPerSm);
+    const Span t_span{Tout, (size_t)ntiles * (g ? 2 * 8192 + 256 : 8192)};
+    const Span b_span{beta, (size_t)Z * Tdim * 2}, g_span{g, (size_t)Z * Tdim * 4};
     cudaError_t e;
     if (g) {
         static std::atomic<uint64_t> smem_set_g{0};
         e = set_smem_limit_once(ut_kernel<true>, (int)SMEM_BYTES_G, smem_set_g);
         if (e != cudaSuccess) return e;
         ut_kernel<true><<<(unsigned)grid, kThreads, SMEM_BYTES_G, stream>>>(
-            mk, (const __nv_bfloat16*)beta, (__nv_bfloat16*)Tout, seqs, Tdim, ntiles, err, limit_ns, rule, g);
+            mk, (const __nv_bfloat16*)beta, (__nv_bfloat16*)Tout, seqs, Tdim, ntiles, err, limit_ns, rule, g, t_span,
+            b_span, g_span);
     } else {
         static std::atomic<uint64_t> smem_set{0};
         e = set_smem_limit_once(ut_kernel<false>, (int)SMEM_BYTES, smem_set);
         if (e != cudaSuccess) return e;
         ut_kernel<false><<<(unsigned)grid, kThreads, SMEM_BYTES, stream>>>(
-            mk, (const __nv_bfloat16*)beta, (__nv_bfloat16*)Tout, seqs, Tdim, ntiles, err, limit_ns, rule, nullptr);
+            mk, (const __nv_bfloat16*)beta, (__nv_bfloat16*)Tout, seqs, Tdim, ntiles, err, limit_ns, rule, nullptr,
+            t_span, b_span, g_span);
     }
     return cudaGetLastError();
 }

@@ -45,7 +45,8 @@ typedef enum {
     EFLA_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, non-positive size, bad workspace */
     EFLA_ERR_UNSUPPORTED = 2,  /* valid but unsupported shape (d_k, d_v, chunk) or dtype */
     EFLA_ERR_CUDA = 3,         /* a CUDA call or kernel launch failed */
-    EFLA_ERR_TIMEOUT = 4       /* a device-side bounded wait ran out (see efla_workspace_status) */
+    EFLA_ERR_TIMEOUT = 4,      /* a device-side bounded wait ran out (see efla_workspace_status) */
+    EFLA_ERR_BOUNDS = 5        /* a checked build (libefla_checked.so) recorded an out-of-range access */
 } efla_status;
 
 typedef enum {
@@ -268,7 +269,11 @@ int efla_noalloc_status(int clear, efla_stream_t stream);
 /*
  * efla_workspace_status -- waits for `stream`, then returns EFLA_ERR_TIMEOUT if any
  * efla_chunk_fwd that used `workspace` gave up on a device wait since the word was last
- * cleared (its outputs are then invalid), else EFLA_OK.  clear != 0 resets the word.
+ * cleared (its outputs are then invalid), EFLA_ERR_BOUNDS if a checked build of the
+ * library (libefla_checked.so: the same entry points, built with EFLA_CHECKED=1, whose
+ * tensor-core forward kernels test every direct global access and computed shared-memory
+ * store against its buffer and skip it when out of range) recorded an out-of-range
+ * access, else EFLA_OK.  clear != 0 resets the word.
  * This is the one call that synchronises the host.
  */
 int efla_workspace_status(void *workspace, int clear, efla_stream_t stream);

@@ -22,13 +22,13 @@ def oracle_lib():
     return oracle.load()
 
 
-def _build_library():
+def _build_library(checked: bool = False):
     import importlib.util
     spec = importlib.util.spec_from_file_location(
         "efla_build", os.path.join(ROOT, "delta_rule_linear_02_b200", "build.py"))
     mod = importlib.util.module_from_spec(spec)
     spec.loader.exec_module(mod)
-    return mod.build()
+    return mod.build(checked=checked)
 
 
 @pytest.fixture(scope="session")
@@ -46,3 +46,16 @@ def cuda(efla):
         pytest.fail("GPU test selected but no CUDA device is visible")
     torch.backends.cuda.matmul.allow_tf32 = False
     return torch.device("cuda", 0)
+
+
+@pytest.fixture
+def efla_checked(efla, cuda):
+    """The binding with its `lib` swapped for the checked build (libefla_checked.so) for the
+    duration of one test."""
+    _build_library(checked=True)
+    saved = efla.lib
+    efla.lib = efla.load_checked()
+    try:
+        yield efla
+    finally:
+        efla.lib = saved

@@ -32,9 +32,21 @@ def test_library_exports_every_declared_symbol(efla):
         assert hasattr(lib, name), f"libefla.so does not export {name}"
 
 
+def test_checked_library_exports_every_declared_symbol(efla):
+    """The EFLA_CHECKED=1 build of the same sources (bounds recorded, accesses skipped)."""
+    from conftest import _build_library
+    path = _build_library(checked=True)
+    assert path == efla.LIB_CHECKED_PATH
+    lib = efla.load_checked()
+    for name in declared_functions():
+        assert hasattr(lib, name), f"libefla_checked.so does not export {name}"
+    assert lib.efla_status_string(efla.EFLA_ERR_BOUNDS) == b"EFLA_ERR_BOUNDS"
+
+
 def test_status_strings(efla):
     assert efla.efla_status_string(0) == "EFLA_OK"
     assert efla.efla_status_string(4) == "EFLA_ERR_TIMEOUT"
+    assert efla.efla_status_string(5) == "EFLA_ERR_BOUNDS"
     assert efla.efla_status_string(99) == "EFLA_ERR_UNKNOWN"
 
 
