@@ -19,14 +19,17 @@
 //      independently), and stores each chunk's dS' (bf16);
 //   3. bwd_tile_kernel: one CTA per (stream, chunk), all chunks at once: every gradient of
 //      the chunk from its S and dS'.
-// Products are warp-level bf16 tensor-core tiles (mma.sync m16n8k16, fp32 accumulation;
-// operands read with ldmatrix from padded shared memory); the triangular solve that gives X
-// again is fp32 on CUDA cores.  Operands pass through bf16 as in the forward, so the
-// gradients carry bf16-operand rounding (relative Frobenius error ~1e-2), not fp32's.
+// The reverse chain's products are warp-level bf16 tiles (mma.sync m16n8k16, fp32
+// accumulation, operands read with ldmatrix from padded shared memory); the per-chunk
+// kernel's are tcgen05 MMAs (see below); the triangular solve that gives X again is fp32 on
+// CUDA cores.  Operands pass through bf16 as in the forward, so the gradients carry
+// bf16-operand rounding (relative Frobenius error ~1e-2), not fp32's.
 #include "efla_common.cuh"
 #include "efla_kernels.h"
 #include "efla_mma_sync.cuh"
+#include "efla_tma.cuh"
 #include "efla_ut_solve.cuh"
+#include "sm100.cuh"
 
 namespace efla {
 
@@ -35,7 +38,6 @@ using namespace mmas;
 constexpr int kD = 128, kC = 64;
 constexpr int LW = kD + 8;     // bf16 row stride of 128-wide tiles (272 B: conflict-free ldmatrix rows)
 constexpr int LH = 64 + 8;     // bf16 row stride of 64-wide tiles (144 B)
-constexpr int LF = 65;         // fp32 row stride of the solve's 64 x 64 tiles
 
 // ============================================================================ reverse chain
 // One CTA (8 warps) per (stream, d_v half).  Per chunk, walking backwards:
@@ -140,224 +142,486 @@ bwd_chain_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const b
 }
 
 // ============================================================================ per-chunk gradients
-// One CTA (8 warps) per (stream, chunk).  64 x 128 products: warp w -> rows 16 (w % 4), columns
-// 64 (w / 4); 64 x 64 products: columns 32 (w / 4).  Shared memory: the S tile's bytes host
-// the solve's fp32 A and scratch before S is loaded, and dT and dX X^T after its last use.
-struct TileSmem {
-    // bf16 tiles (element offsets)
-    static constexpr int K = 0, Q = K + kC * LW, VR = Q + kC * LW, DO = VR + kC * LW, DEL = DO + kC * LW;
-    static constexpr int S = DEL + kC * LW;              // 128 x LW: S (fp32 A and scratch around it)
-    static constexpr int DSP = S + kD * LW;              // 128 x LW: dS', later dDelta (rows 0-63), -dR (64-127)
-    static constexpr int TB = DSP + kD * LW;             // 64 x LH: T
-    static constexpr int PB = TB + kC * LH;              // 64 x LH: P, later dP
-    static constexpr int GB = PB + kC * LH;              // 64 x LH: G, later dG + dG^T
-    static constexpr int BF16_END = GB + kC * LH;
-    // fp32 (float offsets from the end of the bf16 part)
-    static constexpr int FX = 0;
-    static constexpr int ALPHA = FX + kC * LF, BETA = ALPHA + kC, DALPHA = BETA + kC, LAM = DALPHA + kC, ONES = LAM + kC;
-    static constexpr int F32_END = ONES + kC;
-    static constexpr size_t BYTES = sizeof(bf16) * BF16_END + sizeof(float) * F32_END;
-    static_assert(2 * kC * LF * sizeof(float) <= kD * LW * sizeof(bf16), "fp32 A and scratch fit in the S tile");
-    static_assert(BYTES <= 232448, "shared memory");
-};
+// One CTA (8 warps) per (stream, chunk), every product on the 5th-generation tensor cores
+// (tcgen05, bf16 operands in shared memory, fp32 accumulators in tensor memory).
+//
+// Products whose rows index d are computed transposed (M = 128 = d, N = 64 tokens): the
+// accumulator then fills all 128 TMEM lanes, an N = 64 MMA costs less than an N = 128 one,
+// and each epilogue thread owns one d-row of 64 tokens, which it writes as one 128-byte
+// swizzled row (bf16) or, for the fp32 gradients, as one column of dq / dk / dv (a warp's
+// 32 lanes are 32 consecutive d: 128 contiguous bytes per token).  Token x token products
+// (G, P, dP, dT) are M = 64 or ride in the rows 64-127 of a stacked M = 128 product.
+// Operand shapes (row convention, t and s tokens, i = d_k, j = d_v):
+//   [G; P~] = [K; Q] K^T          R^T = V^T - S^T K^T          dQ^T = S dO^T + K^T dP^T
+//   Delta^T = R^T T^T             dDelta^T = dO^T P + dS'^T K^T
+//   dK^T = dS' Delta^T + S (-dR^T) + Q^T dP + K^T (dG + dG^T)
+//   dR^T = dDelta^T T (= dV^T)    dP = tril_incl(dO Delta^T)   dT = dDelta R^T
+// Shared-memory tiles are 128-byte swizzled rows of 64 elements: token-major tiles (K, Q, V,
+// dO: 64 rows per 64-column atom) serve as K-major operands over d or MN-major ones over
+// tokens, d-major tiles (S, dS', R^T, Delta^T, dDelta^T, -dR^T: 128 rows) the other way
+// round, so no operand is ever transposed in memory.  The triangular solve for
+// X = (I + A)^{-1} and the two 64^3 products of dA = strict_tril(-X^T dX X^T) stay fp32 on
+// CUDA cores (their accuracy sets dbeta's).  Phases are sequential: one warp issues a
+// phase's MMAs and commits them to one mbarrier; all warps wait (bounded), run the
+// epilogue, and meet at a block barrier.
+namespace tb {
+constexpr uint32_t TILE = 8192;
+constexpr uint32_t KQ = 0;                 // [K a0 | Q a0 | K a1 | Q a1]: rows 0-63 K, 64-127 Q of [K; Q]
+constexpr uint32_t V = 32768;              // [V a0 | V a1]; later dT^T, dX^T, dA (fp32)
+constexpr uint32_t DO = 49152;             // [dO a0 | dO a1]
+constexpr uint32_t DSP = 65536;            // dS' [a0 | a1] (128 rows each); later dDelta^T and -dR^T
+constexpr uint32_t SS = 98304;             // S [a0 | a1]
+constexpr uint32_t TT = 131072;            // T (bf16 [t][s]); later X^T (fp32)
+constexpr uint32_t PP = 139264;            // P, later dP (bf16 [t][s])
+constexpr uint32_t RT = 147456;            // the solve's A (fp32); then R^T (128 rows)
+constexpr uint32_t DL = 163840;            // the solve's scratch; then Delta^T (128 rows)
+constexpr uint32_t DG = 180224;            // G (bf16 [t][s]), later dG + dG^T
+constexpr int LA = 64;                     // row stride (floats) of the solve's A and scratch
+constexpr int LX = 68;                     // row stride of the other fp32 64 x 64 tiles (16-byte rows)
+constexpr uint32_t F32 = 64 * LX * 4;      // bytes of one of them
+constexpr uint32_t FX = 188416;            // X (fp32)
+constexpr uint32_t FXT = TT;               // X^T
+constexpr uint32_t FW = TT + F32;          // W = dX X^T
+constexpr uint32_t FDT = V;                // dT^T, then dX^T, then dA
+constexpr uint32_t SMALL = FX + F32;       // alpha, beta, dalpha, lambda, ones (fp32 [64] each)
+constexpr uint32_t BAR = SMALL + 5 * 256;  // mbarriers: loads, MMA commits
+constexpr uint32_t MISC = BAR + 2 * 8;     // TMEM base, abort flag
+constexpr uint32_t SMEM_BYTES = MISC + 16 + 1024;
+static_assert(64 * LA * 4 <= 16384, "the solve's A and scratch fit R^T's and Delta^T's regions");
+static_assert(FDT + F32 <= DSP && FW + F32 <= DG, "fp32 tiles stay inside dead regions");
+static_assert(SMEM_BYTES <= 232448, "shared memory");
+// TMEM columns (fp32 accumulators, 64 columns each)
+constexpr uint32_t C_GP = 0, C_SK = 64, C_DQ = 128, C_DL = 192, C_DD = 256, C_DK = 320, C_DR = 384, C_COLS = 512;
+constexpr uint32_t LOAD_BYTES = 131072;    // K, Q, V, dO, dS', S
 
-__global__ void __launch_bounds__(256, 1)
-bwd_tile_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16* __restrict__ v,
-                const bf16* __restrict__ beta, const bf16* __restrict__ dO, const bf16* __restrict__ states,
-                const bf16* __restrict__ dSp, float* __restrict__ dq, float* __restrict__ dk, float* __restrict__ dv,
-                float* __restrict__ dbeta, int T, int rule) {
-    extern __shared__ __align__(16) uint8_t smem_raw[];
-    using L = TileSmem;
-    bf16* sh = reinterpret_cast<bf16*>(smem_raw);
-    float* sf = reinterpret_cast<float*>(smem_raw + sizeof(bf16) * L::BF16_END);
-    float* fA = reinterpret_cast<float*>(sh + L::S);      // aliases the S tile (see above)
-    float* fY = fA + kC * LF;
-    float* fX = sf + L::FX;
-    float *al = sf + L::ALPHA, *bt = sf + L::BETA, *dal = sf + L::DALPHA, *lam = sf + L::LAM, *ones = sf + L::ONES;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int nchunks = (T + kC - 1) / kC;
-    const long tile = blockIdx.x;
-    const long bh = tile / nchunks;
-    const int c = (int)(tile % nchunks);
-    const int nv = min(kC, T - c * kC);
-    const size_t row0 = (size_t)bh * T + (size_t)c * kC;
-    const int wm = 16 * (warp & 3);                  // this warp's row block
-    const int wn = 64 * (warp >> 2), wn64 = 32 * (warp >> 2);
+// nk k-steps of K = 16 with A and B in shared memory; operand k-step ks starts at
+// base + (ks / 4) * atom + (ks % 4) * step (K-major: step 32 bytes inside a 64-column atom;
+// MN-major: step 16 rows = 2048 bytes, atom 64 rows = 8192 bytes; lbo = distance between
+// 64-element MN blocks of an MN-major operand).
+__device__ __forceinline__ void mma_ss(uint32_t d, uint32_t a, uint32_t a_atom, uint32_t a_step, uint32_t a_lbo,
+                                       uint32_t b, uint32_t b_atom, uint32_t b_step, uint32_t b_lbo, uint32_t idesc,
+                                       int nk, bool acc) {
+    const uint64_t da = sm100::sdesc_sw128(a, a_lbo, 1024), db = sm100::sdesc_sw128(b, b_lbo, 1024);
+#pragma unroll
+    for (int ks = 0; ks < nk; ++ks)
+        sm100::mma_bf16_elect(d, da + (((ks >> 2) * a_atom + (ks & 3) * a_step) >> 4),
+                              db + (((ks >> 2) * b_atom + (ks & 3) * b_step) >> 4), idesc, acc || ks > 0);
+}
+constexpr uint32_t K_MAJ = 0, MN_MAJ = 1;
+__host__ __device__ constexpr uint32_t idesc(int M, uint32_t a, uint32_t b) {
+    return sm100::idesc_bf16(M, 64, a == MN_MAJ, b == MN_MAJ);
+}
 
-    load_tile(sh + L::K, LW, k + row0 * kD, kD, kC, kD, nv, tid, 256);
-    cp_async_commit();
-    load_tile(sh + L::Q, LW, q + row0 * kD, kD, kC, kD, nv, tid, 256);
-    load_tile(sh + L::VR, LW, v + row0 * kD, kD, kC, kD, nv, tid, 256);
-    load_tile(sh + L::DO, LW, dO + row0 * kD, kD, kC, kD, nv, tid, 256);
-    load_tile(sh + L::DSP, LW, dSp + (size_t)tile * kD * kD, kD, kD, kD, kD, tid, 256);
-    cp_async_commit();
-    if (tid < kC) {
-        bt[tid] = tid < nv ? __bfloat162float(beta[row0 + tid]) : 0.f;
-        ones[tid] = 1.f;
-        dal[tid] = 0.f;
-    }
-    cp_async_wait<1>();
-    __syncthreads();                                 // K landed
-    {   // G = K K^T (fp32 into fY), lambda from its diagonal
-        float acc[4][4];
-        zero_acc(acc);
-        warp_mma<4, false, false>(acc, sh + L::K, LW, sh + L::K, LW, wm, wn64, kD, lane);
-        for_acc(acc, wm, wn64, lane, [&](int r, int c2, float& x) {
-            fY[r * LF + c2] = x;
-            sh[L::GB + r * LH + c2] = __float2bfloat16_rn(x);
-        });
-    }
-    __syncthreads();
-    if (tid < kC) {
-        lam[tid] = fY[tid * LF + tid];
-        al[tid] = rule_alpha(rule, bt[tid], lam[tid]);
-    }
-    __syncthreads();
-    for (int e = tid; e < kC * kC; e += 256) {       // A = strict_tril(diag(alpha) G)
-        const int r = e >> 6, s2 = e & 63;
-        fA[r * LF + s2] = s2 < r ? al[r] * fY[r * LF + s2] : 0.f;
-    }
-    __syncthreads();
-    ut_inverse64<256>(fA, ones, fX, fY, LF, tid);    // X = (I + A)^{-1} (ends with a barrier)
-    // the S tile is free of the solve: load the chunk's entering state
-    load_tile(sh + L::S, LW, states + (size_t)tile * kD * kD, kD, kD, kD, kD, tid, 256);
-    cp_async_commit();
-    for (int e = tid; e < kC * kC; e += 256) {       // T = X diag(alpha), bf16
-        const int r = e >> 6, s2 = e & 63;
-        sh[L::TB + r * LH + s2] = __float2bfloat16_rn(fX[r * LF + s2] * al[s2]);
-    }
-    cp_async_wait<0>();
-    __syncthreads();                                 // everything landed, T written
-    float dqa[8][4], dka[8][4];
-    zero_acc(dqa);
-    zero_acc(dka);
-    {   // R = V - K S (bf16 over V);  dQ = dO S^T (+ dP K below)
-        float acc[8][4];
-        zero_acc(acc);
-        warp_mma<8, false, true>(acc, sh + L::K, LW, sh + L::S, LW, wm, wn, kD, lane);
-        warp_mma<8, false, false>(dqa, sh + L::DO, LW, sh + L::S, LW, wm, wn, kD, lane);
-        for_acc(acc, wm, wn, lane, [&](int r, int c2, float& x) {
-            bf16* p = sh + L::VR + r * LW + c2;
-            *p = __float2bfloat16_rn(__bfloat162float(*p) - x);
-        });
-    }
-    {   // P = tril_incl(Q K^T)
-        float acc[4][4];
-        zero_acc(acc);
-        warp_mma<4, false, false>(acc, sh + L::Q, LW, sh + L::K, LW, wm, wn64, kD, lane);
-        for_acc(acc, wm, wn64, lane, [&](int r, int c2, float& x) {
-            sh[L::PB + r * LH + c2] = __float2bfloat16_rn(c2 <= r ? x : 0.f);
-        });
-    }
-    __syncthreads();
-    {   // Delta = T R
-        float acc[8][4];
-        zero_acc(acc);
-        warp_mma<8, false, true>(acc, sh + L::TB, LH, sh + L::VR, LW, wm, wn, kC, lane);
-        for_acc(acc, wm, wn, lane, [&](int r, int c2, float& x) { sh[L::DEL + r * LW + c2] = __float2bfloat16_rn(x); });
-    }
-    __syncthreads();
-    {   // dDelta = P^T dO + K dS';  dK = Delta dS'^T (+ more below).  dS' is then dead.
-        float acc[8][4];
-        zero_acc(acc);
-        warp_mma<8, true, true>(acc, sh + L::PB, LH, sh + L::DO, LW, wm, wn, kC, lane);
-        warp_mma<8, false, true>(acc, sh + L::K, LW, sh + L::DSP, LW, wm, wn, kD, lane);
-        warp_mma<8, false, false>(dka, sh + L::DEL, LW, sh + L::DSP, LW, wm, wn, kD, lane);
-        __syncthreads();
-        for_acc(acc, wm, wn, lane, [&](int r, int c2, float& x) { sh[L::DSP + r * LW + c2] = __float2bfloat16_rn(x); });
-    }
-    __syncthreads();
-    const bf16* dD = sh + L::DSP;                    // dDelta, rows 0-63 of the old dS' tile
-    bf16* nR = sh + L::DSP + kC * LW;                // -dR, rows 64-127 of the old dS' tile
-    {   // dR = T^T dDelta = dV, and -dR (bf16) for dK -= dR S^T
-        float acc[8][4];
-        zero_acc(acc);
-        warp_mma<8, true, true>(acc, sh + L::TB, LH, dD, LW, wm, wn, kC, lane);
-        for_acc(acc, wm, wn, lane, [&](int r, int c2, float& x) {
-            if (r < nv) dv[(row0 + r) * kD + c2] = x;
-            nR[r * LW + c2] = __float2bfloat16_rn(-x);
-        });
-    }
-    {   // dP = tril_incl(dO Delta^T) over P (dead since dDelta)
-        float acc[4][4];
-        zero_acc(acc);
-        warp_mma<4, false, false>(acc, sh + L::DO, LW, sh + L::DEL, LW, wm, wn64, kD, lane);
-        for_acc(acc, wm, wn64, lane, [&](int r, int c2, float& x) {
-            sh[L::PB + r * LH + c2] = __float2bfloat16_rn(c2 <= r ? x : 0.f);
-        });
-    }
-    __syncthreads();
-    // dK -= dR S^T (S's last use);  dQ += dP K
-    warp_mma<8, false, false>(dka, nR, LW, sh + L::S, LW, wm, wn, kD, lane);
-    warp_mma<8, false, true>(dqa, sh + L::PB, LH, sh + L::K, LW, wm, wn, kC, lane);
-    for_acc(dqa, wm, wn, lane, [&](int r, int c2, float& x) {
-        if (r < nv) dq[(row0 + r) * kD + c2] = x;
-    });
-    float dta[4][4];                                 // dT = dDelta R^T
-    zero_acc(dta);
-    warp_mma<4, false, false>(dta, dD, LW, sh + L::VR, LW, wm, wn64, kD, lane);
-    __syncthreads();                                 // S is dead: fp32 dT over it
-    for_acc(dta, wm, wn64, lane, [&](int r, int c2, float& x) { fA[r * LF + c2] = x; });
-    __syncthreads();
-    // ---- through T = X diag(alpha) and X = (I + A)^{-1}, fp32 on CUDA cores
-    if (tid < kC) {                                  // dalpha_j = sum_i dT_ij X_ij
-        float sacc = 0.f;
-        for (int i = 0; i < kC; ++i) sacc = fmaf(fA[i * LF + tid], fX[i * LF + tid], sacc);
-        dal[tid] = sacc;
-    }
-    __syncthreads();
-    for (int e = tid; e < kC * kC; e += 256) {       // dX = dT diag(alpha), in place
-        const int r = e >> 6, s2 = e & 63;
-        fA[r * LF + s2] *= al[s2];
-    }
-    __syncthreads();
-    // 64 x 64 x 64 fp32 products on CUDA cores, 4 x 4 outputs per thread (rows 4 (tid / 16),
-    // columns 4 (tid % 16)): per k, 4 + 4 shared loads for 16 FMAs
-    const int r4 = 4 * (tid >> 4), c4 = 4 * (tid & 15);
-    {   // W = dX X^T into fY:  W[r][c] = sum_m dX[r][m] X[c][m]
-        float w[4][4] = {};
-        for (int m = 0; m < kC; ++m) {
-            float a[4], b[4];
+__device__ __forceinline__ uint32_t pack2(float a, float b) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+// 32 floats -> row `r`, 16-byte chunks c0 .. c0 + 3 of a 128-byte-swizzled tile at `tile`
+__device__ __forceinline__ void st_row32(uint8_t* tile, uint32_t r, uint32_t c0, const float* v) {
 #pragma unroll
-            for (int i = 0; i < 4; ++i) a[i] = fA[(r4 + i) * LF + m];
+    for (int m = 0; m < 4; ++m) {
+        uint4 u;
+        u.x = pack2(v[8 * m], v[8 * m + 1]);
+        u.y = pack2(v[8 * m + 2], v[8 * m + 3]);
+        u.z = pack2(v[8 * m + 4], v[8 * m + 5]);
+        u.w = pack2(v[8 * m + 6], v[8 * m + 7]);
+        *reinterpret_cast<uint4*>(tile + sm100::sw128_off(r, c0 + m)) = u;
+    }
+}
+// 16 floats -> row `r`, chunks c0, c0 + 1
+__device__ __forceinline__ void st_row16(uint8_t* tile, uint32_t r, uint32_t c0, const float* v) {
 #pragma unroll
-            for (int j = 0; j < 4; ++j) b[j] = fX[(c4 + j) * LF + m];
+    for (int m = 0; m < 2; ++m) {
+        uint4 u;
+        u.x = pack2(v[8 * m], v[8 * m + 1]);
+        u.y = pack2(v[8 * m + 2], v[8 * m + 3]);
+        u.z = pack2(v[8 * m + 4], v[8 * m + 5]);
+        u.w = pack2(v[8 * m + 6], v[8 * m + 7]);
+        *reinterpret_cast<uint4*>(tile + sm100::sw128_off(r, c0 + m)) = u;
+    }
+}
+// element (r, c) of a token-major tile of 64-column atoms `atom` bytes apart
+__device__ __forceinline__ float ld_tok(const uint8_t* tile, uint32_t atom, int r, int c) {
+    const uint8_t* p = tile + (c >> 6) * atom + sm100::sw128_off(r, (c & 63) >> 3) + (c & 7) * 2;
+    return __bfloat162float(*reinterpret_cast<const bf16*>(p));
+}
+
+// X = (I + A)^{-1} for the 64 x 64 strictly-lower A (row stride LA; only its strictly-lower
+// part is read), written in full into X (row stride LX; zeros above the diagonal), Y scratch
+// (row stride LA).  Block doubling: the four 16 x 16 diagonal blocks by forward
+// substitution (one thread per column), then merges X21 = -X22 (A21 X11) at 32 and 64.  In
+// the 64 merge each thread keeps four rows of one column in registers (one operand load
+// per four FMAs).  256 threads; ends with a barrier.
+__device__ __forceinline__ void unit_lower_inverse64(const float* __restrict__ A, float* __restrict__ X,
+                                                     float* __restrict__ Y, int tid) {
+    if (tid < 64) {
+        const int b = tid >> 4, c = tid & 15;
+        const float* Ab = A + (16 * b) * LA + 16 * b;
+        float x[16];
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
+        for (int i = 0; i < 16; ++i) x[i] = (i == c) ? 1.f : 0.f;
 #pragma unroll
-                for (int j = 0; j < 4; ++j) w[i][j] = fmaf(a[i], b[j], w[i][j]);
+        for (int i = 1; i < 16; ++i) {
+            float s = 0.f;
+#pragma unroll
+            for (int j = 0; j < i; ++j) s = fmaf(Ab[i * LA + j], x[j], s);
+            if (i > c) x[i] = -s;
         }
+        float* Xb = X + (16 * b) * LX + 16 * b + c;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) Xb[i * LX] = x[i];
+    } else {
+        for (int e = tid - 64; e < 64 * 64; e += 192) {   // the strictly-upper 16 x 16 blocks
+            const int i = e >> 6, c = e & 63;
+            if ((c >> 4) > (i >> 4)) X[i * LX + c] = 0.f;
+        }
+    }
+    __syncthreads();
+    {   // 32 x 32 blocks s = 0, 1:  Y21 = A21 X11, then X21 = -X22 Y21 (16 x 16 blocks)
+        const int s = tid >> 7, i = (tid >> 4) & 7, c = tid & 15;     // rows i and i + 8
+        const int r0 = 32 * s + 16, c0 = 32 * s;
+        float y0 = 0.f, y1 = 0.f;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            const float xv = X[(c0 + j) * LX + c0 + c];
+            y0 = fmaf(A[(r0 + i) * LA + c0 + j], xv, y0);
+            y1 = fmaf(A[(r0 + i + 8) * LA + c0 + j], xv, y1);
+        }
+        Y[(r0 + i) * LA + c0 + c] = y0;
+        Y[(r0 + i + 8) * LA + c0 + c] = y1;
+    }
+    __syncthreads();
+    {
+        const int s = tid >> 7, i = (tid >> 4) & 7, c = tid & 15;
+        const int r0 = 32 * s + 16, c0 = 32 * s;
+        float x0 = 0.f, x1 = 0.f;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            const float yv = Y[(r0 + j) * LA + c0 + c];
+            x0 = fmaf(X[(r0 + i) * LX + r0 + j], yv, x0);
+            x1 = fmaf(X[(r0 + i + 8) * LX + r0 + j], yv, x1);
+        }
+        X[(r0 + i) * LX + c0 + c] = -x0;
+        X[(r0 + i + 8) * LX + c0 + c] = -x1;
+    }
+    __syncthreads();
+    const int c = tid & 31, i0 = tid >> 5;            // column c, rows i0 + 8 k of the 32 x 32 blocks
+    {   // Y21 = A21 X11
+        float y[4] = {};
+#pragma unroll 8
+        for (int j = 0; j < 32; ++j) {
+            const float xv = X[j * LX + c];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) y[k] = fmaf(A[(32 + i0 + 8 * k) * LA + j], xv, y[k]);
+        }
+#pragma unroll
+        for (int k = 0; k < 4; ++k) Y[(32 + i0 + 8 * k) * LA + c] = y[k];
+    }
+    __syncthreads();
+    {   // X21 = -X22 Y21
+        float x[4] = {};
+#pragma unroll 8
+        for (int j = 0; j < 32; ++j) {
+            const float yv = Y[(32 + j) * LA + c];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) x[k] = fmaf(X[(32 + i0 + 8 * k) * LX + 32 + j], yv, x[k]);
+        }
+#pragma unroll
+        for (int k = 0; k < 4; ++k) X[(32 + i0 + 8 * k) * LX + c] = -x[k];
+    }
+    __syncthreads();
+}
+
+// C (64 x 64, row stride LX) = sum_m P[m][r] Q[m][c] for the fp32 tiles P, Q (row stride LX):
+// thread -> 4 x 4 outputs (rows 4 (tid / 16), columns 4 (tid % 16)), two 16-byte loads per m.
+__device__ __forceinline__ void gemm_tn64(const float* __restrict__ P, const float* __restrict__ Q, float (&w)[4][4],
+                                          int r4, int c4) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) w[i][j] = 0.f;
+#pragma unroll 4
+    for (int m = 0; m < 64; ++m) {
+        const float4 a = *reinterpret_cast<const float4*>(P + m * LX + r4);
+        const float4 b = *reinterpret_cast<const float4*>(Q + m * LX + c4);
+        const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
         for (int i = 0; i < 4; ++i)
 #pragma unroll
-            for (int j = 0; j < 4; ++j) fY[(r4 + i) * LF + c4 + j] = w[i][j];
+            for (int j = 0; j < 4; ++j) w[i][j] = fmaf(av[i], bv[j], w[i][j]);
+    }
+}
+}  // namespace tb
+
+__global__ void __launch_bounds__(256, 1)
+bwd_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                const __grid_constant__ CUtensorMap tm_s, const __grid_constant__ CUtensorMap tm_dsp,
+                const bf16* __restrict__ beta, float* __restrict__ dq, float* __restrict__ dk, float* __restrict__ dv,
+                float* __restrict__ dbeta, int T, int rule, uint32_t* __restrict__ err, unsigned long long limit_ns) {
+    using namespace tb;
+    using namespace sm100;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sb = smem_u32(sm);
+    uint64_t* bar = reinterpret_cast<uint64_t*>(sm + BAR);    // 0: the tile's loads, 1: MMA commits
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + MISC);
+    volatile int* abort = reinterpret_cast<volatile int*>(sm + MISC + 4);
+    float* fA = reinterpret_cast<float*>(sm + RT);
+    float* fY = reinterpret_cast<float*>(sm + DL);
+    float* fX = reinterpret_cast<float*>(sm + FX);
+    float* fXT = reinterpret_cast<float*>(sm + FXT);
+    float* fW = reinterpret_cast<float*>(sm + FW);
+    float* fdT = reinterpret_cast<float*>(sm + FDT);
+    float* al = reinterpret_cast<float*>(sm + SMALL);
+    float *bt = al + 64, *dal = al + 128, *lam = al + 192, *ones = al + 256;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int q = warp & 3, h = warp >> 2;                    // TMEM lane quarter, column half
+    const uint32_t lane_off = static_cast<uint32_t>(32 * q) << 16;
+    const int row = 32 * q + lane;                            // accumulator row (M = 128)
+    const int nchunks = (T + 63) / 64;
+    const long tile = blockIdx.x;
+    const long bh = tile / nchunks;
+    const int c = (int)(tile % nchunks), t0 = c * 64;
+    const int nv = min(64, T - t0);
+    const size_t row0 = (size_t)bh * T + t0;
+
+    if (tid == 0) {
+        mbar_init(bar, 1);
+        mbar_init(bar + 1, 1);
+        *abort = 0;
+        fence_mbar_init();
+        mbar_arrive_expect_tx(bar, LOAD_BYTES);
+        tma_load_3d(sm + KQ, &tm_k, bar, 0, t0, (int)bh);
+        tma_load_3d(sm + KQ + 2 * TILE, &tm_k, bar, 64, t0, (int)bh);
+        tma_load_3d(sm + KQ + TILE, &tm_q, bar, 0, t0, (int)bh);
+        tma_load_3d(sm + KQ + 3 * TILE, &tm_q, bar, 64, t0, (int)bh);
+        tma_load_3d(sm + V, &tm_v, bar, 0, t0, (int)bh);
+        tma_load_3d(sm + V + TILE, &tm_v, bar, 64, t0, (int)bh);
+        tma_load_3d(sm + DO, &tm_do, bar, 0, t0, (int)bh);
+        tma_load_3d(sm + DO + TILE, &tm_do, bar, 64, t0, (int)bh);
+        tma_load_2d(sm + DSP, &tm_dsp, bar, 0, (int)(tile * 128));
+        tma_load_2d(sm + DSP + 2 * TILE, &tm_dsp, bar, 64, (int)(tile * 128));
+        tma_load_2d(sm + SS, &tm_s, bar, 0, (int)(tile * 128));
+        tma_load_2d(sm + SS + 2 * TILE, &tm_s, bar, 64, (int)(tile * 128));
+    }
+    const float beta_t = tid < nv ? __bfloat162float(beta[row0 + tid]) : 0.f;   // in flight during the setup
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, C_COLS);
+        tmem_relinquish();
+    }
+    if (tid < 64) {
+        bt[tid] = beta_t;
+        ones[tid] = 1.f;
+        dal[tid] = 0.f;
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tm = *tmem_slot;
+    // bounded waits; once one has run out every later wait is skipped (the outputs are then
+    // invalid and the error word says so), so the block still reaches every barrier
+    auto wait = [&](int i, uint32_t parity) {
+        if (*abort) return;
+        if (!mbar_wait(bar + i, parity, limit_ns)) *abort = 1;
+        tc_fence_after();
+    };
+    uint32_t mma_phase = 0;
+    auto wait_mma = [&]() { wait(1, mma_phase & 1); ++mma_phase; };
+    auto commit = [&]() { mma_commit_elect(bar + 1); };
+    // the next phase's operands written by this block's threads -> visible to the tensor core
+    auto handoff = [&]() {
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+    };
+
+    // ---- 1. [G; P~] = [K; Q] K^T;  dDelta^T = dS'^T K^T (+ dO^T P below);  S^T K^T;  dQ^T = S dO^T
+    wait(0, 0);
+    if (warp == 0) {
+        mma_ss(tm + C_GP, sb + KQ, 2 * TILE, 32, 16, sb + KQ, 2 * TILE, 32, 16, idesc(128, K_MAJ, K_MAJ), 8, false);
+        mma_ss(tm + C_DD, sb + DSP, TILE, 2048, 2 * TILE, sb + KQ, 2 * TILE, 32, 16, idesc(128, MN_MAJ, K_MAJ), 8,
+               false);
+        mma_ss(tm + C_SK, sb + SS, TILE, 2048, 2 * TILE, sb + KQ, 2 * TILE, 32, 16, idesc(128, MN_MAJ, K_MAJ), 8,
+               false);
+        mma_ss(tm + C_DQ, sb + SS, 2 * TILE, 32, 16, sb + DO, TILE, 32, 16, idesc(128, K_MAJ, K_MAJ), 8, false);
+        commit();
+    }
+    wait_mma();
+    float g[32];
+    tmem_ld32_wait(tm + lane_off + C_GP + 32 * h, g);
+    if (q < 2) {          // G row `row`: bf16 copy, lambda and alpha from its diagonal
+        st_row32(sm + DG, row, 4 * h, g);
+        if (q == h) {
+            float dg = 0.f;
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+                if (j == lane) dg = g[j];
+            lam[row] = dg;
+            al[row] = rule_alpha(rule, bt[row], dg);
+        }
+    } else {              // P = tril_incl(Q K^T), query row t = row - 64
+        const int t = row - 64;
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+            if (32 * h + j > t) g[j] = 0.f;
+        st_row32(sm + PP, t, 4 * h, g);
     }
     __syncthreads();
-    {   // dA = strict_tril(-X^T W) over fA:  dA[r][c] = -sum_m X[m][r] W[m][c];  dalpha_r += sum_{s<r} dA_rs G_rs
-        float w[4][4] = {};
-        for (int m = 0; m < kC; ++m) {
-            float a[4], b[4];
+    if (q < 2) {          // A = strict_tril(diag(alpha) G), fp32, for the solve
+        const float a = al[row];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) a[i] = fX[m * LF + r4 + i];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) b[j] = fY[m * LF + c4 + j];
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-#pragma unroll
-                for (int j = 0; j < 4; ++j) w[i][j] = fmaf(a[i], b[j], w[i][j]);
+        for (int j = 0; j < 32; ++j) {
+            const int s = 32 * h + j;
+            fA[row * LA + s] = s < row ? a * g[j] : 0.f;
         }
-        // (fA, the dX tile, is not read here: it is overwritten at once)
+    }
+    handoff();
+    // ---- 2. dDelta^T += dO^T P, while the CUDA cores solve for X = (I + A)^{-1}
+    if (warp == 0) {
+        mma_ss(tm + C_DD, sb + DO, TILE, 2048, TILE, sb + PP, TILE, 2048, TILE, idesc(128, MN_MAJ, MN_MAJ), 4, true);
+        commit();
+    }
+    unit_lower_inverse64(fA, fX, fY, tid);            // ends with a barrier: A and the scratch are dead
+    {   // T = X diag(alpha), bf16 [t][s]: thread -> row tid / 4, 16 columns;  R^T = V^T - S^T K^T
+        const int t = tid >> 2, s0 = 16 * (tid & 3);
+        float x[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) x[j] = fX[t * LX + s0 + j] * al[s0 + j];
+        st_row16(sm + TT, t, 2 * (tid & 3), x);
+        float r[32];
+        tmem_ld32_wait(tm + lane_off + C_SK + 32 * h, r);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) r[j] = ld_tok(sm + V, TILE, 32 * h + j, row) - r[j];
+        st_row32(sm + RT, row, 4 * h, r);
+    }
+    wait_mma();           // dO^T P has landed (read in step 4)
+    handoff();
+    // ---- 3. Delta^T = R^T T^T
+    if (warp == 0) {
+        mma_ss(tm + C_DL, sb + RT, 0, 32, 16, sb + TT, 0, 32, 16, idesc(128, K_MAJ, K_MAJ), 4, false);
+        commit();
+    }
+    wait_mma();
+    {
+        float x[32];
+        tmem_ld32_wait(tm + lane_off + C_DL + 32 * h, x);
+        st_row32(sm + DL, row, 4 * h, x);
+    }
+    handoff();
+    // ---- 4. dK^T = dS' Delta^T;  dP~ = dO Delta^T (M = 64)
+    if (warp == 0) {
+        mma_ss(tm + C_DK, sb + DSP, 2 * TILE, 32, 16, sb + DL, TILE, 2048, TILE, idesc(128, K_MAJ, MN_MAJ), 8, false);
+        mma_ss(tm + C_GP, sb + DO, TILE, 32, 16, sb + DL, TILE, 2048, TILE, idesc(64, K_MAJ, MN_MAJ), 8, false);
+        commit();
+    }
+    wait_mma();
+    {   // dDelta^T (dS' is dead) -> DSP rows 0-127;  dP = tril_incl(dP~) (rows 16 q + lane, lanes < 16)
+        float x[32];
+        tmem_ld32_wait(tm + lane_off + C_DD + 32 * h, x);
+        st_row32(sm + DSP, row, 4 * h, x);
+        tmem_ld32_wait(tm + lane_off + C_GP + 32 * h, x);
+        if (lane < 16) {
+            const int t = 16 * q + lane;
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+                if (32 * h + j > t) x[j] = 0.f;
+            st_row32(sm + PP, t, 4 * h, x);
+        }
+    }
+    handoff();
+    // ---- 5. dR^T = dDelta^T T;  dT = dDelta R^T (M = 64);  dQ^T += K^T dP^T;  dK^T += Q^T dP
+    if (warp == 0) {
+        mma_ss(tm + C_DR, sb + DSP, 0, 32, 16, sb + TT, 0, 2048, TILE, idesc(128, K_MAJ, MN_MAJ), 4, false);
+        mma_ss(tm + C_SK, sb + DSP, TILE, 2048, TILE, sb + RT, TILE, 2048, TILE, idesc(64, MN_MAJ, MN_MAJ), 8, false);
+        mma_ss(tm + C_DQ, sb + KQ, 0, 2048, 2 * TILE, sb + PP, 0, 32, 16, idesc(128, MN_MAJ, K_MAJ), 4, true);
+        mma_ss(tm + C_DK, sb + KQ + TILE, 0, 2048, 2 * TILE, sb + PP, 0, 2048, TILE, idesc(128, MN_MAJ, MN_MAJ), 4,
+               true);
+        commit();
+    }
+    wait_mma();
+    {
+        float x[32];
+        // dV = dR: dv[token][j] for this thread's j = row (a warp stores 32 consecutive floats)
+        tmem_ld32_wait(tm + lane_off + C_DR + 32 * h, x);
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+            if (32 * h + j < nv) dv[(row0 + 32 * h + j) * 128 + row] = x[j];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) x[j] = -x[j];
+        st_row32(sm + DSP + 2 * TILE, row, 4 * h, x);   // -dR^T, over dS' atom 1
+        // dQ = (S dO^T + K^T dP^T)^T
+        tmem_ld32_wait(tm + lane_off + C_DQ + 32 * h, x);
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+            if (32 * h + j < nv) dq[(row0 + 32 * h + j) * 128 + row] = x[j];
+        // dT, stored transposed (fp32): dT^T[s][t] for this thread's row t = 16 q + lane
+        tmem_ld32_wait(tm + lane_off + C_SK + 32 * h, x);
+        if (lane < 16) {
+            const int t = 16 * q + lane;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) fdT[(32 * h + j) * LX + t] = x[j];
+        }
+    }
+    {   // X^T (fp32): thread -> a 4 x 4 block
+        const int r4 = 4 * (tid >> 4), c4 = 4 * (tid & 15);
+        float4 xr[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) xr[i] = *reinterpret_cast<const float4*>(fX + (r4 + i) * LX + c4);
+        *reinterpret_cast<float4*>(fXT + (c4 + 0) * LX + r4) = make_float4(xr[0].x, xr[1].x, xr[2].x, xr[3].x);
+        *reinterpret_cast<float4*>(fXT + (c4 + 1) * LX + r4) = make_float4(xr[0].y, xr[1].y, xr[2].y, xr[3].y);
+        *reinterpret_cast<float4*>(fXT + (c4 + 2) * LX + r4) = make_float4(xr[0].z, xr[1].z, xr[2].z, xr[3].z);
+        *reinterpret_cast<float4*>(fXT + (c4 + 3) * LX + r4) = make_float4(xr[0].w, xr[1].w, xr[2].w, xr[3].w);
+    }
+    handoff();
+    // ---- 6. dK^T += S (-dR^T), while the CUDA cores go through T = X diag(alpha)
+    if (warp == 0) {
+        mma_ss(tm + C_DK, sb + SS, 2 * TILE, 32, 16, sb + DSP + 2 * TILE, TILE, 2048, TILE,
+               idesc(128, K_MAJ, MN_MAJ), 8, true);
+        commit();
+    }
+    // ---- 7. through T = X diag(alpha) and X = (I + A)^{-1}, fp32 on CUDA cores
+    if (tid < 64) {       // dalpha_s = sum_t dT_ts X_ts;  dX^T = diag(alpha) dT^T, in place
+        const float a = al[tid];
+        float sacc = 0.f;
+#pragma unroll 4
+        for (int t = 0; t < 64; t += 4) {
+            float4 d4 = *reinterpret_cast<const float4*>(fdT + tid * LX + t);
+            const float4 x4 = *reinterpret_cast<const float4*>(fXT + tid * LX + t);
+            sacc = fmaf(d4.x, x4.x, fmaf(d4.y, x4.y, fmaf(d4.z, x4.z, fmaf(d4.w, x4.w, sacc))));
+            d4.x *= a; d4.y *= a; d4.z *= a; d4.w *= a;
+            *reinterpret_cast<float4*>(fdT + tid * LX + t) = d4;
+        }
+        dal[tid] = sacc;
+    }
+    __syncthreads();
+    const int r4 = 4 * (tid >> 4), c4 = 4 * (tid & 15);
+    {   // W = dX X^T:  W[r][c] = sum_m dX^T[m][r] X^T[m][c]
+        float w[4][4];
+        gemm_tn64(fdT, fXT, w, r4, c4);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            *reinterpret_cast<float4*>(fW + (r4 + i) * LX + c4) = make_float4(w[i][0], w[i][1], w[i][2], w[i][3]);
+    }
+    __syncthreads();
+    {   // dA = strict_tril(-X^T W) over dX^T:  dA[r][c] = -sum_m X[m][r] W[m][c];
+        // dalpha_r += sum_{s<r} dA_rs G_rs
+        float w[4][4];
+        gemm_tn64(fX, fW, w, r4, c4);
         float part[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             part[i] = 0.f;
+            float da[4];
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 const int r = r4 + i, s2 = c4 + j;
-                const float da = s2 < r ? -w[i][j] : 0.f;
-                fA[r * LF + s2] = da;
-                part[i] = fmaf(da, __bfloat162float(sh[L::GB + r * LH + s2]), part[i]);
+                da[j] = s2 < r ? -w[i][j] : 0.f;
+                part[i] = fmaf(da[j], ld_tok(sm + DG, 0, r, s2), part[i]);
             }
+            *reinterpret_cast<float4*>(fdT + (r4 + i) * LX + c4) = make_float4(da[0], da[1], da[2], da[3]);
         }
         // the 16 column blocks of a row block sit in 16 consecutive lanes: sum over them
 #pragma unroll
@@ -371,27 +635,71 @@ bwd_tile_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf
         }
     }
     __syncthreads();
-    for (int e = tid; e < kC * kC; e += 256) {       // dG + dG^T with dG = diag(alpha) dA, bf16 over G
-        const int r = e >> 6, s2 = e & 63;
-        const float x = (s2 < r ? al[r] * fA[r * LF + s2] : 0.f) + (r < s2 ? al[s2] * fA[s2 * LF + r] : 0.f);
-        sh[L::GB + r * LH + s2] = __float2bfloat16_rn(x);
+    {   // dG + dG^T with dG = diag(alpha) dA, bf16 over G: thread -> row tid / 4, 16 columns
+        const int r = tid >> 2, s0 = 16 * (tid & 3);
+        float x[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            const int s2 = s0 + j;
+            x[j] = (s2 < r ? al[r] * fdT[r * LX + s2] : 0.f) + (r < s2 ? al[s2] * fdT[s2 * LX + r] : 0.f);
+        }
+        st_row16(sm + DG, r, 2 * (tid & 3), x);
     }
-    __syncthreads();
-    // dK += dP^T Q + (dG + dG^T) K, then the gate's lambda term; dbeta
-    warp_mma<8, true, true>(dka, sh + L::PB, LH, sh + L::Q, LW, wm, wn, kC, lane);
-    warp_mma<8, false, true>(dka, sh + L::GB, LH, sh + L::K, LW, wm, wn, kC, lane);
-    if (tid < kC) {
+    if (tid < 64) {   // dbeta; the coefficient of k in dk's gate term
         float dadb, dadl;
         gate_derivatives(rule, bt[tid], lam[tid], al[tid], &dadb, &dadl);
         if (tid < nv) dbeta[row0 + tid] = dal[tid] * dadb;
-        lam[tid] = 2.f * dal[tid] * dadl;            // the coefficient of k in dk's gate term
+        lam[tid] = 2.f * dal[tid] * dadl;
     }
+    wait_mma();           // dK^T += S (-dR^T) is done (the commits are waited on in order)
+    handoff();
+    // ---- 8. dK^T += K^T (dG + dG^T)
+    if (warp == 0) {
+        mma_ss(tm + C_DK, sb + KQ, 0, 2048, 2 * TILE, sb + DG, 0, 2048, TILE, idesc(128, MN_MAJ, MN_MAJ), 4, true);
+        commit();
+    }
+    wait_mma();
+    {   // dk[token][i] = dK^T[i][token] + coef[token] k[token][i]
+        float x[32];
+        tmem_ld32_wait(tm + lane_off + C_DK + 32 * h, x);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            const int s = 32 * h + j;
+            if (s < nv) dk[(row0 + s) * 128 + row] = x[j] + lam[s] * ld_tok(sm + KQ, 2 * TILE, s, row);
+        }
+    }
+    tc_fence_before();
     __syncthreads();
-    for_acc(dka, wm, wn, lane, [&](int r, int c2, float& x) {
-        if (r < nv) dk[(row0 + r) * kD + c2] = x + lam[r] * __bfloat162float(sh[L::K + r * LW + c2]);
-    });
+    if (*abort) {         // a wait ran out: record it, and let every issued MMA finish before
+        if (tid == 0) atomicOr(err, kDevTimeout);   // the tensor memory is released
+        if (warp == 0) {
+            commit();
+            if (lane == 0) mbar_wait(bar + 1, mma_phase & 1, limit_ns);
+            __syncwarp();
+        }
+    }
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tm, C_COLS);
+    }
 }
 }  // namespace
+
+// rows x 128 bf16 row-major (the per-chunk S and dS' tiles) as a 2-D tensor: 64-column x
+// 128-row boxes, 128-byte swizzle (one box is one 64-column atom of a 128 x 128 tile).
+static bool tma_map_rows128(CUtensorMap* map, const void* ptr, long rows) {
+    auto fn = tma_encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {128, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {256};
+    cuuint32_t box[2] = {64, 128};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+constexpr unsigned long long kTileWaitNs = 2000000000ull;   // 2 s per wait
 
 size_t bwd_chunk_workspace_bytes(long BH, int T) {
     const long ntiles = BH * ((T + kC - 1) / kC);
@@ -421,11 +729,15 @@ cudaError_t launch_bwd_chunk(const void* q, const void* k, const void* v, const 
         (const bf16*)q, (const bf16*)k, (const bf16*)dO, Tt, dST, dSp, dS0, T);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     // 3. every chunk's gradients
-    e = set_smem_limit_once(bwd_tile_kernel, (int)TileSmem::BYTES, smem_tile);
+    CUtensorMap mq, mk, mv, mdo, ms, mdsp;
+    if (!tma_map_tokens(&mq, q, kD, T, BH) || !tma_map_tokens(&mk, k, kD, T, BH) || !tma_map_tokens(&mv, v, kD, T, BH) ||
+        !tma_map_tokens(&mdo, dO, kD, T, BH) || !tma_map_rows128(&ms, states, ntiles * kD) ||
+        !tma_map_rows128(&mdsp, dSp, ntiles * kD))
+        return cudaErrorInvalidValue;
+    e = set_smem_limit_once(bwd_tile_kernel, (int)tb::SMEM_BYTES, smem_tile);
     if (e != cudaSuccess) return e;
-    bwd_tile_kernel<<<(unsigned)ntiles, 256, TileSmem::BYTES, stream>>>(
-        (const bf16*)q, (const bf16*)k, (const bf16*)v, (const bf16*)beta, (const bf16*)dO, states, dSp, dq, dk, dv,
-        dbeta, T, rule);
+    bwd_tile_kernel<<<(unsigned)ntiles, 256, tb::SMEM_BYTES, stream>>>(
+        mq, mk, mv, mdo, ms, mdsp, (const bf16*)beta, dq, dk, dv, dbeta, T, rule, err, kTileWaitNs);
     return cudaGetLastError();
 }
 
