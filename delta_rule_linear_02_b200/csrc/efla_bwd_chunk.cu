@@ -29,6 +29,7 @@
 #include "efla_mma_sync.cuh"
 #include "efla_tma.cuh"
 #include "efla_ut_solve.cuh"
+#include "efla_ut_tf32.cuh"
 #include "sm100.cuh"
 
 namespace efla {
@@ -183,16 +184,16 @@ constexpr uint32_t FX = 188416;            // X (fp32)
 constexpr uint32_t FXT = TT;               // X^T
 constexpr uint32_t FW = TT + F32;          // W = dX X^T
 constexpr uint32_t FDT = V;                // dT^T, then dX^T, then dA
-constexpr uint32_t SMALL = FX + F32;       // alpha, beta, dalpha, lambda, ones (fp32 [64] each)
-constexpr uint32_t BAR = SMALL + 5 * 256;  // mbarriers: loads, MMA commits
-constexpr uint32_t MISC = BAR + 2 * 8;     // TMEM base, abort flag
+constexpr uint32_t SMALL = FX + F32;       // alpha, beta, dalpha, lambda, ones, two partial sums (fp32 [64] each)
+constexpr uint32_t BAR = SMALL + 7 * 256;  // mbarriers: K and Q, MMA commits, the other inputs
+constexpr uint32_t MISC = BAR + 3 * 8;     // TMEM base, abort flag
 constexpr uint32_t SMEM_BYTES = MISC + 16 + 1024;
 static_assert(64 * LA * 4 <= 16384, "the solve's A and scratch fit R^T's and Delta^T's regions");
 static_assert(FDT + F32 <= DSP && FW + F32 <= DG, "fp32 tiles stay inside dead regions");
 static_assert(SMEM_BYTES <= 232448, "shared memory");
 // TMEM columns (fp32 accumulators, 64 columns each)
 constexpr uint32_t C_GP = 0, C_SK = 64, C_DQ = 128, C_DL = 192, C_DD = 256, C_DK = 320, C_DR = 384, C_COLS = 512;
-constexpr uint32_t LOAD_BYTES = 131072;    // K, Q, V, dO, dS', S
+constexpr uint32_t KQ_BYTES = 32768, REST_BYTES = 98304;   // K and Q; V, dO, dS', S
 
 // nk k-steps of K = 16 with A and B in shared memory; operand k-step ks starts at
 // base + (ks / 4) * atom + (ks % 4) * step (K-major: step 32 bytes inside a 64-column atom;
@@ -246,9 +247,15 @@ __device__ __forceinline__ float ld_tok(const uint8_t* tile, uint32_t atom, int 
     return __bfloat162float(*reinterpret_cast<const bf16*>(p));
 }
 
-// X = (I + A)^{-1} for the 64 x 64 strictly-lower A (row stride LA; only its strictly-lower
-// part is read), written in full into X (row stride LX; zeros above the diagonal), Y scratch
-// (row stride LA).  Block doubling: the four 16 x 16 diagonal blocks by forward
+// Element (r, j) of the solve's A and scratch (row stride LA): the column is XOR-swizzled
+// with the row's low five bits, so a warp writing one column of 32 consecutive rows hits 32
+// banks, while every read of the solve (one row's element broadcast to the warp, or one
+// row's consecutive columns) stays a single wavefront.
+__device__ __forceinline__ int sa(int r, int j) { return r * LA + (j ^ (r & 31)); }
+
+// X = (I + A)^{-1} for the 64 x 64 strictly-lower A (swizzled, see sa; only its
+// strictly-lower part is read), written in full into X (row stride LX; zeros above the
+// diagonal), Y scratch (swizzled like A).  Block doubling: the four 16 x 16 diagonal blocks by forward
 // substitution (one thread per column), then merges X21 = -X22 (A21 X11) at 32 and 64.  In
 // the 64 merge each thread keeps four rows of one column in registers (one operand load
 // per four FMAs).  256 threads; ends with a barrier.
@@ -256,7 +263,6 @@ __device__ __forceinline__ void unit_lower_inverse64(const float* __restrict__ A
                                                      float* __restrict__ Y, int tid) {
     if (tid < 64) {
         const int b = tid >> 4, c = tid & 15;
-        const float* Ab = A + (16 * b) * LA + 16 * b;
         float x[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) x[i] = (i == c) ? 1.f : 0.f;
@@ -264,7 +270,7 @@ __device__ __forceinline__ void unit_lower_inverse64(const float* __restrict__ A
         for (int i = 1; i < 16; ++i) {
             float s = 0.f;
 #pragma unroll
-            for (int j = 0; j < i; ++j) s = fmaf(Ab[i * LA + j], x[j], s);
+            for (int j = 0; j < i; ++j) s = fmaf(A[sa(16 * b + i, 16 * b + j)], x[j], s);
             if (i > c) x[i] = -s;
         }
         float* Xb = X + (16 * b) * LX + 16 * b + c;
@@ -284,11 +290,11 @@ __device__ __forceinline__ void unit_lower_inverse64(const float* __restrict__ A
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
             const float xv = X[(c0 + j) * LX + c0 + c];
-            y0 = fmaf(A[(r0 + i) * LA + c0 + j], xv, y0);
-            y1 = fmaf(A[(r0 + i + 8) * LA + c0 + j], xv, y1);
+            y0 = fmaf(A[sa(r0 + i, c0 + j)], xv, y0);
+            y1 = fmaf(A[sa(r0 + i + 8, c0 + j)], xv, y1);
         }
-        Y[(r0 + i) * LA + c0 + c] = y0;
-        Y[(r0 + i + 8) * LA + c0 + c] = y1;
+        Y[sa(r0 + i, c0 + c)] = y0;
+        Y[sa(r0 + i + 8, c0 + c)] = y1;
     }
     __syncthreads();
     {
@@ -297,7 +303,7 @@ __device__ __forceinline__ void unit_lower_inverse64(const float* __restrict__ A
         float x0 = 0.f, x1 = 0.f;
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
-            const float yv = Y[(r0 + j) * LA + c0 + c];
+            const float yv = Y[sa(r0 + j, c0 + c)];
             x0 = fmaf(X[(r0 + i) * LX + r0 + j], yv, x0);
             x1 = fmaf(X[(r0 + i + 8) * LX + r0 + j], yv, x1);
         }
@@ -312,17 +318,17 @@ __device__ __forceinline__ void unit_lower_inverse64(const float* __restrict__ A
         for (int j = 0; j < 32; ++j) {
             const float xv = X[j * LX + c];
 #pragma unroll
-            for (int k = 0; k < 4; ++k) y[k] = fmaf(A[(32 + i0 + 8 * k) * LA + j], xv, y[k]);
+            for (int k = 0; k < 4; ++k) y[k] = fmaf(A[sa(32 + i0 + 8 * k, j)], xv, y[k]);
         }
 #pragma unroll
-        for (int k = 0; k < 4; ++k) Y[(32 + i0 + 8 * k) * LA + c] = y[k];
+        for (int k = 0; k < 4; ++k) Y[sa(32 + i0 + 8 * k, c)] = y[k];
     }
     __syncthreads();
     {   // X21 = -X22 Y21
         float x[4] = {};
 #pragma unroll 8
         for (int j = 0; j < 32; ++j) {
-            const float yv = Y[(32 + j) * LA + c];
+            const float yv = Y[sa(32 + j, c)];
 #pragma unroll
             for (int k = 0; k < 4; ++k) x[k] = fmaf(X[(32 + i0 + 8 * k) * LX + 32 + j], yv, x[k]);
         }
@@ -332,23 +338,34 @@ __device__ __forceinline__ void unit_lower_inverse64(const float* __restrict__ A
     __syncthreads();
 }
 
-// C (64 x 64, row stride LX) = sum_m P[m][r] Q[m][c] for the fp32 tiles P, Q (row stride LX):
-// thread -> 4 x 4 outputs (rows 4 (tid / 16), columns 4 (tid % 16)), two 16-byte loads per m.
-__device__ __forceinline__ void gemm_tn64(const float* __restrict__ P, const float* __restrict__ Q, float (&w)[4][4],
-                                          int r4, int c4) {
+// C (64 x 64) = sum_m P[m][r] Q[m][c] for the fp32 tiles P, Q (row stride LX), on the TF32
+// tensor path (mma.sync m16n8k8; operands rounded to TF32, 10-bit mantissa, finer than the
+// bf16 operands of the other products).  Warp w: rows 16 (w % 4) .. + 15, columns
+// 32 (w / 4) .. + 31 (four 8-column tiles); acc[nt] holds C[r0 + g][c] and C[r0 + g + 8][c]
+// for c = c0 + 8 nt + 2 t, + 1 (g = lane / 4, t = lane % 4).  The k slots t and t + 4 of a
+// k-step take m = 2 t and 2 t + 1: with LX = 4 (mod 32) every operand load of a warp then
+// hits 32 distinct banks.
+__device__ __forceinline__ void gemm_tn64_tc(const float* __restrict__ P, const float* __restrict__ Q,
+                                             float (&acc)[4][4], int warp, int lane) {
+    const int g = lane >> 2, t = lane & 3;
+    const int r0 = 16 * (warp & 3), c0 = 32 * (warp >> 2);
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) w[i][j] = 0.f;
-#pragma unroll 4
-    for (int m = 0; m < 64; ++m) {
-        const float4 a = *reinterpret_cast<const float4*>(P + m * LX + r4);
-        const float4 b = *reinterpret_cast<const float4*>(Q + m * LX + c4);
-        const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+        for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
+#pragma unroll 2
+    for (int k0 = 0; k0 < 64; k0 += 8) {
+        const float* p0 = P + (k0 + 2 * t) * LX + r0 + g;
+        const float av[4] = {p0[0], p0[8], p0[LX], p0[LX + 8]};
+        uint32_t a[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
+        for (int e = 0; e < 4; ++e) a[e] = ut::to_tf32(av[e]);
 #pragma unroll
-            for (int j = 0; j < 4; ++j) w[i][j] = fmaf(av[i], bv[j], w[i][j]);
+        for (int nt = 0; nt < 4; ++nt) {
+            const float* q0 = Q + (k0 + 2 * t) * LX + c0 + 8 * nt + g;
+            uint32_t b[2] = {ut::to_tf32(q0[0]), ut::to_tf32(q0[LX])};
+            ut::mma_tf32(acc[nt], a, b);
+        }
     }
 }
 }  // namespace tb
@@ -364,7 +381,7 @@ bwd_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sb = smem_u32(sm);
-    uint64_t* bar = reinterpret_cast<uint64_t*>(sm + BAR);    // 0: the tile's loads, 1: MMA commits
+    uint64_t* bar = reinterpret_cast<uint64_t*>(sm + BAR);    // 0: K and Q, 1: MMA commits, 2: V, dO, dS', S
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + MISC);
     volatile int* abort = reinterpret_cast<volatile int*>(sm + MISC + 4);
     float* fA = reinterpret_cast<float*>(sm + RT);
@@ -374,7 +391,7 @@ bwd_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     float* fW = reinterpret_cast<float*>(sm + FW);
     float* fdT = reinterpret_cast<float*>(sm + FDT);
     float* al = reinterpret_cast<float*>(sm + SMALL);
-    float *bt = al + 64, *dal = al + 128, *lam = al + 192, *ones = al + 256;
+    float *bt = al + 64, *dal = al + 128, *lam = al + 192, *ones = al + 256, *part = al + 320;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int q = warp & 3, h = warp >> 2;                    // TMEM lane quarter, column half
@@ -390,21 +407,24 @@ bwd_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     if (tid == 0) {
         mbar_init(bar, 1);
         mbar_init(bar + 1, 1);
+        mbar_init(bar + 2, 1);
         *abort = 0;
         fence_mbar_init();
-        mbar_arrive_expect_tx(bar, LOAD_BYTES);
+        mbar_arrive_expect_tx(bar, KQ_BYTES);
         tma_load_3d(sm + KQ, &tm_k, bar, 0, t0, (int)bh);
         tma_load_3d(sm + KQ + 2 * TILE, &tm_k, bar, 64, t0, (int)bh);
         tma_load_3d(sm + KQ + TILE, &tm_q, bar, 0, t0, (int)bh);
         tma_load_3d(sm + KQ + 3 * TILE, &tm_q, bar, 64, t0, (int)bh);
-        tma_load_3d(sm + V, &tm_v, bar, 0, t0, (int)bh);
-        tma_load_3d(sm + V + TILE, &tm_v, bar, 64, t0, (int)bh);
-        tma_load_3d(sm + DO, &tm_do, bar, 0, t0, (int)bh);
-        tma_load_3d(sm + DO + TILE, &tm_do, bar, 64, t0, (int)bh);
-        tma_load_2d(sm + DSP, &tm_dsp, bar, 0, (int)(tile * 128));
-        tma_load_2d(sm + DSP + 2 * TILE, &tm_dsp, bar, 64, (int)(tile * 128));
-        tma_load_2d(sm + SS, &tm_s, bar, 0, (int)(tile * 128));
-        tma_load_2d(sm + SS + 2 * TILE, &tm_s, bar, 64, (int)(tile * 128));
+        uint64_t* rest = bar + 2;
+        mbar_arrive_expect_tx(rest, REST_BYTES);
+        tma_load_3d(sm + V, &tm_v, rest, 0, t0, (int)bh);
+        tma_load_3d(sm + V + TILE, &tm_v, rest, 64, t0, (int)bh);
+        tma_load_3d(sm + DO, &tm_do, rest, 0, t0, (int)bh);
+        tma_load_3d(sm + DO + TILE, &tm_do, rest, 64, t0, (int)bh);
+        tma_load_2d(sm + DSP, &tm_dsp, rest, 0, (int)(tile * 128));
+        tma_load_2d(sm + DSP + 2 * TILE, &tm_dsp, rest, 64, (int)(tile * 128));
+        tma_load_2d(sm + SS, &tm_s, rest, 0, (int)(tile * 128));
+        tma_load_2d(sm + SS + 2 * TILE, &tm_s, rest, 64, (int)(tile * 128));
     }
     const float beta_t = tid < nv ? __bfloat162float(beta[row0 + tid]) : 0.f;   // in flight during the setup
     if (warp == 0) {
@@ -438,15 +458,10 @@ bwd_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         tc_fence_after();
     };
 
-    // ---- 1. [G; P~] = [K; Q] K^T;  dDelta^T = dS'^T K^T (+ dO^T P below);  S^T K^T;  dQ^T = S dO^T
+    // ---- 1. [G; P~] = [K; Q] K^T, as soon as K and Q have landed
     wait(0, 0);
     if (warp == 0) {
         mma_ss(tm + C_GP, sb + KQ, 2 * TILE, 32, 16, sb + KQ, 2 * TILE, 32, 16, idesc(128, K_MAJ, K_MAJ), 8, false);
-        mma_ss(tm + C_DD, sb + DSP, TILE, 2048, 2 * TILE, sb + KQ, 2 * TILE, 32, 16, idesc(128, MN_MAJ, K_MAJ), 8,
-               false);
-        mma_ss(tm + C_SK, sb + SS, TILE, 2048, 2 * TILE, sb + KQ, 2 * TILE, 32, 16, idesc(128, MN_MAJ, K_MAJ), 8,
-               false);
-        mma_ss(tm + C_DQ, sb + SS, 2 * TILE, 32, 16, sb + DO, TILE, 32, 16, idesc(128, K_MAJ, K_MAJ), 8, false);
         commit();
     }
     wait_mma();
@@ -475,13 +490,20 @@ bwd_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
             const int s = 32 * h + j;
-            fA[row * LA + s] = s < row ? a * g[j] : 0.f;
+            fA[sa(row, s)] = s < row ? a * g[j] : 0.f;
         }
     }
     handoff();
-    // ---- 2. dDelta^T += dO^T P, while the CUDA cores solve for X = (I + A)^{-1}
+    // ---- 2. while the CUDA cores solve for X = (I + A)^{-1}:
+    //         dDelta^T = dS'^T K^T + dO^T P;  S^T K^T;  dQ^T = S dO^T
+    wait(2, 0);
     if (warp == 0) {
+        mma_ss(tm + C_DD, sb + DSP, TILE, 2048, 2 * TILE, sb + KQ, 2 * TILE, 32, 16, idesc(128, MN_MAJ, K_MAJ), 8,
+               false);
         mma_ss(tm + C_DD, sb + DO, TILE, 2048, TILE, sb + PP, TILE, 2048, TILE, idesc(128, MN_MAJ, MN_MAJ), 4, true);
+        mma_ss(tm + C_SK, sb + SS, TILE, 2048, 2 * TILE, sb + KQ, 2 * TILE, 32, 16, idesc(128, MN_MAJ, K_MAJ), 8,
+               false);
+        mma_ss(tm + C_DQ, sb + SS, 2 * TILE, 32, 16, sb + DO, TILE, 32, 16, idesc(128, K_MAJ, K_MAJ), 8, false);
         commit();
     }
     unit_lower_inverse64(fA, fX, fY, tid);            // ends with a barrier: A and the scratch are dead
@@ -491,13 +513,13 @@ bwd_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
         for (int j = 0; j < 16; ++j) x[j] = fX[t * LX + s0 + j] * al[s0 + j];
         st_row16(sm + TT, t, 2 * (tid & 3), x);
+        wait_mma();       // the products of step 2 have landed
         float r[32];
         tmem_ld32_wait(tm + lane_off + C_SK + 32 * h, r);
 #pragma unroll
         for (int j = 0; j < 32; ++j) r[j] = ld_tok(sm + V, TILE, 32 * h + j, row) - r[j];
         st_row32(sm + RT, row, 4 * h, r);
     }
-    wait_mma();           // dO^T P has landed (read in step 4)
     handoff();
     // ---- 3. Delta^T = R^T T^T
     if (warp == 0) {
@@ -597,44 +619,46 @@ bwd_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         dal[tid] = sacc;
     }
     __syncthreads();
-    const int r4 = 4 * (tid >> 4), c4 = 4 * (tid & 15);
+    const int g8 = lane >> 2, t4 = lane & 3, r0 = 16 * (warp & 3), c0 = 32 * (warp >> 2);
     {   // W = dX X^T:  W[r][c] = sum_m dX^T[m][r] X^T[m][c]
         float w[4][4];
-        gemm_tn64(fdT, fXT, w, r4, c4);
+        gemm_tn64_tc(fdT, fXT, w, warp, lane);
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-            *reinterpret_cast<float4*>(fW + (r4 + i) * LX + c4) = make_float4(w[i][0], w[i][1], w[i][2], w[i][3]);
+        for (int nt = 0; nt < 4; ++nt) {
+            const int cc = c0 + 8 * nt + 2 * t4;
+            *reinterpret_cast<float2*>(fW + (r0 + g8) * LX + cc) = make_float2(w[nt][0], w[nt][1]);
+            *reinterpret_cast<float2*>(fW + (r0 + g8 + 8) * LX + cc) = make_float2(w[nt][2], w[nt][3]);
+        }
     }
     __syncthreads();
     {   // dA = strict_tril(-X^T W) over dX^T:  dA[r][c] = -sum_m X[m][r] W[m][c];
-        // dalpha_r += sum_{s<r} dA_rs G_rs
+        // dalpha_r += sum_{s<r} dA_rs G_rs (this warp's 32 columns, then the two halves)
         float w[4][4];
-        gemm_tn64(fX, fW, w, r4, c4);
-        float part[4];
+        gemm_tn64_tc(fX, fW, w, warp, lane);
+        float p0 = 0.f, p1 = 0.f;
+        const int ra = r0 + g8, rb = r0 + g8 + 8;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            part[i] = 0.f;
-            float da[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int r = r4 + i, s2 = c4 + j;
-                da[j] = s2 < r ? -w[i][j] : 0.f;
-                part[i] = fmaf(da[j], ld_tok(sm + DG, 0, r, s2), part[i]);
-            }
-            *reinterpret_cast<float4*>(fdT + (r4 + i) * LX + c4) = make_float4(da[0], da[1], da[2], da[3]);
+        for (int nt = 0; nt < 4; ++nt) {
+            const int cc = c0 + 8 * nt + 2 * t4;
+            const float a0 = cc < ra ? -w[nt][0] : 0.f, a1 = cc + 1 < ra ? -w[nt][1] : 0.f;
+            const float b0 = cc < rb ? -w[nt][2] : 0.f, b1 = cc + 1 < rb ? -w[nt][3] : 0.f;
+            *reinterpret_cast<float2*>(fdT + ra * LX + cc) = make_float2(a0, a1);
+            *reinterpret_cast<float2*>(fdT + rb * LX + cc) = make_float2(b0, b1);
+            p0 = fmaf(a0, ld_tok(sm + DG, 0, ra, cc), fmaf(a1, ld_tok(sm + DG, 0, ra, cc + 1), p0));
+            p1 = fmaf(b0, ld_tok(sm + DG, 0, rb, cc), fmaf(b1, ld_tok(sm + DG, 0, rb, cc + 1), p1));
         }
-        // the 16 column blocks of a row block sit in 16 consecutive lanes: sum over them
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-#pragma unroll
-            for (int off = 1; off < 16; off <<= 1) part[i] += __shfl_xor_sync(0xffffffffu, part[i], off);
-        }
-        if ((tid & 15) == 0) {
-#pragma unroll
-            for (int i = 0; i < 4; ++i) dal[r4 + i] += part[i];
+        // the four lanes of a row group hold its 32 columns: sum over them
+        p0 += __shfl_xor_sync(0xffffffffu, p0, 1);
+        p0 += __shfl_xor_sync(0xffffffffu, p0, 2);
+        p1 += __shfl_xor_sync(0xffffffffu, p1, 1);
+        p1 += __shfl_xor_sync(0xffffffffu, p1, 2);
+        if (t4 == 0) {
+            part[(warp >> 2) * 64 + ra] = p0;
+            part[(warp >> 2) * 64 + rb] = p1;
         }
     }
     __syncthreads();
+    if (tid < 64) dal[tid] += part[tid] + part[64 + tid];
     {   // dG + dG^T with dG = diag(alpha) dA, bf16 over G: thread -> row tid / 4, 16 columns
         const int r = tid >> 2, s0 = 16 * (tid & 3);
         float x[16];
