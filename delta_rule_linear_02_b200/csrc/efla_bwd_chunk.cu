@@ -26,7 +26,6 @@
 // bf16-operand rounding (relative Frobenius error ~1e-2), not fp32's.
 #include "efla_common.cuh"
 #include "efla_kernels.h"
-#include "efla_mma_sync.cuh"
 #include "efla_tma.cuh"
 #include "efla_ut_solve.cuh"
 #include "efla_ut_tf32.cuh"
@@ -35,112 +34,8 @@
 namespace efla {
 
 namespace {
-using namespace mmas;
+using bf16 = __nv_bfloat16;
 constexpr int kD = 128, kC = 64;
-constexpr int LW = kD + 8;     // bf16 row stride of 128-wide tiles (272 B: conflict-free ldmatrix rows)
-constexpr int LH = 64 + 8;     // bf16 row stride of 64-wide tiles (144 B)
-
-// ============================================================================ reverse chain
-// One CTA (8 warps) per (stream, d_v half).  Per chunk, walking backwards:
-//   store dS' (the carried gradient, bf16) for the tile kernel;
-//   P = tril(Q K^T);  dDelta = P^T dO + K dS';  -dR = -(T^T dDelta);  dS += Q^T dO + K^T (-dR).
-// Warp w carries rows 16 w .. 16 w + 15 of the dS half in its accumulators.
-struct ChainSmem {
-    static constexpr int Q = 0;                          // per stage: Q, K (64 x LW), T (64 x LH), dO (64 x LH)
-    static constexpr int K = Q + kC * LW;
-    static constexpr int T = K + kC * LW;
-    static constexpr int DO = T + kC * LH;
-    static constexpr int STAGE = DO + kC * LH;           // bf16 elements per stage
-    static constexpr int P = 2 * STAGE;
-    static constexpr int DD = P + kC * LH;               // dDelta
-    static constexpr int NR = DD + kC * LH;              // -dR
-    static constexpr int DS = NR + kC * LH;              // dS (bf16), 128 x LH
-    static constexpr int ELEMS = DS + kD * LH;
-    static constexpr size_t BYTES = sizeof(bf16) * ELEMS;
-};
-
-__global__ void __launch_bounds__(256, 1)
-bwd_chain_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16* __restrict__ dO,
-                 const bf16* __restrict__ Tt, const float* __restrict__ dST, bf16* __restrict__ dSp,
-                 float* __restrict__ dS0, int T) {
-    extern __shared__ __align__(16) bf16 sh[];
-    using L = ChainSmem;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const long bh = blockIdx.x >> 1;
-    const int col0 = (blockIdx.x & 1) * 64;
-    const int nchunks = (T + kC - 1) / kC;
-    const long tile0 = bh * nchunks;
-    auto stage = [&](int c) { return sh + (c & 1) * L::STAGE; };
-    auto issue = [&](int c) {   // chunk c's Q, K, T and dO half into its stage
-        bf16* st = stage(c);
-        const int nv = min(kC, T - c * kC);
-        const size_t row0 = (size_t)bh * T + (size_t)c * kC;
-        load_tile(st + L::Q, LW, q + row0 * kD, kD, kC, kD, nv, tid, 256);
-        load_tile(st + L::K, LW, k + row0 * kD, kD, kC, kD, nv, tid, 256);
-        load_tile(st + L::T, LH, Tt + (size_t)(tile0 + c) * kC * kC, kC, kC, kC, kC, tid, 256);
-        load_tile(st + L::DO, LH, dO + row0 * kD + col0, kD, kC, 64, nv, tid, 256);
-        cp_async_commit();
-    };
-    // the carried gradient: dS_T's half (or zero)
-    float ds[8][4];
-    zero_acc(ds);
-    if (dST) for_acc(ds, 16 * warp, 0, lane, [&](int r, int c, float& v) { v = dST[((size_t)bh * kD + r) * kD + col0 + c]; });
-    bf16* dsb = sh + L::DS;
-    auto write_ds = [&]() {
-        for_acc(ds, 16 * warp, 0, lane, [&](int r, int c, float& v) { dsb[r * LH + c] = __float2bfloat16_rn(v); });
-    };
-    write_ds();
-    issue(nchunks - 1);
-    for (int c = nchunks - 1; c >= 0; --c) {
-        if (c > 0) {
-            issue(c - 1);
-            cp_async_wait<1>();
-        } else {
-            cp_async_wait<0>();
-        }
-        __syncthreads();                                   // stage c landed, dS' (bf16) complete
-        const bf16* st = stage(c);
-        // dS' for the tile kernel (this half's 64 columns of the 128 x 128 matrix)
-        for (int e = tid; e < kD * 8; e += 256) {
-            const int rr = e >> 3, cc = (e & 7) * 8;
-            *reinterpret_cast<uint4*>(dSp + ((size_t)(tile0 + c) * kD + rr) * kD + col0 + cc) =
-                *reinterpret_cast<const uint4*>(dsb + rr * LH + cc);
-        }
-        {   // P = tril_incl(Q K^T): warp w -> rows 16 (w % 4), columns 32 (w / 4)
-            float acc[4][4];
-            zero_acc(acc);
-            const int m0 = 16 * (warp & 3), n0 = 32 * (warp >> 2);
-            warp_mma<4, false, false>(acc, st + L::Q, LW, st + L::K, LW, m0, n0, kD, lane);
-            for_acc(acc, m0, n0, lane, [&](int r, int c2, float& v) {
-                sh[L::P + r * LH + c2] = __float2bfloat16_rn(c2 <= r ? v : 0.f);
-            });
-        }
-        __syncthreads();
-        {   // dDelta = P^T dO + K dS'
-            float acc[4][4];
-            zero_acc(acc);
-            const int m0 = 16 * (warp & 3), n0 = 32 * (warp >> 2);
-            warp_mma<4, true, true>(acc, sh + L::P, LH, st + L::DO, LH, m0, n0, kC, lane);
-            warp_mma<4, false, true>(acc, st + L::K, LW, dsb, LH, m0, n0, kD, lane);
-            for_acc(acc, m0, n0, lane, [&](int r, int c2, float& v) { sh[L::DD + r * LH + c2] = __float2bfloat16_rn(v); });
-        }
-        __syncthreads();
-        {   // -dR = -(T^T dDelta)
-            float acc[4][4];
-            zero_acc(acc);
-            const int m0 = 16 * (warp & 3), n0 = 32 * (warp >> 2);
-            warp_mma<4, true, true>(acc, st + L::T, LH, sh + L::DD, LH, m0, n0, kC, lane);
-            for_acc(acc, m0, n0, lane, [&](int r, int c2, float& v) { sh[L::NR + r * LH + c2] = __float2bfloat16_rn(-v); });
-        }
-        __syncthreads();
-        // dS += Q^T dO + K^T (-dR): rows 16 w .. of the 128 x 64 half
-        warp_mma<8, true, true>(ds, st + L::Q, LW, st + L::DO, LH, 16 * warp, 0, kC, lane);
-        warp_mma<8, true, true>(ds, st + L::K, LW, sh + L::NR, LH, 16 * warp, 0, kC, lane);
-        __syncthreads();                                   // every read of dS' and of stage c is done
-        write_ds();
-    }
-    if (dS0) for_acc(ds, 16 * warp, 0, lane, [&](int r, int c, float& v) { dS0[((size_t)bh * kD + r) * kD + col0 + c] = v; });
-}
 
 // ============================================================================ per-chunk gradients
 // One CTA (8 warps) per (stream, chunk), every product on the 5th-generation tensor cores
@@ -698,7 +593,11 @@ bwd_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (tid == 0) atomicOr(err, kDevTimeout);   // the tensor memory is released
         if (warp == 0) {
             commit();
-            if (lane == 0) mbar_wait(bar + 1, mma_phase & 1, limit_ns);
+            if (lane == 0) {
+                mbar_wait(bar + 1, mma_phase & 1, limit_ns);
+                mbar_wait(bar, 0, limit_ns);        // and no copy may land after the block exits
+                mbar_wait(bar + 2, 0, limit_ns);
+            }
             __syncwarp();
         }
     }
@@ -707,6 +606,247 @@ bwd_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         tmem_dealloc(tm, C_COLS);
     }
 }
+// ============================================================================ reverse chain
+// One CTA (8 warps) per (stream, 64-column half of d_v) walks the chunks backwards with its
+// half of dS in tensor memory (the columns of dS evolve independently).  Per chunk c:
+//   store dS' (the carried gradient, bf16) for the per-chunk kernel;
+//   dDelta = P^T dO + K dS'   (M = 64)        dR = T^T dDelta   (M = 64)
+//   dS += Q^T dO + K^T (-dR)  (M = 128, the accumulator)
+// with P = tril_incl(Q K^T) of chunk c - 1 formed in the same MMA batch as the dS update.
+// Q, K, T and the dO half of three chunks are in flight by TMA; every product is a tcgen05
+// MMA (bf16 operands in shared memory, fp32 accumulators in tensor memory); between the
+// products the eight warps convert the accumulator to the next bf16 operand.
+namespace rc {
+constexpr uint32_t TILE = 8192;
+constexpr int kStages = 3;
+constexpr uint32_t ST_Q = 0, ST_K = 2 * TILE, ST_T = 4 * TILE, ST_DO = 5 * TILE, STAGE = 6 * TILE;
+constexpr uint32_t P = kStages * STAGE;    // P (bf16 [t][s])
+constexpr uint32_t DSB = P + TILE;         // dS' (bf16, 128 rows i x 64 columns j)
+constexpr uint32_t DD = DSB + 2 * TILE;    // dDelta (bf16 [s][j])
+constexpr uint32_t NR = DD + TILE;         // -dR (bf16 [s][j])
+constexpr uint32_t BAR = NR + TILE;        // stage full [3], MMA commits
+constexpr uint32_t MISC = BAR + 4 * 8;     // TMEM base, abort flag, loads issued per stage [3]
+constexpr uint32_t SMEM_BYTES = MISC + 32 + 1024;
+static_assert(SMEM_BYTES <= 232448, "shared memory");
+constexpr uint32_t C_DS = 0, C_P = 64, C_DD = 128, C_DR = 192, C_COLS = 256;
+
+// 2-D tiled store of one box from shared memory (bulk-group completion; no multicast)
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src, int c0, int c1) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(sm100::smem_u32(src)), "r"(c0), "r"(c1)
+                 : "memory");
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// the shared-memory source of every earlier store has been read / every earlier store is done
+__device__ __forceinline__ void tma_store_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void tma_store_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+}  // namespace rc
+
+__global__ void __launch_bounds__(256, 1)
+bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                 const __grid_constant__ CUtensorMap tm_do, const __grid_constant__ CUtensorMap tm_t,
+                 const __grid_constant__ CUtensorMap tm_dsp, const float* __restrict__ dST, float* __restrict__ dS0,
+                 int T, uint32_t* __restrict__ err, unsigned long long limit_ns) {
+    using namespace rc;
+    using namespace sm100;
+    using tb::K_MAJ;
+    using tb::MN_MAJ;
+    using tb::idesc;
+    using tb::mma_ss;
+    using tb::st_row32;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sb = smem_u32(sm);
+    uint64_t* bar = reinterpret_cast<uint64_t*>(sm + BAR);    // 0-2: stage full, 3: MMA commits
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + MISC);
+    volatile int* abort = reinterpret_cast<volatile int*>(sm + MISC + 4);
+    int* issued = reinterpret_cast<int*>(sm + MISC + 8);      // written by thread 0 only
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int q = warp & 3, h = warp >> 2;                    // TMEM lane quarter, column half
+    const uint32_t lane_off = static_cast<uint32_t>(32 * q) << 16;
+    const int row = 32 * q + lane;                            // row of dS (d_k index)
+    const int trow = 16 * q + lane;                           // row of an M = 64 product (lanes < 16)
+    const long bh = blockIdx.x >> 1;
+    const int col0 = (blockIdx.x & 1) * 64;
+    const int nc = (T + 63) / 64;
+    const long tile0 = bh * nc;
+    const size_t srow = ((size_t)bh * 128 + row) * 128 + col0 + 32 * h;   // this thread's 32 entries of dS
+
+    if (nc == 0) {        // no tokens: dS0 = dS_T
+        if (dS0)
+            for (int j = 0; j < 32; ++j) dS0[srow + j] = dST ? dST[srow + j] : 0.f;
+        return;
+    }
+    auto load = [&](int c) {   // chunk c's Q, K, T and dO half into stage c % 3 (one thread)
+        uint8_t* st = sm + (c % kStages) * STAGE;
+        uint64_t* full = bar + c % kStages;
+        ++issued[c % kStages];
+        mbar_arrive_expect_tx(full, STAGE);
+        tma_load_3d(st + ST_Q, &tm_q, full, 0, c * 64, (int)bh);
+        tma_load_3d(st + ST_Q + TILE, &tm_q, full, 64, c * 64, (int)bh);
+        tma_load_3d(st + ST_K, &tm_k, full, 0, c * 64, (int)bh);
+        tma_load_3d(st + ST_K + TILE, &tm_k, full, 64, c * 64, (int)bh);
+        tma_load_2d(st + ST_T, &tm_t, full, 0, (int)((tile0 + c) * 64));
+        tma_load_3d(st + ST_DO, &tm_do, full, col0, c * 64, (int)bh);
+    };
+    if (tid == 0) {
+        for (int i = 0; i < 4; ++i) mbar_init(bar + i, 1);
+        *abort = 0;
+        for (int i = 0; i < kStages; ++i) issued[i] = 0;
+        fence_mbar_init();
+        for (int i = 0; i < kStages && i < nc; ++i) load(nc - 1 - i);
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, C_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tm = *tmem_slot;
+    auto wait = [&](int i, uint32_t parity) {
+        if (*abort) return;
+        if (!mbar_wait(bar + i, parity, limit_ns)) *abort = 1;
+        tc_fence_after();
+    };
+    auto wait_stage = [&](int c) { wait(c % kStages, ((nc - 1 - c) / kStages) & 1); };
+    uint32_t mma_phase = 0;
+    auto wait_mma = [&]() { wait(3, mma_phase & 1); ++mma_phase; };
+    auto commit = [&]() { mma_commit_elect(bar + 3); };
+    auto handoff = [&]() {
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+    };
+    auto stage = [&](int c) { return sb + (uint32_t)(c % kStages) * STAGE; };
+    // dS (fp32, tensor memory) -> dS' of the next chunk, the bf16 operand; the per-chunk
+    // kernel's copy is stored from it by TMA at the start of that chunk's step
+    auto emit_dsp = [&](const float (&x)[32]) { st_row32(sm + DSB, row, 4 * h, x); };
+    // P~ (M = 64, rows trow) -> P = tril_incl, bf16 [t][s]
+    auto emit_p = [&]() {
+        float x[32];
+        tmem_ld32_wait(tm + lane_off + C_P + 32 * h, x);
+        if (lane < 16) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+                if (32 * h + j > trow) x[j] = 0.f;
+            st_row32(sm + P, trow, 4 * h, x);
+        }
+    };
+
+    {   // the carried gradient starts as dS_T's half (or zero)
+        float x[32];
+#pragma unroll
+        for (int j = 0; j < 32; j += 4) {
+            const float4 v = dST ? *reinterpret_cast<const float4*>(dST + srow + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+            x[j] = v.x; x[j + 1] = v.y; x[j + 2] = v.z; x[j + 3] = v.w;
+        }
+        float lo[16], hi[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            lo[j] = x[j];
+            hi[j] = x[16 + j];
+        }
+        tmem_st16(tm + lane_off + C_DS + 32 * h, lo);
+        tmem_st16(tm + lane_off + C_DS + 32 * h + 16, hi);
+        tmem_wait_st();
+        emit_dsp(x);
+    }
+    wait_stage(nc - 1);
+    handoff();            // dS' (bf16) is an MMA operand from here on
+    if (warp == 0) {
+        const uint32_t st = stage(nc - 1);
+        mma_ss(tm + C_P, st + ST_Q, TILE, 32, 16, st + ST_K, TILE, 32, 16, idesc(64, K_MAJ, K_MAJ), 8, false);
+        commit();
+    }
+    wait_mma();
+    emit_p();
+    handoff();
+    for (int c = nc - 1; c >= 0; --c) {
+        const uint32_t st = stage(c);
+        // ---- dDelta = P^T dO + K dS'
+        if (warp == 0) {
+            mma_ss(tm + C_DD, sb + P, 0, 2048, TILE, st + ST_DO, 0, 2048, TILE, idesc(64, MN_MAJ, MN_MAJ), 4, false);
+            mma_ss(tm + C_DD, st + ST_K, TILE, 32, 16, sb + DSB, TILE, 2048, TILE, idesc(64, K_MAJ, MN_MAJ), 8, true);
+            commit();
+        }
+        if (warp == 1 && lane == 0) {
+            tma_store_2d(&tm_dsp, sm + DSB, col0, (int)((tile0 + c) * 128));   // dS' of chunk c
+            if (c + 1 - kStages >= 0 && c + 1 < nc && !*abort)
+                load(c + 1 - kStages);   // into the stage chunk c + 1 no longer reads
+        }
+        wait_mma();
+        {
+            float x[32];
+            tmem_ld32_wait(tm + lane_off + C_DD + 32 * h, x);
+            if (lane < 16) st_row32(sm + DD, trow, 4 * h, x);
+        }
+        handoff();
+        // ---- dR = T^T dDelta
+        if (warp == 0) {
+            mma_ss(tm + C_DR, st + ST_T, 0, 2048, TILE, sb + DD, 0, 2048, TILE, idesc(64, MN_MAJ, MN_MAJ), 4, false);
+            commit();
+        }
+        wait_mma();
+        {
+            float x[32];
+            tmem_ld32_wait(tm + lane_off + C_DR + 32 * h, x);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) x[j] = -x[j];
+            if (lane < 16) st_row32(sm + NR, trow, 4 * h, x);
+        }
+        if (warp == 1 && lane == 0) tma_store_wait_read();   // dS' may be overwritten below
+        handoff();
+        // ---- dS += Q^T dO + K^T (-dR);  P~ of chunk c - 1
+        if (c > 0) wait_stage(c - 1);
+        if (warp == 0) {
+            mma_ss(tm + C_DS, st + ST_Q, 0, 2048, TILE, st + ST_DO, 0, 2048, TILE, idesc(128, MN_MAJ, MN_MAJ), 4, true);
+            mma_ss(tm + C_DS, st + ST_K, 0, 2048, TILE, sb + NR, 0, 2048, TILE, idesc(128, MN_MAJ, MN_MAJ), 4, true);
+            if (c > 0) {
+                const uint32_t sp = stage(c - 1);
+                mma_ss(tm + C_P, sp + ST_Q, TILE, 32, 16, sp + ST_K, TILE, 32, 16, idesc(64, K_MAJ, K_MAJ), 8, false);
+            }
+            commit();
+        }
+        wait_mma();
+        {
+            float x[32];
+            tmem_ld32_wait(tm + lane_off + C_DS + 32 * h, x);
+            if (c > 0) {
+                emit_dsp(x);
+            } else if (dS0) {
+#pragma unroll
+                for (int j = 0; j < 32; j += 4)
+                    *reinterpret_cast<float4*>(dS0 + srow + j) = make_float4(x[j], x[j + 1], x[j + 2], x[j + 3]);
+            }
+        }
+        if (c > 0) emit_p();
+        handoff();
+    }
+    if (warp == 1 && lane == 0) tma_store_wait_all();
+    tc_fence_before();
+    __syncthreads();
+    if (*abort) {         // a wait ran out: record it, and let every issued MMA finish before
+        if (tid == 0) atomicOr(err, kDevTimeout);   // the tensor memory is released
+        if (warp == 0) {
+            commit();
+            if (lane == 0) {
+                mbar_wait(bar + 3, mma_phase & 1, limit_ns);
+                for (int i = 0; i < kStages; ++i)   // and no copy may land after the block exits
+                    if (issued[i] > 0) mbar_wait(bar + i, (issued[i] - 1) & 1, limit_ns);
+            }
+            __syncwarp();
+        }
+    }
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tm, C_COLS);
+    }
+}
+
 }  // namespace
 
 // rows x 128 bf16 row-major (the per-chunk S and dS' tiles) as a 2-D tensor: 64-column x
@@ -746,18 +886,20 @@ cudaError_t launch_bwd_chunk(const void* q, const void* k, const void* v, const 
                                     stream, nullptr, plan);
     if (e != cudaSuccess) return e;
     // 2. the reverse chain
+    CUtensorMap mq, mk, mv, mdo, mt, ms, mdsp;
+    if (!tma_map_tokens(&mq, q, kD, T, BH) || !tma_map_tokens(&mk, k, kD, T, BH) || !tma_map_tokens(&mv, v, kD, T, BH) ||
+        !tma_map_tokens(&mdo, dO, kD, T, BH) || !tma_map_rows64(&mt, Tt, std::max<long>(1, ntiles) * kC) ||
+        !tma_map_rows128(&ms, states, std::max<long>(1, ntiles) * kD) ||
+        !tma_map_rows128(&mdsp, dSp, std::max<long>(1, ntiles) * kD))
+        return cudaErrorInvalidValue;
     static std::atomic<uint64_t> smem_chain{0}, smem_tile{0};
-    e = set_smem_limit_once(bwd_chain_kernel, (int)ChainSmem::BYTES, smem_chain);
+    e = set_smem_limit_once(bwd_chain_kernel, (int)rc::SMEM_BYTES, smem_chain);
     if (e != cudaSuccess) return e;
-    bwd_chain_kernel<<<(unsigned)(BH * 2), 256, ChainSmem::BYTES, stream>>>(
-        (const bf16*)q, (const bf16*)k, (const bf16*)dO, Tt, dST, dSp, dS0, T);
+    bwd_chain_kernel<<<(unsigned)(BH * 2), 256, rc::SMEM_BYTES, stream>>>(mq, mk, mdo, mt, mdsp, dST, dS0, T, err,
+                                                                          kTileWaitNs);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     // 3. every chunk's gradients
-    CUtensorMap mq, mk, mv, mdo, ms, mdsp;
-    if (!tma_map_tokens(&mq, q, kD, T, BH) || !tma_map_tokens(&mk, k, kD, T, BH) || !tma_map_tokens(&mv, v, kD, T, BH) ||
-        !tma_map_tokens(&mdo, dO, kD, T, BH) || !tma_map_rows128(&ms, states, ntiles * kD) ||
-        !tma_map_rows128(&mdsp, dSp, ntiles * kD))
-        return cudaErrorInvalidValue;
+    if (ntiles == 0) return cudaSuccess;
     e = set_smem_limit_once(bwd_tile_kernel, (int)tb::SMEM_BYTES, smem_tile);
     if (e != cudaSuccess) return e;
     bwd_tile_kernel<<<(unsigned)ntiles, 256, tb::SMEM_BYTES, stream>>>(
