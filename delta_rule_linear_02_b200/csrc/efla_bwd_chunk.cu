@@ -37,6 +37,12 @@ namespace {
 using bf16 = __nv_bfloat16;
 constexpr int kD = 128, kC = 64;
 
+// The extents of the buffers the two backward kernels address directly (checked builds test
+// each access against them; see efla_common.cuh).
+struct BwdSpans {
+    Span beta, dq, dk, dv, dbeta, dst, ds0;
+};
+
 // ============================================================================ per-chunk gradients
 // One CTA (8 warps) per (stream, chunk), every product on the 5th-generation tensor cores
 // (tcgen05, bf16 operands in shared memory, fp32 accumulators in tensor memory).
@@ -270,7 +276,8 @@ bwd_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                 const __grid_constant__ CUtensorMap tm_s, const __grid_constant__ CUtensorMap tm_dsp,
                 const bf16* __restrict__ beta, float* __restrict__ dq, float* __restrict__ dk, float* __restrict__ dv,
-                float* __restrict__ dbeta, int T, int rule, uint32_t* __restrict__ err, unsigned long long limit_ns) {
+                float* __restrict__ dbeta, int T, int rule, uint32_t* __restrict__ err, unsigned long long limit_ns,
+                BwdSpans spans) {
     using namespace tb;
     using namespace sm100;
     extern __shared__ uint8_t smem_raw[];
@@ -321,7 +328,8 @@ bwd_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         tma_load_2d(sm + SS, &tm_s, rest, 0, (int)(tile * 128));
         tma_load_2d(sm + SS + 2 * TILE, &tm_s, rest, 64, (int)(tile * 128));
     }
-    const float beta_t = tid < nv ? __bfloat162float(beta[row0 + tid]) : 0.f;   // in flight during the setup
+    const float beta_t = tid < nv && span_ok(err, spans.beta, beta + row0 + tid, 2)   // in flight during the setup
+                             ? __bfloat162float(beta[row0 + tid]) : 0.f;
     if (warp == 0) {
         tmem_alloc(tmem_slot, C_COLS);
         tmem_relinquish();
@@ -465,7 +473,8 @@ bwd_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         tmem_ld32_wait(tm + lane_off + C_DR + 32 * h, x);
 #pragma unroll
         for (int j = 0; j < 32; ++j)
-            if (32 * h + j < nv) dv[(row0 + 32 * h + j) * 128 + row] = x[j];
+            if (32 * h + j < nv && span_ok(err, spans.dv, dv + (row0 + 32 * h + j) * 128 + row, 4))
+                dv[(row0 + 32 * h + j) * 128 + row] = x[j];
 #pragma unroll
         for (int j = 0; j < 32; ++j) x[j] = -x[j];
         st_row32(sm + DSP + 2 * TILE, row, 4 * h, x);   // -dR^T, over dS' atom 1
@@ -473,7 +482,8 @@ bwd_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         tmem_ld32_wait(tm + lane_off + C_DQ + 32 * h, x);
 #pragma unroll
         for (int j = 0; j < 32; ++j)
-            if (32 * h + j < nv) dq[(row0 + 32 * h + j) * 128 + row] = x[j];
+            if (32 * h + j < nv && span_ok(err, spans.dq, dq + (row0 + 32 * h + j) * 128 + row, 4))
+                dq[(row0 + 32 * h + j) * 128 + row] = x[j];
         // dT, stored transposed (fp32): dT^T[s][t] for this thread's row t = 16 q + lane
         tmem_ld32_wait(tm + lane_off + C_SK + 32 * h, x);
         if (lane < 16) {
@@ -567,7 +577,7 @@ bwd_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     if (tid < 64) {   // dbeta; the coefficient of k in dk's gate term
         float dadb, dadl;
         gate_derivatives(rule, bt[tid], lam[tid], al[tid], &dadb, &dadl);
-        if (tid < nv) dbeta[row0 + tid] = dal[tid] * dadb;
+        if (tid < nv && span_ok(err, spans.dbeta, dbeta + row0 + tid, 4)) dbeta[row0 + tid] = dal[tid] * dadb;
         lam[tid] = 2.f * dal[tid] * dadl;
     }
     wait_mma();           // dK^T += S (-dR^T) is done (the commits are waited on in order)
@@ -584,7 +594,8 @@ bwd_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
             const int s = 32 * h + j;
-            if (s < nv) dk[(row0 + s) * 128 + row] = x[j] + lam[s] * ld_tok(sm + KQ, 2 * TILE, s, row);
+            if (s < nv && span_ok(err, spans.dk, dk + (row0 + s) * 128 + row, 4))
+                dk[(row0 + s) * 128 + row] = x[j] + lam[s] * ld_tok(sm + KQ, 2 * TILE, s, row);
         }
     }
     tc_fence_before();
@@ -647,7 +658,7 @@ __global__ void __launch_bounds__(256, 1)
 bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_do, const __grid_constant__ CUtensorMap tm_t,
                  const __grid_constant__ CUtensorMap tm_dsp, const float* __restrict__ dST, float* __restrict__ dS0,
-                 int T, uint32_t* __restrict__ err, unsigned long long limit_ns) {
+                 int T, uint32_t* __restrict__ err, unsigned long long limit_ns, BwdSpans spans) {
     using namespace rc;
     using namespace sm100;
     using tb::K_MAJ;
@@ -676,7 +687,9 @@ bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 
     if (nc == 0) {        // no tokens: dS0 = dS_T
         if (dS0)
-            for (int j = 0; j < 32; ++j) dS0[srow + j] = dST ? dST[srow + j] : 0.f;
+            for (int j = 0; j < 32; ++j)
+                if (span_ok(err, spans.ds0, dS0 + srow + j, 4))
+                    dS0[srow + j] = dST && span_ok(err, spans.dst, dST + srow + j, 4) ? dST[srow + j] : 0.f;
         return;
     }
     auto load = [&](int c) {   // chunk c's Q, K, T and dO half into stage c % 3 (one thread)
@@ -741,7 +754,8 @@ bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         float x[32];
 #pragma unroll
         for (int j = 0; j < 32; j += 4) {
-            const float4 v = dST ? *reinterpret_cast<const float4*>(dST + srow + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+            const float4 v = dST && span_ok(err, spans.dst, dST + srow + j, 16)
+                                 ? *reinterpret_cast<const float4*>(dST + srow + j) : make_float4(0.f, 0.f, 0.f, 0.f);
             x[j] = v.x; x[j + 1] = v.y; x[j + 2] = v.z; x[j + 3] = v.w;
         }
         float lo[16], hi[16];
@@ -820,7 +834,8 @@ bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             } else if (dS0) {
 #pragma unroll
                 for (int j = 0; j < 32; j += 4)
-                    *reinterpret_cast<float4*>(dS0 + srow + j) = make_float4(x[j], x[j + 1], x[j + 2], x[j + 3]);
+                    if (span_ok(err, spans.ds0, dS0 + srow + j, 16))
+                        *reinterpret_cast<float4*>(dS0 + srow + j) = make_float4(x[j], x[j + 1], x[j + 2], x[j + 3]);
             }
         }
         if (c > 0) emit_p();
@@ -892,18 +907,27 @@ cudaError_t launch_bwd_chunk(const void* q, const void* k, const void* v, const 
         !tma_map_rows128(&ms, states, std::max<long>(1, ntiles) * kD) ||
         !tma_map_rows128(&mdsp, dSp, std::max<long>(1, ntiles) * kD))
         return cudaErrorInvalidValue;
+    BwdSpans sp;
+    const size_t tok = (size_t)BH * T, sbytes = (size_t)BH * kD * kD * 4;
+    sp.beta = Span{beta, tok * 2};
+    sp.dq = Span{dq, tok * kD * 4};
+    sp.dk = Span{dk, tok * kD * 4};
+    sp.dv = Span{dv, tok * kD * 4};
+    sp.dbeta = Span{dbeta, tok * 4};
+    sp.dst = Span{dST, sbytes};
+    sp.ds0 = Span{dS0, sbytes};
     static std::atomic<uint64_t> smem_chain{0}, smem_tile{0};
     e = set_smem_limit_once(bwd_chain_kernel, (int)rc::SMEM_BYTES, smem_chain);
     if (e != cudaSuccess) return e;
     bwd_chain_kernel<<<(unsigned)(BH * 2), 256, rc::SMEM_BYTES, stream>>>(mq, mk, mdo, mt, mdsp, dST, dS0, T, err,
-                                                                          kTileWaitNs);
+                                                                          kTileWaitNs, sp);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     // 3. every chunk's gradients
     if (ntiles == 0) return cudaSuccess;
     e = set_smem_limit_once(bwd_tile_kernel, (int)tb::SMEM_BYTES, smem_tile);
     if (e != cudaSuccess) return e;
     bwd_tile_kernel<<<(unsigned)ntiles, 256, tb::SMEM_BYTES, stream>>>(
-        mq, mk, mv, mdo, ms, mdsp, (const bf16*)beta, dq, dk, dv, dbeta, T, rule, err, kTileWaitNs);
+        mq, mk, mv, mdo, ms, mdsp, (const bf16*)beta, dq, dk, dv, dbeta, T, rule, err, kTileWaitNs, sp);
     return cudaGetLastError();
 }
 

@@ -120,3 +120,20 @@ def test_backward_full_shape_every_stream(efla, cuda):
         e = rel_frob(g, r)
         print(f"full shape {nme}: {e:.3e}")
         assert e <= 2e-2, (nme, e)
+
+
+def test_chunked_backward_repeats_bitwise_and_reports_ok(efla, cuda):
+    """The chunkwise backward has no atomics and no order-dependent sums: two calls on the same
+    inputs give the same bits, and the workspace's error word stays EFLA_OK."""
+    w = W["lm1p3b_bf16"].replace(B=1, H=3, T=300)
+    inp = workloads.make_chunk_inputs(w)
+    cot = workloads.make_cotangents(w, with_state_grad=True)
+    S0 = 0.1 * torch.randn(w.B, w.H, w.dk, w.dv, generator=torch.Generator().manual_seed(w.seed + 7))
+    d = {k: (None if v is None else v.to(cuda)) for k, v in dict(inp, S0=S0, **cot).items()}
+    n = efla.efla_backward_workspace_bytes(w.B, w.H, w.T, w.dk, w.dv, torch.bfloat16)
+    ws = torch.zeros(n, dtype=torch.uint8, device=cuda)
+    a = efla.efla_backward(d["q"], d["k"], d["v"], d["beta"], d["dO"], S0=d["S0"], dS_T=d["dS_T"], workspace=ws)
+    b = efla.efla_backward(d["q"], d["k"], d["v"], d["beta"], d["dO"], S0=d["S0"], dS_T=d["dS_T"], workspace=ws)
+    assert efla.efla_workspace_status(ws) == efla.EFLA_OK
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)

@@ -1,12 +1,13 @@
-"""The checked build (libefla_checked.so, EFLA_CHECKED=1) on the tensor-core forward.
+"""The checked build (libefla_checked.so, EFLA_CHECKED=1) of the tensor-core forward and of
+the chunkwise backward.
 
 In that build the UT and chain kernels test every direct global access (loads of beta and
 the log-decay, stores of T, o, S_T, the chunk states and the segment products, loads of
-S0) and every computed shared-memory store against its buffer's extent; an access out of
+S0) and every computed shared-memory store against its buffer's extent, and the backward's
+kernels test their direct accesses (beta, dS_T, dS0 and the gradients); an access out of
 range is skipped and recorded, and efla_workspace_status then returns EFLA_ERR_BOUNDS.
-Each case below runs one path of the forward through the checked library and asserts
-that nothing was recorded and that the outputs still match the fp64 oracle (2e-2,
-relative Frobenius, bf16).
+Each case below runs one path through the checked library and asserts that nothing was
+recorded and that the outputs still match the fp64 oracle (2e-2, relative Frobenius, bf16).
 """
 import ctypes
 
@@ -115,3 +116,21 @@ def test_checked_segmented(efla_checked, cuda, segments, gated):
     else:
         o_ref, S_ref = oracle.fwd(inp["q"], inp["k"], inp["v"], inp["beta"], inp["S0"])
     assert rel_frob(o, o_ref) <= TOL[w.dtype] and rel_frob(ST, S_ref) <= TOL[w.dtype]
+
+
+def test_checked_backward(efla_checked, cuda):
+    """The chunkwise backward (bf16, d = 128) through the checked library: the reverse chain's
+    dS_T / dS0 accesses and the per-chunk kernel's beta loads and gradient stores are tested
+    against their buffers, on top of the forward kernels it reuses."""
+    efla = efla_checked
+    w = W["lm1p3b_bf16"].replace(B=1, H=2, T=150)
+    inp = workloads.make_chunk_inputs(w)
+    cot = workloads.make_cotangents(w, with_state_grad=True)
+    S0 = 0.1 * torch.randn(w.B, w.H, w.dk, w.dv, generator=torch.Generator().manual_seed(w.seed + 7))
+    d = {k: (None if v is None else v.to(cuda)) for k, v in dict(inp, S0=S0, **cot).items()}
+    ws = zeroed(efla.efla_backward_workspace_bytes(w.B, w.H, w.T, w.dk, w.dv, torch.bfloat16), cuda)
+    got = efla.efla_backward(d["q"], d["k"], d["v"], d["beta"], d["dO"], S0=d["S0"], dS_T=d["dS_T"], workspace=ws)
+    assert_clean(efla, ws)
+    ref = oracle.bwd(inp["q"], inp["k"], inp["v"], inp["beta"], cot["dO"], S0=S0, dS_T=cot["dS_T"])
+    for g, r in zip(got, ref):
+        assert rel_frob(g.cpu(), r) <= 2e-2
