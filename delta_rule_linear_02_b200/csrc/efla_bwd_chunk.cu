@@ -76,25 +76,27 @@ constexpr uint32_t SS = 98304;             // S [a0 | a1]
 constexpr uint32_t TT = 131072;            // T (bf16 [t][s]); later X^T (fp32)
 constexpr uint32_t PP = 139264;            // P, later dP (bf16 [t][s])
 constexpr uint32_t RT = 147456;            // the solve's A (fp32); then R^T (128 rows)
-constexpr uint32_t DL = 163840;            // the solve's scratch; then Delta^T (128 rows)
-constexpr uint32_t DG = 180224;            // G (bf16 [t][s]), later dG + dG^T
-constexpr int LA = 64;                     // row stride (floats) of the solve's A and scratch
+constexpr uint32_t DL = 164864;            // the solve's scratch; then Delta^T (128 rows)
+constexpr uint32_t DG = 181248;            // G (bf16 [t][s]), later dG + dG^T
+constexpr int LAA = 65;                    // row stride (floats) of the solve's A: the G epilogue writes
+                                           // one column of 32 consecutive rows per warp, conflict-free
+constexpr int LA = 64;                     // row stride of the solve's scratch
 constexpr int LX = 68;                     // row stride of the other fp32 64 x 64 tiles (16-byte rows)
 constexpr uint32_t F32 = 64 * LX * 4;      // bytes of one of them
-constexpr uint32_t FX = 188416;            // X (fp32)
+constexpr uint32_t FX = 189440;            // X (fp32)
 constexpr uint32_t FXT = TT;               // X^T
 constexpr uint32_t FW = TT + F32;          // W = dX X^T
 constexpr uint32_t FDT = V;                // dT^T, then dX^T, then dA
 constexpr uint32_t SMALL = FX + F32;       // alpha, beta, dalpha, lambda, ones, two partial sums (fp32 [64] each)
-constexpr uint32_t BAR = SMALL + 7 * 256;  // mbarriers: K and Q, MMA commits, the other inputs
-constexpr uint32_t MISC = BAR + 3 * 8;     // TMEM base, abort flag
+constexpr uint32_t BAR = SMALL + 7 * 256;  // mbarriers: the tile's inputs, MMA commits
+constexpr uint32_t MISC = BAR + 2 * 8;     // TMEM base, abort flag
 constexpr uint32_t SMEM_BYTES = MISC + 16 + 1024;
-static_assert(64 * LA * 4 <= 16384, "the solve's A and scratch fit R^T's and Delta^T's regions");
+static_assert(RT + 64 * LAA * 4 <= DL && DL + 64 * LA * 4 <= DG, "the solve's A and scratch fit R^T's and Delta^T's regions");
 static_assert(FDT + F32 <= DSP && FW + F32 <= DG, "fp32 tiles stay inside dead regions");
 static_assert(SMEM_BYTES <= 232448, "shared memory");
 // TMEM columns (fp32 accumulators, 64 columns each)
 constexpr uint32_t C_GP = 0, C_SK = 64, C_DQ = 128, C_DL = 192, C_DD = 256, C_DK = 320, C_DR = 384, C_COLS = 512;
-constexpr uint32_t KQ_BYTES = 32768, REST_BYTES = 98304;   // K and Q; V, dO, dS', S
+constexpr uint32_t LOAD_BYTES = 131072;    // K, Q, V, dO, dS', S
 
 // nk k-steps of K = 16 with A and B in shared memory; operand k-step ks starts at
 // base + (ks / 4) * atom + (ks % 4) * step (K-major: step 32 bytes inside a 64-column atom;
@@ -148,15 +150,9 @@ __device__ __forceinline__ float ld_tok(const uint8_t* tile, uint32_t atom, int 
     return __bfloat162float(*reinterpret_cast<const bf16*>(p));
 }
 
-// Element (r, j) of the solve's A and scratch (row stride LA): the column is XOR-swizzled
-// with the row's low five bits, so a warp writing one column of 32 consecutive rows hits 32
-// banks, while every read of the solve (one row's element broadcast to the warp, or one
-// row's consecutive columns) stays a single wavefront.
-__device__ __forceinline__ int sa(int r, int j) { return r * LA + (j ^ (r & 31)); }
-
-// X = (I + A)^{-1} for the 64 x 64 strictly-lower A (swizzled, see sa; only its
-// strictly-lower part is read), written in full into X (row stride LX; zeros above the
-// diagonal), Y scratch (swizzled like A).  Block doubling: the four 16 x 16 diagonal blocks by forward
+// X = (I + A)^{-1} for the 64 x 64 strictly-lower A (row stride LAA; only its strictly-lower
+// part is read), written in full into X (row stride LX; zeros above the diagonal), Y scratch
+// (row stride LA).  Block doubling: the four 16 x 16 diagonal blocks by forward
 // substitution (one thread per column), then merges X21 = -X22 (A21 X11) at 32 and 64.  In
 // the 64 merge each thread keeps four rows of one column in registers (one operand load
 // per four FMAs).  256 threads; ends with a barrier.
@@ -171,7 +167,7 @@ __device__ __forceinline__ void unit_lower_inverse64(const float* __restrict__ A
         for (int i = 1; i < 16; ++i) {
             float s = 0.f;
 #pragma unroll
-            for (int j = 0; j < i; ++j) s = fmaf(A[sa(16 * b + i, 16 * b + j)], x[j], s);
+            for (int j = 0; j < i; ++j) s = fmaf(A[(16 * b + i) * LAA + 16 * b + j], x[j], s);
             if (i > c) x[i] = -s;
         }
         float* Xb = X + (16 * b) * LX + 16 * b + c;
@@ -191,11 +187,11 @@ __device__ __forceinline__ void unit_lower_inverse64(const float* __restrict__ A
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
             const float xv = X[(c0 + j) * LX + c0 + c];
-            y0 = fmaf(A[sa(r0 + i, c0 + j)], xv, y0);
-            y1 = fmaf(A[sa(r0 + i + 8, c0 + j)], xv, y1);
+            y0 = fmaf(A[(r0 + i) * LAA + c0 + j], xv, y0);
+            y1 = fmaf(A[(r0 + i + 8) * LAA + c0 + j], xv, y1);
         }
-        Y[sa(r0 + i, c0 + c)] = y0;
-        Y[sa(r0 + i + 8, c0 + c)] = y1;
+        Y[(r0 + i) * LA + c0 + c] = y0;
+        Y[(r0 + i + 8) * LA + c0 + c] = y1;
     }
     __syncthreads();
     {
@@ -204,7 +200,7 @@ __device__ __forceinline__ void unit_lower_inverse64(const float* __restrict__ A
         float x0 = 0.f, x1 = 0.f;
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
-            const float yv = Y[sa(r0 + j, c0 + c)];
+            const float yv = Y[(r0 + j) * LA + c0 + c];
             x0 = fmaf(X[(r0 + i) * LX + r0 + j], yv, x0);
             x1 = fmaf(X[(r0 + i + 8) * LX + r0 + j], yv, x1);
         }
@@ -219,17 +215,17 @@ __device__ __forceinline__ void unit_lower_inverse64(const float* __restrict__ A
         for (int j = 0; j < 32; ++j) {
             const float xv = X[j * LX + c];
 #pragma unroll
-            for (int k = 0; k < 4; ++k) y[k] = fmaf(A[sa(32 + i0 + 8 * k, j)], xv, y[k]);
+            for (int k = 0; k < 4; ++k) y[k] = fmaf(A[(32 + i0 + 8 * k) * LAA + j], xv, y[k]);
         }
 #pragma unroll
-        for (int k = 0; k < 4; ++k) Y[sa(32 + i0 + 8 * k, c)] = y[k];
+        for (int k = 0; k < 4; ++k) Y[(32 + i0 + 8 * k) * LA + c] = y[k];
     }
     __syncthreads();
     {   // X21 = -X22 Y21
         float x[4] = {};
 #pragma unroll 8
         for (int j = 0; j < 32; ++j) {
-            const float yv = Y[sa(32 + j, c)];
+            const float yv = Y[(32 + j) * LA + c];
 #pragma unroll
             for (int k = 0; k < 4; ++k) x[k] = fmaf(X[(32 + i0 + 8 * k) * LX + 32 + j], yv, x[k]);
         }
@@ -283,7 +279,7 @@ bwd_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sb = smem_u32(sm);
-    uint64_t* bar = reinterpret_cast<uint64_t*>(sm + BAR);    // 0: K and Q, 1: MMA commits, 2: V, dO, dS', S
+    uint64_t* bar = reinterpret_cast<uint64_t*>(sm + BAR);    // 0: the tile's inputs, 1: MMA commits
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + MISC);
     volatile int* abort = reinterpret_cast<volatile int*>(sm + MISC + 4);
     float* fA = reinterpret_cast<float*>(sm + RT);
@@ -309,16 +305,14 @@ bwd_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     if (tid == 0) {
         mbar_init(bar, 1);
         mbar_init(bar + 1, 1);
-        mbar_init(bar + 2, 1);
         *abort = 0;
         fence_mbar_init();
-        mbar_arrive_expect_tx(bar, KQ_BYTES);
+        mbar_arrive_expect_tx(bar, LOAD_BYTES);
         tma_load_3d(sm + KQ, &tm_k, bar, 0, t0, (int)bh);
         tma_load_3d(sm + KQ + 2 * TILE, &tm_k, bar, 64, t0, (int)bh);
         tma_load_3d(sm + KQ + TILE, &tm_q, bar, 0, t0, (int)bh);
         tma_load_3d(sm + KQ + 3 * TILE, &tm_q, bar, 64, t0, (int)bh);
-        uint64_t* rest = bar + 2;
-        mbar_arrive_expect_tx(rest, REST_BYTES);
+        uint64_t* rest = bar;   // one barrier for all of the tile's inputs
         tma_load_3d(sm + V, &tm_v, rest, 0, t0, (int)bh);
         tma_load_3d(sm + V + TILE, &tm_v, rest, 64, t0, (int)bh);
         tma_load_3d(sm + DO, &tm_do, rest, 0, t0, (int)bh);
@@ -361,10 +355,15 @@ bwd_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         tc_fence_after();
     };
 
-    // ---- 1. [G; P~] = [K; Q] K^T, as soon as K and Q have landed
+    // ---- 1. [G; P~] = [K; Q] K^T;  dDelta^T = dS'^T K^T (+ dO^T P below);  S^T K^T;  dQ^T = S dO^T
     wait(0, 0);
     if (warp == 0) {
         mma_ss(tm + C_GP, sb + KQ, 2 * TILE, 32, 16, sb + KQ, 2 * TILE, 32, 16, idesc(128, K_MAJ, K_MAJ), 8, false);
+        mma_ss(tm + C_DD, sb + DSP, TILE, 2048, 2 * TILE, sb + KQ, 2 * TILE, 32, 16, idesc(128, MN_MAJ, K_MAJ), 8,
+               false);
+        mma_ss(tm + C_SK, sb + SS, TILE, 2048, 2 * TILE, sb + KQ, 2 * TILE, 32, 16, idesc(128, MN_MAJ, K_MAJ), 8,
+               false);
+        mma_ss(tm + C_DQ, sb + SS, 2 * TILE, 32, 16, sb + DO, TILE, 32, 16, idesc(128, K_MAJ, K_MAJ), 8, false);
         commit();
     }
     wait_mma();
@@ -393,20 +392,13 @@ bwd_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
             const int s = 32 * h + j;
-            fA[sa(row, s)] = s < row ? a * g[j] : 0.f;
+            fA[row * LAA + s] = s < row ? a * g[j] : 0.f;
         }
     }
     handoff();
-    // ---- 2. while the CUDA cores solve for X = (I + A)^{-1}:
-    //         dDelta^T = dS'^T K^T + dO^T P;  S^T K^T;  dQ^T = S dO^T
-    wait(2, 0);
+    // ---- 2. dDelta^T += dO^T P, while the CUDA cores solve for X = (I + A)^{-1}
     if (warp == 0) {
-        mma_ss(tm + C_DD, sb + DSP, TILE, 2048, 2 * TILE, sb + KQ, 2 * TILE, 32, 16, idesc(128, MN_MAJ, K_MAJ), 8,
-               false);
         mma_ss(tm + C_DD, sb + DO, TILE, 2048, TILE, sb + PP, TILE, 2048, TILE, idesc(128, MN_MAJ, MN_MAJ), 4, true);
-        mma_ss(tm + C_SK, sb + SS, TILE, 2048, 2 * TILE, sb + KQ, 2 * TILE, 32, 16, idesc(128, MN_MAJ, K_MAJ), 8,
-               false);
-        mma_ss(tm + C_DQ, sb + SS, 2 * TILE, 32, 16, sb + DO, TILE, 32, 16, idesc(128, K_MAJ, K_MAJ), 8, false);
         commit();
     }
     unit_lower_inverse64(fA, fX, fY, tid);            // ends with a barrier: A and the scratch are dead
@@ -416,7 +408,7 @@ bwd_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
         for (int j = 0; j < 16; ++j) x[j] = fX[t * LX + s0 + j] * al[s0 + j];
         st_row16(sm + TT, t, 2 * (tid & 3), x);
-        wait_mma();       // the products of step 2 have landed
+        wait_mma();       // dO^T P has landed
         float r[32];
         tmem_ld32_wait(tm + lane_off + C_SK + 32 * h, r);
 #pragma unroll
@@ -607,7 +599,6 @@ bwd_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if (lane == 0) {
                 mbar_wait(bar + 1, mma_phase & 1, limit_ns);
                 mbar_wait(bar, 0, limit_ns);        // and no copy may land after the block exits
-                mbar_wait(bar + 2, 0, limit_ns);
             }
             __syncwarp();
         }
