@@ -631,18 +631,6 @@ constexpr uint32_t MISC = BAR + 4 * 8;     // TMEM base, abort flag, loads issue
 constexpr uint32_t SMEM_BYTES = MISC + 32 + 1024;
 static_assert(SMEM_BYTES <= 232448, "shared memory");
 constexpr uint32_t C_DS = 0, C_P = 64, C_DD = 128, C_DR = 192, C_COLS = 256;
-
-// 2-D tiled store of one box from shared memory (bulk-group completion; no multicast)
-__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src, int c0, int c1) {
-    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
-                     reinterpret_cast<uint64_t>(map)),
-                 "r"(sm100::smem_u32(src)), "r"(c0), "r"(c1)
-                 : "memory");
-    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-}
-// the shared-memory source of every earlier store has been read / every earlier store is done
-__device__ __forceinline__ void tma_store_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
-__device__ __forceinline__ void tma_store_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 }  // namespace rc
 
 __global__ void __launch_bounds__(256, 1)
@@ -854,20 +842,6 @@ bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 }
 
 }  // namespace
-
-// rows x 128 bf16 row-major (the per-chunk S and dS' tiles) as a 2-D tensor: 64-column x
-// 128-row boxes, 128-byte swizzle (one box is one 64-column atom of a 128 x 128 tile).
-static bool tma_map_rows128(CUtensorMap* map, const void* ptr, long rows) {
-    auto fn = tma_encode_fn();
-    if (!fn) return false;
-    cuuint64_t dims[2] = {128, (cuuint64_t)rows};
-    cuuint64_t strides[1] = {256};
-    cuuint32_t box[2] = {64, 128};
-    cuuint32_t estr[2] = {1, 1};
-    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
 
 constexpr unsigned long long kTileWaitNs = 2000000000ull;   // 2 s per wait
 

@@ -222,6 +222,7 @@ template <bool kGated>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_t,
+                const __grid_constant__ CUtensorMap tm_st,
                 const float* __restrict__ S0, __nv_bfloat16* __restrict__ o, float* __restrict__ S_T,
                 Seqs seqs, int Tdim, uint32_t* __restrict__ err, unsigned long long limit_ns,
                 const float* __restrict__ gl_all, long ntiles, SegPlan seg, ChainSpans spans) {
@@ -419,12 +420,20 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             tc_fence_after();
             mma_ts(tmem + TM_X, tmem + TM_AWQ, sb + OFF_SB, 4 * 2048, 2048, TILE, ID_N64, 8, 0);
             mma_commit_elect(ctl.b(B_XS_FULL));
+            if (seg.states && lane == 0) {   // chunk c's entering state, for the backward: one TMA store
+                const long srow = (jb.tile0 + c) * kD;
+                if (span_ok(err, spans.states, seg.states + (srow + kD) * kD - 1, 2))
+                    tma_store_2d(&tm_st, sm + OFF_SB, col0, (int)srow);
+            }
+            __syncwarp();
             // this chunk's Q K^T (its Q has been in place since the last chunk) runs while
             // Delta is formed
             if (!(ok = c == 0 || wait(B_GP_FREE, (c - 1) & 1))) break;
             issue_qk(c, 0, 8);
             // S += K^T Delta (state chain)
             if (!(ok = wait(B_D_READY, c & 1))) break;
+            if (seg.states && lane == 0) tma_store_wait_read();   // the bf16 S is rewritten after this product
+            __syncwarp();
             tc_fence_after();
             mma_ss(tmem + TM_S, sb + kvt(c) + KVT_K, 4 * 2048, 2048, TILE, sb + L::OFF_DL2, 4 * 2048, 2048, TILE,
                    ID_S, 4, 1);
@@ -444,7 +453,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
         }
         mma_commit_elect(ctl.b(B_DRAIN));
-        if (lane == 0) mbar_wait(ctl.b(B_DRAIN), 0, limit_ns);
+        if (lane == 0) {
+            mbar_wait(ctl.b(B_DRAIN), 0, limit_ns);
+            if (seg.states) tma_store_wait_all();
+        }
         __syncwarp();
     } else if (warp == 4 || warp == 5) {
         // ================================================================ W -> A operand (quarters 0-1)
@@ -637,13 +649,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     st_chunk(sm + OFF_SB + sw128_off(ct, 4 * ch + 2 * qd), s16);
                     st_chunk(sm + OFF_SB + sw128_off(ct, 4 * ch + 2 * qd + 1), s16 + 8);
                 }
-                if (seg.states) {   // chunk 0's entering state, for the backward
-                    uint8_t* dst = reinterpret_cast<uint8_t*>(seg.states + ((size_t)jb.tile0 * kD + ct) * kD + col0 + cc + 16 * qd);
-                    if (span_ok(err, spans.states, dst, 32)) {
-                        st_chunk(dst, s16);
-                        st_chunk(dst + 16, s16 + 8);
-                    }
-                }
                 if constexpr (kGated) {
 #pragma unroll
                     for (int j = 0; j < 16; ++j) s16[j] *= dec0;
@@ -702,13 +707,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 for (int j = 0; j < 4; ++j)
                     if (smem_ok(err, OFF_SB + sw128_off(ct, 4 * ch + j), 16, OFF_SB + 2 * TILE))
                         st_chunk(sm + OFF_SB + sw128_off(ct, 4 * ch + j), t + 8 * j);
-                if (seg.states && c + 1 < nchunks) {   // chunk c+1's entering state, for the backward
-                    uint8_t* dst = reinterpret_cast<uint8_t*>(seg.states + ((size_t)(jb.tile0 + c + 1) * kD + ct) * kD + col0 + cc);
-                    if (span_ok(err, spans.states, dst, 64)) {
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) st_chunk(dst + 16 * j, t + 8 * j);
-                    }
-                }
                 if (c == nchunks - 1 && stp && span_ok(err, st_span, stp + (size_t)ct * kD + col0 + cc, 128)) {
                     float* dst = stp + (size_t)ct * kD + col0 + cc;
 #pragma unroll
@@ -787,9 +785,10 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const v
     sp.states = Span{seg.states, (size_t)ntiles * kD * kD * 2};
     sp.gl = Span{g ? static_cast<const char*>(scratch) + ntiles * 8192 * 2 : nullptr, (size_t)ntiles * 256};
     sp.t_rows = (g ? 2 : 1) * ntiles * 64;
-    CUtensorMap mq, mk, mv, mt;
+    CUtensorMap mq, mk, mv, mt, mst;
     if (!tma_map_tokens(&mq, q, kD, Tdim, Z) || !tma_map_tokens(&mk, k, kD, Tdim, Z) ||
-        !tma_map_tokens(&mv, v, kD, Tdim, Z) || !tma_map_rows64(&mt, scratch, std::max<long>(1, (g ? 2 : 1) * ntiles) * 64))
+        !tma_map_tokens(&mv, v, kD, Tdim, Z) || !tma_map_rows64(&mt, scratch, std::max<long>(1, (g ? 2 : 1) * ntiles) * 64) ||
+        !(seg.states ? tma_map_rows128(&mst, seg.states, std::max<long>(1, ntiles) * kD) : (mst = mt, true)))
         return cudaErrorInvalidValue;
     if (g) {
         const float* gl = reinterpret_cast<const float*>(static_cast<const char*>(scratch) + ntiles * 8192 * 2);
@@ -797,14 +796,14 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const v
         e = set_smem_limit_once(chunk_tc_kernel<true>, (int)Lay<true>::SMEM_BYTES, smem_set_g);
         if (e != cudaSuccess) return e;
         chunk_tc_kernel<true><<<(unsigned)ctas, kThreads, Lay<true>::SMEM_BYTES, stream>>>(
-            mq, mk, mv, mt, S0, (__nv_bfloat16*)o, S_T, seqs, Tdim, err, kWaitLimitNs, gl, ntiles, seg, sp);
+            mq, mk, mv, mt, mst, S0, (__nv_bfloat16*)o, S_T, seqs, Tdim, err, kWaitLimitNs, gl, ntiles, seg, sp);
         return cudaGetLastError();
     }
     static std::atomic<uint64_t> smem_set{0};
     e = set_smem_limit_once(chunk_tc_kernel<false>, (int)Lay<false>::SMEM_BYTES, smem_set);
     if (e != cudaSuccess) return e;
     chunk_tc_kernel<false><<<(unsigned)ctas, kThreads, Lay<false>::SMEM_BYTES, stream>>>(
-        mq, mk, mv, mt, S0, (__nv_bfloat16*)o, S_T, seqs, Tdim, err, kWaitLimitNs, nullptr, ntiles, seg, sp);
+        mq, mk, mv, mt, mst, S0, (__nv_bfloat16*)o, S_T, seqs, Tdim, err, kWaitLimitNs, nullptr, ntiles, seg, sp);
     return cudaGetLastError();
 }
 

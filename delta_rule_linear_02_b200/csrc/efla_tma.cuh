@@ -45,4 +45,18 @@ inline bool tma_map_rows64(CUtensorMap* map, const void* ptr, long rows) {
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// rows x 128 bf16 row-major (per-chunk 128 x 128 tiles stacked) as a 2-D tensor, 64-column x
+// 128-row boxes, 128-byte swizzle: one box is one 64-column half of a 128 x 128 tile.
+inline bool tma_map_rows128(CUtensorMap* map, const void* ptr, long rows) {
+    auto fn = tma_encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {128, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {256};
+    cuuint32_t box[2] = {64, 128};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace efla
