@@ -603,7 +603,43 @@ def main():
                # bf16, d = 128: the UT kernel, the forward chain storing states, the reverse chain and
                # the per-chunk gradient kernel per call
                "gpu_launches": 4 * args.bwd_steps}
-        del xb, dOb, gb, wsb
+        # training with saved residuals: the forward keeps T and every chunk's entering state
+        # (efla_chunk_fwd_save) and the backward reads them instead of recomputing them
+        ob = torch.empty(B, H, T, d, device=dev, dtype=wb.dtype)
+        _, _, saved = efla.efla_chunk_fwd_save(xb["q"], xb["k"], xb["v"], xb["beta"], o=ob, want_state=False,
+                                               stream=stream)
+        wss = torch.zeros(efla.lib.efla_backward_saved_workspace_bytes(B, H, T, d, d, efla.EFLA_DTYPE_BF16),
+                          dtype=torch.uint8, device=dev)
+        call_fs = lambda: efla.efla_chunk_fwd_save(xb["q"], xb["k"], xb["v"], xb["beta"], o=ob, want_state=False,
+                                                   saved=saved, stream=stream)
+        call_bs = lambda: efla.efla_backward_saved(xb["q"], xb["k"], xb["v"], xb["beta"], dOb, saved, grads=gb,
+                                                   workspace=wss, stream=stream)
+
+        def timed(fn, steps):
+            for _ in range(args.warmup):
+                fn()
+            barrier(world)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(steps):
+                fn()
+            e1.record(stream)
+            barrier(world)
+            return max_over_ranks(e0.elapsed_time(e1), world) / steps
+
+        bs_ms = timed(call_bs, args.bwd_steps)
+        ts_ms = timed(lambda: (call_fs(), call_bs()), args.bwd_steps)
+        bsrf = roofline_record(bbytes, bflops, bs_ms * 1e-3, hbm, tc, peak_kind)
+        bwd["saved_residuals"] = {
+            "what": "efla_backward_saved: the same gradients from T and the chunk states that "
+                    "efla_chunk_fwd_save kept (no forward recompute)",
+            "ms_per_step": bs_ms, "value": wb.tokens * world / (bs_ms * 1e-3), "unit": "tokens/s",
+            "roofline": bsrf, "gpu_launches": 2 * args.bwd_steps}
+        bwd["train_step"] = {
+            "what": "efla_chunk_fwd_save then efla_backward_saved, one training step of the layer's recurrence",
+            "ms_per_step": ts_ms, "value": wb.tokens * world / (ts_ms * 1e-3), "unit": "tokens/s",
+            "gpu_launches": 4 * args.bwd_steps}
+        del xb, dOb, gb, wsb, ob, saved, wss
 
     # ---- the other forward workloads (long context, stiff keys): tokens/s and roofline
     # fraction of a few forwards each, inputs resident in HBM, CUDA events around the calls

@@ -82,6 +82,14 @@ def _load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.efla_backward.restype = I
     lib.efla_backward_ex.argtypes = [vp] * 12 + [I, I, I, I, I, I, I, vp, Z, vp]
     lib.efla_backward_ex.restype = I
+    lib.efla_train_saved_bytes.argtypes = [I, I, I, I, I, I, I]
+    lib.efla_train_saved_bytes.restype = Z
+    lib.efla_chunk_fwd_save.argtypes = [vp] * 7 + [I] * 8 + [vp, Z, vp]
+    lib.efla_chunk_fwd_save.restype = I
+    lib.efla_backward_saved_workspace_bytes.argtypes = [I, I, I, I, I, I]
+    lib.efla_backward_saved_workspace_bytes.restype = Z
+    lib.efla_backward_saved.argtypes = [vp] * 11 + [I] * 7 + [vp, Z, vp, Z, vp]
+    lib.efla_backward_saved.restype = I
     return lib
 
 
@@ -297,6 +305,71 @@ def efla_chunk_fwd_varlen(q, k, v, beta, cu_seqlens, S0=None, g=None, chunk: int
     return o, S_T
 
 
+def efla_train_saved_bytes(B, H, T, d_k, d_v, chunk=CHUNK, dtype=torch.bfloat16) -> int:
+    return int(lib.efla_train_saved_bytes(B, H, T, d_k, d_v, chunk, _DTYPES.get(dtype, -1)))
+
+
+def efla_chunk_fwd_save(q, k, v, beta, S0=None, saved=None, o=None, S_T=None, want_state: bool = True,
+                        stream=None, rule: int = EFLA_RULE_EXACT):
+    """efla_chunk_fwd that also keeps the residuals efla_backward_saved needs (bf16, d = 128).
+    Returns (o, S_T or None, saved); `saved` is a uint8 tensor of efla_train_saved_bytes."""
+    dt = k.dtype
+    for t, nme in ((q, "q"), (k, "k"), (v, "v"), (beta, "beta")):
+        _check(t, nme, dt)
+    B, H, T, d_k = k.shape
+    d_v = v.shape[-1]
+    if S0 is not None:
+        _check(S0, "S0", torch.float32)
+    if o is None:
+        o = torch.empty((B, H, T, d_v), device=k.device, dtype=dt)
+    _check(o, "o", dt)
+    if S_T is None and want_state:
+        S_T = torch.empty((B, H, d_k, d_v), device=k.device, dtype=torch.float32)
+    if S_T is not None:
+        _check(S_T, "S_T", torch.float32)
+    if saved is None:
+        n = efla_train_saved_bytes(B, H, T, d_k, d_v, CHUNK, dt)
+        if n == 0:
+            raise EflaError(EFLA_ERR_UNSUPPORTED, "efla_train_saved_bytes")
+        saved = torch.zeros(n, dtype=torch.uint8, device=k.device)
+    st = lib.efla_chunk_fwd_save(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(S0), _ptr(o), _ptr(S_T),
+                                 B, H, T, d_k, d_v, CHUNK, _DTYPES.get(dt, -1), int(rule), _ptr(saved),
+                                 saved.numel(), _stream(stream))
+    _raise(st, "efla_chunk_fwd_save")
+    return o, S_T, saved
+
+
+def efla_backward_saved(q, k, v, beta, dO, saved, dS_T=None, want_dS0: bool = True, grads=None,
+                        workspace=None, stream=None, rule: int = EFLA_RULE_EXACT):
+    """efla_backward from the residuals efla_chunk_fwd_save kept (no forward recompute).
+    Returns (dq, dk, dv, dbeta, dS0 or None), all float32."""
+    dt = k.dtype
+    for t, nme in ((q, "q"), (k, "k"), (v, "v"), (beta, "beta"), (dO, "dO")):
+        _check(t, nme, dt)
+    B, H, T, d_k = k.shape
+    d_v = v.shape[-1]
+    if dS_T is not None:
+        _check(dS_T, "dS_T", torch.float32)
+    f32 = dict(device=k.device, dtype=torch.float32)
+    if grads is None:
+        grads = (torch.empty((B, H, T, d_k), **f32), torch.empty((B, H, T, d_k), **f32),
+                 torch.empty((B, H, T, d_v), **f32), torch.empty((B, H, T), **f32),
+                 torch.empty((B, H, d_k, d_v), **f32) if want_dS0 else None)
+    for t, nme in zip(grads, ("dq", "dk", "dv", "dbeta", "dS0")):
+        if t is not None:
+            _check(t, nme, torch.float32)
+    if workspace is None:
+        n = int(lib.efla_backward_saved_workspace_bytes(B, H, T, d_k, d_v, _DTYPES.get(dt, -1)))
+        if n == 0:
+            raise EflaError(EFLA_ERR_UNSUPPORTED, "efla_backward_saved_workspace_bytes")
+        workspace = torch.zeros(n, dtype=torch.uint8, device=k.device)
+    st = lib.efla_backward_saved(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(dO), _ptr(dS_T),
+                                 *(_ptr(g) for g in grads), B, H, T, d_k, d_v, _DTYPES.get(dt, -1), int(rule),
+                                 _ptr(saved), saved.numel(), _ptr(workspace), workspace.numel(), _stream(stream))
+    _raise(st, "efla_backward_saved")
+    return grads
+
+
 def efla_chunk_fwd_noalloc(q, k, v, beta, S0=None, chunk: int = CHUNK, o=None, S_T=None,
                            want_state: bool = True, stream=None
                            ) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
@@ -394,6 +467,6 @@ def efla_backward(q, k, v, beta, dO, S0=None, dS_T=None, want_dS0: bool = True, 
     return grads
 
 
-__all__ = ["efla_chunk_fwd_segmented", "efla_chunk_fwd_varlen", "efla_chunk_fwd_gated", "efla_recurrent_step_gated", "efla_backward", "efla_backward_workspace_bytes", "EFLA_RULE_EXACT", "EFLA_RULE_EULER", "efla_gate", "efla_chunk_fwd", "efla_chunk_fwd_noalloc", "efla_chunk_fwd_workspace_bytes", "efla_recurrent_step",
+__all__ = ["efla_train_saved_bytes", "efla_chunk_fwd_save", "efla_backward_saved", "efla_chunk_fwd_segmented", "efla_chunk_fwd_varlen", "efla_chunk_fwd_gated", "efla_recurrent_step_gated", "efla_backward", "efla_backward_workspace_bytes", "EFLA_RULE_EXACT", "EFLA_RULE_EULER", "efla_gate", "efla_chunk_fwd", "efla_chunk_fwd_noalloc", "efla_chunk_fwd_workspace_bytes", "efla_recurrent_step",
            "efla_workspace_status", "efla_noalloc_status", "efla_status_string", "load_checked", "efla_selftest_wait_timeout", "new_workspace", "EflaError", "lib",
            "LIB_PATH", "CHUNK"]

@@ -79,12 +79,14 @@ size_t efla_chunk_fwd_gated_workspace_bytes(int B, int H, int T, int d_k, int d_
 static int chunk_fwd_impl(const void* q, const void* k, const void* v, const void* beta, const float* g,
                           const float* S0, void* o, float* S_T, int B, int H, int T, int d_k, int d_v,
                           int chunk, int dtype, int rule, void* workspace, size_t workspace_bytes,
-                          efla_stream_t stream) {
+                          efla_stream_t stream, bool save = false) {
     int st = check_chunk_shape(B, H, T, d_k, d_v, chunk, dtype);
     if (st != EFLA_OK) return st;
     if (rule != EFLA_RULE_EXACT && rule != EFLA_RULE_EULER) return EFLA_ERR_INVALID_ARG;
-    const size_t need = g ? efla_chunk_fwd_gated_workspace_bytes(B, H, T, d_k, d_v, chunk, dtype)
-                          : efla_chunk_fwd_workspace_bytes(B, H, T, d_k, d_v, chunk, dtype);
+    if (save && (g || dtype != EFLA_DTYPE_BF16 || d_k != 128)) return EFLA_ERR_UNSUPPORTED;
+    const size_t need = save ? efla_train_saved_bytes(B, H, T, d_k, d_v, chunk, dtype)
+                      : g    ? efla_chunk_fwd_gated_workspace_bytes(B, H, T, d_k, d_v, chunk, dtype)
+                             : efla_chunk_fwd_workspace_bytes(B, H, T, d_k, d_v, chunk, dtype);
     if (!workspace || !aligned16(workspace) || workspace_bytes < need) return EFLA_ERR_INVALID_ARG;
     const long BH = (long)B * H;
     if (BH == 0) return EFLA_OK;
@@ -119,10 +121,13 @@ static int chunk_fwd_impl(const void* q, const void* k, const void* v, const voi
         overlaps(workspace, workspace_bytes, g, ng))
         return EFLA_ERR_INVALID_ARG;
     efla::Seqs seqs{nullptr, nullptr, 0, 0, T, 0};
-    if (dtype == EFLA_DTYPE_BF16 && d_k == 128)
+    if (dtype == EFLA_DTYPE_BF16 && d_k == 128) {
+        char* scratch = static_cast<char*>(workspace) + kWorkspaceHeader;
+        efla::SegPlan plan;   // training: every chunk's entering state after the transforms
+        if (save) plan.states = reinterpret_cast<__nv_bfloat16*>(scratch + efla::bwd_saved_t_bytes(BH, T));
         return from_cuda(efla::launch_chunk_tc(q, k, v, beta, S0, o, S_T, seqs, BH, BH, T, BH * ((T + 63) / 64),
-                                               static_cast<uint32_t*>(workspace),
-                                               static_cast<char*>(workspace) + kWorkspaceHeader, rule, s, g));
+                                               static_cast<uint32_t*>(workspace), scratch, rule, s, g, plan));
+    }
     return from_cuda(efla::launch_chunk_simt(q, k, v, beta, S0, o, S_T, seqs, BH, T, d_k,
                                              dtype == EFLA_DTYPE_BF16, rule, s, g));
 }
@@ -509,6 +514,75 @@ int efla_backward_ex(const void* q, const void* k, const void* v, const void* be
                                                 static_cast<char*>(workspace) + kWorkspaceHeader, s));
     return from_cuda(efla::launch_bwd(q, k, v, beta, S0, dO, dS_T, dq, dk, dv, dbeta, dS0, BH, T, d_k,
                                       dtype == EFLA_DTYPE_BF16, rule, workspace, s));
+}
+
+// ---------------------------------------------------------------- training: saved residuals
+size_t efla_train_saved_bytes(int B, int H, int T, int d_k, int d_v, int chunk, int dtype) {
+    if (check_chunk_shape(B, H, T, d_k, d_v, chunk, dtype) != EFLA_OK) return 0;
+    if (dtype != EFLA_DTYPE_BF16 || d_k != 128) return 0;
+    const long BH = (long)B * H;
+    return kWorkspaceHeader + efla::bwd_saved_t_bytes(BH, T) + efla::bwd_saved_state_bytes(BH, T);
+}
+
+int efla_chunk_fwd_save(const void* q, const void* k, const void* v, const void* beta, const float* S0, void* o,
+                        float* S_T, int B, int H, int T, int d_k, int d_v, int chunk, int dtype, int rule,
+                        void* saved, size_t saved_bytes, efla_stream_t stream) {
+    if (check_chunk_shape(B, H, T, d_k, d_v, chunk, dtype) == EFLA_OK && (dtype != EFLA_DTYPE_BF16 || d_k != 128))
+        return EFLA_ERR_UNSUPPORTED;
+    return chunk_fwd_impl(q, k, v, beta, nullptr, S0, o, S_T, B, H, T, d_k, d_v, chunk, dtype, rule, saved,
+                          saved_bytes, stream, true);
+}
+
+size_t efla_backward_saved_workspace_bytes(int B, int H, int T, int d_k, int d_v, int dtype) {
+    if (check_bwd_shape(B, H, T, d_k, d_v, dtype) != EFLA_OK || !bwd_chunked(d_k, dtype)) return 0;
+    return kWorkspaceHeader + efla::bwd_saved_state_bytes((long)B * H, T);   // every chunk's dS'
+}
+
+int efla_backward_saved(const void* q, const void* k, const void* v, const void* beta, const void* dO,
+                        const float* dS_T, float* dq, float* dk, float* dv, float* dbeta, float* dS0, int B, int H,
+                        int T, int d_k, int d_v, int dtype, int rule, const void* saved, size_t saved_bytes,
+                        void* workspace, size_t workspace_bytes, efla_stream_t stream) {
+    int st = check_bwd_shape(B, H, T, d_k, d_v, dtype);
+    if (st != EFLA_OK) return st;
+    if (!bwd_chunked(d_k, dtype)) return EFLA_ERR_UNSUPPORTED;
+    if (rule != EFLA_RULE_EXACT && rule != EFLA_RULE_EULER) return EFLA_ERR_INVALID_ARG;
+    const long BH = (long)B * H;
+    const size_t ns = (size_t)BH * d_k * d_v * sizeof(float);
+    cudaStream_t s = (cudaStream_t)stream;
+    if ((dS_T && !aligned16(dS_T)) || (dS0 && !aligned16(dS0))) return EFLA_ERR_INVALID_ARG;
+    if (BH == 0) return EFLA_OK;
+    if (T == 0) {   // no token: the state gradient passes through
+        if (!dS0 || dS0 == dS_T) return EFLA_OK;
+        return from_cuda(dS_T ? cudaMemcpyAsync(dS0, dS_T, ns, cudaMemcpyDeviceToDevice, s)
+                              : cudaMemsetAsync(dS0, 0, ns, s));
+    }
+    const size_t need_ws = efla_backward_saved_workspace_bytes(B, H, T, d_k, d_v, dtype);
+    const size_t need_saved = efla_train_saved_bytes(B, H, T, d_k, d_v, 64, dtype);
+    if (!workspace || !aligned16(workspace) || workspace_bytes < need_ws) return EFLA_ERR_INVALID_ARG;
+    if (!saved || !aligned16(saved) || saved_bytes < need_saved) return EFLA_ERR_INVALID_ARG;
+    if (!q || !k || !v || !beta || !dO || !dq || !dk || !dv || !dbeta) return EFLA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(beta) || !aligned16(dO) ||
+        !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(dbeta))
+        return EFLA_ERR_INVALID_ARG;
+    const size_t es = elem_size(dtype);
+    const size_t nqk = (size_t)BH * T * d_k * es, nv = (size_t)BH * T * d_v * es, nb = (size_t)BH * T * es;
+    const size_t gqk = (size_t)BH * T * d_k * 4, gv = (size_t)BH * T * d_v * 4, gb = (size_t)BH * T * 4;
+    // every output and the workspace must be disjoint from every input and from each other
+    const void* outs[6] = {dq, dk, dv, dbeta, dS0, workspace};
+    const size_t outn[6] = {gqk, gqk, gv, gb, ns, workspace_bytes};
+    const void* ins[7] = {q, k, v, beta, dO, dS_T, saved};
+    const size_t inn[7] = {nqk, nqk, nv, nb, nv, ns, saved_bytes};
+    for (int i = 0; i < 6; ++i) {
+        for (int j = 0; j < 7; ++j)
+            if (overlaps(outs[i], outn[i], ins[j], inn[j])) return EFLA_ERR_INVALID_ARG;
+        for (int j = i + 1; j < 6; ++j)
+            if (overlaps(outs[i], outn[i], outs[j], outn[j])) return EFLA_ERR_INVALID_ARG;
+    }
+    const char* sv = static_cast<const char*>(saved) + kWorkspaceHeader;
+    return from_cuda(efla::launch_bwd_chunk_saved(q, k, v, beta, dO, dS_T, dq, dk, dv, dbeta, dS0, BH, T, rule,
+                                                  static_cast<uint32_t*>(workspace), sv,
+                                                  sv + efla::bwd_saved_t_bytes(BH, T),
+                                                  static_cast<char*>(workspace) + kWorkspaceHeader, s));
 }
 
 int efla_backward(const void* q, const void* k, const void* v, const void* beta, const float* S0,

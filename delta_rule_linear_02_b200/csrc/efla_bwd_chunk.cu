@@ -502,18 +502,22 @@ bwd_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         commit();
     }
     // ---- 7. through T = X diag(alpha) and X = (I + A)^{-1}, fp32 on CUDA cores
-    if (tid < 64) {       // dalpha_s = sum_t dT_ts X_ts;  dX^T = diag(alpha) dT^T, in place
-        const float a = al[tid];
+    {   // dalpha_s = sum_t dT_ts X_ts;  dX^T = diag(alpha) dT^T, in place.  Row s = tid / 4,
+        // a quarter of its 64 entries per thread, the four partial sums added by shuffles.
+        const int srow = tid >> 2, t0q = 16 * (tid & 3);
+        const float a = al[srow];
         float sacc = 0.f;
-#pragma unroll 4
-        for (int t = 0; t < 64; t += 4) {
-            float4 d4 = *reinterpret_cast<const float4*>(fdT + tid * LX + t);
-            const float4 x4 = *reinterpret_cast<const float4*>(fXT + tid * LX + t);
+#pragma unroll
+        for (int t = t0q; t < t0q + 16; t += 4) {
+            float4 d4 = *reinterpret_cast<const float4*>(fdT + srow * LX + t);
+            const float4 x4 = *reinterpret_cast<const float4*>(fXT + srow * LX + t);
             sacc = fmaf(d4.x, x4.x, fmaf(d4.y, x4.y, fmaf(d4.z, x4.z, fmaf(d4.w, x4.w, sacc))));
             d4.x *= a; d4.y *= a; d4.z *= a; d4.w *= a;
-            *reinterpret_cast<float4*>(fdT + tid * LX + t) = d4;
+            *reinterpret_cast<float4*>(fdT + srow * LX + t) = d4;
         }
-        dal[tid] = sacc;
+        sacc += __shfl_xor_sync(0xffffffffu, sacc, 1);
+        sacc += __shfl_xor_sync(0xffffffffu, sacc, 2);
+        if ((tid & 3) == 0) dal[srow] = sacc;
     }
     __syncthreads();
     const int g8 = lane >> 2, t4 = lane & 3, r0 = 16 * (warp & 3), c0 = 32 * (warp >> 2);
@@ -850,6 +854,9 @@ size_t bwd_chunk_workspace_bytes(long BH, int T) {
     return (size_t)ntiles * (kC * kC + 2 * kD * kD) * sizeof(bf16);   // T, S and dS' per tile
 }
 
+size_t bwd_saved_t_bytes(long BH, int T) { return (size_t)BH * ((T + kC - 1) / kC) * kC * kC * sizeof(bf16); }
+size_t bwd_saved_state_bytes(long BH, int T) { return (size_t)BH * ((T + kC - 1) / kC) * kD * kD * sizeof(bf16); }
+
 cudaError_t launch_bwd_chunk(const void* q, const void* k, const void* v, const void* beta, const float* S0,
                              const void* dO, const float* dST, float* dq, float* dk, float* dv, float* dbeta,
                              float* dS0, long BH, int T, int rule, uint32_t* err, void* scratch, cudaStream_t stream) {
@@ -865,6 +872,18 @@ cudaError_t launch_bwd_chunk(const void* q, const void* k, const void* v, const 
     cudaError_t e = launch_chunk_tc(q, k, v, beta, S0, nullptr, nullptr, seqs, BH, BH, T, ntiles, err, Tt, rule,
                                     stream, nullptr, plan);
     if (e != cudaSuccess) return e;
+    // 2, 3. the reverse chain and every chunk's gradients
+    return launch_bwd_chunk_saved(q, k, v, beta, dO, dST, dq, dk, dv, dbeta, dS0, BH, T, rule, err, Tt, states, dSp,
+                                  stream);
+}
+
+cudaError_t launch_bwd_chunk_saved(const void* q, const void* k, const void* v, const void* beta, const void* dO,
+                                   const float* dST, float* dq, float* dk, float* dv, float* dbeta, float* dS0,
+                                   long BH, int T, int rule, uint32_t* err, const void* Tt, const void* states,
+                                   void* dSp, cudaStream_t stream) {
+    const int nchunks = (T + kC - 1) / kC;
+    const long ntiles = BH * nchunks;
+    cudaError_t e;
     // 2. the reverse chain
     CUtensorMap mq, mk, mv, mdo, mt, ms, mdsp;
     if (!tma_map_tokens(&mq, q, kD, T, BH) || !tma_map_tokens(&mk, k, kD, T, BH) || !tma_map_tokens(&mv, v, kD, T, BH) ||

@@ -86,6 +86,16 @@ size_t bwd_chunk_workspace_bytes(long BH, int T);
 cudaError_t launch_bwd_chunk(const void* q, const void* k, const void* v, const void* beta, const float* S0,
                              const void* dO, const float* dST, float* dq, float* dk, float* dv, float* dbeta,
                              float* dS0, long BH, int T, int rule, uint32_t* err, void* scratch, cudaStream_t stream);
+// the same from saved residuals (training): T of every chunk (Tt, ntiles x 64 x 64 bf16) and every
+// chunk's entering state (states, ntiles x 128 x 128 bf16) as the forward left them; dSp: the
+// per-chunk dS' scratch (ntiles x 128 x 128 bf16)
+cudaError_t launch_bwd_chunk_saved(const void* q, const void* k, const void* v, const void* beta, const void* dO,
+                                   const float* dST, float* dq, float* dk, float* dv, float* dbeta, float* dS0,
+                                   long BH, int T, int rule, uint32_t* err, const void* Tt, const void* states,
+                                   void* dSp, cudaStream_t stream);
+// bytes of T and of the entering states kept for the backward (bf16, d = 128)
+size_t bwd_saved_t_bytes(long BH, int T);
+size_t bwd_saved_state_bytes(long BH, int T);
 
 cudaError_t launch_wait_timeout_selftest(uint32_t* err, unsigned long long limit_ns, cudaStream_t stream);
 

@@ -313,9 +313,12 @@ int efla_recurrent_step_ex(const void *q, const void *k, const void *v, const vo
                            int rule, efla_stream_t stream);
 
 /*
- * efla_backward_workspace_bytes -- bytes of device workspace efla_backward needs:
- * B*H*T*d_v + B*H*T floats (the residuals r_t = S_{t-1}^T k_t - v_t of a forward sweep,
- * and the gate gradient).  0 for an unsupported shape or dtype.
+ * efla_backward_workspace_bytes -- bytes of device workspace efla_backward needs.  bf16 with
+ * d = 128 (the chunkwise form): a 256-byte header (the device error word) and, per 64-token
+ * chunk, its UT transform (bf16 64 x 64), its entering state and its dS' (bf16 128 x 128
+ * each).  Otherwise (the token sweep): B*H*T*d_v + B*H*T floats (the residuals
+ * r_t = S_{t-1}^T k_t - v_t of a forward sweep, and the gate gradient).  0 for an
+ * unsupported shape or dtype.
  */
 size_t efla_backward_workspace_bytes(int B, int H, int T, int d_k, int d_v, int dtype);
 
@@ -337,10 +340,15 @@ size_t efla_backward_workspace_bytes(int B, int H, int T, int d_k, int d_v, int 
  * Supported: d_k = d_v in {64, 128}; dtype f32 or bf16; any T >= 0 (T = 0 copies dS_T
  * into dS0).  All pointers 16-byte aligned; no output may overlap an input, the
  * workspace or another output, and no input may overlap the workspace; else
- * EFLA_ERR_INVALID_ARG and nothing is launched.  The
- * state is fp32 throughout; the outputs are accumulated in fp32 (the row sums over d_v
- * columns with atomics, so their last bits depend on arrival order).  Asynchronous on
- * `stream`; launch failures return EFLA_ERR_CUDA.
+ * EFLA_ERR_INVALID_ARG and nothing is launched.
+ * bf16 with d = 128 runs the reverse mode of the chunkwise form (Section 3.3) on tensor
+ * cores: the UT transforms and the chunk states are recomputed, a reverse chain carries
+ * dL/dS across chunks, and every chunk's gradients follow from its state and dS'.  Its
+ * products take bf16 operands (as the forward's do) with fp32 accumulation, and its
+ * results are the same bits on every call.  The token sweep (fp32, d = 64) keeps the state
+ * and the gradients in fp32; its row sums over d_v columns use atomics, so their last bits
+ * depend on arrival order.  Asynchronous on `stream`; launch failures return
+ * EFLA_ERR_CUDA; a device wait that runs out is reported by efla_workspace_status.
  */
 int efla_backward(const void *q, const void *k, const void *v, const void *beta, const float *S0,
                   const void *dO, const float *dS_T, float *dq, float *dk, float *dv, float *dbeta,
@@ -355,6 +363,41 @@ int efla_backward_ex(const void *q, const void *k, const void *v, const void *be
                      const void *dO, const float *dS_T, float *dq, float *dk, float *dv, float *dbeta,
                      float *dS0, int B, int H, int T, int d_k, int d_v, int dtype, int rule,
                      void *workspace, size_t workspace_bytes, efla_stream_t stream);
+
+/*
+ * Training with saved residuals (bf16, d_k = d_v = 128, chunk 64, ungated; the exact or
+ * Euler rule).  The forward keeps what the chunkwise backward needs, and the backward takes
+ * it instead of recomputing it (the recompute is a full forward: the UT transforms and the
+ * state chain).
+ *
+ * efla_train_saved_bytes -- bytes of `saved`: a 256-byte header (the forward's device error
+ *   word), the UT transform T of every 64-token chunk (bf16 64 x 64) and every chunk's
+ *   entering state (bf16 128 x 128).  0 for any other shape, dtype or chunk.
+ *
+ * efla_chunk_fwd_save -- efla_chunk_fwd_ex with `saved` (>= efla_train_saved_bytes,
+ *   16-byte aligned, caller-owned) as its workspace: the same outputs, the same bits, and
+ *   on return `saved` also holds every chunk's entering state.  Unsupported shapes return
+ *   EFLA_ERR_UNSUPPORTED; the other argument rules and errors are efla_chunk_fwd_ex's.
+ *
+ * efla_backward_saved_workspace_bytes -- bytes of workspace efla_backward_saved needs: a
+ *   256-byte header (the device error word) and every chunk's dS' (bf16 128 x 128).
+ *
+ * efla_backward_saved -- efla_backward_ex without the recompute: T and the entering states
+ *   are read from `saved`, written by efla_chunk_fwd_save for the same q, k, v, beta, S0 and
+ *   rule and not modified since (S0 is not an argument: it is the first saved state).
+ *   The gradients are efla_backward_ex's, bit for bit.  No output or the workspace may
+ *   overlap an input, `saved` or each other; else EFLA_ERR_INVALID_ARG and nothing is
+ *   launched.  Asynchronous on `stream`.
+ */
+size_t efla_train_saved_bytes(int B, int H, int T, int d_k, int d_v, int chunk, int dtype);
+int efla_chunk_fwd_save(const void *q, const void *k, const void *v, const void *beta, const float *S0,
+                        void *o, float *S_T, int B, int H, int T, int d_k, int d_v, int chunk, int dtype,
+                        int rule, void *saved, size_t saved_bytes, efla_stream_t stream);
+size_t efla_backward_saved_workspace_bytes(int B, int H, int T, int d_k, int d_v, int dtype);
+int efla_backward_saved(const void *q, const void *k, const void *v, const void *beta, const void *dO,
+                        const float *dS_T, float *dq, float *dk, float *dv, float *dbeta, float *dS0, int B,
+                        int H, int T, int d_k, int d_v, int dtype, int rule, const void *saved,
+                        size_t saved_bytes, void *workspace, size_t workspace_bytes, efla_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -266,3 +266,49 @@ def test_segmented_entry_point_validates_arguments(efla):
     assert call(ws=plain) == INVALID                              # too small for two segments
     assert call(rule=3) == INVALID
     assert call(B=0) == OK
+
+
+def test_training_entry_points_sizes_and_validation(efla):
+    """efla_chunk_fwd_save / efla_backward_saved (bf16, d = 128 only): sizes, and every
+    rejection happens before anything is launched."""
+    L = efla.lib
+    tiles = 4 * 16 * 32
+    assert L.efla_train_saved_bytes(4, 16, 2048, 128, 128, 64, 1) == 256 + tiles * (64 * 64 + 128 * 128) * 2
+    assert L.efla_backward_saved_workspace_bytes(4, 16, 2048, 128, 128, 1) == 256 + tiles * 128 * 128 * 2
+    for args in ((1, 1, 64, 64, 64, 64, 1), (1, 1, 64, 128, 128, 64, 0), (1, 1, 64, 128, 128, 32, 1),
+                 (1, 1, -1, 128, 128, 64, 1)):
+        assert L.efla_train_saved_bytes(*args) == 0, args
+    assert L.efla_backward_saved_workspace_bytes(1, 1, 64, 64, 64, 1) == 0
+    assert L.efla_backward_saved_workspace_bytes(1, 1, 64, 128, 128, 0) == 0
+    q, k, v, b, s0, o, st, sv = GOOD
+    need = L.efla_train_saved_bytes(1, 1, 64, 128, 128, 64, 1)
+
+    def fwd(d=128, dtype=1, rule=0, saved=sv, n=need, out=o):
+        return L.efla_chunk_fwd_save(q, k, v, b, s0, out, st, 1, 1, 64, d, d, 64, dtype, rule, saved, n, None)
+    assert fwd(d=64) == UNSUPPORTED
+    assert fwd(dtype=0) == UNSUPPORTED
+    assert fwd(rule=5) == INVALID
+    assert fwd(n=need - 16) == INVALID
+    assert fwd(saved=None) == INVALID
+    assert fwd(out=q) == INVALID                               # o aliases q
+    assert fwd(saved=ctypes.c_void_p(q.value)) == INVALID      # saved covers q
+
+    P = GOOD_B
+    ws_need = L.efla_backward_saved_workspace_bytes(1, 1, 64, 128, 128, 1)
+
+    def bwd(ptrs=P, d=128, dtype=1, rule=0, saved_n=need, ws_n=ws_need):
+        qq, kk, vv, bb, do, dst, dq, dk, dv, db, ds0, saved, w = ptrs
+        return L.efla_backward_saved(qq, kk, vv, bb, do, dst, dq, dk, dv, db, ds0, 1, 1, 64, d, d, dtype, rule,
+                                     saved, saved_n, w, ws_n, None)
+    assert bwd(d=64) == UNSUPPORTED
+    assert bwd(dtype=0) == UNSUPPORTED
+    assert bwd(rule=7) == INVALID
+    assert bwd(saved_n=need - 16) == INVALID
+    assert bwd(ws_n=ws_need - 16) == INVALID
+    for i in range(13):                           # every pointer must be 16-byte aligned
+        bad = list(P); bad[i] = ctypes.c_void_p(P[i].value + 4)
+        assert bwd(bad) == INVALID, i
+    bad = list(P); bad[6] = P[0]                  # dq aliases q
+    assert bwd(bad) == INVALID
+    bad = list(P); bad[12] = P[11]                # the workspace holds `saved`
+    assert bwd(bad, ws_n=max(ws_need, need)) == INVALID

@@ -137,3 +137,33 @@ def test_chunked_backward_repeats_bitwise_and_reports_ok(efla, cuda):
     assert efla.efla_workspace_status(ws) == efla.EFLA_OK
     for x, y in zip(a, b):
         assert torch.equal(x, y)
+
+
+@pytest.mark.parametrize("name,over,rule", [("lm1p3b_bf16", dict(B=1, H=3, T=300), None),
+                                            ("lm1p3b_bf16", dict(B=1, H=2, T=65), "euler"),
+                                            ("lm1p3b_bf16", {}, None)], ids=str)
+def test_training_saved_path_is_the_recompute_bit_for_bit(efla, cuda, name, over, rule):
+    """efla_chunk_fwd_save gives efla_chunk_fwd's outputs, and efla_backward_saved (fed by it)
+    efla_backward's gradients, bit for bit: the saved T and entering states are the ones the
+    backward would recompute.  The recompute path is itself checked against the oracle above."""
+    w = W[name].replace(**over)
+    inp = workloads.make_chunk_inputs(w)
+    if rule == "euler":
+        k = inp["k"].float()
+        inp["k"] = (k / k.norm(dim=-1, keepdim=True).clamp_min(1e-30)).to(inp["k"].dtype)
+    cot = workloads.make_cotangents(w, with_state_grad=True)
+    S0 = 0.1 * torch.randn(w.B, w.H, w.dk, w.dv, generator=torch.Generator().manual_seed(w.seed + 7))
+    d = {k: (None if v is None else v.to(cuda)) for k, v in dict(inp, S0=S0, **cot).items()}
+    r = efla.EFLA_RULE_EULER if rule == "euler" else efla.EFLA_RULE_EXACT
+    o1, S1 = efla.efla_chunk_fwd(d["q"], d["k"], d["v"], d["beta"], d["S0"], rule=r)
+    o2, S2, saved = efla.efla_chunk_fwd_save(d["q"], d["k"], d["v"], d["beta"], d["S0"], rule=r)
+    assert torch.equal(o1, o2) and torch.equal(S1, S2)
+    g1 = efla.efla_backward(d["q"], d["k"], d["v"], d["beta"], d["dO"], S0=d["S0"], dS_T=d["dS_T"], rule=r)
+    ws = torch.zeros(efla.lib.efla_backward_saved_workspace_bytes(w.B, w.H, w.T, w.dk, w.dv, efla.EFLA_DTYPE_BF16),
+                     dtype=torch.uint8, device=cuda)
+    g2 = efla.efla_backward_saved(d["q"], d["k"], d["v"], d["beta"], d["dO"], saved, dS_T=d["dS_T"], rule=r,
+                                  workspace=ws)
+    assert efla.efla_workspace_status(ws) == efla.EFLA_OK
+    assert efla.efla_workspace_status(saved) == efla.EFLA_OK
+    for nme, x, y in zip(NAMES, g1, g2):
+        assert torch.equal(x, y), nme
