@@ -613,31 +613,43 @@ bwd_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
 }
 // ============================================================================ reverse chain
-// One CTA (8 warps) per (stream, 64-column half of d_v) walks the chunks backwards with its
-// half of dS in tensor memory (the columns of dS evolve independently).  Per chunk c:
-//   store dS' (the carried gradient, bf16) for the per-chunk kernel;
-//   dDelta = P^T dO + K dS'   (M = 64)        dR = T^T dDelta   (M = 64)
-//   dS += Q^T dO + K^T (-dR)  (M = 128, the accumulator)
-// with P = tril_incl(Q K^T) of chunk c - 1 formed in the same MMA batch as the dS update.
-// Q, K, T and the dO half of three chunks are in flight by TMA; every product is a tcgen05
-// MMA (bf16 operands in shared memory, fp32 accumulators in tensor memory); between the
-// products the eight warps convert the accumulator to the next bf16 operand.
 namespace rc {
 constexpr uint32_t TILE = 8192;
 constexpr int kStages = 3;
+constexpr int kThreads = 320;              // warps 0-7 convert, 8 copies (TMA), 9 issues the MMAs
 constexpr uint32_t ST_Q = 0, ST_K = 2 * TILE, ST_T = 4 * TILE, ST_DO = 5 * TILE, STAGE = 6 * TILE;
 constexpr uint32_t P = kStages * STAGE;    // P (bf16 [t][s])
 constexpr uint32_t DSB = P + TILE;         // dS' (bf16, 128 rows i x 64 columns j)
 constexpr uint32_t DD = DSB + 2 * TILE;    // dDelta (bf16 [s][j])
 constexpr uint32_t NR = DD + TILE;         // -dR (bf16 [s][j])
-constexpr uint32_t BAR = NR + TILE;        // stage full [3], MMA commits
-constexpr uint32_t MISC = BAR + 4 * 8;     // TMEM base, abort flag, loads issued per stage [3]
-constexpr uint32_t SMEM_BYTES = MISC + 32 + 1024;
+constexpr uint32_t BAR = NR + TILE;        // mbarriers, see below
+constexpr int NBAR = 16;
+constexpr uint32_t MISC = BAR + NBAR * 8;  // TMEM base, abort flag
+constexpr uint32_t SMEM_BYTES = MISC + 16 + 1024;
 static_assert(SMEM_BYTES <= 232448, "shared memory");
 constexpr uint32_t C_DS = 0, C_P = 64, C_DD = 128, C_DR = 192, C_COLS = 256;
+// mbarriers: stage full (TMA) and free (MMA commit) per stage; each product's commit and the
+// converters' hand-off back (one arrival per converter warp); the first P~; the drain
+enum : int {
+    B_FULL = 0, B_FREE = 3, B_DD_FULL = 6, B_DD_READY, B_DR_FULL, B_DR_READY, B_DS_FULL, B_DS_READY, B_PRO,
+    B_DRAIN
+};
+__host__ __device__ constexpr uint32_t bar_count(int i) {
+    return (i == B_DD_READY || i == B_DR_READY || i == B_DS_READY) ? 8u : 1u;
+}
 }  // namespace rc
 
-__global__ void __launch_bounds__(256, 1)
+// One CTA (10 warps) per (stream, 64-column half of d_v) walks the chunks backwards with its
+// half of dS in tensor memory.  Warp 8 keeps three chunks' Q, K, T and dO half in flight by
+// TMA; warp 9 issues every MMA; warps 0-7 turn each accumulator into the next bf16 operand.
+// The roles hand off through mbarriers only (every wait bounded), so an MMA issue that
+// stalls on a full queue stalls no converter.  Step k (chunk c = nc - 1 - k):
+//   issuer:     [dS'(c), P(c) ready]  store dS'(c) (TMA);  dDelta = P^T dO + K dS'  -> DD_FULL
+//               [dDelta ready]        dR = T^T dDelta  -> DR_FULL;  dS += Q^T dO;  P~(c - 1)
+//               [-dR ready]           dS += K^T (-dR)  -> DS_FULL, stage c free
+//   converters: DD_FULL -> dDelta bf16;  DR_FULL -> -dR bf16;  DS_FULL -> dS'(c - 1) bf16 (or
+//               dS0 after chunk 0) and P(c - 1) = tril_incl(P~) bf16  -> DS_READY
+__global__ void __launch_bounds__(rc::kThreads, 1)
 bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_do, const __grid_constant__ CUtensorMap tm_t,
                  const __grid_constant__ CUtensorMap tm_dsp, const float* __restrict__ dST, float* __restrict__ dS0,
@@ -652,47 +664,30 @@ bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sb = smem_u32(sm);
-    uint64_t* bar = reinterpret_cast<uint64_t*>(sm + BAR);    // 0-2: stage full, 3: MMA commits
+    uint64_t* bar = reinterpret_cast<uint64_t*>(sm + BAR);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + MISC);
     volatile int* abort = reinterpret_cast<volatile int*>(sm + MISC + 4);
-    int* issued = reinterpret_cast<int*>(sm + MISC + 8);      // written by thread 0 only
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int q = warp & 3, h = warp >> 2;                    // TMEM lane quarter, column half
-    const uint32_t lane_off = static_cast<uint32_t>(32 * q) << 16;
-    const int row = 32 * q + lane;                            // row of dS (d_k index)
-    const int trow = 16 * q + lane;                           // row of an M = 64 product (lanes < 16)
     const long bh = blockIdx.x >> 1;
     const int col0 = (blockIdx.x & 1) * 64;
     const int nc = (T + 63) / 64;
     const long tile0 = bh * nc;
-    const size_t srow = ((size_t)bh * 128 + row) * 128 + col0 + 32 * h;   // this thread's 32 entries of dS
 
     if (nc == 0) {        // no tokens: dS0 = dS_T
-        if (dS0)
+        if (dS0 && tid < 256) {
+            const int q = (tid >> 5) & 3, h = tid >> 7, row = 32 * q + (tid & 31);
+            const size_t srow = ((size_t)bh * 128 + row) * 128 + col0 + 32 * h;
             for (int j = 0; j < 32; ++j)
                 if (span_ok(err, spans.ds0, dS0 + srow + j, 4))
                     dS0[srow + j] = dST && span_ok(err, spans.dst, dST + srow + j, 4) ? dST[srow + j] : 0.f;
+        }
         return;
     }
-    auto load = [&](int c) {   // chunk c's Q, K, T and dO half into stage c % 3 (one thread)
-        uint8_t* st = sm + (c % kStages) * STAGE;
-        uint64_t* full = bar + c % kStages;
-        ++issued[c % kStages];
-        mbar_arrive_expect_tx(full, STAGE);
-        tma_load_3d(st + ST_Q, &tm_q, full, 0, c * 64, (int)bh);
-        tma_load_3d(st + ST_Q + TILE, &tm_q, full, 64, c * 64, (int)bh);
-        tma_load_3d(st + ST_K, &tm_k, full, 0, c * 64, (int)bh);
-        tma_load_3d(st + ST_K + TILE, &tm_k, full, 64, c * 64, (int)bh);
-        tma_load_2d(st + ST_T, &tm_t, full, 0, (int)((tile0 + c) * 64));
-        tma_load_3d(st + ST_DO, &tm_do, full, col0, c * 64, (int)bh);
-    };
     if (tid == 0) {
-        for (int i = 0; i < 4; ++i) mbar_init(bar + i, 1);
+        for (int i = 0; i < NBAR; ++i) mbar_init(bar + i, bar_count(i));
         *abort = 0;
-        for (int i = 0; i < kStages; ++i) issued[i] = 0;
         fence_mbar_init();
-        for (int i = 0; i < kStages && i < nc; ++i) load(nc - 1 - i);
     }
     if (warp == 0) {
         tmem_alloc(tmem_slot, C_COLS);
@@ -702,118 +697,156 @@ bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     __syncthreads();
     tc_fence_after();
     const uint32_t tm = *tmem_slot;
-    auto wait = [&](int i, uint32_t parity) {
-        if (*abort) return;
-        if (!mbar_wait(bar + i, parity, limit_ns)) *abort = 1;
-        tc_fence_after();
+    // bounded wait; gives up early once another role has aborted
+    auto wait = [&](int i, uint32_t parity) -> bool {
+        if (*abort) return false;
+        if (mbar_wait(bar + i, parity, limit_ns)) return true;
+        *abort = 1;
+        return false;
     };
-    auto wait_stage = [&](int c) { wait(c % kStages, ((nc - 1 - c) / kStages) & 1); };
-    uint32_t mma_phase = 0;
-    auto wait_mma = [&]() { wait(3, mma_phase & 1); ++mma_phase; };
-    auto commit = [&]() { mma_commit_elect(bar + 3); };
-    auto handoff = [&]() {
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
+    auto wwait = [&](int i, uint32_t parity) { return __all_sync(0xffffffffu, wait(i, parity)); };
+    auto warp_arrive = [&](int i) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar + i);
     };
-    auto stage = [&](int c) { return sb + (uint32_t)(c % kStages) * STAGE; };
-    // dS (fp32, tensor memory) -> dS' of the next chunk, the bf16 operand; the per-chunk
-    // kernel's copy is stored from it by TMA at the start of that chunk's step
-    auto emit_dsp = [&](const float (&x)[32]) { st_row32(sm + DSB, row, 4 * h, x); };
-    // P~ (M = 64, rows trow) -> P = tril_incl, bf16 [t][s]
-    auto emit_p = [&]() {
-        float x[32];
-        tmem_ld32_wait(tm + lane_off + C_P + 32 * h, x);
-        if (lane < 16) {
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-                if (32 * h + j > trow) x[j] = 0.f;
-            st_row32(sm + P, trow, 4 * h, x);
-        }
-    };
+    auto stage = [&](int c) { return (uint32_t)(c % kStages); };
+    auto use = [&](int c) { return (uint32_t)(((nc - 1 - c) / kStages) & 1); };   // phase of chunk c's stage
 
-    {   // the carried gradient starts as dS_T's half (or zero)
-        float x[32];
-#pragma unroll
-        for (int j = 0; j < 32; j += 4) {
-            const float4 v = dST && span_ok(err, spans.dst, dST + srow + j, 16)
-                                 ? *reinterpret_cast<const float4*>(dST + srow + j) : make_float4(0.f, 0.f, 0.f, 0.f);
-            x[j] = v.x; x[j + 1] = v.y; x[j + 2] = v.z; x[j + 3] = v.w;
+    if (warp == 8) {
+        // ================================================================ TMA producer
+        if (lane == 0) {
+            int issued = 0;
+            for (int c = nc - 1; c >= 0; --c, ++issued) {
+                const uint32_t s = stage(c);
+                if (issued >= kStages && !wait(B_FREE + s, use(c + kStages))) break;
+                uint8_t* st = sm + s * STAGE;
+                uint64_t* full = bar + B_FULL + s;
+                mbar_arrive_expect_tx(full, STAGE);
+                tma_load_3d(st + ST_Q, &tm_q, full, 0, c * 64, (int)bh);
+                tma_load_3d(st + ST_Q + TILE, &tm_q, full, 64, c * 64, (int)bh);
+                tma_load_3d(st + ST_K, &tm_k, full, 0, c * 64, (int)bh);
+                tma_load_3d(st + ST_K + TILE, &tm_k, full, 64, c * 64, (int)bh);
+                tma_load_2d(st + ST_T, &tm_t, full, 0, (int)((tile0 + c) * 64));
+                tma_load_3d(st + ST_DO, &tm_do, full, col0, c * 64, (int)bh);
+            }
+            // no copy may land after the block exits
+            for (int c = nc - issued; c < nc - issued + kStages && c < nc; ++c)
+                mbar_wait(bar + B_FULL + stage(c), use(c), limit_ns);
         }
-        float lo[16], hi[16];
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-            lo[j] = x[j];
-            hi[j] = x[16 + j];
+    } else if (warp == 9) {
+        // ================================================================ MMA issuer (whole warp)
+        bool ok = wwait(B_FULL + stage(nc - 1), use(nc - 1));
+        if (ok) {
+            tc_fence_after();
+            const uint32_t st = sb + stage(nc - 1) * STAGE;
+            mma_ss(tm + C_P, st + ST_Q, TILE, 32, 16, st + ST_K, TILE, 32, 16, idesc(64, K_MAJ, K_MAJ), 8, false);
+            mma_commit_elect(bar + B_PRO);
         }
-        tmem_st16(tm + lane_off + C_DS + 32 * h, lo);
-        tmem_st16(tm + lane_off + C_DS + 32 * h + 16, hi);
-        tmem_wait_st();
-        emit_dsp(x);
-    }
-    wait_stage(nc - 1);
-    handoff();            // dS' (bf16) is an MMA operand from here on
-    if (warp == 0) {
-        const uint32_t st = stage(nc - 1);
-        mma_ss(tm + C_P, st + ST_Q, TILE, 32, 16, st + ST_K, TILE, 32, 16, idesc(64, K_MAJ, K_MAJ), 8, false);
-        commit();
-    }
-    wait_mma();
-    emit_p();
-    handoff();
-    for (int c = nc - 1; c >= 0; --c) {
-        const uint32_t st = stage(c);
-        // ---- dDelta = P^T dO + K dS'
-        if (warp == 0) {
+        for (int k = 0; k < nc && ok; ++k) {
+            const int c = nc - 1 - k;
+            const uint32_t st = sb + stage(c) * STAGE, ph = k & 1;
+            if (!(ok = wwait(B_DS_READY, ph))) break;
+            tc_fence_after();
+            if (lane == 0) tma_store_2d(&tm_dsp, sm + DSB, col0, (int)((tile0 + c) * 128));   // dS' of chunk c
+            __syncwarp();
             mma_ss(tm + C_DD, sb + P, 0, 2048, TILE, st + ST_DO, 0, 2048, TILE, idesc(64, MN_MAJ, MN_MAJ), 4, false);
             mma_ss(tm + C_DD, st + ST_K, TILE, 32, 16, sb + DSB, TILE, 2048, TILE, idesc(64, K_MAJ, MN_MAJ), 8, true);
-            commit();
+            mma_commit_elect(bar + B_DD_FULL);
+            if (!(ok = wwait(B_DD_READY, ph))) break;
+            tc_fence_after();
+            mma_ss(tm + C_DR, st + ST_T, 0, 2048, TILE, sb + DD, 0, 2048, TILE, idesc(64, MN_MAJ, MN_MAJ), 4, false);
+            mma_commit_elect(bar + B_DR_FULL);
+            // what does not need -dR: dS += Q^T dO, and the next chunk's P~
+            mma_ss(tm + C_DS, st + ST_Q, 0, 2048, TILE, st + ST_DO, 0, 2048, TILE, idesc(128, MN_MAJ, MN_MAJ), 4, true);
+            if (c > 0) {
+                if (!(ok = wwait(B_FULL + stage(c - 1), use(c - 1)))) break;
+                tc_fence_after();
+                const uint32_t sp = sb + stage(c - 1) * STAGE;
+                mma_ss(tm + C_P, sp + ST_Q, TILE, 32, 16, sp + ST_K, TILE, 32, 16, idesc(64, K_MAJ, K_MAJ), 8, false);
+            }
+            if (!(ok = wwait(B_DR_READY, ph))) break;
+            if (lane == 0) tma_store_wait_read();   // dS' is rewritten once the dS update has landed
+            __syncwarp();
+            tc_fence_after();
+            mma_ss(tm + C_DS, st + ST_K, 0, 2048, TILE, sb + NR, 0, 2048, TILE, idesc(128, MN_MAJ, MN_MAJ), 4, true);
+            mma_commit_elect(bar + B_DS_FULL);
+            mma_commit_elect(bar + B_FREE + stage(c));
         }
-        if (warp == 1 && lane == 0) {
-            tma_store_2d(&tm_dsp, sm + DSB, col0, (int)((tile0 + c) * 128));   // dS' of chunk c
-            if (c + 1 - kStages >= 0 && c + 1 < nc && !*abort)
-                load(c + 1 - kStages);   // into the stage chunk c + 1 no longer reads
+        mma_commit_elect(bar + B_DRAIN);
+        if (lane == 0) {
+            mbar_wait(bar + B_DRAIN, 0, limit_ns);
+            tma_store_wait_all();
         }
-        wait_mma();
-        {
+        __syncwarp();
+    } else {
+        // ================================================================ converters (warps 0-7)
+        const int q = warp & 3, h = warp >> 2;            // TMEM lane quarter, column half
+        const uint32_t lane_off = static_cast<uint32_t>(32 * q) << 16;
+        const int row = 32 * q + lane;                    // row of dS (d_k index)
+        const int trow = 16 * q + lane;                   // row of an M = 64 product (lanes < 16)
+        const size_t srow = ((size_t)bh * 128 + row) * 128 + col0 + 32 * h;   // this thread's 32 entries of dS
+        auto emit_p = [&]() {   // P~ (M = 64) -> P = tril_incl, bf16 [t][s]
             float x[32];
+            tmem_ld32_wait(tm + lane_off + C_P + 32 * h, x);
+            if (lane < 16) {
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                    if (32 * h + j > trow) x[j] = 0.f;
+                st_row32(sm + P, trow, 4 * h, x);
+            }
+        };
+        auto hand_off = [&](int i) {
+            fence_proxy_async_smem();
+            tc_fence_before();
+            warp_arrive(i);
+        };
+        bool ok = true;
+        {   // the carried gradient starts as dS_T's half (or zero); P of the last chunk
+            float x[32];
+#pragma unroll
+            for (int j = 0; j < 32; j += 4) {
+                const float4 v = dST && span_ok(err, spans.dst, dST + srow + j, 16)
+                                     ? *reinterpret_cast<const float4*>(dST + srow + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+                x[j] = v.x; x[j + 1] = v.y; x[j + 2] = v.z; x[j + 3] = v.w;
+            }
+            float lo[16], hi[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                lo[j] = x[j];
+                hi[j] = x[16 + j];
+            }
+            tmem_st16(tm + lane_off + C_DS + 32 * h, lo);
+            tmem_st16(tm + lane_off + C_DS + 32 * h + 16, hi);
+            tmem_wait_st();
+            st_row32(sm + DSB, row, 4 * h, x);
+            ok = wwait(B_PRO, 0);
+            tc_fence_after();
+            emit_p();
+            hand_off(B_DS_READY);
+        }
+        for (int k = 0; k < nc && ok; ++k) {
+            const int c = nc - 1 - k;
+            const uint32_t ph = k & 1;
+            float x[32];
+            if (!(ok = wwait(B_DD_FULL, ph))) break;
+            tc_fence_after();
             tmem_ld32_wait(tm + lane_off + C_DD + 32 * h, x);
             if (lane < 16) st_row32(sm + DD, trow, 4 * h, x);
-        }
-        handoff();
-        // ---- dR = T^T dDelta
-        if (warp == 0) {
-            mma_ss(tm + C_DR, st + ST_T, 0, 2048, TILE, sb + DD, 0, 2048, TILE, idesc(64, MN_MAJ, MN_MAJ), 4, false);
-            commit();
-        }
-        wait_mma();
-        {
-            float x[32];
+            hand_off(B_DD_READY);
+            if (!(ok = wwait(B_DR_FULL, ph))) break;
+            tc_fence_after();
             tmem_ld32_wait(tm + lane_off + C_DR + 32 * h, x);
 #pragma unroll
             for (int j = 0; j < 32; ++j) x[j] = -x[j];
             if (lane < 16) st_row32(sm + NR, trow, 4 * h, x);
-        }
-        if (warp == 1 && lane == 0) tma_store_wait_read();   // dS' may be overwritten below
-        handoff();
-        // ---- dS += Q^T dO + K^T (-dR);  P~ of chunk c - 1
-        if (c > 0) wait_stage(c - 1);
-        if (warp == 0) {
-            mma_ss(tm + C_DS, st + ST_Q, 0, 2048, TILE, st + ST_DO, 0, 2048, TILE, idesc(128, MN_MAJ, MN_MAJ), 4, true);
-            mma_ss(tm + C_DS, st + ST_K, 0, 2048, TILE, sb + NR, 0, 2048, TILE, idesc(128, MN_MAJ, MN_MAJ), 4, true);
-            if (c > 0) {
-                const uint32_t sp = stage(c - 1);
-                mma_ss(tm + C_P, sp + ST_Q, TILE, 32, 16, sp + ST_K, TILE, 32, 16, idesc(64, K_MAJ, K_MAJ), 8, false);
-            }
-            commit();
-        }
-        wait_mma();
-        {
-            float x[32];
+            hand_off(B_DR_READY);
+            if (!(ok = wwait(B_DS_FULL, ph))) break;
+            tc_fence_after();
             tmem_ld32_wait(tm + lane_off + C_DS + 32 * h, x);
             if (c > 0) {
-                emit_dsp(x);
+                st_row32(sm + DSB, row, 4 * h, x);
+                emit_p();
+                hand_off(B_DS_READY);
             } else if (dS0) {
 #pragma unroll
                 for (int j = 0; j < 32; j += 4)
@@ -821,24 +854,10 @@ bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                         *reinterpret_cast<float4*>(dS0 + srow + j) = make_float4(x[j], x[j + 1], x[j + 2], x[j + 3]);
             }
         }
-        if (c > 0) emit_p();
-        handoff();
     }
-    if (warp == 1 && lane == 0) tma_store_wait_all();
     tc_fence_before();
     __syncthreads();
-    if (*abort) {         // a wait ran out: record it, and let every issued MMA finish before
-        if (tid == 0) atomicOr(err, kDevTimeout);   // the tensor memory is released
-        if (warp == 0) {
-            commit();
-            if (lane == 0) {
-                mbar_wait(bar + 3, mma_phase & 1, limit_ns);
-                for (int i = 0; i < kStages; ++i)   // and no copy may land after the block exits
-                    if (issued[i] > 0) mbar_wait(bar + i, (issued[i] - 1) & 1, limit_ns);
-            }
-            __syncwarp();
-        }
-    }
+    if (tid == 0 && *abort) atomicOr(err, kDevTimeout);
     if (warp == 0) {
         tc_fence_after();
         tmem_dealloc(tm, C_COLS);
@@ -903,7 +922,7 @@ cudaError_t launch_bwd_chunk_saved(const void* q, const void* k, const void* v, 
     static std::atomic<uint64_t> smem_chain{0}, smem_tile{0};
     e = set_smem_limit_once(bwd_chain_kernel, (int)rc::SMEM_BYTES, smem_chain);
     if (e != cudaSuccess) return e;
-    bwd_chain_kernel<<<(unsigned)(BH * 2), 256, rc::SMEM_BYTES, stream>>>(mq, mk, mdo, mt, mdsp, dST, dS0, T, err,
+    bwd_chain_kernel<<<(unsigned)(BH * 2), rc::kThreads, rc::SMEM_BYTES, stream>>>(mq, mk, mdo, mt, mdsp, dST, dS0, T, err,
                                                                           kTileWaitNs, sp);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     // 3. every chunk's gradients
