@@ -74,7 +74,7 @@ KERNEL_SOURCES = {
                        "efla_chunk_simt.cu", "efla_common.cuh", "efla_tma.cuh", "sm100.cuh"],
     "efla_recurrent_step": ["efla_decode.cu", "efla_common.cuh"],
     "efla_backward": ["efla_bwd.cu", "efla_bwd_chunk.cu", "efla_chunk_tc.cu", "efla_ut.cu",
-                      "efla_ut_tf32.cuh", "efla_ut_solve.cuh", "efla_common.cuh", "efla_tma.cuh", "sm100.cuh"],
+                      "efla_ut_tf32.cuh", "efla_common.cuh", "efla_tma.cuh", "sm100.cuh"],
 }
 
 

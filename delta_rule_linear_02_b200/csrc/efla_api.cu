@@ -124,7 +124,11 @@ static int chunk_fwd_impl(const void* q, const void* k, const void* v, const voi
     if (dtype == EFLA_DTYPE_BF16 && d_k == 128) {
         char* scratch = static_cast<char*>(workspace) + kWorkspaceHeader;
         efla::SegPlan plan;   // training: every chunk's entering state after the transforms
-        if (save) plan.states = reinterpret_cast<__nv_bfloat16*>(scratch + efla::bwd_saved_t_bytes(BH, T));
+        if (save) {
+            plan.X = reinterpret_cast<float*>(scratch + efla::bwd_saved_t_bytes(BH, T));
+            plan.states = reinterpret_cast<__nv_bfloat16*>(scratch + efla::bwd_saved_t_bytes(BH, T) +
+                                                           efla::bwd_saved_x_bytes(BH, T));
+        }
         return from_cuda(efla::launch_chunk_tc(q, k, v, beta, S0, o, S_T, seqs, BH, BH, T, BH * ((T + 63) / 64),
                                                static_cast<uint32_t*>(workspace), scratch, rule, s, g, plan));
     }
@@ -521,7 +525,8 @@ size_t efla_train_saved_bytes(int B, int H, int T, int d_k, int d_v, int chunk, 
     if (check_chunk_shape(B, H, T, d_k, d_v, chunk, dtype) != EFLA_OK) return 0;
     if (dtype != EFLA_DTYPE_BF16 || d_k != 128) return 0;
     const long BH = (long)B * H;
-    return kWorkspaceHeader + efla::bwd_saved_t_bytes(BH, T) + efla::bwd_saved_state_bytes(BH, T);
+    return kWorkspaceHeader + efla::bwd_saved_t_bytes(BH, T) + efla::bwd_saved_x_bytes(BH, T) +
+           efla::bwd_saved_state_bytes(BH, T);
 }
 
 int efla_chunk_fwd_save(const void* q, const void* k, const void* v, const void* beta, const float* S0, void* o,
@@ -581,7 +586,8 @@ int efla_backward_saved(const void* q, const void* k, const void* v, const void*
     const char* sv = static_cast<const char*>(saved) + kWorkspaceHeader;
     return from_cuda(efla::launch_bwd_chunk_saved(q, k, v, beta, dO, dS_T, dq, dk, dv, dbeta, dS0, BH, T, rule,
                                                   static_cast<uint32_t*>(workspace), sv,
-                                                  sv + efla::bwd_saved_t_bytes(BH, T),
+                                                  reinterpret_cast<const float*>(sv + efla::bwd_saved_t_bytes(BH, T)),
+                                                  sv + efla::bwd_saved_t_bytes(BH, T) + efla::bwd_saved_x_bytes(BH, T),
                                                   static_cast<char*>(workspace) + kWorkspaceHeader, s));
 }
 

@@ -13,21 +13,21 @@
 //             dK = Delta dS'^T + dP^T Q - dR S^T + (dG + dG^T) K + dalpha (dalpha/dlambda) 2 K,
 //             dG = diag(alpha) dA,  dbeta = dalpha dalpha/dbeta.
 // Three launches after the UT transforms (efla_ut.cu):
-//   1. the forward chain (efla_chunk_tc.cu) storing every chunk's entering state S (bf16);
+//   1. the UT transforms keeping X = (I + A)^{-1} (fp32) beside T, and the forward chain
+//      (efla_chunk_tc.cu) storing every chunk's entering state S (bf16) -- or, for training,
+//      the same residuals saved by the forward (efla_chunk_fwd_save);
 //   2. bwd_chain_kernel: one CTA per (stream, 64-column half of d_v) walks the chunks in
 //      reverse, carrying its half of dS in the MMA accumulators (the columns of dS evolve
 //      independently), and stores each chunk's dS' (bf16);
 //   3. bwd_tile_kernel: one CTA per (stream, chunk), all chunks at once: every gradient of
 //      the chunk from its S and dS'.
-// The reverse chain's products are warp-level bf16 tiles (mma.sync m16n8k16, fp32
-// accumulation, operands read with ldmatrix from padded shared memory); the per-chunk
-// kernel's are tcgen05 MMAs (see below); the triangular solve that gives X again is fp32 on
-// CUDA cores.  Operands pass through bf16 as in the forward, so the gradients carry
-// bf16-operand rounding (relative Frobenius error ~1e-2), not fp32's.
+// Both kernels' bf16 products are tcgen05 MMAs (operands in shared memory, fp32 accumulators
+// in tensor memory); only dA's two small fp32 products are TF32 mma.sync tiles.  Operands pass
+// through bf16 as in the forward, so the gradients carry bf16-operand rounding (relative
+// Frobenius error ~1e-2), not fp32's.
 #include "efla_common.cuh"
 #include "efla_kernels.h"
 #include "efla_tma.cuh"
-#include "efla_ut_solve.cuh"
 #include "efla_ut_tf32.cuh"
 #include "sm100.cuh"
 
@@ -40,7 +40,7 @@ constexpr int kD = 128, kC = 64;
 // The extents of the buffers the two backward kernels address directly (checked builds test
 // each access against them; see efla_common.cuh).
 struct BwdSpans {
-    Span beta, dq, dk, dv, dbeta, dst, ds0;
+    Span beta, dq, dk, dv, dbeta, dst, ds0, x;
 };
 
 // ============================================================================ per-chunk gradients
@@ -61,9 +61,9 @@ struct BwdSpans {
 // Shared-memory tiles are 128-byte swizzled rows of 64 elements: token-major tiles (K, Q, V,
 // dO: 64 rows per 64-column atom) serve as K-major operands over d or MN-major ones over
 // tokens, d-major tiles (S, dS', R^T, Delta^T, dDelta^T, -dR^T: 128 rows) the other way
-// round, so no operand is ever transposed in memory.  The triangular solve for
-// X = (I + A)^{-1} and the two 64^3 products of dA = strict_tril(-X^T dX X^T) stay fp32 on
-// CUDA cores (their accuracy sets dbeta's).  Phases are sequential: one warp issues a
+// round, so no operand is ever transposed in memory.  X = (I + A)^{-1} (fp32) and T (bf16)
+// come from the UT transform; the two 64^3 products of dA = strict_tril(-X^T dX X^T) run on
+// the TF32 tensor path, dalpha and dG on CUDA cores.  Phases are sequential: one warp issues a
 // phase's MMAs and commits them to one mbarrier; all warps wait (bounded), run the
 // epilogue, and meet at a block barrier.
 namespace tb {
@@ -75,28 +75,26 @@ constexpr uint32_t DSP = 65536;            // dS' [a0 | a1] (128 rows each); lat
 constexpr uint32_t SS = 98304;             // S [a0 | a1]
 constexpr uint32_t TT = 131072;            // T (bf16 [t][s]); later X^T (fp32)
 constexpr uint32_t PP = 139264;            // P, later dP (bf16 [t][s])
-constexpr uint32_t RT = 147456;            // the solve's A (fp32); then R^T (128 rows)
-constexpr uint32_t DL = 164864;            // the solve's scratch; then Delta^T (128 rows)
+constexpr uint32_t RT = 147456;            // R^T (128 rows)
+constexpr uint32_t DL = 164864;            // Delta^T (128 rows)
 constexpr uint32_t DG = 181248;            // G (bf16 [t][s]), later dG + dG^T
-constexpr int LAA = 65;                    // row stride (floats) of the solve's A: the G epilogue writes
-                                           // one column of 32 consecutive rows per warp, conflict-free
-constexpr int LA = 64;                     // row stride of the solve's scratch
-constexpr int LX = 68;                     // row stride of the other fp32 64 x 64 tiles (16-byte rows)
+constexpr int LX = 68;                     // row stride of the fp32 64 x 64 tiles (16-byte rows; the UT
+                                           // transform's X arrives in this layout)
 constexpr uint32_t F32 = 64 * LX * 4;      // bytes of one of them
 constexpr uint32_t FX = 189440;            // X (fp32)
 constexpr uint32_t FXT = TT;               // X^T
 constexpr uint32_t FW = TT + F32;          // W = dX X^T
 constexpr uint32_t FDT = V;                // dT^T, then dX^T, then dA
-constexpr uint32_t SMALL = FX + F32;       // alpha, beta, dalpha, lambda, ones, two partial sums (fp32 [64] each)
+constexpr uint32_t SMALL = FX + F32;       // alpha, beta, dalpha, lambda, (unused), two partial sums (fp32 [64] each)
 constexpr uint32_t BAR = SMALL + 7 * 256;  // mbarriers: the tile's inputs, MMA commits
 constexpr uint32_t MISC = BAR + 2 * 8;     // TMEM base, abort flag
 constexpr uint32_t SMEM_BYTES = MISC + 16 + 1024;
-static_assert(RT + 64 * LAA * 4 <= DL && DL + 64 * LA * 4 <= DG, "the solve's A and scratch fit R^T's and Delta^T's regions");
+static_assert(64 * LX * 4 == kUtXBytes, "X as the UT transform writes it");
 static_assert(FDT + F32 <= DSP && FW + F32 <= DG, "fp32 tiles stay inside dead regions");
 static_assert(SMEM_BYTES <= 232448, "shared memory");
 // TMEM columns (fp32 accumulators, 64 columns each)
 constexpr uint32_t C_GP = 0, C_SK = 64, C_DQ = 128, C_DL = 192, C_DD = 256, C_DK = 320, C_DR = 384, C_COLS = 512;
-constexpr uint32_t LOAD_BYTES = 131072;    // K, Q, V, dO, dS', S
+constexpr uint32_t LOAD_BYTES = 131072 + 64 * 68 * 4 + 8192;   // K, Q, V, dO, dS', S, X, T
 
 // nk k-steps of K = 16 with A and B in shared memory; operand k-step ks starts at
 // base + (ks / 4) * atom + (ks % 4) * step (K-major: step 32 bytes inside a 64-column atom;
@@ -150,91 +148,6 @@ __device__ __forceinline__ float ld_tok(const uint8_t* tile, uint32_t atom, int 
     return __bfloat162float(*reinterpret_cast<const bf16*>(p));
 }
 
-// X = (I + A)^{-1} for the 64 x 64 strictly-lower A (row stride LAA; only its strictly-lower
-// part is read), written in full into X (row stride LX; zeros above the diagonal), Y scratch
-// (row stride LA).  Block doubling: the four 16 x 16 diagonal blocks by forward
-// substitution (one thread per column), then merges X21 = -X22 (A21 X11) at 32 and 64.  In
-// the 64 merge each thread keeps four rows of one column in registers (one operand load
-// per four FMAs).  256 threads; ends with a barrier.
-__device__ __forceinline__ void unit_lower_inverse64(const float* __restrict__ A, float* __restrict__ X,
-                                                     float* __restrict__ Y, int tid) {
-    if (tid < 64) {
-        const int b = tid >> 4, c = tid & 15;
-        float x[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) x[i] = (i == c) ? 1.f : 0.f;
-#pragma unroll
-        for (int i = 1; i < 16; ++i) {
-            float s = 0.f;
-#pragma unroll
-            for (int j = 0; j < i; ++j) s = fmaf(A[(16 * b + i) * LAA + 16 * b + j], x[j], s);
-            if (i > c) x[i] = -s;
-        }
-        float* Xb = X + (16 * b) * LX + 16 * b + c;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) Xb[i * LX] = x[i];
-    } else {
-        for (int e = tid - 64; e < 64 * 64; e += 192) {   // the strictly-upper 16 x 16 blocks
-            const int i = e >> 6, c = e & 63;
-            if ((c >> 4) > (i >> 4)) X[i * LX + c] = 0.f;
-        }
-    }
-    __syncthreads();
-    {   // 32 x 32 blocks s = 0, 1:  Y21 = A21 X11, then X21 = -X22 Y21 (16 x 16 blocks)
-        const int s = tid >> 7, i = (tid >> 4) & 7, c = tid & 15;     // rows i and i + 8
-        const int r0 = 32 * s + 16, c0 = 32 * s;
-        float y0 = 0.f, y1 = 0.f;
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-            const float xv = X[(c0 + j) * LX + c0 + c];
-            y0 = fmaf(A[(r0 + i) * LAA + c0 + j], xv, y0);
-            y1 = fmaf(A[(r0 + i + 8) * LAA + c0 + j], xv, y1);
-        }
-        Y[(r0 + i) * LA + c0 + c] = y0;
-        Y[(r0 + i + 8) * LA + c0 + c] = y1;
-    }
-    __syncthreads();
-    {
-        const int s = tid >> 7, i = (tid >> 4) & 7, c = tid & 15;
-        const int r0 = 32 * s + 16, c0 = 32 * s;
-        float x0 = 0.f, x1 = 0.f;
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-            const float yv = Y[(r0 + j) * LA + c0 + c];
-            x0 = fmaf(X[(r0 + i) * LX + r0 + j], yv, x0);
-            x1 = fmaf(X[(r0 + i + 8) * LX + r0 + j], yv, x1);
-        }
-        X[(r0 + i) * LX + c0 + c] = -x0;
-        X[(r0 + i + 8) * LX + c0 + c] = -x1;
-    }
-    __syncthreads();
-    const int c = tid & 31, i0 = tid >> 5;            // column c, rows i0 + 8 k of the 32 x 32 blocks
-    {   // Y21 = A21 X11
-        float y[4] = {};
-#pragma unroll 8
-        for (int j = 0; j < 32; ++j) {
-            const float xv = X[j * LX + c];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) y[k] = fmaf(A[(32 + i0 + 8 * k) * LAA + j], xv, y[k]);
-        }
-#pragma unroll
-        for (int k = 0; k < 4; ++k) Y[(32 + i0 + 8 * k) * LA + c] = y[k];
-    }
-    __syncthreads();
-    {   // X21 = -X22 Y21
-        float x[4] = {};
-#pragma unroll 8
-        for (int j = 0; j < 32; ++j) {
-            const float yv = Y[(32 + j) * LA + c];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) x[k] = fmaf(X[(32 + i0 + 8 * k) * LX + 32 + j], yv, x[k]);
-        }
-#pragma unroll
-        for (int k = 0; k < 4; ++k) X[(32 + i0 + 8 * k) * LX + c] = -x[k];
-    }
-    __syncthreads();
-}
-
 // C (64 x 64) = sum_m P[m][r] Q[m][c] for the fp32 tiles P, Q (row stride LX), on the TF32
 // tensor path (mma.sync m16n8k8; operands rounded to TF32, 10-bit mantissa, finer than the
 // bf16 operands of the other products).  Warp w: rows 16 (w % 4) .. + 15, columns
@@ -271,6 +184,7 @@ __global__ void __launch_bounds__(256, 1)
 bwd_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                 const __grid_constant__ CUtensorMap tm_s, const __grid_constant__ CUtensorMap tm_dsp,
+                const __grid_constant__ CUtensorMap tm_t, const float* __restrict__ Xg,
                 const bf16* __restrict__ beta, float* __restrict__ dq, float* __restrict__ dk, float* __restrict__ dv,
                 float* __restrict__ dbeta, int T, int rule, uint32_t* __restrict__ err, unsigned long long limit_ns,
                 BwdSpans spans) {
@@ -282,14 +196,12 @@ bwd_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     uint64_t* bar = reinterpret_cast<uint64_t*>(sm + BAR);    // 0: the tile's inputs, 1: MMA commits
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + MISC);
     volatile int* abort = reinterpret_cast<volatile int*>(sm + MISC + 4);
-    float* fA = reinterpret_cast<float*>(sm + RT);
-    float* fY = reinterpret_cast<float*>(sm + DL);
     float* fX = reinterpret_cast<float*>(sm + FX);
     float* fXT = reinterpret_cast<float*>(sm + FXT);
     float* fW = reinterpret_cast<float*>(sm + FW);
     float* fdT = reinterpret_cast<float*>(sm + FDT);
     float* al = reinterpret_cast<float*>(sm + SMALL);
-    float *bt = al + 64, *dal = al + 128, *lam = al + 192, *ones = al + 256, *part = al + 320;
+    float *bt = al + 64, *dal = al + 128, *lam = al + 192, *part = al + 320;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int q = warp & 3, h = warp >> 2;                    // TMEM lane quarter, column half
@@ -321,6 +233,9 @@ bwd_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         tma_load_2d(sm + DSP + 2 * TILE, &tm_dsp, rest, 64, (int)(tile * 128));
         tma_load_2d(sm + SS, &tm_s, rest, 0, (int)(tile * 128));
         tma_load_2d(sm + SS + 2 * TILE, &tm_s, rest, 64, (int)(tile * 128));
+        tma_load_2d(sm + TT, &tm_t, rest, 0, (int)(tile * 64));
+        const float* xs = Xg + tile * (64 * LX);
+        if (span_ok(err, spans.x, xs, 64 * LX * 4)) bulk_load(sm + FX, xs, 64 * LX * 4, rest);
     }
     const float beta_t = tid < nv && span_ok(err, spans.beta, beta + row0 + tid, 2)   // in flight during the setup
                              ? __bfloat162float(beta[row0 + tid]) : 0.f;
@@ -330,7 +245,6 @@ bwd_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
     if (tid < 64) {
         bt[tid] = beta_t;
-        ones[tid] = 1.f;
         dal[tid] = 0.f;
     }
     tc_fence_before();
@@ -386,28 +300,14 @@ bwd_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if (32 * h + j > t) g[j] = 0.f;
         st_row32(sm + PP, t, 4 * h, g);
     }
-    __syncthreads();
-    if (q < 2) {          // A = strict_tril(diag(alpha) G), fp32, for the solve
-        const float a = al[row];
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-            const int s = 32 * h + j;
-            fA[row * LAA + s] = s < row ? a * g[j] : 0.f;
-        }
-    }
     handoff();
-    // ---- 2. dDelta^T += dO^T P, while the CUDA cores solve for X = (I + A)^{-1}
+    // ---- 2. dDelta^T += dO^T P;  R^T = V^T - S^T K^T.  T and X = (I + A)^{-1} come from the
+    //         UT transform of the forward (its fp32 X and bf16 T), not from a solve here.
     if (warp == 0) {
         mma_ss(tm + C_DD, sb + DO, TILE, 2048, TILE, sb + PP, TILE, 2048, TILE, idesc(128, MN_MAJ, MN_MAJ), 4, true);
         commit();
     }
-    unit_lower_inverse64(fA, fX, fY, tid);            // ends with a barrier: A and the scratch are dead
-    {   // T = X diag(alpha), bf16 [t][s]: thread -> row tid / 4, 16 columns;  R^T = V^T - S^T K^T
-        const int t = tid >> 2, s0 = 16 * (tid & 3);
-        float x[16];
-#pragma unroll
-        for (int j = 0; j < 16; ++j) x[j] = fX[t * LX + s0 + j] * al[s0 + j];
-        st_row16(sm + TT, t, 2 * (tid & 3), x);
+    {
         wait_mma();       // dO^T P has landed
         float r[32];
         tmem_ld32_wait(tm + lane_off + C_SK + 32 * h, r);
@@ -870,10 +770,11 @@ constexpr unsigned long long kTileWaitNs = 2000000000ull;   // 2 s per wait
 
 size_t bwd_chunk_workspace_bytes(long BH, int T) {
     const long ntiles = BH * ((T + kC - 1) / kC);
-    return (size_t)ntiles * (kC * kC + 2 * kD * kD) * sizeof(bf16);   // T, S and dS' per tile
+    return (size_t)ntiles * ((kC * kC + 2 * kD * kD) * sizeof(bf16) + kUtXBytes);   // T, X, S and dS' per tile
 }
 
 size_t bwd_saved_t_bytes(long BH, int T) { return (size_t)BH * ((T + kC - 1) / kC) * kC * kC * sizeof(bf16); }
+size_t bwd_saved_x_bytes(long BH, int T) { return (size_t)BH * ((T + kC - 1) / kC) * kUtXBytes; }
 size_t bwd_saved_state_bytes(long BH, int T) { return (size_t)BH * ((T + kC - 1) / kC) * kD * kD * sizeof(bf16); }
 
 cudaError_t launch_bwd_chunk(const void* q, const void* k, const void* v, const void* beta, const float* S0,
@@ -882,24 +783,26 @@ cudaError_t launch_bwd_chunk(const void* q, const void* k, const void* v, const 
     const int nchunks = (T + kC - 1) / kC;
     const long ntiles = BH * nchunks;
     bf16* Tt = static_cast<bf16*>(scratch);
-    bf16* states = Tt + (size_t)ntiles * kC * kC;
+    float* X = reinterpret_cast<float*>(Tt + (size_t)ntiles * kC * kC);
+    bf16* states = reinterpret_cast<bf16*>(reinterpret_cast<char*>(X) + (size_t)ntiles * kUtXBytes);
     bf16* dSp = states + (size_t)ntiles * kD * kD;
-    // 1. UT transforms and the forward chain, storing every chunk's entering state
+    // 1. UT transforms (keeping X) and the forward chain, storing every chunk's entering state
     SegPlan plan;
     plan.states = states;
+    plan.X = X;
     Seqs seqs{nullptr, nullptr, 0, 0, T, 0};
     cudaError_t e = launch_chunk_tc(q, k, v, beta, S0, nullptr, nullptr, seqs, BH, BH, T, ntiles, err, Tt, rule,
                                     stream, nullptr, plan);
     if (e != cudaSuccess) return e;
     // 2, 3. the reverse chain and every chunk's gradients
-    return launch_bwd_chunk_saved(q, k, v, beta, dO, dST, dq, dk, dv, dbeta, dS0, BH, T, rule, err, Tt, states, dSp,
-                                  stream);
+    return launch_bwd_chunk_saved(q, k, v, beta, dO, dST, dq, dk, dv, dbeta, dS0, BH, T, rule, err, Tt, X, states,
+                                  dSp, stream);
 }
 
 cudaError_t launch_bwd_chunk_saved(const void* q, const void* k, const void* v, const void* beta, const void* dO,
                                    const float* dST, float* dq, float* dk, float* dv, float* dbeta, float* dS0,
-                                   long BH, int T, int rule, uint32_t* err, const void* Tt, const void* states,
-                                   void* dSp, cudaStream_t stream) {
+                                   long BH, int T, int rule, uint32_t* err, const void* Tt, const float* X,
+                                   const void* states, void* dSp, cudaStream_t stream) {
     const int nchunks = (T + kC - 1) / kC;
     const long ntiles = BH * nchunks;
     cudaError_t e;
@@ -919,6 +822,7 @@ cudaError_t launch_bwd_chunk_saved(const void* q, const void* k, const void* v, 
     sp.dbeta = Span{dbeta, tok * 4};
     sp.dst = Span{dST, sbytes};
     sp.ds0 = Span{dS0, sbytes};
+    sp.x = Span{X, (size_t)ntiles * kUtXBytes};
     static std::atomic<uint64_t> smem_chain{0}, smem_tile{0};
     e = set_smem_limit_once(bwd_chain_kernel, (int)rc::SMEM_BYTES, smem_chain);
     if (e != cudaSuccess) return e;
@@ -930,7 +834,7 @@ cudaError_t launch_bwd_chunk_saved(const void* q, const void* k, const void* v, 
     e = set_smem_limit_once(bwd_tile_kernel, (int)tb::SMEM_BYTES, smem_tile);
     if (e != cudaSuccess) return e;
     bwd_tile_kernel<<<(unsigned)ntiles, 256, tb::SMEM_BYTES, stream>>>(
-        mq, mk, mv, mdo, ms, mdsp, (const bf16*)beta, dq, dk, dv, dbeta, T, rule, err, kTileWaitNs, sp);
+        mq, mk, mv, mdo, ms, mdsp, mt, X, (const bf16*)beta, dq, dk, dv, dbeta, T, rule, err, kTileWaitNs, sp);
     return cudaGetLastError();
 }
 

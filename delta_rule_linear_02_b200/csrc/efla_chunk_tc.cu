@@ -771,7 +771,7 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const v
                             void* o, float* S_T, const Seqs& seqs, long nstreams, long Z, int Tdim, long ntiles,
                             uint32_t* err, void* scratch, int rule, cudaStream_t stream, const float* g,
                             const SegPlan& seg) {
-    cudaError_t e = launch_ut(k, beta, scratch, seqs, Z, Tdim, ntiles, err, kWaitLimitNs, rule, stream, g);
+    cudaError_t e = launch_ut(k, beta, scratch, seqs, Z, Tdim, ntiles, err, kWaitLimitNs, rule, stream, g, seg.X);
     if (e != cudaSuccess) return e;
     const long ctas = seg.G > 1 ? nstreams * (2 + 4 * (seg.G - 1)) : nstreams * 2;
     ChainSpans sp;

@@ -38,6 +38,7 @@ size_t chunk_tc_gated_workspace_bytes(long BH, int T);
 // of segment g is S_in(g) = Phi[g-1] S_in(g-1) + Sloc[g-1] and its outputs O_loc + R S_in(g).
 struct SegPlan {
     __nv_bfloat16* states = nullptr;   // if set: the entering state of every chunk, bf16 [tiles][128][128]
+    float* X = nullptr;                // if set: X = (I + A)^{-1} of every chunk, fp32 [tiles][64][68] (ungated)
     int G = 1;                     // 1: no segmentation
     int seg_chunks = 0;
     float* Sloc = nullptr;         // [nstreams][G][128][128]
@@ -68,7 +69,9 @@ cudaError_t launch_seg_correct(const SegPlan& seg, const void* SinT, __nv_bfloat
 // tiles: ntiles of `seqs` (dense: BH * ceil(T / 64); packed: H * tileoff[N]); tensors [Z][Tdim][d]
 cudaError_t launch_ut(const void* k, const void* beta, void* Tout, const Seqs& seqs, long Z, int Tdim,
                       long ntiles, uint32_t* err, unsigned long long limit_ns, int rule, cudaStream_t stream,
-                      const float* g = nullptr);
+                      const float* g = nullptr, float* Xout = nullptr);
+// bytes of one chunk's X as launch_ut writes it (fp32 64 x 64, rows padded to 68 floats)
+constexpr size_t kUtXBytes = 64 * 68 * 4;
 
 // reverse-mode pass (efla_bwd.cu): fp32 gradients; workspace of bwd_workspace_bytes
 size_t bwd_workspace_bytes(long BH, int T, int D);
@@ -86,15 +89,17 @@ size_t bwd_chunk_workspace_bytes(long BH, int T);
 cudaError_t launch_bwd_chunk(const void* q, const void* k, const void* v, const void* beta, const float* S0,
                              const void* dO, const float* dST, float* dq, float* dk, float* dv, float* dbeta,
                              float* dS0, long BH, int T, int rule, uint32_t* err, void* scratch, cudaStream_t stream);
-// the same from saved residuals (training): T of every chunk (Tt, ntiles x 64 x 64 bf16) and every
-// chunk's entering state (states, ntiles x 128 x 128 bf16) as the forward left them; dSp: the
-// per-chunk dS' scratch (ntiles x 128 x 128 bf16)
+// the same from saved residuals (training): T of every chunk (Tt, ntiles x 64 x 64 bf16), its
+// X = (I + A)^{-1} (fp32, kUtXBytes each) and every chunk's entering state (states, ntiles x
+// 128 x 128 bf16) as the forward left them; dSp: the per-chunk dS' scratch (bf16 128 x 128)
 cudaError_t launch_bwd_chunk_saved(const void* q, const void* k, const void* v, const void* beta, const void* dO,
                                    const float* dST, float* dq, float* dk, float* dv, float* dbeta, float* dS0,
-                                   long BH, int T, int rule, uint32_t* err, const void* Tt, const void* states,
-                                   void* dSp, cudaStream_t stream);
-// bytes of T and of the entering states kept for the backward (bf16, d = 128)
+                                   long BH, int T, int rule, uint32_t* err, const void* Tt, const float* X,
+                                   const void* states, void* dSp, cudaStream_t stream);
+// bytes of T (bf16), of X (fp32, launch_ut's padded tiles) and of the entering states (bf16)
+// kept for the backward (d = 128)
 size_t bwd_saved_t_bytes(long BH, int T);
+size_t bwd_saved_x_bytes(long BH, int T);
 size_t bwd_saved_state_bytes(long BH, int T);
 
 cudaError_t launch_wait_timeout_selftest(uint32_t* err, unsigned long long limit_ns, cudaStream_t stream);

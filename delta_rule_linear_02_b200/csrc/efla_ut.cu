@@ -95,7 +95,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 ut_kernel(const __grid_constant__ CUtensorMap tm_k, const __nv_bfloat16* __restrict__ beta,
           __nv_bfloat16* __restrict__ Tout, Seqs seqs, int Tdim, long ntiles, uint32_t* __restrict__ err,
           unsigned long long limit_ns, int rule, const float* __restrict__ gdec, Span t_span, Span b_span,
-          Span g_span) {
+          Span g_span, float* __restrict__ Xout, Span x_span) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sb = smem_u32(sm);
@@ -283,6 +283,7 @@ ut_kernel(const __grid_constant__ CUtensorMap tm_k, const __nv_bfloat16* __restr
                 }
             }
             tc_fence_before();
+            if (Xout && wt == 0) tma_store_wait_read();   // the last tile's X has been copied out
             bar_sync(NB_W, 128);                     // G read, A^T written
             if (wt == 0) mbar_arrive(bar + B_GP_FREE);
             ut::ut_solve<NB_W, 128>(At, X, wt);
@@ -291,6 +292,10 @@ ut_kernel(const __grid_constant__ CUtensorMap tm_k, const __nv_bfloat16* __restr
             fence_proxy_async_smem();
             bar_sync(NB_W, 128);
             if (wt == 0) mbar_arrive(bar + B_AT_FREE);
+            if (Xout && wt == 0) {   // X itself, for the backward: one bulk copy of the padded tile
+                float* dst = Xout + (first + (long)j * step) * 64 * LDX;
+                if (span_ok(err, x_span, dst, F32_TILE)) bulk_store(dst, X, F32_TILE);
+            }
             {   // T = X diag(alpha) -> bf16, 64 bytes per thread (a warp reads 32 consecutive
                 // rows of one column half: conflict-free with the 68-float row stride).
                 // Gated: T_W = X diag(alpha Gam), T_U = X diag(abar), and the row's G log2(e).
@@ -325,6 +330,7 @@ ut_kernel(const __grid_constant__ CUtensorMap tm_k, const __nv_bfloat16* __restr
         }
     }
 
+    if (Xout && tid == 32) tma_store_wait_all();
     tc_fence_before();
     __syncthreads();
     if (tid == 0 && *abort) atomicOr(err, kDevTimeout);
@@ -342,13 +348,14 @@ int sm_count() {
 
 cudaError_t launch_ut(const void* k, const void* beta, void* Tout, const Seqs& seqs, long Z, int Tdim,
                       long ntiles, uint32_t* err, unsigned long long limit_ns, int rule, cudaStream_t stream,
-                      const float* g) {
+                      const float* g, float* Xout) {
     if (ntiles == 0) return cudaSuccess;
     CUtensorMap mk;
     if (!tma_map_tokens(&mk, k, 128, Tdim, Z)) return cudaErrorInvalidValue;
     const long grid = std::min<long>(ntiles, (long)sm_count() * kCtasPerSm);
     const Span t_span{Tout, (size_t)ntiles * (g ? 2 * 8192 + 256 : 8192)};
     const Span b_span{beta, (size_t)Z * Tdim * 2}, g_span{g, (size_t)Z * Tdim * 4};
+    const Span x_span{Xout, (size_t)ntiles * F32_TILE};
     cudaError_t e;
     if (g) {
         static std::atomic<uint64_t> smem_set_g{0};
@@ -356,14 +363,14 @@ cudaError_t launch_ut(const void* k, const void* beta, void* Tout, const Seqs& s
         if (e != cudaSuccess) return e;
         ut_kernel<true><<<(unsigned)grid, kThreads, SMEM_BYTES_G, stream>>>(
             mk, (const __nv_bfloat16*)beta, (__nv_bfloat16*)Tout, seqs, Tdim, ntiles, err, limit_ns, rule, g, t_span,
-            b_span, g_span);
+            b_span, g_span, nullptr, x_span);
     } else {
         static std::atomic<uint64_t> smem_set{0};
         e = set_smem_limit_once(ut_kernel<false>, (int)SMEM_BYTES, smem_set);
         if (e != cudaSuccess) return e;
         ut_kernel<false><<<(unsigned)grid, kThreads, SMEM_BYTES, stream>>>(
             mk, (const __nv_bfloat16*)beta, (__nv_bfloat16*)Tout, seqs, Tdim, ntiles, err, limit_ns, rule, nullptr,
-            t_span, b_span, g_span);
+            t_span, b_span, g_span, Xout, x_span);
     }
     return cudaGetLastError();
 }

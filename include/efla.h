@@ -315,8 +315,8 @@ int efla_recurrent_step_ex(const void *q, const void *k, const void *v, const vo
 /*
  * efla_backward_workspace_bytes -- bytes of device workspace efla_backward needs.  bf16 with
  * d = 128 (the chunkwise form): a 256-byte header (the device error word) and, per 64-token
- * chunk, its UT transform (bf16 64 x 64), its entering state and its dS' (bf16 128 x 128
- * each).  Otherwise (the token sweep): B*H*T*d_v + B*H*T floats (the residuals
+ * chunk, its UT transform T (bf16 64 x 64), X = (I + A)^{-1} (fp32 64 x 64, rows padded
+ * to 68), its entering state and its dS' (bf16 128 x 128 each).  Otherwise (the token sweep): B*H*T*d_v + B*H*T floats (the residuals
  * r_t = S_{t-1}^T k_t - v_t of a forward sweep, and the gate gradient).  0 for an
  * unsupported shape or dtype.
  */
@@ -371,8 +371,9 @@ int efla_backward_ex(const void *q, const void *k, const void *v, const void *be
  * state chain).
  *
  * efla_train_saved_bytes -- bytes of `saved`: a 256-byte header (the forward's device error
- *   word), the UT transform T of every 64-token chunk (bf16 64 x 64) and every chunk's
- *   entering state (bf16 128 x 128).  0 for any other shape, dtype or chunk.
+ *   word), the UT transform T of every 64-token chunk (bf16 64 x 64) with its
+ *   X = (I + A)^{-1} (fp32 64 x 64, rows padded to 68) and every chunk's entering state
+ *   (bf16 128 x 128).  0 for any other shape, dtype or chunk.
  *
  * efla_chunk_fwd_save -- efla_chunk_fwd_ex with `saved` (>= efla_train_saved_bytes,
  *   16-byte aligned, caller-owned) as its workspace: the same outputs, the same bits, and

@@ -164,8 +164,10 @@ GOOD_B = [ctypes.c_void_p(0x10000000 + 0x1000000 * i) for i in range(13)]
 
 def test_backward_workspace_bytes(efla):
     L = efla.lib
-    # bf16, d = 128 (the chunkwise path): error word + per tile T (64 x 64), S and dS' (128 x 128), bf16
-    assert L.efla_backward_workspace_bytes(4, 16, 2048, 128, 128, 1) == 256 + 64 * 32 * (64 * 64 + 2 * 128 * 128) * 2
+    # bf16, d = 128 (the chunkwise path): error word + per tile T (64 x 64 bf16), X (64 x 68 fp32),
+    # S and dS' (128 x 128 bf16)
+    assert L.efla_backward_workspace_bytes(4, 16, 2048, 128, 128, 1) == \
+        256 + 64 * 32 * ((64 * 64 + 2 * 128 * 128) * 2 + 64 * 68 * 4)
     # the reverse sweep: residuals and the gate gradient, fp32
     assert L.efla_backward_workspace_bytes(4, 16, 2048, 128, 128, 0) == 4 * 16 * 2048 * (128 + 1) * 4
     assert L.efla_backward_workspace_bytes(1, 1, 1, 96, 96, 0) == 0      # unsupported d
@@ -273,7 +275,8 @@ def test_training_entry_points_sizes_and_validation(efla):
     rejection happens before anything is launched."""
     L = efla.lib
     tiles = 4 * 16 * 32
-    assert L.efla_train_saved_bytes(4, 16, 2048, 128, 128, 64, 1) == 256 + tiles * (64 * 64 + 128 * 128) * 2
+    assert L.efla_train_saved_bytes(4, 16, 2048, 128, 128, 64, 1) == \
+        256 + tiles * ((64 * 64 + 128 * 128) * 2 + 64 * 68 * 4)
     assert L.efla_backward_saved_workspace_bytes(4, 16, 2048, 128, 128, 1) == 256 + tiles * 128 * 128 * 2
     for args in ((1, 1, 64, 64, 64, 64, 1), (1, 1, 64, 128, 128, 64, 0), (1, 1, 64, 128, 128, 32, 1),
                  (1, 1, -1, 128, 128, 64, 1)):
