@@ -75,6 +75,7 @@ KERNEL_SOURCES = {
     "efla_recurrent_step": ["efla_decode.cu", "efla_common.cuh"],
     "efla_backward": ["efla_bwd.cu", "efla_bwd_chunk.cu", "efla_chunk_tc.cu", "efla_ut.cu",
                       "efla_ut_tf32.cuh", "efla_common.cuh", "efla_tma.cuh", "sm100.cuh"],
+    "efla_backward_saved": ["efla_bwd_chunk.cu", "efla_common.cuh", "efla_tma.cuh", "sm100.cuh"],
 }
 
 
@@ -129,6 +130,7 @@ ENTRY_KERNELS = {
     "efla_chunk_fwd": ("ut_kernel", "chunk_tc_kernel"),
     "efla_recurrent_step": ("decode_kernel",),
     "efla_backward": ("ut_kernel", "chunk_tc_kernel", "bwd_chain_kernel", "bwd_tile_kernel"),
+    "efla_backward_saved": ("bwd_chain_kernel", "bwd_tile_kernel"),
 }
 
 
@@ -389,10 +391,19 @@ def profile_call(args):
             f32 = dict(device=dev, dtype=torch.float32)
             g = (torch.empty(B, H, T, d, **f32), torch.empty(B, H, T, d, **f32), torch.empty(B, H, T, d, **f32),
                  torch.empty(B, H, T, **f32), torch.empty(B, H, d, d, **f32))
-            wsb = torch.zeros(efla.efla_backward_workspace_bytes(B, H, T, d, d, w.dtype), dtype=torch.uint8,
-                              device=dev)
-            one = lambda: efla.efla_backward(x["q"], x["k"], x["v"], x["beta"], dO, grads=g, workspace=wsb,
-                                             stream=stream)
+            if args.profile_call == "bwd":
+                wsb = torch.zeros(efla.efla_backward_workspace_bytes(B, H, T, d, d, w.dtype), dtype=torch.uint8,
+                                  device=dev)
+                one = lambda: efla.efla_backward(x["q"], x["k"], x["v"], x["beta"], dO, grads=g, workspace=wsb,
+                                                 stream=stream)
+            else:       # the backward from saved residuals; the forward that saves them runs once first
+                ob = torch.empty(B, H, T, d, dtype=w.dtype, device=dev)
+                _, _, saved = efla.efla_chunk_fwd_save(x["q"], x["k"], x["v"], x["beta"], o=ob, want_state=False,
+                                                       stream=stream)
+                wss = torch.zeros(efla.lib.efla_backward_saved_workspace_bytes(B, H, T, d, d, efla.EFLA_DTYPE_BF16),
+                                  dtype=torch.uint8, device=dev)
+                one = lambda: efla.efla_backward_saved(x["q"], x["k"], x["v"], x["beta"], dO, saved, grads=g,
+                                                       workspace=wss, stream=stream)
         calls = [one] * (args.warmup + args.steps)
     for c in calls:
         c()
@@ -412,7 +423,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--other-steps", type=int, default=10,
                     help="forwards timed on each of the long-context and stiff workloads (0: skip)")
-    ap.add_argument("--profile-call", choices=["fwd", "decode", "bwd", "long", "longseg", "gated"],
+    ap.add_argument("--profile-call", choices=["fwd", "decode", "bwd", "bwd_saved", "long", "longseg", "gated"],
                     help="only run warm-up + steps calls of one entry point (for an ncu capture)")
     ap.add_argument("--traffic-from", metavar="CSV",
                     help="write profiles/traffic.json's record from an ncu --csv log of "
@@ -630,6 +641,7 @@ def main():
         bs_ms = timed(call_bs, args.bwd_steps)
         ts_ms = timed(lambda: (call_fs(), call_bs()), args.bwd_steps)
         bsrf = roofline_record(bbytes, bflops, bs_ms * 1e-3, hbm, tc, peak_kind)
+        bsrf["traffic"] = ncu_traffic("efla_backward_saved")
         bwd["saved_residuals"] = {
             "what": "efla_backward_saved: the same gradients from T and the chunk states that "
                     "efla_chunk_fwd_save kept (no forward recompute)",
