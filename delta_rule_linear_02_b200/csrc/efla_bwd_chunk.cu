@@ -99,15 +99,20 @@ constexpr uint32_t LOAD_BYTES = 131072 + 64 * 68 * 4 + 8192;   // K, Q, V, dO, d
 // nk k-steps of K = 16 with A and B in shared memory; operand k-step ks starts at
 // base + (ks / 4) * atom + (ks % 4) * step (K-major: step 32 bytes inside a 64-column atom;
 // MN-major: step 16 rows = 2048 bytes, atom 64 rows = 8192 bytes; lbo = distance between
-// 64-element MN blocks of an MN-major operand).
+// 64-element MN blocks of an MN-major operand).  Called by a whole converged warp; the lane
+// elect.sync picks builds the descriptors and issues all nk MMAs (one branch per product:
+// about half the code of an elect.sync per MMA, in kernels whose phases each run once).
 __device__ __forceinline__ void mma_ss(uint32_t d, uint32_t a, uint32_t a_atom, uint32_t a_step, uint32_t a_lbo,
                                        uint32_t b, uint32_t b_atom, uint32_t b_step, uint32_t b_lbo, uint32_t idesc,
                                        int nk, bool acc) {
-    const uint64_t da = sm100::sdesc_sw128(a, a_lbo, 1024), db = sm100::sdesc_sw128(b, b_lbo, 1024);
+    if (sm100::elect_one()) {
+        const uint64_t da = sm100::sdesc_sw128(a, a_lbo, 1024), db = sm100::sdesc_sw128(b, b_lbo, 1024);
 #pragma unroll
-    for (int ks = 0; ks < nk; ++ks)
-        sm100::mma_bf16_elect(d, da + (((ks >> 2) * a_atom + (ks & 3) * a_step) >> 4),
-                              db + (((ks >> 2) * b_atom + (ks & 3) * b_step) >> 4), idesc, acc || ks > 0);
+        for (int ks = 0; ks < nk; ++ks)
+            sm100::mma_bf16(d, da + (((ks >> 2) * a_atom + (ks & 3) * a_step) >> 4),
+                            db + (((ks >> 2) * b_atom + (ks & 3) * b_step) >> 4), idesc, acc || ks > 0);
+    }
+    __syncwarp();
 }
 constexpr uint32_t K_MAJ = 0, MN_MAJ = 1;
 __host__ __device__ constexpr uint32_t idesc(int M, uint32_t a, uint32_t b) {

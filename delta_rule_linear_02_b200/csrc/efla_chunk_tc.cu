@@ -218,7 +218,9 @@ __device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a_tmem, uint32_t b, 
                           (acc | ks) != 0);
 }
 
-template <bool kGated>
+// kSeg: the segmented scan's roles (G > 1) and the chunk states kept for the backward are
+// compiled in; the plain forward runs the instantiation without them (a smaller kernel).
+template <bool kGated, bool kSeg>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_t,
@@ -249,7 +251,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     float* stp;                   // final state (128 x 128) or null
     __nv_bfloat16* op = o;        // outputs [.., Tdim, 128]
     bool vzero = false;           // transition product: V = 0
-    if (seg.G <= 1) {
+    if (!kSeg || seg.G <= 1) {
         sidx = blockIdx.x >> 1;
         jb = seqs.job(sidx);
         col0 = (blockIdx.x & 1) * 64;
@@ -286,7 +288,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     // the extents this CTA's pointers must stay inside (checked builds)
     const Span op_span = op == o ? spans.o : spans.r;
     const bool st_in_phi = seg.Phi && stp >= seg.Phi && stp < seg.Phi + spans.phi.bytes / sizeof(float);
-    const Span st_span = seg.G <= 1 ? spans.st : (st_in_phi ? spans.phi : spans.sloc);
+    const Span st_span = (!kSeg || seg.G <= 1) ? spans.st : (st_in_phi ? spans.phi : spans.sloc);
     const Span s0_span = spans.s0;
     if (nchunks == 0) {   // an empty sequence: the state passes through (nothing else runs)
         if (stp) {
@@ -420,7 +422,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             tc_fence_after();
             mma_ts(tmem + TM_X, tmem + TM_AWQ, sb + OFF_SB, 4 * 2048, 2048, TILE, ID_N64, 8, 0);
             mma_commit_elect(ctl.b(B_XS_FULL));
-            if (seg.states && lane == 0) {   // chunk c's entering state, for the backward: one TMA store
+            if (kSeg && seg.states && lane == 0) {   // chunk c's entering state, for the backward: one TMA store
                 const long srow = (jb.tile0 + c) * kD;
                 if (span_ok(err, spans.states, seg.states + (srow + kD) * kD - 1, 2))
                     tma_store_2d(&tm_st, sm + OFF_SB, col0, (int)srow);
@@ -432,7 +434,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             issue_qk(c, 0, 8);
             // S += K^T Delta (state chain)
             if (!(ok = wait(B_D_READY, c & 1))) break;
-            if (seg.states && lane == 0) tma_store_wait_read();   // the bf16 S is rewritten after this product
+            if (kSeg && seg.states && lane == 0) tma_store_wait_read();   // the bf16 S is rewritten after this product
             __syncwarp();
             tc_fence_after();
             mma_ss(tmem + TM_S, sb + kvt(c) + KVT_K, 4 * 2048, 2048, TILE, sb + L::OFF_DL2, 4 * 2048, 2048, TILE,
@@ -455,7 +457,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         mma_commit_elect(ctl.b(B_DRAIN));
         if (lane == 0) {
             mbar_wait(ctl.b(B_DRAIN), 0, limit_ns);
-            if (seg.states) tma_store_wait_all();
+            if (kSeg && seg.states) tma_store_wait_all();
         }
         __syncwarp();
     } else if (warp == 4 || warp == 5) {
@@ -790,20 +792,32 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const v
         !tma_map_tokens(&mv, v, kD, Tdim, Z) || !tma_map_rows64(&mt, scratch, std::max<long>(1, (g ? 2 : 1) * ntiles) * 64) ||
         !(seg.states ? tma_map_rows128(&mst, seg.states, std::max<long>(1, ntiles) * kD) : (mst = mt, true)))
         return cudaErrorInvalidValue;
+    const float* gl = g ? reinterpret_cast<const float*>(static_cast<const char*>(scratch) + ntiles * 8192 * 2)
+                        : nullptr;
+    const bool full = seg.G > 1 || seg.states;
     if (g) {
-        const float* gl = reinterpret_cast<const float*>(static_cast<const char*>(scratch) + ntiles * 8192 * 2);
-        static std::atomic<uint64_t> smem_set_g{0};
-        e = set_smem_limit_once(chunk_tc_kernel<true>, (int)Lay<true>::SMEM_BYTES, smem_set_g);
+        static std::atomic<uint64_t> smem_set_g{0}, smem_set_gs{0};
+        e = full ? set_smem_limit_once(chunk_tc_kernel<true, true>, (int)Lay<true>::SMEM_BYTES, smem_set_gs)
+                 : set_smem_limit_once(chunk_tc_kernel<true, false>, (int)Lay<true>::SMEM_BYTES, smem_set_g);
         if (e != cudaSuccess) return e;
-        chunk_tc_kernel<true><<<(unsigned)ctas, kThreads, Lay<true>::SMEM_BYTES, stream>>>(
-            mq, mk, mv, mt, mst, S0, (__nv_bfloat16*)o, S_T, seqs, Tdim, err, kWaitLimitNs, gl, ntiles, seg, sp);
+        if (full)
+            chunk_tc_kernel<true, true><<<(unsigned)ctas, kThreads, Lay<true>::SMEM_BYTES, stream>>>(
+                mq, mk, mv, mt, mst, S0, (__nv_bfloat16*)o, S_T, seqs, Tdim, err, kWaitLimitNs, gl, ntiles, seg, sp);
+        else
+            chunk_tc_kernel<true, false><<<(unsigned)ctas, kThreads, Lay<true>::SMEM_BYTES, stream>>>(
+                mq, mk, mv, mt, mst, S0, (__nv_bfloat16*)o, S_T, seqs, Tdim, err, kWaitLimitNs, gl, ntiles, seg, sp);
         return cudaGetLastError();
     }
-    static std::atomic<uint64_t> smem_set{0};
-    e = set_smem_limit_once(chunk_tc_kernel<false>, (int)Lay<false>::SMEM_BYTES, smem_set);
+    static std::atomic<uint64_t> smem_set{0}, smem_set_s{0};
+    e = full ? set_smem_limit_once(chunk_tc_kernel<false, true>, (int)Lay<false>::SMEM_BYTES, smem_set_s)
+             : set_smem_limit_once(chunk_tc_kernel<false, false>, (int)Lay<false>::SMEM_BYTES, smem_set);
     if (e != cudaSuccess) return e;
-    chunk_tc_kernel<false><<<(unsigned)ctas, kThreads, Lay<false>::SMEM_BYTES, stream>>>(
-        mq, mk, mv, mt, mst, S0, (__nv_bfloat16*)o, S_T, seqs, Tdim, err, kWaitLimitNs, nullptr, ntiles, seg, sp);
+    if (full)
+        chunk_tc_kernel<false, true><<<(unsigned)ctas, kThreads, Lay<false>::SMEM_BYTES, stream>>>(
+            mq, mk, mv, mt, mst, S0, (__nv_bfloat16*)o, S_T, seqs, Tdim, err, kWaitLimitNs, nullptr, ntiles, seg, sp);
+    else
+        chunk_tc_kernel<false, false><<<(unsigned)ctas, kThreads, Lay<false>::SMEM_BYTES, stream>>>(
+            mq, mk, mv, mt, mst, S0, (__nv_bfloat16*)o, S_T, seqs, Tdim, err, kWaitLimitNs, nullptr, ntiles, seg, sp);
     return cudaGetLastError();
 }
 
