@@ -384,8 +384,15 @@ def profile_call(args):
             ws = efla.new_workspace(B, H, T, d, d, 64, w.dtype, dev)
             o = torch.empty(B, H, T, d, dtype=w.dtype, device=dev)
             ST = torch.empty(B, H, d, d, dtype=torch.float32, device=dev)
-            one = lambda: efla.efla_chunk_fwd(x["q"], x["k"], x["v"], x["beta"], x["S0"], o=o, S_T=ST,
-                                              workspace=ws, stream=stream)
+            # --profile-rotate N: N input sets taken in turn, as in the timed region (so that an
+            # ncu capture with --cache-control none sees the L2 state the timed calls see)
+            xs = [x] + [{k: (None if v is None else v.to(dev))
+                         for k, v in workloads.make_chunk_inputs(w.replace(seed=w.seed + 1 + r)).items()}
+                        for r in range(max(1, args.profile_rotate) - 1)]
+            calls = [lambda xi=xs[i % len(xs)]: efla.efla_chunk_fwd(xi["q"], xi["k"], xi["v"], xi["beta"], xi["S0"],
+                                                                    o=o, S_T=ST, workspace=ws, stream=stream)
+                     for i in range(args.warmup + args.steps)]
+            one = None
         else:
             dO = workloads.make_cotangents(w, with_state_grad=False)["dO"].to(dev)
             f32 = dict(device=dev, dtype=torch.float32)
@@ -404,7 +411,8 @@ def profile_call(args):
                                   dtype=torch.uint8, device=dev)
                 one = lambda: efla.efla_backward_saved(x["q"], x["k"], x["v"], x["beta"], dO, saved, grads=g,
                                                        workspace=wss, stream=stream)
-        calls = [one] * (args.warmup + args.steps)
+        if one is not None:
+            calls = [one] * (args.warmup + args.steps)
     for c in calls:
         c()
     torch.cuda.synchronize(dev)
@@ -425,6 +433,8 @@ def main():
                     help="forwards timed on each of the long-context and stiff workloads (0: skip)")
     ap.add_argument("--profile-call", choices=["fwd", "decode", "bwd", "bwd_saved", "long", "longseg", "gated"],
                     help="only run warm-up + steps calls of one entry point (for an ncu capture)")
+    ap.add_argument("--profile-rotate", type=int, default=1,
+                    help="with --profile-call fwd: input sets taken in turn (the timed region uses %d)" % N_ROTATE)
     ap.add_argument("--traffic-from", metavar="CSV",
                     help="write profiles/traffic.json's record from an ncu --csv log of "
                          "dram__bytes_read.sum and dram__bytes_write.sum, then exit")
