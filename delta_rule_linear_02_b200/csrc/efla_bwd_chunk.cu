@@ -87,15 +87,17 @@ constexpr uint32_t FW = TT + F32;          // W = dX X^T
 constexpr uint32_t FDT = V;                // dT^T, then dX^T, then dA
 constexpr uint32_t SMALL = FX + F32;       // alpha, beta, dalpha, lambda, (unused), two partial sums (fp32 [64] each)
 constexpr uint32_t BAR = SMALL + 7 * 256;  // mbarriers: the tile's inputs, MMA commits
-constexpr uint32_t MISC = BAR + 3 * 8;     // TMEM base, abort flag
+constexpr uint32_t MISC = BAR + 6 * 8;     // TMEM base, abort flag
 constexpr uint32_t SMEM_BYTES = MISC + 16 + 1024;
 static_assert(64 * LX * 4 == kUtXBytes, "X as the UT transform writes it");
 static_assert(FDT + F32 <= DSP && FW + F32 <= DG, "fp32 tiles stay inside dead regions");
 static_assert(SMEM_BYTES <= 232448, "shared memory");
 // TMEM columns (fp32 accumulators, 64 columns each)
 constexpr uint32_t C_GP = 0, C_SK = 64, C_DQ = 128, C_DL = 192, C_DD = 256, C_DK = 320, C_DR = 384, C_COLS = 512;
-constexpr uint32_t LOAD_BYTES = 114688;                         // K, Q, dO, dS', S: the first products' operands
-constexpr uint32_t LOAD2_BYTES = 16384 + 8192 + 64 * 68 * 4;     // V, T, X: needed from the second epilogue on
+// the tile's inputs, on five barriers in the order the first products need them
+enum : int { L_KQ = 0, L_VTX = 2, L_S = 3, L_DSP = 4, L_DO = 5 };   // (1: the MMA commits)
+constexpr uint32_t KQ_BYTES = 32768, S_BYTES = 32768, DSP_BYTES = 32768, DO_BYTES = 16384;
+constexpr uint32_t VTX_BYTES = 16384 + 8192 + 64 * 68 * 4;          // V, T, X: from the second epilogue on
 
 // nk k-steps of K = 16 with A and B in shared memory; operand k-step ks starts at
 // base + (ks / 4) * atom + (ks % 4) * step (K-major: step 32 bytes inside a 64-column atom;
@@ -199,7 +201,7 @@ bwd_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sb = smem_u32(sm);
-    uint64_t* bar = reinterpret_cast<uint64_t*>(sm + BAR);    // 0, 2: the tile's inputs, 1: MMA commits
+    uint64_t* bar = reinterpret_cast<uint64_t*>(sm + BAR);    // 1: MMA commits, the others the tile's inputs
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + MISC);
     volatile int* abort = reinterpret_cast<volatile int*>(sm + MISC + 4);
     float* fX = reinterpret_cast<float*>(sm + FX);
@@ -221,26 +223,27 @@ bwd_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const size_t row0 = (size_t)bh * T + t0;
 
     if (tid == 0) {
-        mbar_init(bar, 1);
-        mbar_init(bar + 1, 1);
-        mbar_init(bar + 2, 1);
+        for (int i = 0; i < 6; ++i) mbar_init(bar + i, 1);
         *abort = 0;
         fence_mbar_init();
-        // the first batch of products' operands on barrier 0, V, T and X on barrier 2 (they
-        // land while the first products run)
-        mbar_arrive_expect_tx(bar, LOAD_BYTES);
-        mbar_arrive_expect_tx(bar + 2, LOAD2_BYTES);
-        tma_load_3d(sm + KQ, &tm_k, bar, 0, t0, (int)bh);
-        tma_load_3d(sm + KQ + 2 * TILE, &tm_k, bar, 64, t0, (int)bh);
-        tma_load_3d(sm + KQ + TILE, &tm_q, bar, 0, t0, (int)bh);
-        tma_load_3d(sm + KQ + 3 * TILE, &tm_q, bar, 64, t0, (int)bh);
-        tma_load_3d(sm + DO, &tm_do, bar, 0, t0, (int)bh);
-        tma_load_3d(sm + DO + TILE, &tm_do, bar, 64, t0, (int)bh);
-        tma_load_2d(sm + DSP, &tm_dsp, bar, 0, (int)(tile * 128));
-        tma_load_2d(sm + DSP + 2 * TILE, &tm_dsp, bar, 64, (int)(tile * 128));
-        tma_load_2d(sm + SS, &tm_s, bar, 0, (int)(tile * 128));
-        tma_load_2d(sm + SS + 2 * TILE, &tm_s, bar, 64, (int)(tile * 128));
-        uint64_t* rest = bar + 2;
+        // each of the first products starts once its operands have landed; V, T and X land
+        // while those products run
+        mbar_arrive_expect_tx(bar + L_KQ, KQ_BYTES);
+        mbar_arrive_expect_tx(bar + L_S, S_BYTES);
+        mbar_arrive_expect_tx(bar + L_DSP, DSP_BYTES);
+        mbar_arrive_expect_tx(bar + L_DO, DO_BYTES);
+        mbar_arrive_expect_tx(bar + L_VTX, VTX_BYTES);
+        tma_load_3d(sm + KQ, &tm_k, bar + L_KQ, 0, t0, (int)bh);
+        tma_load_3d(sm + KQ + 2 * TILE, &tm_k, bar + L_KQ, 64, t0, (int)bh);
+        tma_load_3d(sm + KQ + TILE, &tm_q, bar + L_KQ, 0, t0, (int)bh);
+        tma_load_3d(sm + KQ + 3 * TILE, &tm_q, bar + L_KQ, 64, t0, (int)bh);
+        tma_load_2d(sm + SS, &tm_s, bar + L_S, 0, (int)(tile * 128));
+        tma_load_2d(sm + SS + 2 * TILE, &tm_s, bar + L_S, 64, (int)(tile * 128));
+        tma_load_2d(sm + DSP, &tm_dsp, bar + L_DSP, 0, (int)(tile * 128));
+        tma_load_2d(sm + DSP + 2 * TILE, &tm_dsp, bar + L_DSP, 64, (int)(tile * 128));
+        tma_load_3d(sm + DO, &tm_do, bar + L_DO, 0, t0, (int)bh);
+        tma_load_3d(sm + DO + TILE, &tm_do, bar + L_DO, 64, t0, (int)bh);
+        uint64_t* rest = bar + L_VTX;
         tma_load_3d(sm + V, &tm_v, rest, 0, t0, (int)bh);
         tma_load_3d(sm + V + TILE, &tm_v, rest, 64, t0, (int)bh);
         tma_load_2d(sm + TT, &tm_t, rest, 0, (int)(tile * 64));
@@ -280,13 +283,20 @@ bwd_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     };
 
     // ---- 1. [G; P~] = [K; Q] K^T;  dDelta^T = dS'^T K^T (+ dO^T P below);  S^T K^T;  dQ^T = S dO^T
-    wait(0, 0);
-    if (warp == 0) {
+    //      (every thread waits on each input barrier; warp 0 issues each product as its operands land)
+    wait(L_KQ, 0);
+    if (warp == 0)
         mma_ss(tm + C_GP, sb + KQ, 2 * TILE, 32, 16, sb + KQ, 2 * TILE, 32, 16, idesc(128, K_MAJ, K_MAJ), 8, false);
-        mma_ss(tm + C_DD, sb + DSP, TILE, 2048, 2 * TILE, sb + KQ, 2 * TILE, 32, 16, idesc(128, MN_MAJ, K_MAJ), 8,
-               false);
+    wait(L_S, 0);
+    if (warp == 0)
         mma_ss(tm + C_SK, sb + SS, TILE, 2048, 2 * TILE, sb + KQ, 2 * TILE, 32, 16, idesc(128, MN_MAJ, K_MAJ), 8,
                false);
+    wait(L_DSP, 0);
+    if (warp == 0)
+        mma_ss(tm + C_DD, sb + DSP, TILE, 2048, 2 * TILE, sb + KQ, 2 * TILE, 32, 16, idesc(128, MN_MAJ, K_MAJ), 8,
+               false);
+    wait(L_DO, 0);
+    if (warp == 0) {
         mma_ss(tm + C_DQ, sb + SS, 2 * TILE, 32, 16, sb + DO, TILE, 32, 16, idesc(128, K_MAJ, K_MAJ), 8, false);
         commit();
     }
@@ -319,7 +329,7 @@ bwd_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
     {
         wait_mma();       // dO^T P has landed
-        wait(2, 0);       // V, T and X have landed
+        wait(L_VTX, 0);   // V, T and X have landed
         float r[32];
         tmem_ld32_wait(tm + lane_off + C_SK + 32 * h, r);
 #pragma unroll
