@@ -381,9 +381,10 @@ bwd_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
     wait_mma();
     {
-        float x[32];
+        float x[32], y[32], z[32];
+        tmem_ld32x3_wait(tm + lane_off + C_DR + 32 * h, tm + lane_off + C_DQ + 32 * h, tm + lane_off + C_SK + 32 * h,
+                         x, y, z);
         // dV = dR: dv[token][j] for this thread's j = row (a warp stores 32 consecutive floats)
-        tmem_ld32_wait(tm + lane_off + C_DR + 32 * h, x);
 #pragma unroll
         for (int j = 0; j < 32; ++j)
             if (32 * h + j < nv && span_ok(err, spans.dv, dv + (row0 + 32 * h + j) * 128 + row, 4))
@@ -392,28 +393,25 @@ bwd_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         for (int j = 0; j < 32; ++j) x[j] = -x[j];
         st_row32(sm + DSP + 2 * TILE, row, 4 * h, x);   // -dR^T, over dS' atom 1
         // dQ = (S dO^T + K^T dP^T)^T
-        tmem_ld32_wait(tm + lane_off + C_DQ + 32 * h, x);
 #pragma unroll
         for (int j = 0; j < 32; ++j)
             if (32 * h + j < nv && span_ok(err, spans.dq, dq + (row0 + 32 * h + j) * 128 + row, 4))
-                dq[(row0 + 32 * h + j) * 128 + row] = x[j];
+                dq[(row0 + 32 * h + j) * 128 + row] = y[j];
         // dT, stored transposed (fp32): dT^T[s][t] for this thread's row t = 16 q + lane
-        tmem_ld32_wait(tm + lane_off + C_SK + 32 * h, x);
         if (lane < 16) {
             const int t = 16 * q + lane;
 #pragma unroll
-            for (int j = 0; j < 32; ++j) fdT[(32 * h + j) * LX + t] = x[j];
+            for (int j = 0; j < 32; ++j) fdT[(32 * h + j) * LX + t] = z[j];
         }
     }
-    {   // X^T (fp32): thread -> a 4 x 4 block
-        const int r4 = 4 * (tid >> 4), c4 = 4 * (tid & 15);
-        float4 xr[4];
+    {   // X^T (fp32): thread -> column c of X, rows 16 rb .. + 15; a warp reads 32 consecutive
+        // columns of a row (one wavefront) and writes 16-byte pieces of 32 rows of X^T that are
+        // LX = 4 (mod 32) words apart (conflict-free)
+        const int c = tid & 63, rb = tid >> 6;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) xr[i] = *reinterpret_cast<const float4*>(fX + (r4 + i) * LX + c4);
-        *reinterpret_cast<float4*>(fXT + (c4 + 0) * LX + r4) = make_float4(xr[0].x, xr[1].x, xr[2].x, xr[3].x);
-        *reinterpret_cast<float4*>(fXT + (c4 + 1) * LX + r4) = make_float4(xr[0].y, xr[1].y, xr[2].y, xr[3].y);
-        *reinterpret_cast<float4*>(fXT + (c4 + 2) * LX + r4) = make_float4(xr[0].z, xr[1].z, xr[2].z, xr[3].z);
-        *reinterpret_cast<float4*>(fXT + (c4 + 3) * LX + r4) = make_float4(xr[0].w, xr[1].w, xr[2].w, xr[3].w);
+        for (int r = 16 * rb; r < 16 * rb + 16; r += 4)
+            *reinterpret_cast<float4*>(fXT + c * LX + r) =
+                make_float4(fX[r * LX + c], fX[(r + 1) * LX + c], fX[(r + 2) * LX + c], fX[(r + 3) * LX + c]);
     }
     handoff();
     // ---- 6. dK^T += S (-dR^T), while the CUDA cores go through T = X diag(alpha)
