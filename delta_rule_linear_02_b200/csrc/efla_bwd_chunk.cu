@@ -85,12 +85,14 @@ constexpr uint32_t FX = 189440;            // X (fp32)
 constexpr uint32_t FXT = TT;               // X^T
 constexpr uint32_t FW = TT + F32;          // W = dX X^T
 constexpr uint32_t FDT = V;                // dT^T, then dX^T, then dA
+constexpr uint32_t FDA2 = FDT + F32;       // dA^T (over dO and the first dS' atom, both dead by then)
 constexpr uint32_t SMALL = FX + F32;       // alpha, beta, dalpha, lambda, (unused), two partial sums (fp32 [64] each)
 constexpr uint32_t BAR = SMALL + 7 * 256;  // mbarriers: the tile's inputs, MMA commits
 constexpr uint32_t MISC = BAR + 6 * 8;     // TMEM base, abort flag
 constexpr uint32_t SMEM_BYTES = MISC + 16 + 1024;
 static_assert(64 * LX * 4 == kUtXBytes, "X as the UT transform writes it");
-static_assert(FDT + F32 <= DSP && FW + F32 <= DG, "fp32 tiles stay inside dead regions");
+static_assert(FDT + F32 <= DSP && FW + F32 <= DG && FDA2 + F32 <= DSP + 2 * TILE,
+              "fp32 tiles stay inside dead regions");
 static_assert(SMEM_BYTES <= 232448, "shared memory");
 // TMEM columns (fp32 accumulators, 64 columns each)
 constexpr uint32_t C_GP = 0, C_SK = 64, C_DQ = 128, C_DL = 192, C_DD = 256, C_DK = 320, C_DR = 384, C_COLS = 512;
@@ -130,18 +132,6 @@ __device__ __forceinline__ uint32_t pack2(float a, float b) {
 __device__ __forceinline__ void st_row32(uint8_t* tile, uint32_t r, uint32_t c0, const float* v) {
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
-        uint4 u;
-        u.x = pack2(v[8 * m], v[8 * m + 1]);
-        u.y = pack2(v[8 * m + 2], v[8 * m + 3]);
-        u.z = pack2(v[8 * m + 4], v[8 * m + 5]);
-        u.w = pack2(v[8 * m + 6], v[8 * m + 7]);
-        *reinterpret_cast<uint4*>(tile + sm100::sw128_off(r, c0 + m)) = u;
-    }
-}
-// 16 floats -> row `r`, chunks c0, c0 + 1
-__device__ __forceinline__ void st_row16(uint8_t* tile, uint32_t r, uint32_t c0, const float* v) {
-#pragma unroll
-    for (int m = 0; m < 2; ++m) {
         uint4 u;
         u.x = pack2(v[8 * m], v[8 * m + 1]);
         u.y = pack2(v[8 * m + 2], v[8 * m + 3]);
@@ -208,6 +198,7 @@ bwd_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     float* fXT = reinterpret_cast<float*>(sm + FXT);
     float* fW = reinterpret_cast<float*>(sm + FW);
     float* fdT = reinterpret_cast<float*>(sm + FDT);
+    float* fdA2 = reinterpret_cast<float*>(sm + FDA2);
     float* al = reinterpret_cast<float*>(sm + SMALL);
     float *bt = al + 64, *dal = al + 128, *lam = al + 192, *part = al + 320;
 
@@ -422,12 +413,15 @@ bwd_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
     // ---- 7. through T = X diag(alpha) and X = (I + A)^{-1}, fp32 on CUDA cores
     {   // dalpha_s = sum_t dT_ts X_ts;  dX^T = diag(alpha) dT^T, in place.  Row s = tid / 4,
-        // a quarter of its 64 entries per thread, the four partial sums added by shuffles.
-        const int srow = tid >> 2, t0q = 16 * (tid & 3);
+        // a quarter of its 64 entries per thread (columns 8 u .. 8 u + 7 and 32 more, u = tid % 4:
+        // the 16-byte pieces of the two rows that 8 lanes touch then fall in 8 different bank
+        // groups), the four partial sums added by shuffles.
+        const int srow = tid >> 2, u = tid & 3;
         const float a = al[srow];
         float sacc = 0.f;
 #pragma unroll
-        for (int t = t0q; t < t0q + 16; t += 4) {
+        for (int i = 0; i < 4; ++i) {
+            const int t = 8 * u + 4 * (i & 1) + 32 * (i >> 1);
             float4 d4 = *reinterpret_cast<const float4*>(fdT + srow * LX + t);
             const float4 x4 = *reinterpret_cast<const float4*>(fXT + srow * LX + t);
             sacc = fmaf(d4.x, x4.x, fmaf(d4.y, x4.y, fmaf(d4.z, x4.z, fmaf(d4.w, x4.w, sacc))));
@@ -464,6 +458,10 @@ bwd_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             const float b0 = cc < rb ? -w[nt][2] : 0.f, b1 = cc + 1 < rb ? -w[nt][3] : 0.f;
             *reinterpret_cast<float2*>(fdT + ra * LX + cc) = make_float2(a0, a1);
             *reinterpret_cast<float2*>(fdT + rb * LX + cc) = make_float2(b0, b1);
+            fdA2[cc * LX + ra] = a0;          // the transpose, for dG^T below (a warp's 32 stores
+            fdA2[(cc + 1) * LX + ra] = a1;    // of one instruction hit 32 different banks)
+            fdA2[cc * LX + rb] = b0;
+            fdA2[(cc + 1) * LX + rb] = b1;
             p0 = fmaf(a0, ld_tok(sm + DG, 0, ra, cc), fmaf(a1, ld_tok(sm + DG, 0, ra, cc + 1), p0));
             p1 = fmaf(b0, ld_tok(sm + DG, 0, rb, cc), fmaf(b1, ld_tok(sm + DG, 0, rb, cc + 1), p1));
         }
@@ -479,15 +477,33 @@ bwd_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
     __syncthreads();
     if (tid < 64) dal[tid] += part[tid] + part[64 + tid];
-    {   // dG + dG^T with dG = diag(alpha) dA, bf16 over G: thread -> row tid / 4, 16 columns
-        const int r = tid >> 2, s0 = 16 * (tid & 3);
-        float x[16];
+    {   // dG + dG^T with dG = diag(alpha) dA (dA strictly lower, zero elsewhere), bf16 over G:
+        // thread -> row r = tid / 4, columns 8 u .. 8 u + 7 and 8 u + 32 .. 8 u + 39 (u = tid % 4),
+        // rows of dA and of dA^T read as 16-byte pieces in 8 different bank groups per 8 lanes
+        const int r = tid >> 2, u = tid & 3;
+        const float ar = al[r];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-            const int s2 = s0 + j;
-            x[j] = (s2 < r ? al[r] * fdT[r * LX + s2] : 0.f) + (r < s2 ? al[s2] * fdT[s2 * LX + r] : 0.f);
+        for (int hlf = 0; hlf < 2; ++hlf) {
+            const int sb0 = 8 * u + 32 * hlf;
+            float x[8];
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                const int s2 = sb0 + 4 * i;
+                const float4 a4 = *reinterpret_cast<const float4*>(fdT + r * LX + s2);    // dA[r][s2 ..]
+                const float4 b4 = *reinterpret_cast<const float4*>(fdA2 + r * LX + s2);   // dA[s2 ..][r]
+                const float4 al4 = *reinterpret_cast<const float4*>(al + s2);
+                x[4 * i] = fmaf(ar, a4.x, al4.x * b4.x);
+                x[4 * i + 1] = fmaf(ar, a4.y, al4.y * b4.y);
+                x[4 * i + 2] = fmaf(ar, a4.z, al4.z * b4.z);
+                x[4 * i + 3] = fmaf(ar, a4.w, al4.w * b4.w);
+            }
+            uint4 w;
+            w.x = pack2(x[0], x[1]);
+            w.y = pack2(x[2], x[3]);
+            w.z = pack2(x[4], x[5]);
+            w.w = pack2(x[6], x[7]);
+            *reinterpret_cast<uint4*>(sm + DG + sm100::sw128_off(r, u + 4 * hlf)) = w;
         }
-        st_row16(sm + DG, r, 2 * (tid & 3), x);
     }
     if (tid < 64) {   // dbeta; the coefficient of k in dk's gate term
         float dadb, dadl;
