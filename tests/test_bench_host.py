@@ -82,3 +82,26 @@ def test_cotangents_are_seeded():
     a, b = workloads.make_cotangents(w), workloads.make_cotangents(w)
     assert (a["dO"] == b["dO"]).all() and (a["dS_T"] == b["dS_T"]).all()
     assert workloads.make_cotangents(w, with_state_grad=False)["dS_T"] is None
+
+
+CSV_BWD = """"ID","Process ID","Process Name","Host Name","Kernel Name","Context","Stream","Block Size","Grid Size","Device","CC","Section Name","Metric Name","Metric Unit","Metric Value"
+"0","1","python","h","void efla::<unnamed>::chunk_tc_kernel<0, 1>(CUtensorMap_st)","1","7","(448, 1, 1)","(128, 1, 1)","0","10.0","Command line profiler metrics","dram__bytes_read.sum","byte","9,000"
+"1","1","python","h","void efla::<unnamed>::bwd_chain_kernel(CUtensorMap_st)","1","7","(320, 1, 1)","(128, 1, 1)","0","10.0","Command line profiler metrics","dram__bytes_read.sum","byte","3,000"
+"1","1","python","h","void efla::<unnamed>::bwd_chain_kernel(CUtensorMap_st)","1","7","(320, 1, 1)","(128, 1, 1)","0","10.0","Command line profiler metrics","dram__bytes_write.sum","byte","300"
+"2","1","python","h","void efla::<unnamed>::bwd_tile_kernel(CUtensorMap_st)","1","7","(256, 1, 1)","(2048, 1, 1)","0","10.0","Command line profiler metrics","dram__bytes_read.sum","byte","4,000"
+"2","1","python","h","void efla::<unnamed>::bwd_tile_kernel(CUtensorMap_st)","1","7","(256, 1, 1)","(2048, 1, 1)","0","10.0","Command line profiler metrics","dram__bytes_write.sum","byte","400"
+"""
+
+
+def test_saved_backward_traffic_counts_only_its_own_kernels(tmp_path, monkeypatch):
+    """The saved-residual backward runs the reverse chain and the per-chunk kernel only: a
+    forward launch in the same log (the one that saved the residuals) is not counted, and the
+    record follows its own, smaller set of kernel sources."""
+    csv = tmp_path / "dram.csv"
+    csv.write_text(CSV_BWD)
+    monkeypatch.setattr(bench, "TRAFFIC_JSON", str(tmp_path / "traffic.json"))
+    rec = bench.traffic_from_csv(str(csv), "efla_backward_saved", calls=1)
+    assert rec["bytes_per_call"] == 3_000 + 300 + 4_000 + 400 and rec["launches"] == 2
+    assert rec["kernels"] == ["bwd_chain_kernel", "bwd_tile_kernel"]
+    assert bench.ncu_traffic("efla_backward_saved") == rec["bytes_per_call"]
+    assert set(bench.KERNEL_SOURCES["efla_backward_saved"]) < set(bench.KERNEL_SOURCES["efla_backward"])
